@@ -1,0 +1,204 @@
+/*
+ * pagedattn — single-token decode attention over a paged KV cache, for
+ * NVIDIA B200 (sm_100a).  C ABI of libpagedattn.so.
+ *
+ * The method (all citations are to the surveyed web pages):
+ *  - "KV-Cache Optimization Techniques", section "PagedAttention (vLLM)":
+ *    the cache is kept in fixed-size pages of P tokens in one physical pool;
+ *    each request has a page table mapping its logical KV positions to
+ *    physical pages; pages are allocated on demand. Eq. (1): attention for
+ *    the current query token is softmax(q [K_page1; ...; K_pagen]^T / sqrt(d_k))
+ *    times [V_page1; ...; V_pagen], i.e. ordinary attention over the
+ *    gathered pages.
+ *  - same page, section "Multi-Query and Grouped-Query Caching", Eq. (7):
+ *    H query heads share G groups of K/V; here query head hq reads KV head
+ *    hq / (Hq / Hkv).
+ *  - same page, section "KV-Cache Quantization", Eq. (3): per-token INT8
+ *    codes with one scale/zero-point per row of K or V.
+ *  - same page, section "Prefix Caching": requests that share a prefix point
+ *    their tables at the same physical pages; results must not depend on
+ *    which physical pages a table names ("Understanding KV-Cache Optimization
+ *    in Modern LLM Serving", section "PagedAttention Solution": paging does
+ *    not change the model's output).
+ *
+ * Conventions for every entry point
+ *  - Pointers marked (device) are CUDA device pointers owned by the caller;
+ *    the library allocates nothing, keeps no mutable global state and never
+ *    synchronises a stream. `stream` is a cudaStream_t passed as void*
+ *    (NULL = legacy default stream). Calls are asynchronous on that stream.
+ *  - Host-side checks run before any launch; a failed check returns an error
+ *    status and launches nothing. pa_last_error() then gives a message
+ *    (per host thread).
+ *  - Device-side checks never trap: a kernel that meets a table entry outside
+ *    the pool, an out-of-range context length, sequence index or position
+ *    skips that data (it is neither read nor written) and ORs a PA_DERR_*
+ *    bit into *d_err when d_err is not NULL.
+ */
+#ifndef PAGEDATTN_H
+#define PAGEDATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PA_ABI_VERSION 1
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,  /* null pointer, negative size, mismatched shapes  */
+  PA_ERR_UNSUPPORTED = 2,  /* shape outside the compiled set (D, P, G, dtype)  */
+  PA_ERR_WORKSPACE = 3,    /* workspace too small or misaligned                */
+  PA_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed             */
+  PA_ERR_BAD_TABLE = 5     /* reserved for callers that read d_err back        */
+} pa_status_t;
+
+/* Bits a kernel ORs into *d_err (device int32) when it skips bad input. */
+#define PA_DERR_BAD_PAGE 1 /* a needed table entry is outside [0, num_pages)  */
+#define PA_DERR_BAD_CTX 2  /* context_len < 0 or > max_pages * page_size       */
+#define PA_DERR_BAD_SEQ 4  /* append: seq_idx outside [0, num_seqs)            */
+#define PA_DERR_BAD_POS 8  /* append: pos < 0 or pos / page_size >= max_pages  */
+
+typedef enum {
+  PA_KV_BF16 = 0,         /* K/V stored as bf16                               */
+  PA_KV_U8_PER_TOKEN = 1  /* Eq. (3): uint8 codes + fp32 (scale, zero) per row */
+} pa_kv_dtype_t;
+
+/*
+ * The physical page pool ("PagedAttention (vLLM)", "Architecture").
+ * Layout of one tensor (K or V): [num_pages][num_kv_heads][page_size][head_dim],
+ * row-major, so the page_size x head_dim block of one (page, KV head) is
+ * contiguous. bf16 pools hold 2-byte elements, INT8 pools 1-byte codes plus
+ * k_sz / v_sz = fp32 [num_pages][num_kv_heads][page_size][2] holding
+ * (scale, zero) of each row. Every pointer must be 16-byte aligned.
+ * Supported: page_size in {16, 32}; head_dim in {64, 128}.
+ */
+typedef struct {
+  int32_t num_pages;
+  int32_t page_size;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int32_t dtype;      /* pa_kv_dtype_t */
+  void *k_pool;       /* (device) */
+  void *v_pool;       /* (device) */
+  float *k_sz;        /* (device) INT8 only, else NULL */
+  float *v_sz;        /* (device) INT8 only, else NULL */
+} pa_kv_pool_t;
+
+/*
+ * pa_kv_append — write new tokens' K/V rows into their page slots.
+ * ("PagedAttention (vLLM)", "Architecture": logical position -> physical page
+ * through the request's page table; pages are allocated by the caller on
+ * demand. For an INT8 pool each row is quantised on the way in by Eq. (3):
+ * z = min of the row, s = (max - min) / 255, code = round-half-even((x - z)/s)
+ * clamped to [0, 255], all in IEEE fp32; a constant row stores s = 0, codes 0.
+ * Input rows must be finite; -0 is stored as +0.)
+ *
+ *   k_new, v_new : (device) bf16 [num_tokens][num_kv_heads][head_dim]
+ *   seq_idx, pos : (device) int32 [num_tokens]; token i is position pos[i]
+ *                  (0-based) of sequence seq_idx[i]
+ *   block_tables : (device) int32 [num_seqs][max_pages]
+ * Row i goes to page block_tables[seq_idx[i]][pos[i] / P], slot pos[i] % P.
+ * Two tokens that name the same slot race (the caller must not do that);
+ * writing into a page shared by several tables changes all of them
+ * (copy-on-write is the caller's job). num_tokens == 0 is a no-op.
+ */
+pa_status_t pa_kv_append(const pa_kv_pool_t *pool, const void *k_new,
+                         const void *v_new, const int32_t *seq_idx,
+                         const int32_t *pos, int32_t num_tokens,
+                         const int32_t *block_tables, int32_t num_seqs,
+                         int32_t max_pages, int32_t *d_err, void *stream);
+
+/*
+ * pa_decode_num_splits — the split-KV partition count pa_decode uses.
+ * requested > 0 is clamped to [1, max_pages]; requested == 0 picks one from
+ * the number of (sequence, KV head) units, the table width and the current
+ * device's SM count. Split s covers logical pages
+ * [s * ceil(max_pages / S), (s + 1) * ceil(max_pages / S)) of every sequence.
+ * Returns <= 0 on invalid arguments.
+ */
+int32_t pa_decode_num_splits(int32_t num_seqs, int32_t num_kv_heads,
+                             int32_t max_pages, int32_t page_size,
+                             int32_t requested);
+
+/*
+ * pa_decode_workspace_bytes — device scratch pa_decode needs for
+ * num_splits (already resolved, >= 1): 0 when num_splits == 1, else the
+ * partial outputs fp32 [num_seqs][num_q_heads][num_splits][head_dim] plus
+ * their log-sum-exps fp32 [num_seqs][num_q_heads][num_splits], each part
+ * 256-byte aligned.
+ */
+size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
+                                 int32_t head_dim, int32_t num_splits);
+
+/*
+ * pa_decode — Eq. (1) for one query token per sequence.
+ *
+ *   q            : (device) bf16 [num_seqs][num_q_heads][head_dim]
+ *   block_tables : (device) int32 [num_seqs][max_pages]; entries at or past
+ *                  ceil(context_lens[b] / P) are never read
+ *   context_lens : (device) int32 [num_seqs]; tokens 0..ctx-1 are attended
+ *                  (the token appended for this step included, no mask)
+ *   scale        : multiplies q.k (1 / sqrt(head_dim) for Eq. (1))
+ *   out          : (device) fp32 [num_seqs][num_q_heads][head_dim]
+ *   workspace    : (device) >= pa_decode_workspace_bytes(...) bytes, 256-byte
+ *                  aligned; may be NULL when that is 0
+ *   num_splits   : 0 = automatic (pa_decode_num_splits), else the split count
+ * num_q_heads must be a multiple of pool->num_kv_heads with a ratio of 1..8.
+ * A sequence with context length 0 gets out = 0. When more than one split is
+ * used the partial results are merged by their log-sum-exp in a second
+ * kernel on the same stream (pa_splitkv_reduce). Results are deterministic
+ * and do not depend on the physical page ids.
+ */
+pa_status_t pa_decode(const pa_kv_pool_t *pool, const void *q,
+                      int32_t num_seqs, int32_t num_q_heads,
+                      const int32_t *block_tables, int32_t max_pages,
+                      const int32_t *context_lens, float scale, float *out,
+                      void *workspace, size_t workspace_bytes,
+                      int32_t num_splits, int32_t *d_err, void *stream);
+
+/*
+ * pa_splitkv_reduce — merge split-KV partial results.
+ * (Not on the pages: the exact identity for softmax over disjoint token
+ * ranges. With M = max_s lse_s and w_s = exp(lse_s - M):
+ * out = sum_s w_s o_s / sum_s w_s; a split with lse = -inf has weight 0 and
+ * if every split is empty out = 0.)
+ *   o_part : (device) fp32 [num_seqs][num_q_heads][num_splits][head_dim],
+ *            each o_s already normalised by its own softmax sum
+ *   lse    : (device) fp32 [num_seqs][num_q_heads][num_splits], natural log
+ *            of the split's sum of exp(scale * q.k)
+ *   out    : (device) fp32 [num_seqs][num_q_heads][head_dim]
+ * head_dim must be a multiple of 4 and at most 512; num_splits in [1, 256].
+ */
+pa_status_t pa_splitkv_reduce(const float *o_part, const float *lse,
+                              int32_t num_seqs, int32_t num_q_heads,
+                              int32_t num_splits, int32_t head_dim, float *out,
+                              void *stream);
+
+/*
+ * pa_validate_tables — check the page tables a decode would read.
+ * For each sequence: 0 <= context_lens[b] <= max_pages * page_size, and every
+ * entry in [0, ceil(ctx / page_size)) lies in [0, num_pages). Violations set
+ * PA_DERR_BAD_CTX / PA_DERR_BAD_PAGE in *d_err (device int32, required);
+ * the word is OR-ed into, not cleared. Asynchronous like everything else.
+ */
+pa_status_t pa_validate_tables(const int32_t *block_tables, int32_t num_seqs,
+                               int32_t max_pages, const int32_t *context_lens,
+                               int32_t num_pages, int32_t page_size,
+                               int32_t *d_err, void *stream);
+
+/* Static description of a status code. */
+const char *pa_status_str(pa_status_t status);
+
+/* Message describing the last failed call on this host thread ("" if none). */
+const char *pa_last_error(void);
+
+/* PA_ABI_VERSION of the loaded library. */
+int32_t pa_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PAGEDATTN_H */

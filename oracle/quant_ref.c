@@ -13,6 +13,9 @@
  *     code = clamp(round_half_even((x - z) / s), 0, 255),
  * with every step in IEEE fp32, round-to-nearest-even, in exactly this order,
  * and a row whose max equals its min stored as s = 0, z = min, codes 0.
+ * Signed zero is left open by the pages; -0 and +0 are the same number, so
+ * each input is read as x + 0.0f (which turns -0 into +0 and changes nothing
+ * else) and the stored (s, z) have a single bit pattern.
  * Build with -ffp-contract=off and no fast-math so the compiler keeps the
  * subtraction and the division as two rounded fp32 operations.
  */
@@ -24,7 +27,7 @@ static float bf16_bits_to_f32(uint16_t b) {
   uint32_t u = ((uint32_t)b) << 16;
   float f;
   memcpy(&f, &u, sizeof f);
-  return f;
+  return f + 0.0f; /* -0 -> +0 */
 }
 
 /* x: [n_rows][d] bf16 bits.  codes: [n_rows][d].  sz: [n_rows][2] (s, z). */

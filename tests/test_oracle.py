@@ -284,6 +284,14 @@ def test_quantiser_constant_row():
     assert sz[0, 0] == 0.0 and sz[0, 1] == 3.25 and np.all(codes == 0)
 
 
+def test_quantiser_signed_zero_has_one_pattern():
+    """A row whose minimum is a zero stores z = +0 whatever the zero's sign,
+    and an all-zero row stores s = +0."""
+    for vals in ([-0.0, 0.0, 1.0, 2.0], [0.0, -0.0, 1.0, 2.0], [-0.0] * 4, [0.0, -0.0] * 2):
+        codes, sz = oracle.quantize_rows(_row_bits(vals))
+        assert sz.view(np.uint32)[0, 1] == 0 and sz.view(np.uint32)[0, 0] in (0, np.float32(2 / 255).view(np.uint32))
+
+
 def test_quantiser_endpoints_and_round_trip_bound():
     """min -> code 0, max -> code 255, and |x - (s*code + z)| <= s/2 up to
     fp32 rounding of the ratio (255 ulp-sized steps at most)."""
