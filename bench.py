@@ -1,0 +1,428 @@
+#!/usr/bin/env python
+"""Decode-attention benchmark on B200: one step = append this step's token per
+sequence into the paged cache (pa_kv_append) + paged decode attention
+(pa_decode, with its split-KV merge) over the whole batch.
+
+Workload (default): the Llama-3-70B-shaped single layer — B=32 sequences of
+8192 tokens, Hq=64, Hkv=8, D=128, bf16, pages of P=32 tokens randomly permuted
+over an 8192-page pool (1.07 GB of K/V, larger than the 126 MB L2, so no L2
+flush is needed between steps). Inputs are seeded synthetic data (seed = rank).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the CPU oracle as the reference arm
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own batch
+(weak scaling) — the sequences are independent, so there is no data-path
+collective; only the timing uses a barrier and a max over ranks.
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attention achieved HBM GB/s and % of B200 peak; sequences/sec per layer"
+FALLBACK_HBM_GBS = 6650.0
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+DECODE_SRC = os.path.join(ROOT, "paged_kv_cache_466_b200", "csrc", "decode.cu")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="llama70b",
+                    choices=["llama70b", "llama8b", "int8", "prefix", "tiny"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--splits", type=int, default=0, help="split-KV count (0 = automatic)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ accounting
+def decode_bytes(w) -> int:
+    """Algorithmic bytes of one decode: every cached K/V element of every
+    attended token once, plus q (Eq. 1 reads nothing else)."""
+    tok = int(w.context_lens.astype("int64").sum())
+    per_tok = w.Hkv * 2 * (w.D * 2 if w.kv == "bf16" else w.D + 8)
+    return tok * per_tok + w.B * w.Hq * w.D * 2
+
+
+def append_bytes(w) -> int:
+    n = len(w.step_seq)
+    row = w.D * 2 if w.kv == "bf16" else w.D + 8
+    return n * w.Hkv * 2 * (w.D * 2 + row)
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def recorded_traffic(workload: str):
+    """ncu DRAM bytes per decode launch, if recorded for the current kernel source."""
+    try:
+        rec = json.load(open(TRAFFIC_FILE))
+        src_sha = hashlib.sha256(open(DECODE_SRC, "rb").read()).hexdigest()
+        r = rec.get(workload)
+        if r and r.get("decode_cu_sha256") == src_sha:
+            return int(r["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """NVML sampling of SM clock and clock-event reasons (read-only)."""
+    NAMES = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+             0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+             0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+             0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.ok = False
+        self.samples, self.reasons = [], 0
+        self.period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            uuid = None
+            try:
+                import torch
+                uuid = str(torch.cuda.get_device_properties(index).uuid)
+            except Exception:
+                pass
+            h = None
+            if uuid:
+                for i in range(pynvml.nvmlDeviceGetCount()):
+                    hh = pynvml.nvmlDeviceGetHandleByIndex(i)
+                    u = pynvml.nvmlDeviceGetUUID(hh)
+                    u = u.decode() if isinstance(u, bytes) else u
+                    if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                        h = hh
+                        break
+            self.h = h if h is not None else pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _read(self):
+        nv = self.nv
+        mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+        try:
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        self.samples.append(mhz)
+        self.reasons |= int(r)
+
+    def _loop(self):
+        while not self._stop.is_set():
+            try:
+                self._read()
+            except Exception:
+                pass
+            self._stop.wait(self.period)
+
+    def start(self):
+        if not self.ok:
+            return
+        self._stop = threading.Event()
+        self._t = threading.Thread(target=self._loop, daemon=True)
+        self._t.start()
+
+    def stop(self):
+        if not self.ok:
+            return None
+        self._stop.set()
+        self._t.join()
+        try:
+            self._read()
+        except Exception:
+            pass
+        names = [n for b, n in self.NAMES.items() if self.reasons & b]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ CPU oracle leg
+def cpu_oracle_throughput(w, budget_s: float = 12.0, max_reps: int = 8):
+    """The fp64 oracle, as it stands, on this host's cores: the whole batch,
+    repeated until ~budget_s of work. Returns (GB/s, cores, sample text)."""
+    cores = len(os.sched_getaffinity(0))
+    os.environ.setdefault("OMP_NUM_THREADS", str(cores))
+    import oracle
+    from paged_kv_cache_466_b200.workloads import bits
+    hp = oracle.empty_pool(w.kv, w.num_pages, w.Hkv, w.P, w.D, 0)
+    seq, pos, k, v = w.all_rows()
+    oracle.scatter_rows(hp, w.block_tables, seq, pos, bits(k), bits(v))
+    qb = bits(w.q)
+    reps, t_total = 0, 0.0
+    while reps < max_reps and (t_total < budget_s or reps == 0):
+        t0 = time.perf_counter()
+        oracle.paged_attention(hp, qb, w.block_tables, w.context_lens, w.scale)
+        t_total += time.perf_counter() - t0
+        reps += 1
+    gbs = decode_bytes(w) * reps / t_total / 1e9
+    sample = (f"{reps} full decode(s) of the {w.name} batch ({w.B} seqs x {w.Hq} heads), "
+              f"{t_total:.1f} s total; attention only (no cache write)")
+    return gbs, cores, sample
+
+
+# ------------------------------------------------------------------ arms
+def make_workload(name: str, seed: int):
+    from paged_kv_cache_466_b200 import workloads as W
+    if name == "prefix":
+        return W.prefix(seed=seed)[0]
+    if name == "tiny":
+        return W.tiny(seed=seed)
+    return getattr(W, name)(seed=seed)
+
+
+def config_of(w, args, n, S):
+    c = {"workload": f"{w.name}: B={w.B}, ctx={'U' if len(set(w.context_lens.tolist())) > 1 else ''}"
+                     f"{int(w.context_lens.min())}..{int(w.context_lens.max())}, Hq={w.Hq}, "
+                     f"Hkv={w.Hkv}, D={w.D}, P={w.P}, kv={w.kv}",
+         "global_batch": w.B * n, "seq_len": int(w.context_lens.max()),
+         "parallelism": f"dp{n} (independent sequences, no collective)",
+         "num_splits": S, "pool_pages": w.num_pages,
+         "l2": "inputs larger than the 126 MB L2, not flushed" if decode_bytes(w) > 256e6
+               else "L2 not flushed (working set may be L2-resident)"}
+    return c
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from paged_kv_cache_466_b200 import (KVPool, pa_decode, pa_decode_num_splits,
+                                         pa_decode_workspace_bytes, pa_kv_append)
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = make_workload(args.workload, seed=rank)
+    pool = KVPool(w.num_pages, w.Hkv, w.P, w.D, w.kv, dev, fill_byte=0)
+    bt = torch.from_numpy(w.block_tables).to(dev)
+    ctx = torch.from_numpy(w.context_lens).to(dev)
+    q = w.q.to(dev)
+    chunk = 1 << 18
+    for a in range(0, len(w.prefill_seq), chunk):
+        b = min(a + chunk, len(w.prefill_seq))
+        pa_kv_append(pool, w.prefill_k[a:b].to(dev), w.prefill_v[a:b].to(dev),
+                     torch.from_numpy(w.prefill_seq[a:b]).to(dev),
+                     torch.from_numpy(w.prefill_pos[a:b]).to(dev), bt)
+    sk, sv = w.step_k.to(dev), w.step_v.to(dev)
+    sseq = torch.from_numpy(w.step_seq).to(dev)
+    spos = torch.from_numpy(w.step_pos).to(dev)
+    S = pa_decode_num_splits(pool, w.B, w.max_pages, args.splits)
+    ws = torch.empty(max(pa_decode_workspace_bytes(w.B, w.Hq, w.D, S), 256), dtype=torch.uint8,
+                     device=dev)
+    out = torch.empty((w.B, w.Hq, w.D), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev0=None, ev1=None):
+        pa_kv_append(pool, sk, sv, sseq, spos, bt)
+        if ev0 is not None:
+            ev0.record(stream)
+        pa_decode(pool, q, bt, ctx, w.scale, out=out, workspace=ws, num_splits=S)
+        if ev1 is not None:
+            ev1.record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- device-resident timed region
+    K = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t0.record(stream)
+    for i in range(K):
+        step(*evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier()
+    ms = t0.elapsed_time(t1)
+    dec_ms = [a.elapsed_time(b) for a, b in evs]
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    ms_step = ms / K
+    step_bytes = decode_bytes(w) + append_bytes(w)
+    value = step_bytes * world / (ms_step * 1e-3) / 1e9
+
+    # ---- end to end through the public API, host buffers in pinned memory
+    h_q = w.q.pin_memory()
+    h_k, h_v = w.step_k.pin_memory(), w.step_v.pin_memory()
+    h_seq = torch.from_numpy(w.step_seq).pin_memory()
+    h_pos = torch.from_numpy(w.step_pos).pin_memory()
+    h_ctx = torch.from_numpy(w.context_lens).pin_memory()
+    h_bt = torch.from_numpy(w.block_tables).pin_memory()
+    h_out = torch.empty((w.B, w.Hq, w.D), dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_seq, h_pos, h_ctx, h_bt))
+    d2h = h_out.numel() * h_out.element_size()
+    d_q, d_k, d_v = torch.empty_like(q), torch.empty_like(sk), torch.empty_like(sv)
+    d_seq, d_pos = torch.empty_like(sseq), torch.empty_like(spos)
+    d_ctx, d_bt = torch.empty_like(ctx), torch.empty_like(bt)
+
+    def e2e_step():
+        for d, h in ((d_q, h_q), (d_k, h_k), (d_v, h_v), (d_seq, h_seq), (d_pos, h_pos),
+                     (d_ctx, h_ctx), (d_bt, h_bt)):
+            d.copy_(h, non_blocking=True)
+        pa_kv_append(pool, d_k, d_v, d_seq, d_pos, d_bt)
+        pa_decode(pool, d_q, d_bt, d_ctx, w.scale, out=out, workspace=ws, num_splits=S)
+        h_out.copy_(out, non_blocking=True)
+        stream.synchronize()   # the caller reads the result every step
+
+    for _ in range(max(args.warmup, 3)):
+        e2e_step()
+    Ke = min(K, 500)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(Ke):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ems = e0.elapsed_time(e1)
+    if world > 1:
+        tt = torch.tensor([ems], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ems = float(tt.item())
+    e2e_value = step_bytes * world / (ems / Ke * 1e-3) / 1e9
+
+    peak, peak_kind = measured_peak()
+    dec_avg_ms = statistics.mean(dec_ms)
+    achieved = decode_bytes(w) / (dec_avg_ms * 1e-3) / 1e9
+    traffic = recorded_traffic(w.name)
+    launches_per_step = 2 + (1 if S > 1 else 0)
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16"
+        if w.kv == "bf16" else "u8 codes, fp32 scale/zero; fp32 accumulate",
+        "data": "synthetic (seeded N(0,1) bf16 K/V/q; no weights needed)",
+        "config": config_of(w, args, world, S),
+        "pct_of_peak": round(100.0 * value / world / peak, 2),
+        "peak_gbs": peak, "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+        if peak_kind == "measured" else "fallback 6.65 TB/s",
+        "seq_per_s_per_layer": round(w.B * world / (ms_step * 1e-3), 1),
+        "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": Ke,
+                "ms_per_step": round(ems / Ke, 5)},
+        "roofline": {"bound": "hbm", "kernel": "pa_decode (decode kernel + split merge)",
+                     "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "algorithmic_bytes": decode_bytes(w),
+                     "avg_launch_ms": round(dec_avg_ms, 5)},
+        "gpu_launches": K * launches_per_step,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, cores, sample = cpu_oracle_throughput(w)
+        res["cpu_baseline"] = {"value": round(gbs, 3), "unit": "GB/s", "cores": cores,
+                               "kind": "oracle", "sample": sample}
+    return res
+
+
+def run_reference(args, rank, world):
+    """The CPU oracle as the reference arm: every step a bounded sample of the
+    workload (a fixed set of (sequence, head) rows), timed on the host cores."""
+    import numpy as np
+    if rank != 0:
+        return None
+    cores = len(os.sched_getaffinity(0))
+    os.environ.setdefault("OMP_NUM_THREADS", str(cores))
+    import oracle
+    from paged_kv_cache_466_b200.workloads import bits
+    w = make_workload(args.workload, seed=0)
+    hp = oracle.empty_pool(w.kv, w.num_pages, w.Hkv, w.P, w.D, 0)
+    seq, pos, k, v = w.all_rows()
+    oracle.scatter_rows(hp, w.block_tables, seq, pos, bits(k), bits(v))
+    qb = bits(w.q)
+    # calibrate: rows per step so the whole run takes about 90 s
+    pairs_all = [(b, h) for b in range(w.B) for h in range(w.Hq)]
+    t0 = time.perf_counter()
+    oracle.paged_attention(hp, qb, w.block_tables, w.context_lens, w.scale, pairs=pairs_all[:w.Hq])
+    per_pair = max((time.perf_counter() - t0) / w.Hq, 1e-6)
+    budget = 90.0 / max(args.steps + args.warmup, 1)
+    n = int(min(len(pairs_all), max(1, budget / per_pair)))
+    sample = pairs_all[:n]
+    tok = sum(int(w.context_lens[b]) for b, _ in sample)
+    per_tok = 2 * (w.D * 2 if w.kv == "bf16" else w.D + 8)
+    sample_bytes = tok * per_tok // w.G + n * w.D * 2     # K/V rows are shared by G heads
+    for _ in range(args.warmup):
+        oracle.paged_attention(hp, qb, w.block_tables, w.context_lens, w.scale, pairs=sample)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.paged_attention(hp, qb, w.block_tables, w.context_lens, w.scale, pairs=sample)
+    dt = (time.perf_counter() - t0) / max(args.steps, 1)
+    value = sample_bytes / dt / 1e9
+    desc = (f"{n} (sequence, query head) rows of the {w.name} batch per step "
+            f"({n / len(pairs_all):.1%} of a decode), fp64, OpenMP")
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+            "config": config_of(w, args, 1, 1),
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores,
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    import torch.distributed as dist
+    from datetime import timedelta
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=180))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -112,16 +112,19 @@ pa_status_t pa_kv_append(const pa_kv_pool_t *pool, const void *k_new,
                          int32_t max_pages, int32_t *d_err, void *stream);
 
 /*
- * pa_decode_num_splits — the split-KV partition count pa_decode uses.
- * requested > 0 is clamped to [1, max_pages]; requested == 0 picks one from
- * the number of (sequence, KV head) units, the table width and the current
- * device's SM count. Split s covers logical pages
- * [s * ceil(max_pages / S), (s + 1) * ceil(max_pages / S)) of every sequence.
- * Returns <= 0 on invalid arguments.
+ * pa_decode_num_splits — the split-KV partition count S pa_decode uses for
+ * this pool shape, table width and request. requested == 0 picks S from the
+ * number of (sequence, KV head) units, the table width and how many decode
+ * CTAs fit on the current device; requested > 0 is honoured as far as the
+ * limits allow. Either way S is then clamped to [1, min(max_pages, 256)],
+ * raised to at least ceil(max_pages / 2048) (a split stages at most 2048
+ * table entries), and reduced so no split is empty by construction:
+ * with C = ceil(max_pages / S), split s covers logical pages [s*C, (s+1)*C)
+ * and S = ceil(max_pages / C). Only pool->num_kv_heads, page_size,
+ * head_dim and dtype are read. Returns <= 0 on invalid arguments.
  */
-int32_t pa_decode_num_splits(int32_t num_seqs, int32_t num_kv_heads,
-                             int32_t max_pages, int32_t page_size,
-                             int32_t requested);
+int32_t pa_decode_num_splits(const pa_kv_pool_t *pool, int32_t num_seqs,
+                             int32_t max_pages, int32_t requested);
 
 /*
  * pa_decode_workspace_bytes — device scratch pa_decode needs for
@@ -145,7 +148,8 @@ size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
  *   out          : (device) fp32 [num_seqs][num_q_heads][head_dim]
  *   workspace    : (device) >= pa_decode_workspace_bytes(...) bytes, 256-byte
  *                  aligned; may be NULL when that is 0
- *   num_splits   : 0 = automatic (pa_decode_num_splits), else the split count
+ *   num_splits   : 0 = automatic; the count actually used is always
+ *                  pa_decode_num_splits(pool, num_seqs, max_pages, num_splits)
  * num_q_heads must be a multiple of pool->num_kv_heads with a ratio of 1..8.
  * A sequence with context length 0 gets out = 0. When more than one split is
  * used the partial results are merged by their log-sum-exp in a second

@@ -1,0 +1,189 @@
+"""pagedattn for B200: paged KV-cache decode attention behind a C ABI.
+
+The Python layer only marshals arguments: it takes torch tensors, passes their
+device pointers and torch's current CUDA stream to ``libpagedattn.so``, and
+raises on a non-OK status. Every step of the computation runs in the library's
+CUDA kernels; there is no Python or CPU fallback.
+
+Entry points (same names as the C ABI, see include/pagedattn.h):
+
+* ``pa_kv_append``       — write new tokens' K/V into their page slots
+                           (quantising for an INT8 pool, Eq. 3)
+* ``pa_decode``          — Eq. 1 decode attention over the paged cache
+* ``pa_splitkv_reduce``  — log-sum-exp merge of split-KV partials
+* ``pa_validate_tables`` — device-side page-table check
+* ``pa_decode_num_splits`` / ``pa_decode_workspace_bytes`` — planning helpers
+
+``KVPool`` owns the page pool tensors; ``pages`` holds the host-side page
+allocator and cache-size formulas.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import (PA_DERR_BAD_CTX, PA_DERR_BAD_PAGE, PA_DERR_BAD_POS, PA_DERR_BAD_SEQ,
+                   PA_KV_BF16, PA_KV_U8_PER_TOKEN, PagedAttnError, pa_kv_pool_t)
+
+__all__ = ["KVPool", "pa_kv_append", "pa_decode", "pa_splitkv_reduce", "pa_validate_tables",
+           "pa_decode_num_splits", "pa_decode_workspace_bytes", "PagedAttnError",
+           "PA_KV_BF16", "PA_KV_U8_PER_TOKEN", "PA_DERR_BAD_PAGE", "PA_DERR_BAD_CTX",
+           "PA_DERR_BAD_SEQ", "PA_DERR_BAD_POS", "load_library"]
+
+
+def load_library() -> ctypes.CDLL:
+    return _lib.load()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype, device=None):
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+
+
+class KVPool:
+    """The physical page pool: K and V as [num_pages, Hkv, P, D] tensors
+    (bf16, or uint8 codes plus fp32 [num_pages, Hkv, P, 2] scale/zero)."""
+
+    def __init__(self, num_pages: int, num_kv_heads: int, page_size: int, head_dim: int,
+                 dtype: str = "bf16", device="cuda", fill_byte: Optional[int] = None):
+        self.num_pages, self.num_kv_heads = num_pages, num_kv_heads
+        self.page_size, self.head_dim = page_size, head_dim
+        self.kind = dtype
+        shape = (num_pages, num_kv_heads, page_size, head_dim)
+        tdt = {"bf16": torch.bfloat16, "u8": torch.uint8}[dtype]
+        self.k = torch.empty(shape, dtype=tdt, device=device)
+        self.v = torch.empty(shape, dtype=tdt, device=device)
+        self.k_sz = self.v_sz = None
+        if dtype == "u8":
+            self.k_sz = torch.empty(shape[:3] + (2,), dtype=torch.float32, device=device)
+            self.v_sz = torch.empty(shape[:3] + (2,), dtype=torch.float32, device=device)
+        if fill_byte is not None:
+            for t in self.tensors():
+                t.view(torch.uint8).fill_(fill_byte)
+        self._c = pa_kv_pool_t(num_pages, page_size, num_kv_heads, head_dim,
+                               PA_KV_BF16 if dtype == "bf16" else PA_KV_U8_PER_TOKEN,
+                               self.k.data_ptr(), self.v.data_ptr(),
+                               None if self.k_sz is None else self.k_sz.data_ptr(),
+                               None if self.v_sz is None else self.v_sz.data_ptr())
+
+    def tensors(self):
+        return [t for t in (self.k, self.v, self.k_sz, self.v_sz) if t is not None]
+
+    @property
+    def c(self) -> pa_kv_pool_t:
+        return self._c
+
+    @property
+    def device(self):
+        return self.k.device
+
+
+def pa_decode_num_splits(pool: KVPool, num_seqs: int, max_pages: int, requested: int = 0) -> int:
+    s = _lib.load().pa_decode_num_splits(ctypes.byref(pool.c), num_seqs, max_pages, requested)
+    if s <= 0:
+        raise ValueError("pa_decode_num_splits: invalid arguments")
+    return s
+
+
+def pa_decode_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int,
+                              num_splits: int) -> int:
+    return int(_lib.load().pa_decode_workspace_bytes(num_seqs, num_q_heads, head_dim, num_splits))
+
+
+def pa_kv_append(pool: KVPool, k_new: torch.Tensor, v_new: torch.Tensor, seq_idx: torch.Tensor,
+                 pos: torch.Tensor, block_tables: torch.Tensor,
+                 d_err: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Write rows k_new/v_new [N, Hkv, D] (bf16) of token (seq_idx[i], pos[i])."""
+    dev = pool.device
+    _need(k_new, "k_new", torch.bfloat16, dev)
+    _need(v_new, "v_new", torch.bfloat16, dev)
+    _need(seq_idx, "seq_idx", torch.int32, dev)
+    _need(pos, "pos", torch.int32, dev)
+    _need(block_tables, "block_tables", torch.int32, dev)
+    n = seq_idx.numel()
+    if k_new.shape != (n, pool.num_kv_heads, pool.head_dim) or v_new.shape != k_new.shape \
+            or pos.numel() != n:
+        raise ValueError("pa_kv_append: shape mismatch")
+    st = _lib.load().pa_kv_append(ctypes.byref(pool.c), _ptr(k_new), _ptr(v_new), _ptr(seq_idx),
+                                  _ptr(pos), n, _ptr(block_tables), block_tables.shape[0],
+                                  block_tables.shape[1], _ptr(d_err), _stream(stream))
+    _lib.check(st, "pa_kv_append")
+
+
+def pa_decode(pool: KVPool, q: torch.Tensor, block_tables: torch.Tensor,
+              context_lens: torch.Tensor, scale: float, out: Optional[torch.Tensor] = None,
+              workspace: Optional[torch.Tensor] = None, num_splits: int = 0,
+              d_err: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Eq. 1 decode: q [B, Hq, D] bf16 -> out [B, Hq, D] fp32.
+
+    ``workspace`` (uint8, >= pa_decode_workspace_bytes) is allocated with torch
+    when not given.
+    """
+    dev = pool.device
+    _need(q, "q", torch.bfloat16, dev)
+    _need(block_tables, "block_tables", torch.int32, dev)
+    _need(context_lens, "context_lens", torch.int32, dev)
+    B, Hq, D = q.shape
+    if D != pool.head_dim or block_tables.shape[0] != B or context_lens.numel() != B:
+        raise ValueError("pa_decode: shape mismatch")
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    _need(out, "out", torch.float32, dev)
+    max_pages = block_tables.shape[1]
+    S = pa_decode_num_splits(pool, B, max_pages, num_splits)
+    need = pa_decode_workspace_bytes(B, Hq, D, S)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _lib.load().pa_decode(ctypes.byref(pool.c), _ptr(q), B, Hq, _ptr(block_tables),
+                               max_pages, _ptr(context_lens), float(scale), _ptr(out),
+                               _ptr(workspace), ws_bytes, num_splits, _ptr(d_err),
+                               _stream(stream))
+    _lib.check(st, "pa_decode")
+    return out
+
+
+def pa_splitkv_reduce(o_part: torch.Tensor, lse: torch.Tensor,
+                      out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Merge partials o_part [B, Hq, S, D] with lse [B, Hq, S] -> [B, Hq, D]."""
+    _need(o_part, "o_part", torch.float32)
+    _need(lse, "lse", torch.float32, o_part.device)
+    B, Hq, S, D = o_part.shape
+    if lse.shape != (B, Hq, S):
+        raise ValueError("pa_splitkv_reduce: shape mismatch")
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=o_part.device)
+    _need(out, "out", torch.float32, o_part.device)
+    st = _lib.load().pa_splitkv_reduce(_ptr(o_part), _ptr(lse), B, Hq, S, D, _ptr(out),
+                                       _stream(stream))
+    _lib.check(st, "pa_splitkv_reduce")
+    return out
+
+
+def pa_validate_tables(block_tables: torch.Tensor, context_lens: torch.Tensor, num_pages: int,
+                       page_size: int, d_err: torch.Tensor, stream=None) -> None:
+    """OR PA_DERR_* bits into d_err (int32 device scalar) for bad tables."""
+    _need(block_tables, "block_tables", torch.int32)
+    _need(context_lens, "context_lens", torch.int32, block_tables.device)
+    _need(d_err, "d_err", torch.int32, block_tables.device)
+    st = _lib.load().pa_validate_tables(_ptr(block_tables), block_tables.shape[0],
+                                        block_tables.shape[1], _ptr(context_lens), num_pages,
+                                        page_size, _ptr(d_err), _stream(stream))
+    _lib.check(st, "pa_validate_tables")

@@ -1,0 +1,299 @@
+// extern "C" boundary of libpagedattn.so: argument checks, split-KV planning
+// and kernel launches. See include/pagedattn.h for the contract of each call.
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "pa_internal.h"
+
+namespace pa {
+namespace {
+
+thread_local std::string g_last_error;
+
+pa_status_t fail(pa_status_t st, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+pa_status_t cuda_status(cudaError_t e, const char *what) {
+  if (e == cudaSuccess) return PA_OK;
+  return fail(PA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];
+std::atomic<int> g_ctas[kMaxDevices][2][2][2];  // [dev][D==128][P==32][dtype]
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  return dev;
+}
+
+pa_status_t check_pool(const pa_kv_pool_t *pool) {
+  if (pool == nullptr) return fail(PA_ERR_INVALID_ARG, "pool is NULL");
+  if (pool->num_pages <= 0 || pool->num_kv_heads <= 0)
+    return fail(PA_ERR_INVALID_ARG, "pool: num_pages=%d num_kv_heads=%d must be positive",
+                pool->num_pages, pool->num_kv_heads);
+  if (pool->page_size != 16 && pool->page_size != 32)
+    return fail(PA_ERR_UNSUPPORTED, "pool: page_size=%d (supported: 16, 32)", pool->page_size);
+  if (pool->head_dim != 64 && pool->head_dim != 128)
+    return fail(PA_ERR_UNSUPPORTED, "pool: head_dim=%d (supported: 64, 128)", pool->head_dim);
+  if (pool->dtype != PA_KV_BF16 && pool->dtype != PA_KV_U8_PER_TOKEN)
+    return fail(PA_ERR_UNSUPPORTED, "pool: dtype=%d", pool->dtype);
+  if (pool->k_pool == nullptr || pool->v_pool == nullptr)
+    return fail(PA_ERR_INVALID_ARG, "pool: k_pool/v_pool is NULL");
+  if (!aligned(pool->k_pool, 16) || !aligned(pool->v_pool, 16))
+    return fail(PA_ERR_INVALID_ARG, "pool: k_pool/v_pool must be 16-byte aligned");
+  if (pool->dtype == PA_KV_U8_PER_TOKEN) {
+    if (pool->k_sz == nullptr || pool->v_sz == nullptr)
+      return fail(PA_ERR_INVALID_ARG, "pool: INT8 pool needs k_sz and v_sz");
+    if (!aligned(pool->k_sz, 16) || !aligned(pool->v_sz, 16))
+      return fail(PA_ERR_INVALID_ARG, "pool: k_sz/v_sz must be 16-byte aligned");
+  }
+  const long long rows = (long long)pool->num_pages * pool->num_kv_heads * pool->page_size;
+  if (rows > (1LL << 40)) return fail(PA_ERR_INVALID_ARG, "pool too large");
+  return PA_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
+int device_sm_count() {
+  const int dev = current_device();
+  if (dev < 0) return 148;
+  int v = g_sm_count[dev].load(std::memory_order_relaxed);
+  if (v > 0) return v;
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    n = 148;
+  g_sm_count[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+static int cached_ctas_per_sm(int D, int P, int dtype) {
+  const int dev = current_device();
+  if (dev < 0) return 1;
+  std::atomic<int> &slot = g_ctas[dev][D == 128][P == 32][dtype];
+  int v = slot.load(std::memory_order_relaxed);
+  if (v > 0) return v;
+  v = decode_ctas_per_sm(D, P, dtype);
+  slot.store(v, std::memory_order_relaxed);
+  return v;
+}
+
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" {
+
+const char *pa_status_str(pa_status_t s) {
+  switch (s) {
+    case PA_OK: return "ok";
+    case PA_ERR_INVALID_ARG: return "invalid argument";
+    case PA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case PA_ERR_WORKSPACE: return "workspace too small or misaligned";
+    case PA_ERR_CUDA: return "CUDA error";
+    case PA_ERR_BAD_TABLE: return "bad page table";
+  }
+  return "unknown status";
+}
+
+const char *pa_last_error(void) { return g_last_error.c_str(); }
+
+int32_t pa_abi_version(void) { return PA_ABI_VERSION; }
+
+pa_status_t pa_kv_append(const pa_kv_pool_t *pool, const void *k_new, const void *v_new,
+                         const int32_t *seq_idx, const int32_t *pos, int32_t num_tokens,
+                         const int32_t *block_tables, int32_t num_seqs, int32_t max_pages,
+                         int32_t *d_err, void *stream) {
+  g_last_error.clear();
+  pa_status_t st = check_pool(pool);
+  if (st != PA_OK) return st;
+  if (num_tokens < 0 || num_seqs < 0 || max_pages <= 0)
+    return fail(PA_ERR_INVALID_ARG, "num_tokens=%d num_seqs=%d max_pages=%d", num_tokens,
+                num_seqs, max_pages);
+  if (num_tokens == 0) return PA_OK;
+  if (!k_new || !v_new || !seq_idx || !pos || !block_tables)
+    return fail(PA_ERR_INVALID_ARG, "k_new, v_new, seq_idx, pos and block_tables are required");
+  if (!aligned(k_new, 16) || !aligned(v_new, 16))
+    return fail(PA_ERR_INVALID_ARG, "k_new/v_new must be 16-byte aligned");
+  return cuda_status(launch_kv_append(*pool, k_new, v_new, seq_idx, pos, num_tokens,
+                                      block_tables, num_seqs, max_pages, d_err,
+                                      static_cast<cudaStream_t>(stream)),
+                     "pa_kv_append launch");
+}
+
+int32_t pa_decode_num_splits(const pa_kv_pool_t *pool, int32_t num_seqs, int32_t max_pages,
+                             int32_t requested) {
+  if (pool == nullptr || num_seqs < 0 || max_pages <= 0 || requested < 0) return -1;
+  if ((pool->head_dim != 64 && pool->head_dim != 128) ||
+      (pool->page_size != 16 && pool->page_size != 32) ||
+      (pool->dtype != PA_KV_BF16 && pool->dtype != PA_KV_U8_PER_TOKEN) ||
+      pool->num_kv_heads <= 0)
+    return -1;
+  const int P = pool->page_size;
+  const int hi = max_pages < kMaxSplits ? max_pages : kMaxSplits;
+  int S = requested;
+  if (S == 0) {
+    // Wave model: CTAs of equal length run in waves of R = SMs x CTAs/SM. A
+    // split count is worth its extra partial writes only if it shortens
+    // (#waves x tokens per CTA); ties go to fewer splits.
+    const long long units = (long long)num_seqs * pool->num_kv_heads;
+    if (units == 0) {
+      S = 1;
+    } else {
+      const long long R =
+          (long long)device_sm_count() * cached_ctas_per_sm(pool->head_dim, P, pool->dtype);
+      const double kCtaOverheadTok = 64.0;   // CTA start-up, in tokens of streaming
+      const double kSplitCostTok = 16.0;     // partial write + merge per split, per unit
+      double best = 1e300;
+      for (int s = 1; s <= hi; ++s) {
+        const long long chunk = (max_pages + s - 1) / s;
+        const int s_eff = (int)((max_pages + chunk - 1) / chunk);
+        if (s_eff != s) continue;
+        const long long waves = (units * s + R - 1) / R;
+        double cost = (double)waves * ((double)chunk * P + kCtaOverheadTok);
+        if (s > 1) cost += kSplitCostTok * s * (double)units / (double)R + kCtaOverheadTok;
+        if (cost < best * (1.0 - 1e-9)) {
+          best = cost;
+          S = s;
+        }
+      }
+    }
+  }
+  if (S > hi) S = hi;
+  const int lo = (max_pages + kMaxPagesPerSplit - 1) / kMaxPagesPerSplit;
+  if (S < lo) S = lo;
+  if (S < 1) S = 1;
+  const int chunk = (max_pages + S - 1) / S;
+  return (max_pages + chunk - 1) / chunk;
+}
+
+size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
+                                 int32_t num_splits) {
+  if (num_splits <= 1 || num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0) return 0;
+  const size_t rows = (size_t)num_seqs * num_q_heads;
+  return align256(rows * num_splits * head_dim * sizeof(float)) +
+         align256(rows * num_splits * sizeof(float));
+}
+
+pa_status_t pa_decode(const pa_kv_pool_t *pool, const void *q, int32_t num_seqs,
+                      int32_t num_q_heads, const int32_t *block_tables, int32_t max_pages,
+                      const int32_t *context_lens, float scale, float *out, void *workspace,
+                      size_t workspace_bytes, int32_t num_splits, int32_t *d_err,
+                      void *stream) {
+  g_last_error.clear();
+  pa_status_t st = check_pool(pool);
+  if (st != PA_OK) return st;
+  if (num_seqs < 0 || num_q_heads <= 0 || max_pages <= 0 || num_splits < 0)
+    return fail(PA_ERR_INVALID_ARG, "num_seqs=%d num_q_heads=%d max_pages=%d num_splits=%d",
+                num_seqs, num_q_heads, max_pages, num_splits);
+  if (num_q_heads % pool->num_kv_heads != 0)
+    return fail(PA_ERR_INVALID_ARG, "num_q_heads=%d is not a multiple of num_kv_heads=%d",
+                num_q_heads, pool->num_kv_heads);
+  const int G = num_q_heads / pool->num_kv_heads;
+  if (G > kMaxGroup)
+    return fail(PA_ERR_UNSUPPORTED, "GQA group %d > %d query heads per KV head", G, kMaxGroup);
+  if (num_seqs > 65535 || pool->num_kv_heads > 65535)
+    return fail(PA_ERR_UNSUPPORTED, "num_seqs and num_kv_heads must be <= 65535");
+  if ((long long)max_pages * pool->page_size > (1LL << 30))
+    return fail(PA_ERR_UNSUPPORTED, "max_pages * page_size too large");
+  if (!(scale == scale)) return fail(PA_ERR_INVALID_ARG, "scale is NaN");
+  if (num_seqs == 0) return PA_OK;
+  if (!q || !block_tables || !context_lens || !out)
+    return fail(PA_ERR_INVALID_ARG, "q, block_tables, context_lens and out are required");
+  if (!aligned(q, 16) || !aligned(out, 16))
+    return fail(PA_ERR_INVALID_ARG, "q and out must be 16-byte aligned");
+  const int S = pa_decode_num_splits(pool, num_seqs, max_pages, num_splits);
+  if (S <= 0) return fail(PA_ERR_INVALID_ARG, "could not plan splits");
+  const size_t need = pa_decode_workspace_bytes(num_seqs, num_q_heads, pool->head_dim, S);
+  if (need > 0) {
+    if (workspace == nullptr || workspace_bytes < need)
+      return fail(PA_ERR_WORKSPACE, "workspace: need %zu bytes for %d splits, got %zu", need, S,
+                  workspace == nullptr ? (size_t)0 : workspace_bytes);
+    if (!aligned(workspace, 256))
+      return fail(PA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  }
+  const int chunk = (max_pages + S - 1) / S;
+  const size_t rows = (size_t)num_seqs * num_q_heads;
+  DecodeArgs a;
+  a.k_pool = pool->k_pool;
+  a.v_pool = pool->v_pool;
+  a.k_sz = pool->k_sz;
+  a.v_sz = pool->v_sz;
+  a.num_pages = pool->num_pages;
+  a.hkv = pool->num_kv_heads;
+  a.q = q;
+  a.B = num_seqs;
+  a.hq = num_q_heads;
+  a.block_tables = block_tables;
+  a.max_pages = max_pages;
+  a.ctx = context_lens;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.out = out;
+  a.o_part = S > 1 ? static_cast<float *>(workspace) : nullptr;
+  a.lse = S > 1 ? reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                            align256(rows * S * pool->head_dim * sizeof(float)))
+                : nullptr;
+  a.S = S;
+  a.pages_per_split = chunk;
+  a.d_err = d_err;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = cuda_status(launch_decode(pool->head_dim, pool->page_size, pool->dtype, a, s),
+                   "pa_decode launch");
+  if (st != PA_OK || S == 1) return st;
+  return cuda_status(launch_splitkv_reduce(a.o_part, a.lse, num_seqs, num_q_heads, S,
+                                           pool->head_dim, out, true, s),
+                     "pa_decode merge launch");
+}
+
+pa_status_t pa_splitkv_reduce(const float *o_part, const float *lse, int32_t num_seqs,
+                              int32_t num_q_heads, int32_t num_splits, int32_t head_dim,
+                              float *out, void *stream) {
+  g_last_error.clear();
+  if (num_seqs < 0 || num_q_heads <= 0 || num_splits < 1 || num_splits > kMaxSplits ||
+      head_dim <= 0 || head_dim % 4 != 0 || head_dim > 512)
+    return fail(PA_ERR_INVALID_ARG, "num_seqs=%d num_q_heads=%d num_splits=%d head_dim=%d",
+                num_seqs, num_q_heads, num_splits, head_dim);
+  if (num_seqs == 0) return PA_OK;
+  if (!o_part || !lse || !out) return fail(PA_ERR_INVALID_ARG, "o_part, lse and out are required");
+  if (!aligned(o_part, 16) || !aligned(out, 16))
+    return fail(PA_ERR_INVALID_ARG, "o_part and out must be 16-byte aligned");
+  if ((long long)num_seqs * num_q_heads > (1LL << 31) - 4)
+    return fail(PA_ERR_UNSUPPORTED, "too many rows");
+  return cuda_status(launch_splitkv_reduce(o_part, lse, num_seqs, num_q_heads, num_splits,
+                                           head_dim, out, false,
+                                           static_cast<cudaStream_t>(stream)),
+                     "pa_splitkv_reduce launch");
+}
+
+pa_status_t pa_validate_tables(const int32_t *block_tables, int32_t num_seqs, int32_t max_pages,
+                               const int32_t *context_lens, int32_t num_pages, int32_t page_size,
+                               int32_t *d_err, void *stream) {
+  g_last_error.clear();
+  if (num_seqs < 0 || max_pages <= 0 || num_pages <= 0 || page_size <= 0)
+    return fail(PA_ERR_INVALID_ARG, "num_seqs=%d max_pages=%d num_pages=%d page_size=%d",
+                num_seqs, max_pages, num_pages, page_size);
+  if (d_err == nullptr) return fail(PA_ERR_INVALID_ARG, "d_err is required");
+  if (num_seqs == 0) return PA_OK;
+  if (!block_tables || !context_lens)
+    return fail(PA_ERR_INVALID_ARG, "block_tables and context_lens are required");
+  return cuda_status(launch_validate_tables(block_tables, num_seqs, max_pages, context_lens,
+                                            num_pages, page_size, d_err,
+                                            static_cast<cudaStream_t>(stream)),
+                     "pa_validate_tables launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,509 @@
+// Paged decode attention (Eq. 1 of "KV-Cache Optimization Techniques",
+// section "PagedAttention (vLLM)") for B200 / sm_100a.
+//
+// One CTA serves one (split, KV head, sequence): it walks that sequence's
+// logical pages in [split * pages_per_split, (split + 1) * pages_per_split),
+// looks each up in the request's block table, and reads every K/V row of the
+// page exactly once for all G query heads that share the KV head (GQA, Eq. 7
+// of the same page). The CTA's warps take 16-token blocks round robin; each
+// warp keeps its own online-softmax state and the CTA merges its warps at the
+// end by their running maxima.
+//
+// Per 16-token block a warp does, on the tensor cores (mma.sync m16n8k16):
+//   S[8 heads x 16 tokens]  = Q[heads x D] . K[tokens x D]^T     (A = Q, B = K)
+//   O^T[D x 8 heads]       += V^T[D x tokens] . P^T[tokens x heads]
+// The score fragment S lands in exactly the register layout the second product
+// needs for its B operand, so P never leaves registers. P is split into a bf16
+// (or f16) high part and the residual low part and multiplied twice, which keeps
+// ~16 significant bits of every softmax weight.
+//
+// Data movement: every lane copies its own 16-byte pieces of K and V (cp.async,
+// L1 bypass, zero-fill past the context) into a private slot of a per-warp ring
+// of NSTAGE blocks in shared memory and later reads back only what it copied.
+// No lane ever reads another lane's staging, so the pipeline needs no barrier,
+// mbarrier or spin-wait: cp.async.wait_group per thread is the only wait.
+//
+// The lane -> (token, d) assignment is chosen so that (i) every global access
+// of a warp covers whole 32-byte sectors, (ii) shared-memory accesses are
+// conflict free, and (iii) the loaded registers are already mma fragments:
+//   K: lane (g = lane/4, t = lane%4) loads token g of each 8-token half-block,
+//      16-byte chunks t, t+4, ... of its row. The contraction index (d) is
+//      permuted identically for Q, which is loaded with the same pattern.
+//   V: lane loads tokens {2t, 2t+1, 8+2t, 9+2t} (the B-fragment rows of P^T),
+//      chunks {g, 8+g} (bf16) or chunk g (uint8); the output rows of O^T are
+//      permuted accordingly and un-permuted when stored.
+//
+// INT8 cache (Eq. 3, "KV-Cache Quantization"): with x = s*c + z per row,
+//   q.x = s (q.c) + z sum(q)          and    sum_t p_t x_t = sum_t (p_t s_t) c_t + sum_t p_t z_t,
+// so the codes go through the tensor cores as exact f16 integers and the scale
+// and zero are applied once per (token, head) instead of once per element.
+#include <cfloat>
+#include <cmath>
+
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+namespace {
+
+constexpr float kLn2 = 0.693147180559945309f;
+// Lazy rescaling: the running max is only raised when a block's max exceeds it
+// by more than this many powers of two, so weights stay <= 2^kRescaleLog2.
+constexpr float kRescaleLog2 = 8.0f;
+
+template <int D, int KVT>
+struct Tile {
+  static_assert(D == 64 || D == 128, "head_dim");
+  static constexpr bool kU8 = KVT == PA_KV_U8_PER_TOKEN;
+  static constexpr int kElem = kU8 ? 1 : 2;
+  static constexpr int kRowBytes = D * kElem;
+  // 16-byte K chunks a lane loads per 8-token half-block
+  static constexpr int kKChunks = kU8 ? D / 64 : D / 32;
+  static constexpr int kKItems = 2 * kKChunks;
+  // 16-byte V chunks a lane loads per token (4 tokens per block)
+  static constexpr int kVChunks = kU8 ? 1 : D / 64;
+  static constexpr int kVItems = 4 * kVChunks;
+  static constexpr int kSzItems = kU8 ? 4 : 0;
+  static constexpr int kItems = kKItems + kVItems + kSzItems;
+  static constexpr int kStageBytes = kItems * 32 * 16;
+  static constexpr int kMTiles = D / 16;  // m16 tiles of O^T
+};
+
+template <int D, int KVT, int W, int NSTAGE>
+struct Smem {
+  using T = Tile<D, KVT>;
+  static constexpr int kRingBytesPerWarp = NSTAGE * T::kStageBytes;
+  static constexpr int kRingBytes = W * kRingBytesPerWarp;
+  // per-warp merge record: m[8], l[8], O[8][D]
+  static constexpr int kMergeBytes = (16 + kMaxGroup * D) * 4;
+  static_assert(kMergeBytes <= kRingBytesPerWarp, "merge record must fit the ring");
+  static constexpr size_t bytes(int pages_per_split) {
+    return (size_t)kRingBytes + (size_t)pages_per_split * 4;
+  }
+};
+
+// Row of O^T held in accumulator c0/c1 (row g) of m-tile j; c2/c3 hold d + 1.
+template <int D, int KVT>
+__device__ __forceinline__ int out_col(int j, int g) {
+  if constexpr (KVT == PA_KV_U8_PER_TOKEN) {
+    return (D == 128 ? 16 * g : 8 * g) + 2 * j;
+  } else {
+    return 8 * (8 * (j / 4) + g) + 2 * (j % 4);
+  }
+}
+
+template <int D, int P, int KVT, int W, int NSTAGE>
+__global__ void __launch_bounds__(W * 32, 2) decode_kernel(const DecodeArgs a) {
+  using T = Tile<D, KVT>;
+  using SM = Smem<D, KVT, W, NSTAGE>;
+  static_assert(P % 16 == 0, "a 16-token block must not straddle pages");
+  extern __shared__ __align__(128) unsigned char smem[];
+
+  const int split = blockIdx.x;
+  const int h = blockIdx.y;
+  const int b = blockIdx.z;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2;
+  const int t = lane & 3;
+  const int G = a.hq / a.hkv;
+
+  int *tbl = reinterpret_cast<int *>(smem + SM::kRingBytes);
+
+  // ---- this split's token range --------------------------------------------
+  int ctx = a.ctx[b];
+  if (ctx < 0 || ctx > a.max_pages * P) {
+    if (threadIdx.x == 0) flag_error(a.d_err, PA_DERR_BAD_CTX);
+    ctx = 0;
+  }
+  const int n_pages = (ctx + P - 1) / P;
+  const int lp0 = split * a.pages_per_split;
+  const int lp1 = min(lp0 + a.pages_per_split, n_pages);
+  const int tok0 = lp0 * P;
+  const int tok1 = min(lp1 * P, ctx);
+  const int nblk = tok1 > tok0 ? (tok1 - tok0 + 15) / 16 : 0;
+
+  // ---- stage this split's block-table entries (bounds-checked) --------------
+  for (int i = threadIdx.x; i < lp1 - lp0; i += W * 32) {
+    int pg = __ldg(a.block_tables + (size_t)b * a.max_pages + lp0 + i);
+    if (pg < 0 || pg >= a.num_pages) {
+      flag_error(a.d_err, PA_DERR_BAD_PAGE);
+      pg = -1;
+    }
+    tbl[i] = pg;
+  }
+
+  // ---- query fragments (A operand, rows = heads; rows 8..15 stay zero) -------
+  const bool head_ok = g < G;
+  const size_t q_row = ((size_t)b * a.hq + (size_t)h * G + (head_ok ? g : 0)) * D;
+  const __nv_bfloat16 *qp = reinterpret_cast<const __nv_bfloat16 *>(a.q) + q_row;
+  uint32_t qa[D / 16][2];  // per k-step: a0 (k 2t..2t+1), a2 (k 2t+8..2t+9)
+  float qsum = 0.f;        // sum of this head's q (as the MMA sees it), INT8 only
+  if constexpr (!T::kU8) {
+#pragma unroll
+    for (int i = 0; i < T::kKChunks; ++i) {
+      uint4 v = head_ok ? ldg_nc128(qp + (4 * i + t) * 8) : make_uint4(0, 0, 0, 0);
+      qa[2 * i][0] = v.x;
+      qa[2 * i][1] = v.y;
+      qa[2 * i + 1][0] = v.z;
+      qa[2 * i + 1][1] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < T::kKChunks; ++i) {
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        uint4 v = head_ok ? ldg_nc128(qp + (4 * i + t) * 16 + hf * 8) : make_uint4(0, 0, 0, 0);
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t f = pack_f16(bf16_lo(w4[k]), bf16_hi(w4[k]));
+          qsum += f16_lo(f) + f16_hi(f);
+          // words of this 16-d chunk: k-step 4i + (2hf + k/2), half k%2
+          qa[4 * i + 2 * hf + k / 2][k % 2] = f;
+        }
+      }
+    }
+    qsum += __shfl_xor_sync(0xffffffffu, qsum, 1);
+    qsum += __shfl_xor_sync(0xffffffffu, qsum, 2);
+  }
+  __syncthreads();  // tbl visible
+
+  // ---- per-warp pipeline ---------------------------------------------------------
+  const uint32_t ring = smem_u32(smem) + warp * SM::kRingBytesPerWarp + lane * 16;
+  const unsigned char *kbase = static_cast<const unsigned char *>(a.k_pool);
+  const unsigned char *vbase = static_cast<const unsigned char *>(a.v_pool);
+  const int nmine = nblk > warp ? (nblk - warp + W - 1) / W : 0;
+
+  auto issue = [&](int kb, int st) {
+    const int btok = tok0 + kb * 16;
+    const int lp = btok / P;
+    const int page = tbl[lp - lp0];
+    const int in_page = btok - lp * P;
+    const bool pvalid = page >= 0;
+    const size_t row0 = ((size_t)(pvalid ? page : 0) * a.hkv + h) * P + in_page;
+    const uint32_t dst = ring + st * T::kStageBytes;
+    // K: token g (and 8 + g), chunks t, t+4, ...
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const int toff = nt * 8 + g;
+      const bool ok = pvalid && btok + toff < tok1;
+#pragma unroll
+      for (int i = 0; i < T::kKChunks; ++i) {
+        const unsigned char *src = kbase + (row0 + toff) * T::kRowBytes + (4 * i + t) * 16;
+        cp_async16(dst + (nt * T::kKChunks + i) * 512, ok ? src : kbase, ok ? 16u : 0u);
+      }
+    }
+    // V: tokens 2t, 2t+1, 8+2t, 9+2t
+#pragma unroll
+    for (int tau = 0; tau < 4; ++tau) {
+      const int toff = (tau & 1) + 2 * t + (tau >> 1) * 8;
+      const bool ok = pvalid && btok + toff < tok1;
+#pragma unroll
+      for (int c = 0; c < T::kVChunks; ++c) {
+        const int chunk = T::kU8 ? (D == 128 ? g : (g >> 1)) : 8 * c + g;
+        const unsigned char *src = vbase + (row0 + toff) * T::kRowBytes + chunk * 16;
+        cp_async16(dst + (T::kKItems + tau * T::kVChunks + c) * 512, ok ? src : vbase,
+                   ok ? 16u : 0u);
+      }
+    }
+    if constexpr (T::kU8) {
+      // (scale, zero) pairs of tokens (2t, 2t+1) and (8+2t, 9+2t), K then V
+#pragma unroll
+      for (int kv = 0; kv < 2; ++kv) {
+        const float *szb = kv == 0 ? a.k_sz : a.v_sz;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const int toff = nt * 8 + 2 * t;
+          const int tok = btok + toff;
+          const uint32_t nbytes = !pvalid ? 0u : (tok + 1 < tok1 ? 16u : (tok < tok1 ? 8u : 0u));
+          const float *src = szb + (row0 + toff) * 2;
+          cp_async16(dst + (T::kKItems + T::kVItems + kv * 2 + nt) * 512,
+                     nbytes ? static_cast<const void *>(src) : static_cast<const void *>(szb),
+                     nbytes);
+        }
+      }
+    }
+  };
+
+  float o[T::kMTiles][4];
+#pragma unroll
+  for (int j = 0; j < T::kMTiles; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  float m_run = -INFINITY;  // running max of this head's scores (log2 units)
+  float l_run = 0.f;        // this lane's share of the softmax denominator
+  float zacc = 0.f;         // INT8: this lane's share of sum_t p_t z_t
+
+#pragma unroll
+  for (int st = 0; st < NSTAGE - 1; ++st) {
+    if (st < nmine) issue(warp + st * W, st);
+    cp_async_commit();
+  }
+
+  for (int k = 0; k < nmine; ++k) {
+    __syncwarp();
+    {
+      const int kn = k + NSTAGE - 1;
+      if (kn < nmine) issue(warp + kn * W, kn % NSTAGE);
+      cp_async_commit();
+    }
+    cp_async_wait<NSTAGE - 1>();
+
+    const int kb = warp + k * W;
+    const int btok = tok0 + kb * 16;
+    const bool pvalid = tbl[btok / P - lp0] >= 0;
+    const uint32_t src = ring + (k % NSTAGE) * T::kStageBytes;
+
+    // ---- S = Q K^T -------------------------------------------------------------
+    float s[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+#pragma unroll
+      for (int i = 0; i < T::kKChunks; ++i) {
+        const uint4 kv = lds128(src + (nt * T::kKChunks + i) * 512);
+        if constexpr (!T::kU8) {
+          mma_bf16_16816(s[nt], qa[2 * i][0], 0u, qa[2 * i][1], 0u, kv.x, kv.y);
+          mma_bf16_16816(s[nt], qa[2 * i + 1][0], 0u, qa[2 * i + 1][1], 0u, kv.z, kv.w);
+        } else {
+          const uint32_t w4[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            mma_f16_16816(s[nt], qa[4 * i + w][0], 0u, qa[4 * i + w][1], 0u,
+                          u8x2_to_f16x2(w4[w], 0x4140), u8x2_to_f16x2(w4[w], 0x4342));
+          }
+        }
+      }
+    }
+
+    // ---- online softmax (log2 domain) ---------------------------------------
+    float x[4] = {s[0][0], s[0][1], s[1][0], s[1][1]};  // tokens 2t, 2t+1, 8+2t, 9+2t
+    float vs[4], vz[4];
+    if constexpr (T::kU8) {
+      const uint4 k01 = lds128(src + (T::kKItems + T::kVItems + 0) * 512);
+      const uint4 k89 = lds128(src + (T::kKItems + T::kVItems + 1) * 512);
+      const uint4 v01 = lds128(src + (T::kKItems + T::kVItems + 2) * 512);
+      const uint4 v89 = lds128(src + (T::kKItems + T::kVItems + 3) * 512);
+      const float ks[4] = {__uint_as_float(k01.x), __uint_as_float(k01.z),
+                           __uint_as_float(k89.x), __uint_as_float(k89.z)};
+      const float kz[4] = {__uint_as_float(k01.y), __uint_as_float(k01.w),
+                           __uint_as_float(k89.y), __uint_as_float(k89.w)};
+      vs[0] = __uint_as_float(v01.x); vz[0] = __uint_as_float(v01.y);
+      vs[1] = __uint_as_float(v01.z); vz[1] = __uint_as_float(v01.w);
+      vs[2] = __uint_as_float(v89.x); vz[2] = __uint_as_float(v89.y);
+      vs[3] = __uint_as_float(v89.z); vz[3] = __uint_as_float(v89.w);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) x[e] = fmaf(ks[e], x[e], kz[e] * qsum);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int toff = (e & 1) + 2 * t + (e >> 1) * 8;
+      x[e] = (pvalid && btok + toff < tok1) ? x[e] * a.scale_log2 : -INFINITY;
+    }
+    float mb = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+    mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
+    mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
+    const bool need = mb > m_run + kRescaleLog2 || (m_run == -INFINITY && mb > -INFINITY);
+    if (__any_sync(0xffffffffu, need)) {
+      const float m_new = fmaxf(m_run, mb);
+      const float alpha = m_new == -INFINITY ? 1.f : fast_exp2(m_run - m_new);
+      m_run = m_new;
+      l_run *= alpha;
+      zacc *= alpha;
+      const float al0 = __shfl_sync(0xffffffffu, alpha, 8 * t);      // head 2t
+      const float al1 = __shfl_sync(0xffffffffu, alpha, 8 * t + 4);  // head 2t+1
+#pragma unroll
+      for (int j = 0; j < T::kMTiles; ++j) {
+        o[j][0] *= al0;
+        o[j][1] *= al1;
+        o[j][2] *= al0;
+        o[j][3] *= al1;
+      }
+    }
+    const float mref = m_run == -INFINITY ? 0.f : m_run;
+    float p[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) p[e] = fast_exp2(x[e] - mref);
+    l_run += (p[0] + p[1]) + (p[2] + p[3]);
+
+    // ---- O^T += V^T P^T -------------------------------------------------------
+    uint32_t bh0, bl0, bh1, bl1;
+    if constexpr (!T::kU8) {
+      split_bf16(p[0], p[1], bh0, bl0);
+      split_bf16(p[2], p[3], bh1, bl1);
+#pragma unroll
+      for (int c = 0; c < T::kVChunks; ++c) {
+        const uint4 v0 = lds128(src + (T::kKItems + 0 * T::kVChunks + c) * 512);
+        const uint4 v1 = lds128(src + (T::kKItems + 1 * T::kVChunks + c) * 512);
+        const uint4 v2 = lds128(src + (T::kKItems + 2 * T::kVChunks + c) * 512);
+        const uint4 v3 = lds128(src + (T::kKItems + 3 * T::kVChunks + c) * 512);
+        const uint32_t x0[4] = {v0.x, v0.y, v0.z, v0.w};
+        const uint32_t x1[4] = {v1.x, v1.y, v1.z, v1.w};
+        const uint32_t x2[4] = {v2.x, v2.y, v2.z, v2.w};
+        const uint32_t x3[4] = {v3.x, v3.y, v3.z, v3.w};
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const uint32_t a0 = __byte_perm(x0[w], x1[w], 0x5410);
+          const uint32_t a1 = __byte_perm(x0[w], x1[w], 0x7632);
+          const uint32_t a2 = __byte_perm(x2[w], x3[w], 0x5410);
+          const uint32_t a3 = __byte_perm(x2[w], x3[w], 0x7632);
+          mma_bf16_16816(o[4 * c + w], a0, a1, a2, a3, bh0, bh1);
+          mma_bf16_16816(o[4 * c + w], a0, a1, a2, a3, bl0, bl1);
+        }
+      }
+    } else {
+      float pv[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        pv[e] = p[e] * vs[e];
+        zacc = fmaf(p[e], vz[e], zacc);
+      }
+      split_f16(pv[0], pv[1], bh0, bl0);
+      split_f16(pv[2], pv[3], bh1, bl1);
+      const uint4 v0 = lds128(src + (T::kKItems + 0) * 512);
+      const uint4 v1 = lds128(src + (T::kKItems + 1) * 512);
+      const uint4 v2 = lds128(src + (T::kKItems + 2) * 512);
+      const uint4 v3 = lds128(src + (T::kKItems + 3) * 512);
+      const uint32_t x0[4] = {v0.x, v0.y, v0.z, v0.w};
+      const uint32_t x1[4] = {v1.x, v1.y, v1.z, v1.w};
+      const uint32_t x2[4] = {v2.x, v2.y, v2.z, v2.w};
+      const uint32_t x3[4] = {v3.x, v3.y, v3.z, v3.w};
+#pragma unroll
+      for (int j = 0; j < T::kMTiles; ++j) {
+        const uint32_t sel = (j & 1) ? 0x7362 : 0x5140;
+        // select with a runtime word offset only for D == 64
+        const uint32_t w0 = D == 128 ? x0[j / 2] : ((g & 1) ? x0[2 + j / 2] : x0[j / 2]);
+        const uint32_t w1 = D == 128 ? x1[j / 2] : ((g & 1) ? x1[2 + j / 2] : x1[j / 2]);
+        const uint32_t w2 = D == 128 ? x2[j / 2] : ((g & 1) ? x2[2 + j / 2] : x2[j / 2]);
+        const uint32_t w3 = D == 128 ? x3[j / 2] : ((g & 1) ? x3[2 + j / 2] : x3[j / 2]);
+        const uint32_t xa = __byte_perm(w0, w1, sel);
+        const uint32_t xb = __byte_perm(w2, w3, sel);
+        const uint32_t a0 = u8x2_to_f16x2(xa, 0x4140);
+        const uint32_t a1 = u8x2_to_f16x2(xa, 0x4342);
+        const uint32_t a2 = u8x2_to_f16x2(xb, 0x4140);
+        const uint32_t a3 = u8x2_to_f16x2(xb, 0x4342);
+        mma_f16_16816(o[j], a0, a1, a2, a3, bh0, bh1);
+        mma_f16_16816(o[j], a0, a1, a2, a3, bl0, bl1);
+      }
+    }
+  }
+  cp_async_wait<0>();
+  __syncwarp();
+
+  // ---- finish this warp's state ---------------------------------------------------
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+  if constexpr (T::kU8) {
+    zacc += __shfl_xor_sync(0xffffffffu, zacc, 1);
+    zacc += __shfl_xor_sync(0xffffffffu, zacc, 2);
+    const float z0 = __shfl_sync(0xffffffffu, zacc, 8 * t);
+    const float z1 = __shfl_sync(0xffffffffu, zacc, 8 * t + 4);
+#pragma unroll
+    for (int j = 0; j < T::kMTiles; ++j) {
+      o[j][0] += z0;
+      o[j][1] += z1;
+      o[j][2] += z0;
+      o[j][3] += z1;
+    }
+  }
+
+  // ---- merge the CTA's warps (fixed order: deterministic) --------------------
+  float *rec = reinterpret_cast<float *>(smem + warp * SM::kRingBytesPerWarp);
+  if (t == 0) {
+    rec[g] = m_run;
+    rec[8 + g] = l_run;
+  }
+  {
+    float *O = rec + 16;
+#pragma unroll
+    for (int j = 0; j < T::kMTiles; ++j) {
+      const int d0 = out_col<D, KVT>(j, g);
+      *reinterpret_cast<float2 *>(O + (2 * t) * D + d0) = make_float2(o[j][0], o[j][2]);
+      *reinterpret_cast<float2 *>(O + (2 * t + 1) * D + d0) = make_float2(o[j][1], o[j][3]);
+    }
+  }
+  __syncthreads();
+
+  for (int e = threadIdx.x; e < G * D; e += W * 32) {
+    const int hd = e / D;
+    const int d = e - hd * D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < W; ++w)
+      M = fmaxf(M, reinterpret_cast<const float *>(smem + w * SM::kRingBytesPerWarp)[hd]);
+    float num = 0.f, L = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < W; ++w) {
+        const float *r = reinterpret_cast<const float *>(smem + w * SM::kRingBytesPerWarp);
+        const float f = fast_exp2(r[hd] - M);  // exp2(-inf) = 0 for empty warps
+        num = fmaf(f, r[16 + hd * D + d], num);
+        L = fmaf(f, r[8 + hd], L);
+      }
+    }
+    const size_t row = (size_t)b * a.hq + (size_t)h * G + hd;
+    const float val = L > 0.f ? num / L : 0.f;
+    if (a.S == 1) {
+      a.out[row * D + d] = val;
+    } else {
+      a.o_part[(row * a.S + split) * D + d] = val;
+      if (d == 0) a.lse[row * a.S + split] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+    }
+  }
+  pdl_launch_dependents();
+}
+
+template <int D, int P, int KVT>
+struct Config {
+  static constexpr int W = 4;
+  static constexpr int NSTAGE = KVT == PA_KV_U8_PER_TOKEN ? 4 : 3;
+  using SM = Smem<D, KVT, W, NSTAGE>;
+  static void *fn() { return reinterpret_cast<void *>(&decode_kernel<D, P, KVT, W, NSTAGE>); }
+};
+
+template <int D, int P, int KVT>
+cudaError_t launch_t(const DecodeArgs &a, cudaStream_t stream) {
+  using C = Config<D, P, KVT>;
+  const size_t smem = C::SM::bytes(a.pages_per_split);
+  cudaError_t e = cudaFuncSetAttribute(C::fn(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.S, a.hkv, a.B);
+  decode_kernel<D, P, KVT, C::W, C::NSTAGE><<<grid, C::W * 32, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D, int P, int KVT>
+int ctas_per_sm_t() {
+  using C = Config<D, P, KVT>;
+  const size_t smem = C::SM::bytes(256);
+  if (cudaFuncSetAttribute(C::fn(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, C::fn(), C::W * 32, smem) != cudaSuccess)
+    return 1;
+  return n > 0 ? n : 1;
+}
+
+}  // namespace
+
+#define PA_DISPATCH(D_, P_, K_, CALL)                                  \
+  if (D == D_ && P == P_ && kv_dtype == K_) return CALL<D_, P_, K_>
+
+cudaError_t launch_decode(int D, int P, int kv_dtype, const DecodeArgs &a, cudaStream_t stream) {
+#define PA_L(D_, P_, K_) PA_DISPATCH(D_, P_, K_, launch_t)(a, stream)
+  PA_L(128, 16, 0); PA_L(128, 32, 0); PA_L(64, 16, 0); PA_L(64, 32, 0);
+  PA_L(128, 16, 1); PA_L(128, 32, 1); PA_L(64, 16, 1); PA_L(64, 32, 1);
+#undef PA_L
+  return cudaErrorInvalidValue;
+}
+
+int decode_ctas_per_sm(int D, int P, int kv_dtype) {
+#define PA_O(D_, P_, K_) PA_DISPATCH(D_, P_, K_, ctas_per_sm_t)()
+  PA_O(128, 16, 0); PA_O(128, 32, 0); PA_O(64, 16, 0); PA_O(64, 32, 0);
+  PA_O(128, 16, 1); PA_O(128, 32, 1); PA_O(64, 16, 1); PA_O(64, 32, 1);
+#undef PA_O
+  return 1;
+}
+
+}  // namespace pa

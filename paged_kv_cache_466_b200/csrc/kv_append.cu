@@ -1,0 +1,180 @@
+// Cache write: scatter new tokens' K/V rows into their page slots.
+//
+// "KV-Cache Optimization Techniques", section "PagedAttention (vLLM)",
+// "Architecture": each request's page table maps a logical KV position to a
+// physical page of P tokens; position pos lives in page table[pos / P], slot
+// pos % P. For an INT8 pool every (token, KV head) row is quantised on the way
+// in by Eq. 3 ("KV-Cache Quantization", per-token calibration):
+//   z = min(row), s = (max(row) - min(row)) / 255,
+//   code = clamp(round_half_even((x - z) / s), 0, 255)   (s == 0 -> code 0),
+// every step an IEEE fp32 operation in that order (explicit _rn intrinsics,
+// no contraction), inputs read as x + 0 so that -0 is stored as +0.
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+namespace {
+
+struct AppendArgs {
+  const unsigned char *k_new;
+  const unsigned char *v_new;
+  const int32_t *seq_idx;
+  const int32_t *pos;
+  const int32_t *block_tables;
+  int32_t n;
+  int32_t num_seqs;
+  int32_t max_pages;
+  int32_t num_pages;
+  int32_t hkv;
+  int32_t P;
+  int32_t D;
+  unsigned char *k_pool;
+  unsigned char *v_pool;
+  float *k_sz;
+  float *v_sz;
+  int32_t *d_err;
+};
+
+// Physical row index (page * Hkv + h) * P + slot of token i, KV head h; -1 and
+// an error bit if the token's sequence, position or page is out of range.
+__device__ __forceinline__ long long slot_row(const AppendArgs &a, int i, int h) {
+  const int seq = __ldg(a.seq_idx + i);
+  const int p = __ldg(a.pos + i);
+  if (seq < 0 || seq >= a.num_seqs) {
+    flag_error(a.d_err, PA_DERR_BAD_SEQ);
+    return -1;
+  }
+  if (p < 0 || p / a.P >= a.max_pages) {
+    flag_error(a.d_err, PA_DERR_BAD_POS);
+    return -1;
+  }
+  const int page = __ldg(a.block_tables + (size_t)seq * a.max_pages + p / a.P);
+  if (page < 0 || page >= a.num_pages) {
+    flag_error(a.d_err, PA_DERR_BAD_PAGE);
+    return -1;
+  }
+  return ((long long)page * a.hkv + h) * a.P + p % a.P;
+}
+
+// bf16: one thread per 16-byte chunk of a (token, head) row, K and V.
+__global__ void append_bf16_kernel(const AppendArgs a) {
+  const int chunks = a.D / 8;
+  const long long total = (long long)a.n * a.hkv * chunks;
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int c = (int)(idx % chunks);
+    const long long r = idx / chunks;  // token * hkv + h
+    const int h = (int)(r % a.hkv);
+    const int i = (int)(r / a.hkv);
+    const long long row = slot_row(a, i, h);
+    if (row < 0) continue;
+    const size_t src = ((size_t)r * a.D + c * 8) * 2;
+    const size_t dst = ((size_t)row * a.D + c * 8) * 2;
+    *reinterpret_cast<uint4 *>(a.k_pool + dst) = ldg_nc128(a.k_new + src);
+    *reinterpret_cast<uint4 *>(a.v_pool + dst) = ldg_nc128(a.v_new + src);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void quantise_row(const unsigned char *src_row, unsigned char *dst_codes,
+                                             float *dst_sz, int lane) {
+  constexpr int E = D / 32;  // elements per lane
+  const __nv_bfloat16 *x16 = reinterpret_cast<const __nv_bfloat16 *>(src_row) + lane * E;
+  float x[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) x[e] = __fadd_rn(__bfloat162float(x16[e]), 0.0f);
+  float mn = x[0], mx = x[0];
+#pragma unroll
+  for (int e = 1; e < E; ++e) {
+    mn = fminf(mn, x[e]);
+    mx = fmaxf(mx, x[e]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  const float s = __fdiv_rn(__fsub_rn(mx, mn), 255.0f);
+  const float z = mn;
+  uint32_t packed = 0;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    uint32_t c = 0;
+    if (s != 0.0f) {
+      float r = rintf(__fdiv_rn(__fsub_rn(x[e], z), s));
+      r = fminf(fmaxf(r, 0.0f), 255.0f);
+      c = static_cast<uint32_t>(r);
+    }
+    packed |= c << (8 * e);
+  }
+  if constexpr (E == 4) {
+    *reinterpret_cast<uint32_t *>(dst_codes + lane * 4) = packed;
+  } else {
+    *reinterpret_cast<uint16_t *>(dst_codes + lane * 2) = static_cast<uint16_t>(packed);
+  }
+  if (lane == 0) *reinterpret_cast<float2 *>(dst_sz) = make_float2(s, z);
+}
+
+// INT8: one warp per (token, head) row; K then V.
+template <int D>
+__global__ void append_u8_kernel(const AppendArgs a) {
+  const int lane = threadIdx.x & 31;
+  const long long rows = (long long)a.n * a.hkv;
+  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long r = blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5); r < rows;
+       r += warps) {
+    const int h = (int)(r % a.hkv);
+    const int i = (int)(r / a.hkv);
+    long long row = 0;
+    if (lane == 0) row = slot_row(a, i, h);
+    row = __shfl_sync(0xffffffffu, row, 0);
+    if (row < 0) continue;
+    const size_t src = (size_t)r * D * 2;
+    quantise_row<D>(a.k_new + src, a.k_pool + (size_t)row * D, a.k_sz + (size_t)row * 2, lane);
+    quantise_row<D>(a.v_new + src, a.v_pool + (size_t)row * D, a.v_sz + (size_t)row * 2, lane);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_kv_append(const pa_kv_pool_t &pool, const void *k_new, const void *v_new,
+                             const int32_t *seq_idx, const int32_t *pos, int32_t n,
+                             const int32_t *block_tables, int32_t num_seqs, int32_t max_pages,
+                             int32_t *d_err, cudaStream_t stream) {
+  AppendArgs a;
+  a.k_new = static_cast<const unsigned char *>(k_new);
+  a.v_new = static_cast<const unsigned char *>(v_new);
+  a.seq_idx = seq_idx;
+  a.pos = pos;
+  a.block_tables = block_tables;
+  a.n = n;
+  a.num_seqs = num_seqs;
+  a.max_pages = max_pages;
+  a.num_pages = pool.num_pages;
+  a.hkv = pool.num_kv_heads;
+  a.P = pool.page_size;
+  a.D = pool.head_dim;
+  a.k_pool = static_cast<unsigned char *>(pool.k_pool);
+  a.v_pool = static_cast<unsigned char *>(pool.v_pool);
+  a.k_sz = pool.k_sz;
+  a.v_sz = pool.v_sz;
+  a.d_err = d_err;
+  const int sms = device_sm_count();
+  if (pool.dtype == PA_KV_BF16) {
+    const long long work = (long long)n * a.hkv * (a.D / 8);
+    long long blocks = (work + 255) / 256;
+    blocks = blocks < 1 ? 1 : (blocks > 16LL * sms ? 16LL * sms : blocks);
+    append_bf16_kernel<<<(unsigned)blocks, 256, 0, stream>>>(a);
+  } else {
+    const long long rows = (long long)n * a.hkv;
+    long long blocks = (rows + 7) / 8;
+    blocks = blocks < 1 ? 1 : (blocks > 16LL * sms ? 16LL * sms : blocks);
+    if (a.D == 128)
+      append_u8_kernel<128><<<(unsigned)blocks, 256, 0, stream>>>(a);
+    else
+      append_u8_kernel<64><<<(unsigned)blocks, 256, 0, stream>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace pa

@@ -1,0 +1,65 @@
+// Host-side declarations shared by the pagedattn translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "pagedattn.h"
+
+namespace pa {
+
+// Largest GQA group a decode CTA serves (query heads per KV head).
+constexpr int kMaxGroup = 8;
+// Page-table entries one decode CTA stages in shared memory; a split covers at
+// most this many logical pages.
+constexpr int kMaxPagesPerSplit = 2048;
+// Upper bound on split-KV partitions.
+constexpr int kMaxSplits = 256;
+
+struct DecodeArgs {
+  const void *k_pool;
+  const void *v_pool;
+  const float *k_sz;
+  const float *v_sz;
+  int32_t num_pages;
+  int32_t hkv;
+  const void *q;  // bf16 [B][Hq][D]
+  int32_t B;
+  int32_t hq;
+  const int32_t *block_tables;
+  int32_t max_pages;
+  const int32_t *ctx;
+  float scale_log2;  // scale * log2(e)
+  float *out;        // final output (S == 1)
+  float *o_part;     // partials (S > 1)
+  float *lse;        // partial log-sum-exps (S > 1)
+  int32_t S;
+  int32_t pages_per_split;
+  int32_t *d_err;
+};
+
+cudaError_t launch_decode(int D, int P, int kv_dtype, const DecodeArgs &a,
+                          cudaStream_t stream);
+// CTAs of the decode kernel for (D, P, kv_dtype) that fit on one SM.
+int decode_ctas_per_sm(int D, int P, int kv_dtype);
+
+cudaError_t launch_splitkv_reduce(const float *o_part, const float *lse, int B,
+                                  int hq, int S, int D, float *out,
+                                  bool programmatic, cudaStream_t stream);
+
+cudaError_t launch_kv_append(const pa_kv_pool_t &pool, const void *k_new,
+                             const void *v_new, const int32_t *seq_idx,
+                             const int32_t *pos, int32_t n,
+                             const int32_t *block_tables, int32_t num_seqs,
+                             int32_t max_pages, int32_t *d_err,
+                             cudaStream_t stream);
+
+cudaError_t launch_validate_tables(const int32_t *block_tables, int32_t B,
+                                   int32_t max_pages, const int32_t *ctx,
+                                   int32_t num_pages, int32_t page_size,
+                                   int32_t *d_err, cudaStream_t stream);
+
+int device_sm_count();
+
+}  // namespace pa

@@ -1,0 +1,115 @@
+"""The C ABI without a GPU: the library loads, exports every function the
+header declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from paged_kv_cache_466_b200 import _lib
+from paged_kv_cache_466_b200._lib import (PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED,
+                                          PA_ERR_WORKSPACE, PA_OK, pa_kv_pool_t)
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", f)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", src))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from paged_kv_cache_466_b200 import build
+    build.build()
+    return _lib.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    declared = _declared()
+    assert {"pa_kv_append", "pa_decode", "pa_splitkv_reduce"} <= declared
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(_lib.SIGNATURES) == declared
+
+
+def test_version_and_status_strings(lib):
+    assert lib.pa_abi_version() == 1
+    for s in range(6):
+        assert lib.pa_status_str(s)
+    assert lib.pa_status_str(99) == b"unknown status"
+
+
+def _pool(**kw):
+    p = dict(num_pages=8, page_size=16, num_kv_heads=2, head_dim=128, dtype=0,
+             k_pool=0x1000, v_pool=0x2000, k_sz=None, v_sz=None)
+    p.update(kw)
+    return pa_kv_pool_t(**p)
+
+
+def _decode(lib, pool, B=2, Hq=4, max_pages=4, ws=None, ws_bytes=0, splits=0, q=0x3000,
+            out=0x4000, scale=0.1):
+    return lib.pa_decode(ctypes.byref(pool) if pool is not None else None, q, B, Hq, 0x5000,
+                         max_pages, 0x6000, scale, out, ws, ws_bytes, splits, None, None)
+
+
+def test_decode_rejects_bad_arguments(lib):
+    assert _decode(lib, None) == PA_ERR_INVALID_ARG
+    assert _decode(lib, _pool(head_dim=96)) == PA_ERR_UNSUPPORTED
+    assert _decode(lib, _pool(page_size=8)) == PA_ERR_UNSUPPORTED
+    assert _decode(lib, _pool(dtype=7)) == PA_ERR_UNSUPPORTED
+    assert _decode(lib, _pool(dtype=1)) == PA_ERR_INVALID_ARG          # no k_sz / v_sz
+    assert _decode(lib, _pool(k_pool=0x1001)) == PA_ERR_INVALID_ARG    # misaligned
+    assert _decode(lib, _pool(), Hq=5) == PA_ERR_INVALID_ARG           # 5 % 2 != 0
+    assert _decode(lib, _pool(), Hq=18) == PA_ERR_UNSUPPORTED          # group of 9
+    assert _decode(lib, _pool(), q=None) == PA_ERR_INVALID_ARG
+    assert _decode(lib, _pool(), out=0x4004) == PA_ERR_INVALID_ARG
+    assert _decode(lib, _pool(), scale=float("nan")) == PA_ERR_INVALID_ARG
+    assert _decode(lib, _pool(), splits=-1) == PA_ERR_INVALID_ARG
+    assert b"multiple" in lib.pa_last_error() or lib.pa_last_error()
+    # more than one split needs a workspace
+    assert _decode(lib, _pool(), splits=2) == PA_ERR_WORKSPACE
+    need = lib.pa_decode_workspace_bytes(2, 4, 128, 2)
+    assert _decode(lib, _pool(), splits=2, ws=0x10010, ws_bytes=need) == PA_ERR_WORKSPACE
+    assert _decode(lib, _pool(), splits=2, ws=0x10000, ws_bytes=need - 1) == PA_ERR_WORKSPACE
+    assert _decode(lib, _pool(), B=0) == PA_OK                          # nothing to do
+
+
+def test_append_and_reduce_reject_bad_arguments(lib):
+    pool = _pool()
+    args = [ctypes.byref(pool), 0x1000, 0x2000, 0x3000, 0x4000, 4, 0x5000, 2, 4, None, None]
+    bad = list(args); bad[1] = None
+    assert lib.pa_kv_append(*bad) == PA_ERR_INVALID_ARG
+    bad = list(args); bad[5] = -1
+    assert lib.pa_kv_append(*bad) == PA_ERR_INVALID_ARG
+    bad = list(args); bad[2] = 0x2002
+    assert lib.pa_kv_append(*bad) == PA_ERR_INVALID_ARG
+    bad = list(args); bad[5] = 0
+    assert lib.pa_kv_append(*bad) == PA_OK                              # empty append
+    assert lib.pa_splitkv_reduce(0x1000, 0x2000, 2, 4, 0, 128, 0x3000, None) == PA_ERR_INVALID_ARG
+    assert lib.pa_splitkv_reduce(0x1000, 0x2000, 2, 4, 2, 130, 0x3000, None) == PA_ERR_INVALID_ARG
+    assert lib.pa_splitkv_reduce(None, 0x2000, 2, 4, 2, 128, 0x3000, None) == PA_ERR_INVALID_ARG
+    assert lib.pa_splitkv_reduce(0x1000, 0x2000, 0, 4, 2, 128, 0x3000, None) == PA_OK
+    assert lib.pa_validate_tables(0x1000, 2, 4, 0x2000, 8, 16, None, None) == PA_ERR_INVALID_ARG
+
+
+def test_split_planning_and_workspace_size(lib):
+    pool = _pool(page_size=32)
+    for B, mp, req in [(32, 256, 0), (1, 1, 0), (64, 256, 5), (3, 4000, 1), (2, 100, 1000)]:
+        S = lib.pa_decode_num_splits(ctypes.byref(pool), B, mp, req)
+        assert 1 <= S <= min(mp, 256)
+        C = -(-mp // S)
+        assert -(-mp // C) == S                       # no empty split by construction
+        assert C <= 2048
+    assert lib.pa_decode_num_splits(ctypes.byref(pool), 4, 4000, 1) == 2   # 2048-entry cap
+    assert lib.pa_decode_num_splits(ctypes.byref(pool), 4, 0, 0) <= 0
+    assert lib.pa_decode_workspace_bytes(32, 64, 128, 1) == 0
+    ws = lib.pa_decode_workspace_bytes(32, 64, 128, 8)
+    o = 32 * 64 * 8 * 128 * 4
+    l = 32 * 64 * 8 * 4
+    assert ws == -(-o // 256) * 256 + -(-l // 256) * 256
