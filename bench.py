@@ -46,6 +46,8 @@ def parse():
                     choices=["llama70b", "llama8b", "int8", "prefix", "tiny"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--splits", type=int, default=0, help="split-KV count (0 = automatic)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's number of sequences (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
@@ -85,6 +87,22 @@ def recorded_traffic(workload: str):
     except Exception:
         pass
     return None
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Max of a per-rank number over all ranks (timing only; no data path)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(step_bytes_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Aggregate throughput: every rank's bytes over the slowest rank's time."""
+    return step_bytes_per_rank * world / (ms_per_step * 1e-3) / 1e9
 
 
 # ------------------------------------------------------------------ clocks
@@ -164,7 +182,7 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ CPU oracle leg
-def cpu_oracle_throughput(w, budget_s: float = 12.0, max_reps: int = 8):
+def cpu_oracle_throughput(w, budget_s: float = 12.0, max_reps: int = 40):
     """The fp64 oracle, as it stands, on this host's cores: the whole batch,
     repeated until ~budget_s of work. Returns (GB/s, cores, sample text)."""
     cores = len(os.sched_getaffinity(0))
@@ -188,13 +206,14 @@ def cpu_oracle_throughput(w, budget_s: float = 12.0, max_reps: int = 8):
 
 
 # ------------------------------------------------------------------ arms
-def make_workload(name: str, seed: int):
+def make_workload(name: str, seed: int, batch: int = 0):
     from paged_kv_cache_466_b200 import workloads as W
+    kw = {"B": batch} if batch else {}
     if name == "prefix":
-        return W.prefix(seed=seed)[0]
+        return W.prefix(seed=seed, **kw)[0]
     if name == "tiny":
         return W.tiny(seed=seed)
-    return getattr(W, name)(seed=seed)
+    return getattr(W, name)(seed=seed, **kw)
 
 
 def config_of(w, args, n, S):
@@ -217,7 +236,7 @@ def run_ours(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w = make_workload(args.workload, seed=rank)
+    w = make_workload(args.workload, seed=rank, batch=args.batch)
     pool = KVPool(w.num_pages, w.Hkv, w.P, w.D, w.kv, dev, fill_byte=0)
     bt = torch.from_numpy(w.block_tables).to(dev)
     ctx = torch.from_numpy(w.context_lens).to(dev)
@@ -269,15 +288,11 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     clk = clocks.stop()
     barrier()
-    ms = t0.elapsed_time(t1)
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
     dec_ms = [a.elapsed_time(b) for a, b in evs]
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
     ms_step = ms / K
     step_bytes = decode_bytes(w) + append_bytes(w)
-    value = step_bytes * world / (ms_step * 1e-3) / 1e9
+    value = whole_job_gbs(step_bytes, world, ms_step)
 
     # ---- end to end through the public API, host buffers in pinned memory
     h_q = w.q.pin_memory()
@@ -314,12 +329,8 @@ def run_ours(args, rank, world, local_rank):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    ems = e0.elapsed_time(e1)
-    if world > 1:
-        tt = torch.tensor([ems], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ems = float(tt.item())
-    e2e_value = step_bytes * world / (ems / Ke * 1e-3) / 1e9
+    ems = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = whole_job_gbs(step_bytes, world, ems / Ke)
 
     peak, peak_kind = measured_peak()
     dec_avg_ms = statistics.mean(dec_ms)
@@ -365,7 +376,7 @@ def run_reference(args, rank, world):
     os.environ.setdefault("OMP_NUM_THREADS", str(cores))
     import oracle
     from paged_kv_cache_466_b200.workloads import bits
-    w = make_workload(args.workload, seed=0)
+    w = make_workload(args.workload, seed=0, batch=args.batch)
     hp = oracle.empty_pool(w.kv, w.num_pages, w.Hkv, w.P, w.D, 0)
     seq, pos, k, v = w.all_rows()
     oracle.scatter_rows(hp, w.block_tables, seq, pos, bits(k), bits(v))
