@@ -164,6 +164,45 @@ pa_status_t pa_decode(const pa_kv_pool_t *pool, const void *q,
                       int32_t num_splits, int32_t *d_err, void *stream);
 
 /*
+ * pa_decode_noalloc — pa_decode for callers that cannot allocate device memory.
+ * The pages have no counterpart to this entry point: it only changes where
+ * pa_decode's split-KV scratch lives.
+ *
+ * Some callers have no way to obtain the workspace pa_decode asks for: a
+ * plugin or C host that is handed only its input and output buffers, a
+ * server that reserved all device memory up front for its own pool, or a
+ * latency-critical loop that must not pay the implicit synchronisation of
+ * cudaMalloc. This entry point takes the same arguments as pa_decode minus
+ * the workspace, and keeps the partial results and their log-sum-exps in a
+ * buffer that belongs to the library itself: a file-scope device array of
+ * PA_NOALLOC_SCRATCH_BYTES bytes, which every GPU that loads the library
+ * holds until the process exits. It calls no cudaMalloc, cudaFree or other
+ * allocating routine.
+ *
+ *   num_splits : 0 = automatic, lowered if needed until the partials fit the
+ *                scratch; an explicit count whose partials
+ *                (pa_decode_workspace_bytes) exceed PA_NOALLOC_SCRATCH_BYTES
+ *                is rejected with PA_ERR_WORKSPACE before any launch.
+ *
+ * Set-up: the first call on each device (with that device current) looks up
+ * the array's device address with cudaGetSymbolAddress; make that first call
+ * before any stream capture. Every call on a device shares the one array and
+ * it keeps the last call's contents; nothing in it needs to start at zero
+ * (each split writes its whole partial before the merge reads it). Calls
+ * that overlap on the GPU — on different streams or from different host
+ * threads without ordering between them — race on the array and must be
+ * serialised by the caller. Results equal pa_decode's for the same split count.
+ */
+#define PA_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+pa_status_t pa_decode_noalloc(const pa_kv_pool_t *pool, const void *q,
+                              int32_t num_seqs, int32_t num_q_heads,
+                              const int32_t *block_tables, int32_t max_pages,
+                              const int32_t *context_lens, float scale,
+                              float *out, int32_t num_splits, int32_t *d_err,
+                              void *stream);
+
+/*
  * pa_splitkv_reduce — merge split-KV partial results.
  * (Not on the pages: the exact identity for softmax over disjoint token
  * ranges. With M = max_s lse_s and w_s = exp(lse_s - M):

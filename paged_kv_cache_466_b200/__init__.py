@@ -13,6 +13,9 @@ Entry points (same names as the C ABI, see include/pagedattn.h):
 * ``pa_splitkv_reduce``  — log-sum-exp merge of split-KV partials
 * ``pa_validate_tables`` — device-side page-table check
 * ``pa_decode_num_splits`` / ``pa_decode_workspace_bytes`` — planning helpers
+* ``pa_decode_noalloc``  — pa_decode without a caller workspace, for callers
+                           that cannot allocate device memory (the scratch is
+                           a fixed-size array owned by the library)
 
 ``KVPool`` owns the page pool tensors; ``pages`` holds the host-side page
 allocator and cache-size formulas.
@@ -28,7 +31,8 @@ from . import _lib
 from ._lib import (PA_DERR_BAD_CTX, PA_DERR_BAD_PAGE, PA_DERR_BAD_POS, PA_DERR_BAD_SEQ,
                    PA_KV_BF16, PA_KV_U8_PER_TOKEN, PagedAttnError, pa_kv_pool_t)
 
-__all__ = ["KVPool", "pa_kv_append", "pa_decode", "pa_splitkv_reduce", "pa_validate_tables",
+__all__ = ["KVPool", "pa_kv_append", "pa_decode", "pa_decode_noalloc", "pa_splitkv_reduce",
+           "pa_validate_tables",
            "pa_decode_num_splits", "pa_decode_workspace_bytes", "PagedAttnError",
            "PA_KV_BF16", "PA_KV_U8_PER_TOKEN", "PA_DERR_BAD_PAGE", "PA_DERR_BAD_CTX",
            "PA_DERR_BAD_SEQ", "PA_DERR_BAD_POS", "load_library"]
@@ -157,6 +161,30 @@ def pa_decode(pool: KVPool, q: torch.Tensor, block_tables: torch.Tensor,
                                _ptr(workspace), ws_bytes, num_splits, _ptr(d_err),
                                _stream(stream))
     _lib.check(st, "pa_decode")
+    return out
+
+
+def pa_decode_noalloc(pool: KVPool, q: torch.Tensor, block_tables: torch.Tensor,
+                      context_lens: torch.Tensor, scale: float, out: torch.Tensor,
+                      num_splits: int = 0, d_err: Optional[torch.Tensor] = None,
+                      stream=None) -> torch.Tensor:
+    """pa_decode for callers that cannot allocate: the split-KV scratch is the
+    library's own fixed-size device array, so ``out`` must be given and nothing
+    is allocated here either. Calls that overlap on the GPU share that array
+    and must be ordered by the caller."""
+    dev = pool.device
+    _need(q, "q", torch.bfloat16, dev)
+    _need(block_tables, "block_tables", torch.int32, dev)
+    _need(context_lens, "context_lens", torch.int32, dev)
+    _need(out, "out", torch.float32, dev)
+    B, Hq, D = q.shape
+    if D != pool.head_dim or block_tables.shape[0] != B or context_lens.numel() != B \
+            or tuple(out.shape) != (B, Hq, D):
+        raise ValueError("pa_decode_noalloc: shape mismatch")
+    st = _lib.load().pa_decode_noalloc(ctypes.byref(pool.c), _ptr(q), B, Hq, _ptr(block_tables),
+                                       block_tables.shape[1], _ptr(context_lens), float(scale),
+                                       _ptr(out), num_splits, _ptr(d_err), _stream(stream))
+    _lib.check(st, "pa_decode_noalloc")
     return out
 
 

@@ -26,6 +26,8 @@ PA_DERR_BAD_POS = 8
 PA_KV_BF16 = 0
 PA_KV_U8_PER_TOKEN = 1
 
+PA_NOALLOC_SCRATCH_BYTES = 16 << 20
+
 
 class pa_kv_pool_t(ctypes.Structure):
     _fields_ = [
@@ -51,6 +53,7 @@ SIGNATURES = {
     "pa_decode_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "pa_decode": (_I, [_POOL, _P, _I, _I, _P, _I, _P, ctypes.c_float, _P, _P, ctypes.c_size_t,
                        _I, _P, _P]),
+    "pa_decode_noalloc": (_I, [_POOL, _P, _I, _I, _P, _I, _P, ctypes.c_float, _P, _I, _P, _P]),
     "pa_splitkv_reduce": (_I, [_P, _P, _I, _I, _I, _I, _P, _P]),
     "pa_validate_tables": (_I, [_P, _I, _I, _P, _I, _I, _P, _P]),
     "pa_status_str": (ctypes.c_char_p, [_I]),

@@ -69,6 +69,8 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
 
+void set_last_error_message(const char *msg) { g_last_error = msg; }
+
 int device_sm_count() {
   const int dev = current_device();
   if (dev < 0) return 148;
