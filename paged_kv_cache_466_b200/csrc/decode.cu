@@ -17,21 +17,24 @@
 // (or f16) high part and the residual low part and multiplied twice, which keeps
 // ~16 significant bits of every softmax weight.
 //
-// Data movement: every lane copies its own 16-byte pieces of K and V (cp.async,
-// L1 bypass, zero-fill past the context) into a private slot of a per-warp ring
-// of NSTAGE blocks in shared memory and later reads back only what it copied.
-// No lane ever reads another lane's staging, so the pipeline needs no barrier,
-// mbarrier or spin-wait: cp.async.wait_group per thread is the only wait.
+// Data movement: per warp, a ring of NSTAGE 16-token blocks in shared memory.
+// The warp copies each block with 16-byte cp.async (L1 bypass, zero-fill past
+// the context) such that every copy instruction moves 512 contiguous bytes of
+// a page, then waits for its own copies and joins the warp (__syncwarp) before
+// the lanes read the block back in mma-fragment order. No CTA barrier, mbarrier
+// or spin-wait is involved: cp.async.wait_group on the thread's own copies is
+// the only wait, and it always completes.
 //
-// The lane -> (token, d) assignment is chosen so that (i) every global access
-// of a warp covers whole 32-byte sectors, (ii) shared-memory accesses are
-// conflict free, and (iii) the loaded registers are already mma fragments:
-//   K: lane (g = lane/4, t = lane%4) loads token g of each 8-token half-block,
+// Fragment order (what each lane reads back), chosen so that the registers are
+// mma operands without shuffles:
+//   K: lane (g = lane/4, t = lane%4) reads token g of each 8-token half-block,
 //      16-byte chunks t, t+4, ... of its row. The contraction index (d) is
 //      permuted identically for Q, which is loaded with the same pattern.
-//   V: lane loads tokens {2t, 2t+1, 8+2t, 9+2t} (the B-fragment rows of P^T),
+//   V: lane reads tokens {2t, 2t+1, 8+2t, 9+2t} (the B-fragment rows of P^T),
 //      chunks {g, 8+g} (bf16) or chunk g (uint8); the output rows of O^T are
 //      permuted accordingly and un-permuted when stored.
+// Rows are stored with their 16-byte chunks XOR-permuted (staged_off) so that
+// both read patterns are free of shared-memory bank conflicts.
 //
 // INT8 cache (Eq. 3, "KV-Cache Quantization"): with x = s*c + z per row,
 //   q.x = s (q.c) + z sum(q)          and    sum_t p_t x_t = sum_t (p_t s_t) c_t + sum_t p_t z_t,
@@ -42,6 +45,21 @@
 
 #include "pa_device.cuh"
 #include "pa_internal.h"
+
+// Tile configuration (warps per CTA, pipeline depth per warp, CTAs per SM the
+// register allocation must allow); overridable at build time for tuning.
+#ifndef PA_DECODE_WARPS
+#define PA_DECODE_WARPS 4
+#endif
+#ifndef PA_DECODE_STAGES_BF16
+#define PA_DECODE_STAGES_BF16 2
+#endif
+#ifndef PA_DECODE_STAGES_U8
+#define PA_DECODE_STAGES_U8 4
+#endif
+#ifndef PA_DECODE_MIN_CTAS
+#define PA_DECODE_MIN_CTAS 3
+#endif
 
 namespace pa {
 namespace {
@@ -57,17 +75,33 @@ struct Tile {
   static constexpr bool kU8 = KVT == PA_KV_U8_PER_TOKEN;
   static constexpr int kElem = kU8 ? 1 : 2;
   static constexpr int kRowBytes = D * kElem;
-  // 16-byte K chunks a lane loads per 8-token half-block
+  // one 16-token block of K (or V) is 16 contiguous rows of the page
+  static constexpr int kBlockBytes = 16 * kRowBytes;
+  static constexpr int kCopies = kBlockBytes / 512;  // 16-byte copies per lane per tensor
+  static constexpr int kSzBytes = kU8 ? 16 * 8 : 0;  // (scale, zero) of 16 rows
+  static constexpr int kVOff = kBlockBytes;
+  static constexpr int kKSzOff = 2 * kBlockBytes;
+  static constexpr int kVSzOff = 2 * kBlockBytes + kSzBytes;
+  static constexpr int kStageBytes = 2 * kBlockBytes + 2 * kSzBytes;
+  // 16-byte K chunks a lane reads per 8-token half-block (fragment layout)
   static constexpr int kKChunks = kU8 ? D / 64 : D / 32;
-  static constexpr int kKItems = 2 * kKChunks;
-  // 16-byte V chunks a lane loads per token (4 tokens per block)
+  // 16-byte V chunks a lane reads per token
   static constexpr int kVChunks = kU8 ? 1 : D / 64;
-  static constexpr int kVItems = 4 * kVChunks;
-  static constexpr int kSzItems = kU8 ? 4 : 0;
-  static constexpr int kItems = kKItems + kVItems + kSzItems;
-  static constexpr int kStageBytes = kItems * 32 * 16;
   static constexpr int kMTiles = D / 16;  // m16 tiles of O^T
+  // rows of at least 128 bytes are stored with their 16-byte chunks permuted
+  // (chunk ^ swz(row)), which makes both fragment read patterns conflict free
+  static constexpr bool kSwizzle = kRowBytes >= 128;
 };
+
+// Shared-memory byte offset of 16-byte chunk `chunk` of row `row` in a staged
+// block. swz(row) = 2*((row >> 1) & 3) ^ 4*(row & 1) keeps the chunk inside its
+// 128-byte group; lanes reading (row g, chunk 4i+t) for K and (row 2t+e, chunk
+// g) for V then touch 8 distinct bank groups per quarter warp.
+template <class T>
+__device__ __forceinline__ int staged_off(int row, int chunk) {
+  const int swz = T::kSwizzle ? ((2 * ((row >> 1) & 3)) ^ (4 * (row & 1))) : 0;
+  return row * T::kRowBytes + ((chunk ^ swz) << 4);
+}
 
 template <int D, int KVT, int W, int NSTAGE>
 struct Smem {
@@ -93,7 +127,7 @@ __device__ __forceinline__ int out_col(int j, int g) {
 }
 
 template <int D, int P, int KVT, int W, int NSTAGE>
-__global__ void __launch_bounds__(W * 32, 2) decode_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(const DecodeArgs a) {
   using T = Tile<D, KVT>;
   using SM = Smem<D, KVT, W, NSTAGE>;
   static_assert(P % 16 == 0, "a 16-token block must not straddle pages");
@@ -170,7 +204,10 @@ __global__ void __launch_bounds__(W * 32, 2) decode_kernel(const DecodeArgs a) {
   __syncthreads();  // tbl visible
 
   // ---- per-warp pipeline ---------------------------------------------------------
-  const uint32_t ring = smem_u32(smem) + warp * SM::kRingBytesPerWarp + lane * 16;
+  // Each lane copies 16-byte pieces of a block so that every copy instruction
+  // of the warp moves 512 contiguous bytes; after the wait, lanes read the
+  // pieces in mma-fragment order (cross-lane, hence the __syncwarp).
+  const uint32_t ring = smem_u32(smem) + warp * SM::kRingBytesPerWarp;
   const unsigned char *kbase = static_cast<const unsigned char *>(a.k_pool);
   const unsigned char *vbase = static_cast<const unsigned char *>(a.v_pool);
   const int nmine = nblk > warp ? (nblk - warp + W - 1) / W : 0;
@@ -180,51 +217,49 @@ __global__ void __launch_bounds__(W * 32, 2) decode_kernel(const DecodeArgs a) {
     const int lp = btok / P;
     const int page = tbl[lp - lp0];
     const int in_page = btok - lp * P;
-    const bool pvalid = page >= 0;
-    const size_t row0 = ((size_t)(pvalid ? page : 0) * a.hkv + h) * P + in_page;
+    const int nvalid = page >= 0 ? min(16, tok1 - btok) : 0;  // rows holding tokens
+    const size_t row0 = ((size_t)(page >= 0 ? page : 0) * a.hkv + h) * P + in_page;
     const uint32_t dst = ring + st * T::kStageBytes;
-    // K: token g (and 8 + g), chunks t, t+4, ...
+    const unsigned char *ksrc = kbase + row0 * T::kRowBytes;
+    const unsigned char *vsrc = vbase + row0 * T::kRowBytes;
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      const int toff = nt * 8 + g;
-      const bool ok = pvalid && btok + toff < tok1;
-#pragma unroll
-      for (int i = 0; i < T::kKChunks; ++i) {
-        const unsigned char *src = kbase + (row0 + toff) * T::kRowBytes + (4 * i + t) * 16;
-        cp_async16(dst + (nt * T::kKChunks + i) * 512, ok ? src : kbase, ok ? 16u : 0u);
-      }
-    }
-    // V: tokens 2t, 2t+1, 8+2t, 9+2t
-#pragma unroll
-    for (int tau = 0; tau < 4; ++tau) {
-      const int toff = (tau & 1) + 2 * t + (tau >> 1) * 8;
-      const bool ok = pvalid && btok + toff < tok1;
-#pragma unroll
-      for (int c = 0; c < T::kVChunks; ++c) {
-        const int chunk = T::kU8 ? (D == 128 ? g : (g >> 1)) : 8 * c + g;
-        const unsigned char *src = vbase + (row0 + toff) * T::kRowBytes + chunk * 16;
-        cp_async16(dst + (T::kKItems + tau * T::kVChunks + c) * 512, ok ? src : vbase,
-                   ok ? 16u : 0u);
-      }
+    for (int j = 0; j < T::kCopies; ++j) {
+      const int o = j * 512 + lane * 16;
+      const int r = o / T::kRowBytes;
+      const int so = staged_off<T>(r, (o % T::kRowBytes) >> 4);
+      const bool ok = r < nvalid;
+      cp_async16(dst + so, ok ? ksrc + o : kbase, ok ? 16u : 0u);
+      cp_async16(dst + T::kVOff + so, ok ? vsrc + o : vbase, ok ? 16u : 0u);
     }
     if constexpr (T::kU8) {
-      // (scale, zero) pairs of tokens (2t, 2t+1) and (8+2t, 9+2t), K then V
-#pragma unroll
-      for (int kv = 0; kv < 2; ++kv) {
-        const float *szb = kv == 0 ? a.k_sz : a.v_sz;
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          const int toff = nt * 8 + 2 * t;
-          const int tok = btok + toff;
-          const uint32_t nbytes = !pvalid ? 0u : (tok + 1 < tok1 ? 16u : (tok < tok1 ? 8u : 0u));
-          const float *src = szb + (row0 + toff) * 2;
-          cp_async16(dst + (T::kKItems + T::kVItems + kv * 2 + nt) * 512,
-                     nbytes ? static_cast<const void *>(src) : static_cast<const void *>(szb),
-                     nbytes);
-        }
+      // lanes 0..7: K (scale, zero) of rows 2l, 2l+1; lanes 8..15: V
+      if (lane < 16) {
+        const int l = lane & 7;
+        const float *szb = lane < 8 ? a.k_sz : a.v_sz;
+        const uint32_t nbytes = 2 * l + 1 < nvalid ? 16u : (2 * l < nvalid ? 8u : 0u);
+        cp_async16(dst + (lane < 8 ? T::kKSzOff : T::kVSzOff) + l * 16,
+                   nbytes ? static_cast<const void *>(szb + (row0 + 2 * l) * 2)
+                          : static_cast<const void *>(szb),
+                   nbytes);
       }
     }
   };
+
+  // per-lane offsets of the fragment reads within a stage
+  int koff[2][T::kKChunks];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int i = 0; i < T::kKChunks; ++i) koff[nt][i] = staged_off<T>(nt * 8 + g, 4 * i + t);
+  int voff[4][T::kVChunks];
+#pragma unroll
+  for (int tau = 0; tau < 4; ++tau)
+#pragma unroll
+    for (int c = 0; c < T::kVChunks; ++c) {
+      const int row = (tau & 1) + 2 * t + (tau >> 1) * 8;
+      const int chunk = T::kU8 ? (D == 128 ? g : (g >> 1)) : 8 * c + g;
+      voff[tau][c] = T::kVOff + staged_off<T>(row, chunk);
+    }
 
   float o[T::kMTiles][4];
 #pragma unroll
@@ -247,6 +282,7 @@ __global__ void __launch_bounds__(W * 32, 2) decode_kernel(const DecodeArgs a) {
       cp_async_commit();
     }
     cp_async_wait<NSTAGE - 1>();
+    __syncwarp();  // every lane's pieces of this block are now visible to the warp
 
     const int kb = warp + k * W;
     const int btok = tok0 + kb * 16;
@@ -260,7 +296,7 @@ __global__ void __launch_bounds__(W * 32, 2) decode_kernel(const DecodeArgs a) {
       s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
 #pragma unroll
       for (int i = 0; i < T::kKChunks; ++i) {
-        const uint4 kv = lds128(src + (nt * T::kKChunks + i) * 512);
+        const uint4 kv = lds128(src + koff[nt][i]);
         if constexpr (!T::kU8) {
           mma_bf16_16816(s[nt], qa[2 * i][0], 0u, qa[2 * i][1], 0u, kv.x, kv.y);
           mma_bf16_16816(s[nt], qa[2 * i + 1][0], 0u, qa[2 * i + 1][1], 0u, kv.z, kv.w);
@@ -279,10 +315,10 @@ __global__ void __launch_bounds__(W * 32, 2) decode_kernel(const DecodeArgs a) {
     float x[4] = {s[0][0], s[0][1], s[1][0], s[1][1]};  // tokens 2t, 2t+1, 8+2t, 9+2t
     float vs[4], vz[4];
     if constexpr (T::kU8) {
-      const uint4 k01 = lds128(src + (T::kKItems + T::kVItems + 0) * 512);
-      const uint4 k89 = lds128(src + (T::kKItems + T::kVItems + 1) * 512);
-      const uint4 v01 = lds128(src + (T::kKItems + T::kVItems + 2) * 512);
-      const uint4 v89 = lds128(src + (T::kKItems + T::kVItems + 3) * 512);
+      const uint4 k01 = lds128(src + T::kKSzOff + 16 * t);
+      const uint4 k89 = lds128(src + T::kKSzOff + 16 * (4 + t));
+      const uint4 v01 = lds128(src + T::kVSzOff + 16 * t);
+      const uint4 v89 = lds128(src + T::kVSzOff + 16 * (4 + t));
       const float ks[4] = {__uint_as_float(k01.x), __uint_as_float(k01.z),
                            __uint_as_float(k89.x), __uint_as_float(k89.z)};
       const float kz[4] = {__uint_as_float(k01.y), __uint_as_float(k01.w),
@@ -332,10 +368,10 @@ __global__ void __launch_bounds__(W * 32, 2) decode_kernel(const DecodeArgs a) {
       split_bf16(p[2], p[3], bh1, bl1);
 #pragma unroll
       for (int c = 0; c < T::kVChunks; ++c) {
-        const uint4 v0 = lds128(src + (T::kKItems + 0 * T::kVChunks + c) * 512);
-        const uint4 v1 = lds128(src + (T::kKItems + 1 * T::kVChunks + c) * 512);
-        const uint4 v2 = lds128(src + (T::kKItems + 2 * T::kVChunks + c) * 512);
-        const uint4 v3 = lds128(src + (T::kKItems + 3 * T::kVChunks + c) * 512);
+        const uint4 v0 = lds128(src + voff[0][c]);
+        const uint4 v1 = lds128(src + voff[1][c]);
+        const uint4 v2 = lds128(src + voff[2][c]);
+        const uint4 v3 = lds128(src + voff[3][c]);
         const uint32_t x0[4] = {v0.x, v0.y, v0.z, v0.w};
         const uint32_t x1[4] = {v1.x, v1.y, v1.z, v1.w};
         const uint32_t x2[4] = {v2.x, v2.y, v2.z, v2.w};
@@ -359,10 +395,10 @@ __global__ void __launch_bounds__(W * 32, 2) decode_kernel(const DecodeArgs a) {
       }
       split_f16(pv[0], pv[1], bh0, bl0);
       split_f16(pv[2], pv[3], bh1, bl1);
-      const uint4 v0 = lds128(src + (T::kKItems + 0) * 512);
-      const uint4 v1 = lds128(src + (T::kKItems + 1) * 512);
-      const uint4 v2 = lds128(src + (T::kKItems + 2) * 512);
-      const uint4 v3 = lds128(src + (T::kKItems + 3) * 512);
+      const uint4 v0 = lds128(src + voff[0][0]);
+      const uint4 v1 = lds128(src + voff[1][0]);
+      const uint4 v2 = lds128(src + voff[2][0]);
+      const uint4 v3 = lds128(src + voff[3][0]);
       const uint32_t x0[4] = {v0.x, v0.y, v0.z, v0.w};
       const uint32_t x1[4] = {v1.x, v1.y, v1.z, v1.w};
       const uint32_t x2[4] = {v2.x, v2.y, v2.z, v2.w};
@@ -454,8 +490,9 @@ __global__ void __launch_bounds__(W * 32, 2) decode_kernel(const DecodeArgs a) {
 
 template <int D, int P, int KVT>
 struct Config {
-  static constexpr int W = 4;
-  static constexpr int NSTAGE = KVT == PA_KV_U8_PER_TOKEN ? 4 : 3;
+  static constexpr int W = PA_DECODE_WARPS;
+  static constexpr int NSTAGE =
+      KVT == PA_KV_U8_PER_TOKEN ? PA_DECODE_STAGES_U8 : PA_DECODE_STAGES_BF16;
   using SM = Smem<D, KVT, W, NSTAGE>;
   static void *fn() { return reinterpret_cast<void *>(&decode_kernel<D, P, KVT, W, NSTAGE>); }
 };

@@ -17,8 +17,8 @@ namespace {
 constexpr int kWarps = 4;
 
 __global__ void __launch_bounds__(kWarps * 32) splitkv_reduce_kernel(
-    const float *__restrict__ o_part, const float *__restrict__ lse, int rows, int S,
-    int D, float *__restrict__ out) {
+    const float *__restrict__ o_part, const float *__restrict__ lse, int rows, int S, int D,
+    float *__restrict__ out) {
   pdl_wait_primary();  // partials come from the kernel just before us
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -32,28 +32,35 @@ __global__ void __launch_bounds__(kWarps * 32) splitkv_reduce_kernel(
   const float4 *op = reinterpret_cast<const float4 *>(o_part + (size_t)row * S * D);
   float4 *dst = reinterpret_cast<float4 *>(out + (size_t)row * D);
   const int D4 = D / 4;
-  for (int i = lane; i < D4; i += 32) {
+  for (int i0 = 0; i0 < D4; i0 += 32) {
+    const int i = i0 + lane;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float den = 0.f;
-    if (M != -INFINITY) {
-      for (int s = 0; s < S; ++s) {
-        const float w = expf(ls[s] - M);  // lse = -inf (empty split) -> 0
-        const float4 v = op[(size_t)s * D4 + i];
-        acc.x = fmaf(w, v.x, acc.x);
-        acc.y = fmaf(w, v.y, acc.y);
-        acc.z = fmaf(w, v.z, acc.z);
-        acc.w = fmaf(w, v.w, acc.w);
-        den += w;
+    // splits in chunks of 32: lane s holds the weight of split s0 + s, and
+    // every lane then issues its loads for the whole chunk back to back
+    for (int s0 = 0; s0 < S; s0 += 32) {
+      const int n = min(32, S - s0);
+      const float wl =
+          (lane < n && M != -INFINITY) ? expf(ls[s0 + lane] - M) : 0.f;  // -inf -> 0
+      den += wl;
+#pragma unroll 8
+      for (int s = 0; s < n; ++s) {
+        const float w = __shfl_sync(0xffffffffu, wl, s);
+        if (i < D4) {
+          const float4 v = op[(size_t)(s0 + s) * D4 + i];
+          acc.x = fmaf(w, v.x, acc.x);
+          acc.y = fmaf(w, v.y, acc.y);
+          acc.z = fmaf(w, v.z, acc.z);
+          acc.w = fmaf(w, v.w, acc.w);
+        }
       }
     }
-    if (den > 0.f) {
-      const float r = 1.f / den;
-      acc.x *= r;
-      acc.y *= r;
-      acc.z *= r;
-      acc.w *= r;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    if (i < D4) {
+      const float r = den > 0.f ? 1.f / den : 0.f;
+      dst[i] = make_float4(acc.x * r, acc.y * r, acc.z * r, acc.w * r);
     }
-    dst[i] = acc;
   }
 }
 
