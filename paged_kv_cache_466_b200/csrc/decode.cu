@@ -157,6 +157,20 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
   const int tok1 = min(lp1 * P, ctx);
   const int nblk = tok1 > tok0 ? (tok1 - tok0 + 15) / 16 : 0;
 
+  if (nblk == 0) {
+    // Nothing to attend in this split: an empty partial (lse = -inf; the merge
+    // gives it weight 0 and never reads its o) or, for an empty context, 0.
+    for (int e = threadIdx.x; e < (a.S == 1 ? G * D : G); e += W * 32) {
+      if (a.S == 1) {
+        a.out[((size_t)b * a.hq + (size_t)h * G) * D + e] = 0.f;
+      } else {
+        a.lse[((size_t)b * a.hq + (size_t)h * G + e) * a.S + split] = -INFINITY;
+      }
+    }
+    pdl_launch_dependents();
+    return;
+  }
+
   // ---- stage this split's block-table entries (bounds-checked) --------------
   for (int i = threadIdx.x; i < lp1 - lp0; i += W * 32) {
     int pg = __ldg(a.block_tables + (size_t)b * a.max_pages + lp0 + i);
@@ -212,35 +226,41 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
   const unsigned char *vbase = static_cast<const unsigned char *>(a.v_pool);
   const int nmine = nblk > warp ? (nblk - warp + W - 1) / W : 0;
 
+  // lane-constant parts of the copies: byte offset in the block, its row and
+  // its swizzled place in the stage
+  int cp_row[T::kCopies], cp_soff[T::kCopies];
+#pragma unroll
+  for (int j = 0; j < T::kCopies; ++j) {
+    const int o = j * 512 + lane * 16;
+    cp_row[j] = o / T::kRowBytes;
+    cp_soff[j] = staged_off<T>(cp_row[j], (o % T::kRowBytes) >> 4);
+  }
+  const float *sz_base = lane < 8 ? a.k_sz : a.v_sz;
+  const int sz_dst = (lane < 8 ? T::kKSzOff : T::kVSzOff) + (lane & 7) * 16;
+
   auto issue = [&](int kb, int st) {
     const int btok = tok0 + kb * 16;
     const int lp = btok / P;
     const int page = tbl[lp - lp0];
     const int in_page = btok - lp * P;
     const int nvalid = page >= 0 ? min(16, tok1 - btok) : 0;  // rows holding tokens
+    // rows of an invalid page are zero-filled; the address stays inside page 0
     const size_t row0 = ((size_t)(page >= 0 ? page : 0) * a.hkv + h) * P + in_page;
     const uint32_t dst = ring + st * T::kStageBytes;
-    const unsigned char *ksrc = kbase + row0 * T::kRowBytes;
-    const unsigned char *vsrc = vbase + row0 * T::kRowBytes;
+    const unsigned char *ksrc = kbase + row0 * T::kRowBytes + lane * 16;
+    const unsigned char *vsrc = vbase + row0 * T::kRowBytes + lane * 16;
 #pragma unroll
     for (int j = 0; j < T::kCopies; ++j) {
-      const int o = j * 512 + lane * 16;
-      const int r = o / T::kRowBytes;
-      const int so = staged_off<T>(r, (o % T::kRowBytes) >> 4);
-      const bool ok = r < nvalid;
-      cp_async16(dst + so, ok ? ksrc + o : kbase, ok ? 16u : 0u);
-      cp_async16(dst + T::kVOff + so, ok ? vsrc + o : vbase, ok ? 16u : 0u);
+      const uint32_t n = cp_row[j] < nvalid ? 16u : 0u;
+      cp_async16(dst + cp_soff[j], ksrc + j * 512, n);
+      cp_async16(dst + T::kVOff + cp_soff[j], vsrc + j * 512, n);
     }
     if constexpr (T::kU8) {
       // lanes 0..7: K (scale, zero) of rows 2l, 2l+1; lanes 8..15: V
       if (lane < 16) {
         const int l = lane & 7;
-        const float *szb = lane < 8 ? a.k_sz : a.v_sz;
         const uint32_t nbytes = 2 * l + 1 < nvalid ? 16u : (2 * l < nvalid ? 8u : 0u);
-        cp_async16(dst + (lane < 8 ? T::kKSzOff : T::kVSzOff) + l * 16,
-                   nbytes ? static_cast<const void *>(szb + (row0 + 2 * l) * 2)
-                          : static_cast<const void *>(szb),
-                   nbytes);
+        cp_async16(dst + sz_dst, sz_base + (row0 + 2 * l) * 2, nbytes);
       }
     }
   };
@@ -330,10 +350,15 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
 #pragma unroll
       for (int e = 0; e < 4; ++e) x[e] = fmaf(ks[e], x[e], kz[e] * qsum);
     }
+    if (pvalid && btok + 16 <= tok1) {  // warp-uniform: a full block needs no mask
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int toff = (e & 1) + 2 * t + (e >> 1) * 8;
-      x[e] = (pvalid && btok + toff < tok1) ? x[e] * a.scale_log2 : -INFINITY;
+      for (int e = 0; e < 4; ++e) x[e] *= a.scale_log2;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int toff = (e & 1) + 2 * t + (e >> 1) * 8;
+        x[e] = (pvalid && btok + toff < tok1) ? x[e] * a.scale_log2 : -INFINITY;
+      }
     }
     float mb = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
     mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));

@@ -46,7 +46,7 @@ __global__ void __launch_bounds__(kWarps * 32) splitkv_reduce_kernel(
 #pragma unroll 8
       for (int s = 0; s < n; ++s) {
         const float w = __shfl_sync(0xffffffffu, wl, s);
-        if (i < D4) {
+        if (i < D4 && w != 0.f) {  // weight-0 (empty) splits are never read
           const float4 v = op[(size_t)(s0 + s) * D4 + i];
           acc.x = fmaf(w, v.x, acc.x);
           acc.y = fmaf(w, v.y, acc.y);
