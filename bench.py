@@ -251,7 +251,7 @@ def run_ours(args, rank, world, local_rank):
     sseq = torch.from_numpy(w.step_seq).to(dev)
     spos = torch.from_numpy(w.step_pos).to(dev)
     S = pa_decode_num_splits(pool, w.B, w.max_pages, args.splits)
-    ws = torch.empty(max(pa_decode_workspace_bytes(w.B, w.Hq, w.D, S), 256), dtype=torch.uint8,
+    ws = torch.zeros(max(pa_decode_workspace_bytes(w.B, w.Hq, w.D, S), 256), dtype=torch.uint8,
                      device=dev)
     out = torch.empty((w.B, w.Hq, w.D), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()

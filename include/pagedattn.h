@@ -129,9 +129,11 @@ int32_t pa_decode_num_splits(const pa_kv_pool_t *pool, int32_t num_seqs,
 /*
  * pa_decode_workspace_bytes — device scratch pa_decode needs for
  * num_splits (already resolved, >= 1): 0 when num_splits == 1, else the
- * partial outputs fp32 [num_seqs][num_q_heads][num_splits][head_dim] plus
- * their log-sum-exps fp32 [num_seqs][num_q_heads][num_splits], each part
- * 256-byte aligned.
+ * partial outputs fp32 [num_seqs][num_q_heads][num_splits][head_dim], their
+ * log-sum-exps fp32 [num_seqs][num_q_heads][num_splits] and one int32 split
+ * counter per (sequence, KV head) (num_seqs * num_q_heads are reserved), each
+ * part 256-byte aligned. The counters must be zero before a workspace's first
+ * use (allocate it zero-filled); every completed pa_decode leaves them zero.
  */
 size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
                                  int32_t head_dim, int32_t num_splits);
@@ -151,10 +153,14 @@ size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
  *   num_splits   : 0 = automatic; the count actually used is always
  *                  pa_decode_num_splits(pool, num_seqs, max_pages, num_splits)
  * num_q_heads must be a multiple of pool->num_kv_heads with a ratio of 1..8.
- * A sequence with context length 0 gets out = 0. When more than one split is
- * used the partial results are merged by their log-sum-exp in a second
- * kernel on the same stream (pa_splitkv_reduce). Results are deterministic
- * and do not depend on the physical page ids.
+ * A sequence with context length 0 gets out = 0. When a sequence spans more
+ * than one split, each split writes a partial result and its log-sum-exp to
+ * the workspace and the split that finishes last merges them (in split order,
+ * the same arithmetic as pa_splitkv_reduce) — one kernel launch in all.
+ * The kernel is launched as a programmatic dependent of the previous kernel
+ * on the stream and waits for it before reading any input. Results are
+ * deterministic and do not depend on the physical page ids. Two calls that
+ * share a workspace must not overlap on the GPU.
  */
 pa_status_t pa_decode(const pa_kv_pool_t *pool, const void *q,
                       int32_t num_seqs, int32_t num_q_heads,
@@ -187,11 +193,12 @@ pa_status_t pa_decode(const pa_kv_pool_t *pool, const void *q,
  * Set-up: the first call on each device (with that device current) looks up
  * the array's device address with cudaGetSymbolAddress; make that first call
  * before any stream capture. Every call on a device shares the one array and
- * it keeps the last call's contents; nothing in it needs to start at zero
- * (each split writes its whole partial before the merge reads it). Calls
- * that overlap on the GPU — on different streams or from different host
- * threads without ordering between them — race on the array and must be
- * serialised by the caller. Results equal pa_decode's for the same split count.
+ * it keeps the last call's contents. The only part that must start at zero is
+ * the split counters, which the array holds from load time and which every
+ * completed call returns to zero. Calls that overlap on the GPU — on
+ * different streams or from different host threads without ordering between
+ * them — race on the array and must be serialised by the caller. Results
+ * equal pa_decode's for the same split count.
  */
 #define PA_NOALLOC_SCRATCH_BYTES (16u << 20)
 

@@ -137,8 +137,8 @@ def pa_decode(pool: KVPool, q: torch.Tensor, block_tables: torch.Tensor,
               d_err: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """Eq. 1 decode: q [B, Hq, D] bf16 -> out [B, Hq, D] fp32.
 
-    ``workspace`` (uint8, >= pa_decode_workspace_bytes) is allocated with torch
-    when not given.
+    ``workspace`` (uint8, >= pa_decode_workspace_bytes, zero-filled before its
+    first use) is allocated zero-filled with torch when not given.
     """
     dev = pool.device
     _need(q, "q", torch.bfloat16, dev)
@@ -151,10 +151,11 @@ def pa_decode(pool: KVPool, q: torch.Tensor, block_tables: torch.Tensor,
         out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
     _need(out, "out", torch.float32, dev)
     max_pages = block_tables.shape[1]
-    S = pa_decode_num_splits(pool, B, max_pages, num_splits)
-    need = pa_decode_workspace_bytes(B, Hq, D, S)
-    if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if workspace is None:
+        S = pa_decode_num_splits(pool, B, max_pages, num_splits)
+        need = pa_decode_workspace_bytes(B, Hq, D, S)
+        if need > 0:
+            workspace = torch.zeros(need, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = _lib.load().pa_decode(ctypes.byref(pool.c), _ptr(q), B, Hq, _ptr(block_tables),
                                max_pages, _ptr(context_lens), float(scale), _ptr(out),

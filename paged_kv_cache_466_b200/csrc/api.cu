@@ -188,7 +188,7 @@ size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t 
   if (num_splits <= 1 || num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0) return 0;
   const size_t rows = (size_t)num_seqs * num_q_heads;
   return align256(rows * num_splits * head_dim * sizeof(float)) +
-         align256(rows * num_splits * sizeof(float));
+         align256(rows * num_splits * sizeof(float)) + align256(rows * sizeof(int32_t));
 }
 
 pa_status_t pa_decode(const pa_kv_pool_t *pool, const void *q, int32_t num_seqs,
@@ -246,19 +246,18 @@ pa_status_t pa_decode(const pa_kv_pool_t *pool, const void *q, int32_t num_seqs,
   a.scale_log2 = scale * 1.4426950408889634f;
   a.out = out;
   a.o_part = S > 1 ? static_cast<float *>(workspace) : nullptr;
-  a.lse = S > 1 ? reinterpret_cast<float *>(static_cast<char *>(workspace) +
-                                            align256(rows * S * pool->head_dim * sizeof(float)))
-                : nullptr;
+  const size_t o_bytes = align256(rows * S * pool->head_dim * sizeof(float));
+  const size_t l_bytes = align256(rows * S * sizeof(float));
+  a.lse = S > 1 ? reinterpret_cast<float *>(static_cast<char *>(workspace) + o_bytes) : nullptr;
+  a.counters = S > 1 ? reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + o_bytes +
+                                                   l_bytes)
+                     : nullptr;
   a.S = S;
   a.pages_per_split = chunk;
   a.d_err = d_err;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  st = cuda_status(launch_decode(pool->head_dim, pool->page_size, pool->dtype, a, s),
-                   "pa_decode launch");
-  if (st != PA_OK || S == 1) return st;
-  return cuda_status(launch_splitkv_reduce(a.o_part, a.lse, num_seqs, num_q_heads, S,
-                                           pool->head_dim, out, true, s),
-                     "pa_decode merge launch");
+  return cuda_status(launch_decode(pool->head_dim, pool->page_size, pool->dtype, a,
+                                   static_cast<cudaStream_t>(stream)),
+                     "pa_decode launch");
 }
 
 pa_status_t pa_splitkv_reduce(const float *o_part, const float *lse, int32_t num_seqs,

@@ -40,6 +40,7 @@
 //   q.x = s (q.c) + z sum(q)          and    sum_t p_t x_t = sum_t (p_t s_t) c_t + sum_t p_t z_t,
 // so the codes go through the tensor cores as exact f16 integers and the scale
 // and zero are applied once per (token, head) instead of once per element.
+#include <atomic>
 #include <cfloat>
 #include <cmath>
 
@@ -59,6 +60,9 @@
 #endif
 #ifndef PA_DECODE_MIN_CTAS
 #define PA_DECODE_MIN_CTAS 3
+#endif
+#ifndef PA_DECODE_PDL
+#define PA_DECODE_PDL 1
 #endif
 
 namespace pa {
@@ -133,6 +137,10 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
   static_assert(P % 16 == 0, "a 16-token block must not straddle pages");
   extern __shared__ __align__(128) unsigned char smem[];
 
+  // Launched as a programmatic dependent: wait until the previous kernel on
+  // the stream (e.g. the cache write) has finished and its writes are visible.
+  pdl_wait_primary();
+
   const int split = blockIdx.x;
   const int h = blockIdx.y;
   const int b = blockIdx.z;
@@ -157,17 +165,13 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
   const int tok1 = min(lp1 * P, ctx);
   const int nblk = tok1 > tok0 ? (tok1 - tok0 + 15) / 16 : 0;
 
+  // splits [0, n_live) of this sequence hold tokens; the others have no work
+  const int n_live = (n_pages + a.pages_per_split - 1) / a.pages_per_split;
   if (nblk == 0) {
-    // Nothing to attend in this split: an empty partial (lse = -inf; the merge
-    // gives it weight 0 and never reads its o) or, for an empty context, 0.
-    for (int e = threadIdx.x; e < (a.S == 1 ? G * D : G); e += W * 32) {
-      if (a.S == 1) {
+    if (split == 0 && n_live == 0) {  // empty context: the output is 0
+      for (int e = threadIdx.x; e < G * D; e += W * 32)
         a.out[((size_t)b * a.hq + (size_t)h * G) * D + e] = 0.f;
-      } else {
-        a.lse[((size_t)b * a.hq + (size_t)h * G + e) * a.S + split] = -INFINITY;
-      }
     }
-    pdl_launch_dependents();
     return;
   }
 
@@ -503,14 +507,73 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
     }
     const size_t row = (size_t)b * a.hq + (size_t)h * G + hd;
     const float val = L > 0.f ? num / L : 0.f;
-    if (a.S == 1) {
+    if (n_live == 1) {
       a.out[row * D + d] = val;
     } else {
       a.o_part[(row * a.S + split) * D + d] = val;
       if (d == 0) a.lse[row * a.S + split] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
     }
   }
-  pdl_launch_dependents();
+  if (n_live == 1) return;
+
+  // ---- split-KV merge, done by whichever CTA of this (sequence, KV head)
+  // finishes last. Partials are made visible device-wide before the ticket is
+  // taken; the merge visits splits in index order, so the result does not
+  // depend on which CTA merges. The last CTA also re-arms the counter.
+  __shared__ int s_last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int ticket = atomicAdd(a.counters + (size_t)b * a.hkv + h, 1);
+    s_last = ticket == n_live - 1;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // weights exp(lse_s - M) / sum, per head, staged in shared memory (the warp
+  // records are no longer needed); then each thread streams its float4 columns
+  // of every split's partial, all loads independent
+  float *wts = reinterpret_cast<float *>(smem);  // [G][n_live]
+  for (int i = threadIdx.x; i < G * n_live; i += W * 32) {
+    const int hd = i / n_live;
+    const int sp = i - hd * n_live;
+    wts[i] = __ldcg(a.lse + ((size_t)b * a.hq + (size_t)h * G + hd) * a.S + sp);
+  }
+  __syncthreads();
+  if (threadIdx.x < G) {
+    float *wh = wts + threadIdx.x * n_live;
+    float M = -INFINITY;
+    for (int sp = 0; sp < n_live; ++sp) M = fmaxf(M, wh[sp]);
+    float den = 0.f;
+    for (int sp = 0; sp < n_live; ++sp) {
+      const float wv = M == -INFINITY ? 0.f : expf(wh[sp] - M);
+      wh[sp] = wv;
+      den += wv;
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    for (int sp = 0; sp < n_live; ++sp) wh[sp] *= inv;
+  }
+  __syncthreads();
+  constexpr int D4 = D / 4;
+  for (int i = threadIdx.x; i < G * D4; i += W * 32) {
+    const int hd = i / D4;
+    const int d4 = i - hd * D4;
+    const size_t row = (size_t)b * a.hq + (size_t)h * G + hd;
+    const float4 *op = reinterpret_cast<const float4 *>(a.o_part + row * a.S * D) + d4;
+    const float *wh = wts + hd * n_live;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int sp = 0; sp < n_live; ++sp) {  // every live split wrote a finite partial
+      const float wv = wh[sp];
+      const float4 v = __ldcg(op + (size_t)sp * D4);
+      acc.x = fmaf(wv, v.x, acc.x);
+      acc.y = fmaf(wv, v.y, acc.y);
+      acc.z = fmaf(wv, v.z, acc.z);
+      acc.w = fmaf(wv, v.w, acc.w);
+    }
+    reinterpret_cast<float4 *>(a.out + row * D)[d4] = acc;
+  }
+  if (threadIdx.x == 0) a.counters[(size_t)b * a.hkv + h] = 0;
 }
 
 template <int D, int P, int KVT>
@@ -522,25 +585,49 @@ struct Config {
   static void *fn() { return reinterpret_cast<void *>(&decode_kernel<D, P, KVT, W, NSTAGE>); }
 };
 
+// Largest dynamic shared memory a decode CTA may request (ring + table slice).
+template <class C>
+constexpr int max_smem() {
+  return (int)C::SM::bytes(kMaxPagesPerSplit);
+}
+
+// Opt each kernel instance in to its dynamic shared memory once per device.
+template <class C>
+cudaError_t ensure_smem_attr() {
+  static std::atomic<uint64_t> done{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(C::fn(), cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem<C>());
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
 template <int D, int P, int KVT>
 cudaError_t launch_t(const DecodeArgs &a, cudaStream_t stream) {
   using C = Config<D, P, KVT>;
-  const size_t smem = C::SM::bytes(a.pages_per_split);
-  cudaError_t e = cudaFuncSetAttribute(C::fn(), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = ensure_smem_attr<C>();
   if (e != cudaSuccess) return e;
-  dim3 grid(a.S, a.hkv, a.B);
-  decode_kernel<D, P, KVT, C::W, C::NSTAGE><<<grid, C::W * 32, smem, stream>>>(a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.S, a.hkv, a.B);
+  cfg.blockDim = dim3(C::W * 32);
+  cfg.dynamicSmemBytes = C::SM::bytes(a.pages_per_split);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = PA_DECODE_PDL ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, decode_kernel<D, P, KVT, C::W, C::NSTAGE>, a);
 }
 
 template <int D, int P, int KVT>
 int ctas_per_sm_t() {
   using C = Config<D, P, KVT>;
   const size_t smem = C::SM::bytes(256);
-  if (cudaFuncSetAttribute(C::fn(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-      cudaSuccess)
-    return 1;
+  if (ensure_smem_attr<C>() != cudaSuccess) return 1;
   int n = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, C::fn(), C::W * 32, smem) != cudaSuccess)
     return 1;

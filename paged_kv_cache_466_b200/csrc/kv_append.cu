@@ -58,6 +58,8 @@ __device__ __forceinline__ long long slot_row(const AppendArgs &a, int i, int h)
 
 // bf16: one thread per 16-byte chunk of a (token, head) row, K and V.
 __global__ void append_bf16_kernel(const AppendArgs a) {
+  pdl_launch_dependents();  // the decode that follows may be scheduled now;
+                            // it waits for this grid before reading anything
   const int chunks = a.D / 8;
   const long long total = (long long)a.n * a.hkv * chunks;
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
@@ -118,6 +120,7 @@ __device__ __forceinline__ void quantise_row(const unsigned char *src_row, unsig
 // INT8: one warp per (token, head) row; K then V.
 template <int D>
 __global__ void append_u8_kernel(const AppendArgs a) {
+  pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const long long rows = (long long)a.n * a.hkv;
   const long long warps = (long long)gridDim.x * (blockDim.x >> 5);

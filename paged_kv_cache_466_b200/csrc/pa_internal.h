@@ -34,6 +34,7 @@ struct DecodeArgs {
   float *out;        // final output (S == 1)
   float *o_part;     // partials (S > 1)
   float *lse;        // partial log-sum-exps (S > 1)
+  int32_t *counters; // per (sequence, KV head) split-arrival counters (S > 1)
   int32_t S;
   int32_t pages_per_split;
   int32_t *d_err;

@@ -112,4 +112,5 @@ def test_split_planning_and_workspace_size(lib):
     ws = lib.pa_decode_workspace_bytes(32, 64, 128, 8)
     o = 32 * 64 * 8 * 128 * 4
     l = 32 * 64 * 8 * 4
-    assert ws == -(-o // 256) * 256 + -(-l // 256) * 256
+    c = 32 * 64 * 4
+    assert ws == -(-o // 256) * 256 + -(-l // 256) * 256 + -(-c // 256) * 256

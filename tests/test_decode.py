@@ -109,6 +109,21 @@ def test_deterministic_and_page_permutation_invariant():
     np.testing.assert_array_equal(a, b)
 
 
+def test_workspace_reuse_across_calls():
+    """The split counters in a workspace are re-armed by every call: one
+    zero-filled workspace serves many decodes (different batches, split
+    counts) with results identical to fresh workspaces."""
+    ws = torch.zeros(1 << 24, dtype=torch.uint8, device=DEV)
+    for seed, S in [(0, 8), (1, 3), (2, 8), (3, 16)]:
+        w = W.llama8b(B=6, ctx_range=(50, 1500), seed=seed)
+        pool, bt, ctx, q = device_inputs(w)
+        device_append(pool, w, bt)
+        fresh = pa_decode(pool, q, bt, ctx, w.scale, num_splits=S)
+        reused = pa_decode(pool, q, bt, ctx, w.scale, num_splits=S, workspace=ws)
+        torch.cuda.synchronize()
+        assert torch.equal(fresh, reused)
+
+
 def test_shared_prefix_equals_unshared_copy_bitwise():
     shared, unshared = W.prefix(B=16, prefix_tokens=160, suffix_range=(1, 100))
     a, _ = _run(shared)
