@@ -170,6 +170,46 @@ pa_status_t pa_decode(const pa_kv_pool_t *pool, const void *q,
                       int32_t num_splits, int32_t *d_err, void *stream);
 
 /*
+ * pa_decode_shared_prefix — cascade decode for a batch whose requests all
+ * begin with the same prompt prefix stored once in shared pages
+ * ("KV-Cache Optimization Techniques", section "Prefix Caching", Eq. 2).
+ * Computes exactly what pa_decode computes when every request's logical pages
+ * [0, prefix_len / P) are prefix_pages, in two passes: (1) attention of all
+ * num_seqs * num_q_heads query rows over the prefix, as dense tensor-core tiles
+ * that read each prefix K/V row once per 64 query rows instead of once per
+ * request; (2) the paged decode over each request's own tokens
+ * [prefix_len, context_lens[b]), which merges (1) into its log-sum-exp merge.
+ *
+ *   prefix_pages : (device) int32 [prefix_len / P] physical pages of the prefix
+ *   prefix_len   : tokens in the prefix; a multiple of the page size (0 falls
+ *                  back to pa_decode)
+ *   block_tables : (device) int32 [num_seqs][max_pages]; entries for logical
+ *                  pages < prefix_len / P are not read
+ *   context_lens : (device) int32 [num_seqs], each >= prefix_len (a shorter
+ *                  one is flagged PA_DERR_BAD_CTX and treated as prefix_len)
+ *   workspace    : (device) >= pa_decode_shared_prefix_workspace_bytes(...)
+ *                  bytes, 256-byte aligned, zero-filled before its first use
+ * Other arguments as for pa_decode. bf16 pools only. Two kernel launches.
+ */
+size_t pa_decode_shared_prefix_workspace_bytes(const pa_kv_pool_t *pool,
+                                               int32_t num_seqs,
+                                               int32_t num_q_heads,
+                                               int32_t max_pages,
+                                               int32_t prefix_len,
+                                               int32_t num_splits);
+
+pa_status_t pa_decode_shared_prefix(const pa_kv_pool_t *pool, const void *q,
+                                    int32_t num_seqs, int32_t num_q_heads,
+                                    const int32_t *prefix_pages,
+                                    int32_t prefix_len,
+                                    const int32_t *block_tables,
+                                    int32_t max_pages,
+                                    const int32_t *context_lens, float scale,
+                                    float *out, void *workspace,
+                                    size_t workspace_bytes, int32_t num_splits,
+                                    int32_t *d_err, void *stream);
+
+/*
  * pa_decode_noalloc — pa_decode for callers that cannot allocate device memory.
  * The pages have no counterpart to this entry point: it only changes where
  * pa_decode's split-KV scratch lives.

@@ -13,6 +13,9 @@ Entry points (same names as the C ABI, see include/pagedattn.h):
 * ``pa_splitkv_reduce``  — log-sum-exp merge of split-KV partials
 * ``pa_validate_tables`` — device-side page-table check
 * ``pa_decode_num_splits`` / ``pa_decode_workspace_bytes`` — planning helpers
+* ``pa_decode_shared_prefix`` — cascade decode for requests sharing a prefix:
+                           the prefix as one tensor-core pass for all requests,
+                           then the paged decode of each request's own tokens
 * ``pa_decode_noalloc``  — pa_decode without a caller workspace, for callers
                            that cannot allocate device memory (the scratch is
                            a fixed-size array owned by the library)
@@ -32,6 +35,7 @@ from ._lib import (PA_DERR_BAD_CTX, PA_DERR_BAD_PAGE, PA_DERR_BAD_POS, PA_DERR_B
                    PA_KV_BF16, PA_KV_U8_PER_TOKEN, PagedAttnError, pa_kv_pool_t)
 
 __all__ = ["KVPool", "pa_kv_append", "pa_decode", "pa_decode_noalloc", "pa_splitkv_reduce",
+           "pa_decode_shared_prefix", "pa_decode_shared_prefix_workspace_bytes",
            "pa_validate_tables",
            "pa_decode_num_splits", "pa_decode_workspace_bytes", "PagedAttnError",
            "PA_KV_BF16", "PA_KV_U8_PER_TOKEN", "PA_DERR_BAD_PAGE", "PA_DERR_BAD_CTX",
@@ -162,6 +166,46 @@ def pa_decode(pool: KVPool, q: torch.Tensor, block_tables: torch.Tensor,
                                _ptr(workspace), ws_bytes, num_splits, _ptr(d_err),
                                _stream(stream))
     _lib.check(st, "pa_decode")
+    return out
+
+
+def pa_decode_shared_prefix_workspace_bytes(pool: KVPool, num_seqs: int, num_q_heads: int,
+                                            max_pages: int, prefix_len: int,
+                                            num_splits: int = 0) -> int:
+    return int(_lib.load().pa_decode_shared_prefix_workspace_bytes(
+        ctypes.byref(pool.c), num_seqs, num_q_heads, max_pages, prefix_len, num_splits))
+
+
+def pa_decode_shared_prefix(pool: KVPool, q: torch.Tensor, prefix_pages: torch.Tensor,
+                            prefix_len: int, block_tables: torch.Tensor,
+                            context_lens: torch.Tensor, scale: float,
+                            out: Optional[torch.Tensor] = None,
+                            workspace: Optional[torch.Tensor] = None, num_splits: int = 0,
+                            d_err: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Cascade decode: every request's first ``prefix_len`` tokens are the
+    shared pages ``prefix_pages``; result equals pa_decode on full tables."""
+    dev = pool.device
+    _need(q, "q", torch.bfloat16, dev)
+    _need(prefix_pages, "prefix_pages", torch.int32, dev)
+    _need(block_tables, "block_tables", torch.int32, dev)
+    _need(context_lens, "context_lens", torch.int32, dev)
+    B, Hq, D = q.shape
+    if D != pool.head_dim or block_tables.shape[0] != B or context_lens.numel() != B:
+        raise ValueError("pa_decode_shared_prefix: shape mismatch")
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    _need(out, "out", torch.float32, dev)
+    max_pages = block_tables.shape[1]
+    if workspace is None:
+        need = pa_decode_shared_prefix_workspace_bytes(pool, B, Hq, max_pages, prefix_len,
+                                                       num_splits)
+        workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = _lib.load().pa_decode_shared_prefix(
+        ctypes.byref(pool.c), _ptr(q), B, Hq, _ptr(prefix_pages), int(prefix_len),
+        _ptr(block_tables), max_pages, _ptr(context_lens), float(scale), _ptr(out),
+        _ptr(workspace), ws_bytes, num_splits, _ptr(d_err), _stream(stream))
+    _lib.check(st, "pa_decode_shared_prefix")
     return out
 
 

@@ -254,10 +254,166 @@ pa_status_t pa_decode(const pa_kv_pool_t *pool, const void *q, int32_t num_seqs,
                      : nullptr;
   a.S = S;
   a.pages_per_split = chunk;
+  a.tok_begin = 0;
+  a.prior_o = nullptr;
+  a.prior_lse = nullptr;
+  a.n_prior = 0;
   a.d_err = d_err;
   return cuda_status(launch_decode(pool->head_dim, pool->page_size, pool->dtype, a,
                                    static_cast<cudaStream_t>(stream)),
                      "pa_decode launch");
+}
+
+// ---------------------------------------------------------------- shared prefix
+namespace {
+
+struct PrefixPlan {
+  int n_psplits, tiles_per_split;  // prefix kernel
+  int S, chunk;                    // suffix decode
+  size_t o_pre, lse_pre, o_part, lse, counters, total;  // workspace offsets / size
+};
+
+bool plan_prefix(const pa_kv_pool_t *pool, int B, int Hq, int max_pages, int prefix_len,
+                 int num_splits, PrefixPlan *pl) {
+  const int P = pool->page_size;
+  const int G = Hq / pool->num_kv_heads;
+  const int lpb = prefix_len / P;
+  const int sfx_pages = max_pages - lpb;
+  if (sfx_pages < 1) return false;
+  // prefix: enough CTAs to cover the GPU twice, splits of whole 64-token tiles
+  const int tiles = (prefix_len + prefix_tile_tokens() - 1) / prefix_tile_tokens();
+  const int mtiles = (B * G + prefix_rows_per_cta() - 1) / prefix_rows_per_cta();
+  const long long base = (long long)mtiles * pool->num_kv_heads;
+  int ns = (int)((2LL * device_sm_count() + base - 1) / base);
+  if (ns > tiles) ns = tiles;
+  if (ns > kMaxSplits) ns = kMaxSplits;
+  if (ns < 1) ns = 1;
+  pl->tiles_per_split = tiles > 0 ? (tiles + ns - 1) / ns : 1;
+  pl->n_psplits = tiles > 0 ? (tiles + pl->tiles_per_split - 1) / pl->tiles_per_split : 0;
+  // suffix: the plain decode's split planning over the suffix pages
+  pl->S = pa_decode_num_splits(pool, B, sfx_pages, num_splits);
+  if (pl->S <= 0) return false;
+  pl->chunk = (sfx_pages + pl->S - 1) / pl->S;
+  const size_t R = (size_t)B * Hq, D = pool->head_dim;
+  size_t off = 0;
+  pl->o_pre = off;    off += align256(pl->n_psplits * R * D * sizeof(float));
+  pl->lse_pre = off;  off += align256(pl->n_psplits * R * sizeof(float));
+  pl->o_part = off;   off += align256(R * pl->S * D * sizeof(float));
+  pl->lse = off;      off += align256(R * pl->S * sizeof(float));
+  pl->counters = off; off += align256(R * sizeof(int32_t));
+  pl->total = off;
+  return true;
+}
+
+}  // namespace
+
+size_t pa_decode_shared_prefix_workspace_bytes(const pa_kv_pool_t *pool, int32_t num_seqs,
+                                               int32_t num_q_heads, int32_t max_pages,
+                                               int32_t prefix_len, int32_t num_splits) {
+  if (pool == nullptr || num_seqs <= 0 || num_q_heads <= 0 || pool->num_kv_heads <= 0 ||
+      pool->page_size <= 0 || prefix_len < 0 || prefix_len % pool->page_size != 0 ||
+      num_q_heads % pool->num_kv_heads != 0)
+    return 0;
+  PrefixPlan pl;
+  if (!plan_prefix(pool, num_seqs, num_q_heads, max_pages, prefix_len, num_splits, &pl)) return 0;
+  return pl.total;
+}
+
+pa_status_t pa_decode_shared_prefix(const pa_kv_pool_t *pool, const void *q, int32_t num_seqs,
+                                    int32_t num_q_heads, const int32_t *prefix_pages,
+                                    int32_t prefix_len, const int32_t *block_tables,
+                                    int32_t max_pages, const int32_t *context_lens, float scale,
+                                    float *out, void *workspace, size_t workspace_bytes,
+                                    int32_t num_splits, int32_t *d_err, void *stream) {
+  g_last_error.clear();
+  pa_status_t st = check_pool(pool);
+  if (st != PA_OK) return st;
+  if (pool->dtype != PA_KV_BF16)
+    return fail(PA_ERR_UNSUPPORTED, "shared-prefix decode supports bf16 pools only");
+  if (prefix_len < 0 || prefix_len % pool->page_size != 0)
+    return fail(PA_ERR_INVALID_ARG, "prefix_len=%d must be a non-negative multiple of %d",
+                prefix_len, pool->page_size);
+  if (prefix_len == 0)
+    return pa_decode(pool, q, num_seqs, num_q_heads, block_tables, max_pages, context_lens, scale,
+                     out, workspace, workspace_bytes, num_splits, d_err, stream);
+  if (num_seqs < 0 || num_q_heads <= 0 || max_pages <= 0 || num_splits < 0)
+    return fail(PA_ERR_INVALID_ARG, "num_seqs=%d num_q_heads=%d max_pages=%d num_splits=%d",
+                num_seqs, num_q_heads, max_pages, num_splits);
+  if (num_q_heads % pool->num_kv_heads != 0)
+    return fail(PA_ERR_INVALID_ARG, "num_q_heads=%d is not a multiple of num_kv_heads=%d",
+                num_q_heads, pool->num_kv_heads);
+  const int G = num_q_heads / pool->num_kv_heads;
+  if (G > kMaxGroup)
+    return fail(PA_ERR_UNSUPPORTED, "GQA group %d > %d query heads per KV head", G, kMaxGroup);
+  if (prefix_len / pool->page_size >= max_pages)
+    return fail(PA_ERR_INVALID_ARG, "prefix of %d pages leaves no room in tables of %d pages",
+                prefix_len / pool->page_size, max_pages);
+  if (num_seqs > 65535 || (long long)max_pages * pool->page_size > (1LL << 30))
+    return fail(PA_ERR_UNSUPPORTED, "too many sequences or pages");
+  if (!(scale == scale)) return fail(PA_ERR_INVALID_ARG, "scale is NaN");
+  if (num_seqs == 0) return PA_OK;
+  if (!q || !prefix_pages || !block_tables || !context_lens || !out)
+    return fail(PA_ERR_INVALID_ARG,
+                "q, prefix_pages, block_tables, context_lens and out are required");
+  if (!aligned(q, 16) || !aligned(out, 16))
+    return fail(PA_ERR_INVALID_ARG, "q and out must be 16-byte aligned");
+  PrefixPlan pl;
+  if (!plan_prefix(pool, num_seqs, num_q_heads, max_pages, prefix_len, num_splits, &pl))
+    return fail(PA_ERR_INVALID_ARG, "could not plan the shared-prefix decode");
+  if (workspace == nullptr || workspace_bytes < pl.total)
+    return fail(PA_ERR_WORKSPACE, "workspace: need %zu bytes, got %zu", pl.total,
+                workspace == nullptr ? (size_t)0 : workspace_bytes);
+  if (!aligned(workspace, 256)) return fail(PA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  char *ws = static_cast<char *>(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  PrefixArgs pa;
+  pa.k_pool = pool->k_pool;
+  pa.v_pool = pool->v_pool;
+  pa.num_pages = pool->num_pages;
+  pa.hkv = pool->num_kv_heads;
+  pa.q = q;
+  pa.B = num_seqs;
+  pa.hq = num_q_heads;
+  pa.prefix_pages = prefix_pages;
+  pa.prefix_len = prefix_len;
+  pa.tiles_per_split = pl.tiles_per_split;
+  pa.n_psplits = pl.n_psplits;
+  pa.scale_log2 = scale * 1.4426950408889634f;
+  pa.o_pre = reinterpret_cast<float *>(ws + pl.o_pre);
+  pa.lse_pre = reinterpret_cast<float *>(ws + pl.lse_pre);
+  pa.d_err = d_err;
+  st = cuda_status(launch_prefix(pool->head_dim, pool->page_size, pa, s),
+                   "pa_decode_shared_prefix prefix launch");
+  if (st != PA_OK) return st;
+
+  DecodeArgs a;
+  a.k_pool = pool->k_pool;
+  a.v_pool = pool->v_pool;
+  a.k_sz = pool->k_sz;
+  a.v_sz = pool->v_sz;
+  a.num_pages = pool->num_pages;
+  a.hkv = pool->num_kv_heads;
+  a.q = q;
+  a.B = num_seqs;
+  a.hq = num_q_heads;
+  a.block_tables = block_tables;
+  a.max_pages = max_pages;
+  a.ctx = context_lens;
+  a.scale_log2 = pa.scale_log2;
+  a.out = out;
+  a.o_part = reinterpret_cast<float *>(ws + pl.o_part);
+  a.lse = reinterpret_cast<float *>(ws + pl.lse);
+  a.counters = reinterpret_cast<int32_t *>(ws + pl.counters);
+  a.S = pl.S;
+  a.pages_per_split = pl.chunk;
+  a.tok_begin = prefix_len;
+  a.prior_o = pa.o_pre;
+  a.prior_lse = pa.lse_pre;
+  a.n_prior = pl.n_psplits;
+  a.d_err = d_err;
+  return cuda_status(launch_decode(pool->head_dim, pool->page_size, pool->dtype, a, s),
+                     "pa_decode_shared_prefix suffix launch");
 }
 
 pa_status_t pa_splitkv_reduce(const float *o_part, const float *lse, int32_t num_seqs,

@@ -130,6 +130,68 @@ __device__ __forceinline__ int out_col(int j, int g) {
   }
 }
 
+// Final log-sum-exp merge for the G query heads of one (sequence, KV head):
+// nl partials of this call's splits (workspace slots 0..nl-1) plus the
+// caller's prior partials (e.g. a shared prefix), in that fixed order. Every
+// thread of the CTA must call it; `wts` is shared scratch of
+// G * (nl + n_prior) floats. Writes out[b][h*G + hd][:].
+template <int D>
+__device__ void merge_rows(const DecodeArgs &a, int b, int h, int G, int nl, float *wts) {
+  const int nw = nl + a.n_prior;
+  const size_t R = (size_t)a.B * a.hq;
+  for (int i = threadIdx.x; i < G * nw; i += blockDim.x) {
+    const int hd = i / nw;
+    const int sp = i - hd * nw;
+    const size_t row = (size_t)b * a.hq + (size_t)h * G + hd;
+    wts[i] = sp < nl ? __ldcg(a.lse + row * a.S + sp)
+                     : __ldcg(a.prior_lse + (size_t)(sp - nl) * R + row);
+  }
+  __syncthreads();
+  if ((int)threadIdx.x < G) {
+    float *wh = wts + threadIdx.x * nw;
+    float M = -INFINITY;
+    for (int sp = 0; sp < nw; ++sp) M = fmaxf(M, wh[sp]);
+    float den = 0.f;
+    for (int sp = 0; sp < nw; ++sp) {
+      const float wv = M == -INFINITY ? 0.f : expf(wh[sp] - M);
+      wh[sp] = wv;
+      den += wv;
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    for (int sp = 0; sp < nw; ++sp) wh[sp] *= inv;
+  }
+  __syncthreads();
+  constexpr int D4 = D / 4;
+  for (int i = threadIdx.x; i < G * D4; i += blockDim.x) {
+    const int hd = i / D4;
+    const int d4 = i - hd * D4;
+    const size_t row = (size_t)b * a.hq + (size_t)h * G + hd;
+    const float *wh = wts + hd * nw;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 *op = reinterpret_cast<const float4 *>(a.o_part + row * a.S * D) + d4;
+#pragma unroll 4
+    for (int sp = 0; sp < nl; ++sp) {  // every live split wrote a finite partial
+      const float wv = wh[sp];
+      const float4 v = __ldcg(op + (size_t)sp * D4);
+      acc.x = fmaf(wv, v.x, acc.x);
+      acc.y = fmaf(wv, v.y, acc.y);
+      acc.z = fmaf(wv, v.z, acc.z);
+      acc.w = fmaf(wv, v.w, acc.w);
+    }
+    for (int sp = 0; sp < a.n_prior; ++sp) {
+      const float wv = wh[nl + sp];
+      if (wv == 0.f) continue;
+      const float4 v = __ldcg(reinterpret_cast<const float4 *>(
+                                  a.prior_o + ((size_t)sp * R + row) * D) + d4);
+      acc.x = fmaf(wv, v.x, acc.x);
+      acc.y = fmaf(wv, v.y, acc.y);
+      acc.z = fmaf(wv, v.z, acc.z);
+      acc.w = fmaf(wv, v.w, acc.w);
+    }
+    reinterpret_cast<float4 *>(a.out + row * D)[d4] = acc;
+  }
+}
+
 template <int D, int P, int KVT, int W, int NSTAGE>
 __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(const DecodeArgs a) {
   using T = Tile<D, KVT>;
@@ -153,24 +215,34 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
   int *tbl = reinterpret_cast<int *>(smem + SM::kRingBytes);
 
   // ---- this split's token range --------------------------------------------
+  // Tokens [tok_begin, ctx) are attended here (tok_begin > 0 when the caller
+  // supplies the shared-prefix part as prior partials); tok_begin is page aligned.
   int ctx = a.ctx[b];
   if (ctx < 0 || ctx > a.max_pages * P) {
     if (threadIdx.x == 0) flag_error(a.d_err, PA_DERR_BAD_CTX);
-    ctx = 0;
+    ctx = a.tok_begin;
+  } else if (ctx < a.tok_begin) {
+    if (threadIdx.x == 0) flag_error(a.d_err, PA_DERR_BAD_CTX);
+    ctx = a.tok_begin;
   }
   const int n_pages = (ctx + P - 1) / P;
-  const int lp0 = split * a.pages_per_split;
+  const int lpb = a.tok_begin / P;
+  const int lp0 = lpb + split * a.pages_per_split;
   const int lp1 = min(lp0 + a.pages_per_split, n_pages);
   const int tok0 = lp0 * P;
   const int tok1 = min(lp1 * P, ctx);
   const int nblk = tok1 > tok0 ? (tok1 - tok0 + 15) / 16 : 0;
 
   // splits [0, n_live) of this sequence hold tokens; the others have no work
-  const int n_live = (n_pages + a.pages_per_split - 1) / a.pages_per_split;
+  const int n_live = (n_pages - lpb + a.pages_per_split - 1) / a.pages_per_split;
   if (nblk == 0) {
-    if (split == 0 && n_live == 0) {  // empty context: the output is 0
-      for (int e = threadIdx.x; e < G * D; e += W * 32)
-        a.out[((size_t)b * a.hq + (size_t)h * G) * D + e] = 0.f;
+    if (split == 0 && n_live == 0) {
+      if (a.n_prior > 0) {  // nothing of our own: the output is the priors' merge
+        merge_rows<D>(a, b, h, G, 0, reinterpret_cast<float *>(smem));
+      } else {  // empty context: the output is 0
+        for (int e = threadIdx.x; e < G * D; e += W * 32)
+          a.out[((size_t)b * a.hq + (size_t)h * G) * D + e] = 0.f;
+      }
     }
     return;
   }
@@ -507,14 +579,19 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
     }
     const size_t row = (size_t)b * a.hq + (size_t)h * G + hd;
     const float val = L > 0.f ? num / L : 0.f;
-    if (n_live == 1) {
+    if (n_live == 1 && a.n_prior == 0) {
       a.out[row * D + d] = val;
     } else {
       a.o_part[(row * a.S + split) * D + d] = val;
       if (d == 0) a.lse[row * a.S + split] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
     }
   }
-  if (n_live == 1) return;
+  if (n_live == 1) {
+    if (a.n_prior == 0) return;
+    __syncthreads();  // our own partial is visible to the whole CTA
+    merge_rows<D>(a, b, h, G, 1, reinterpret_cast<float *>(smem));
+    return;
+  }
 
   // ---- split-KV merge, done by whichever CTA of this (sequence, KV head)
   // finishes last. Partials are made visible device-wide before the ticket is
@@ -530,49 +607,7 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  // weights exp(lse_s - M) / sum, per head, staged in shared memory (the warp
-  // records are no longer needed); then each thread streams its float4 columns
-  // of every split's partial, all loads independent
-  float *wts = reinterpret_cast<float *>(smem);  // [G][n_live]
-  for (int i = threadIdx.x; i < G * n_live; i += W * 32) {
-    const int hd = i / n_live;
-    const int sp = i - hd * n_live;
-    wts[i] = __ldcg(a.lse + ((size_t)b * a.hq + (size_t)h * G + hd) * a.S + sp);
-  }
-  __syncthreads();
-  if (threadIdx.x < G) {
-    float *wh = wts + threadIdx.x * n_live;
-    float M = -INFINITY;
-    for (int sp = 0; sp < n_live; ++sp) M = fmaxf(M, wh[sp]);
-    float den = 0.f;
-    for (int sp = 0; sp < n_live; ++sp) {
-      const float wv = M == -INFINITY ? 0.f : expf(wh[sp] - M);
-      wh[sp] = wv;
-      den += wv;
-    }
-    const float inv = den > 0.f ? 1.f / den : 0.f;
-    for (int sp = 0; sp < n_live; ++sp) wh[sp] *= inv;
-  }
-  __syncthreads();
-  constexpr int D4 = D / 4;
-  for (int i = threadIdx.x; i < G * D4; i += W * 32) {
-    const int hd = i / D4;
-    const int d4 = i - hd * D4;
-    const size_t row = (size_t)b * a.hq + (size_t)h * G + hd;
-    const float4 *op = reinterpret_cast<const float4 *>(a.o_part + row * a.S * D) + d4;
-    const float *wh = wts + hd * n_live;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-    for (int sp = 0; sp < n_live; ++sp) {  // every live split wrote a finite partial
-      const float wv = wh[sp];
-      const float4 v = __ldcg(op + (size_t)sp * D4);
-      acc.x = fmaf(wv, v.x, acc.x);
-      acc.y = fmaf(wv, v.y, acc.y);
-      acc.z = fmaf(wv, v.z, acc.z);
-      acc.w = fmaf(wv, v.w, acc.w);
-    }
-    reinterpret_cast<float4 *>(a.out + row * D)[d4] = acc;
-  }
+  merge_rows<D>(a, b, h, G, n_live, reinterpret_cast<float *>(smem));
   if (threadIdx.x == 0) a.counters[(size_t)b * a.hkv + h] = 0;
 }
 

@@ -60,6 +60,21 @@ __device__ __forceinline__ uint4 ldg_nc128(const void *p) {
   return v;
 }
 
+// Four 8x8 b16 matrices from shared memory; lane l supplies the address of
+// row (l % 8) of matrix (l / 8). The .trans form transposes each matrix.
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1,
+                                        uint32_t &r2, uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t &r0, uint32_t &r1,
+                                              uint32_t &r2, uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
 // ------------------------------------------------------------ tensor cores
 // D = A(16x16, row) * B(16x8, col) + D, fp32 accumulators.
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0,

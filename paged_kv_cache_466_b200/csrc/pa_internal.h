@@ -37,8 +37,34 @@ struct DecodeArgs {
   int32_t *counters; // per (sequence, KV head) split-arrival counters (S > 1)
   int32_t S;
   int32_t pages_per_split;
+  int32_t tok_begin;        // first attended token (page aligned); 0 for plain decode
+  const float *prior_o;     // [n_prior][B*Hq][D] partials merged into the output
+  const float *prior_lse;   // [n_prior][B*Hq]
+  int32_t n_prior;
   int32_t *d_err;
 };
+
+struct PrefixArgs {
+  const void *k_pool;
+  const void *v_pool;
+  int32_t num_pages;
+  int32_t hkv;
+  const void *q;  // bf16 [B][Hq][D]
+  int32_t B;
+  int32_t hq;
+  const int32_t *prefix_pages;  // [ceil(prefix_len / P)]
+  int32_t prefix_len;
+  int32_t tiles_per_split;      // 64-token tiles per prefix split
+  int32_t n_psplits;
+  float scale_log2;
+  float *o_pre;    // [n_psplits][B*Hq][D]
+  float *lse_pre;  // [n_psplits][B*Hq]
+  int32_t *d_err;
+};
+
+cudaError_t launch_prefix(int D, int P, const PrefixArgs &a, cudaStream_t stream);
+int prefix_rows_per_cta();
+int prefix_tile_tokens();
 
 cudaError_t launch_decode(int D, int P, int kv_dtype, const DecodeArgs &a,
                           cudaStream_t stream);
