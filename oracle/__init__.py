@@ -14,6 +14,8 @@ Contents, each written from the pages ("KV-Cache Optimization Techniques",
   ``pos % P`` (section "PagedAttention (vLLM)", "Architecture").
 * ``quantize_rows``        — Eq. 3 per-token INT8 quantiser (C, fp32 IEEE).
 * ``paged_attention``      — Eq. 1 over gathered pages (C, fp64).
+* ``paged_attention_window`` — Eq. 1 over the StreamingLLM token set of Eq. 5
+  (attention sinks + last w tokens) / the sliding window of Eq. 6 (C, fp64).
 * ``lse_merge``            — merging attention results of disjoint token
   ranges by their log-sum-exp. The pages do not describe split-KV; this is the
   plain identity softmax(x ∪ y) = weights exp(lse_x - M), exp(lse_y - M).
@@ -47,6 +49,13 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(path)
         L.oracle_paged_attention.restype = ctypes.c_int
         L.oracle_paged_attention.argtypes = [
+            ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_int,
+            ctypes.c_void_p, ctypes.c_double, ctypes.c_int, ctypes.c_int,
+            ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+        L.oracle_paged_attention_window.restype = ctypes.c_int
+        L.oracle_paged_attention_window.argtypes = [
             ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
             ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_int,
@@ -188,6 +197,33 @@ def paged_attention(pool: HostPool, q_bits: np.ndarray, block_tables: np.ndarray
         _ptr(pr), 0 if pr is None else pr.shape[0], _ptr(out), _ptr(lse))
     if st != 0:
         raise ValueError(f"oracle_paged_attention failed with status {st}")
+    return out, lse
+
+
+def paged_attention_window(pool: HostPool, q_bits: np.ndarray, block_tables: np.ndarray,
+                           context_lens: np.ndarray, scale: float, sinks: int, window: int,
+                           pairs: Optional[Sequence[Sequence[int]]] = None):
+    """fp64 attention over {first `sinks`} U {last `window`} tokens of each
+    sequence (Eq. 5; sinks = 0 is the sliding window of Eq. 6; window = 0
+    means the whole context). Returns (out [n, D], lse [n])."""
+    q = _c(q_bits, np.uint16)
+    B, Hq, D = q.shape
+    bt = _c(block_tables, np.int32)
+    ctx = _c(context_lens, np.int32)
+    pr = None if pairs is None else _c(np.asarray(pairs).reshape(-1, 2), np.int32)
+    n = B * Hq if pr is None else pr.shape[0]
+    out = np.zeros((n, D), np.float64)
+    lse = np.zeros((n,), np.float64)
+    kind = 0 if pool.kind == "bf16" else 1
+    st = lib().oracle_paged_attention_window(
+        kind, _ptr(_c(pool.k, pool.k.dtype)), _ptr(_c(pool.v, pool.v.dtype)),
+        _ptr(None if pool.k_sz is None else _c(pool.k_sz, np.float32)),
+        _ptr(None if pool.v_sz is None else _c(pool.v_sz, np.float32)),
+        pool.num_pages, pool.page_size, pool.num_kv_heads, D, _ptr(q), B, Hq,
+        _ptr(bt), bt.shape[1], _ptr(ctx), float(scale), int(sinks), int(window),
+        _ptr(pr), 0 if pr is None else pr.shape[0], _ptr(out), _ptr(lse))
+    if st != 0:
+        raise ValueError(f"oracle_paged_attention_window failed with status {st}")
     return out, lse
 
 

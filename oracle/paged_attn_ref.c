@@ -140,3 +140,86 @@ int oracle_paged_attention(int kind, const void *k_pool, const void *v_pool,
   }
   return status;
 }
+
+/*
+ * Eq. 5 and Eq. 6 of "KV-Cache Optimization Techniques" (sections "Token
+ * Eviction Strategies", StreamingLLM, and "Sliding Window Cache"): attention
+ * over the cached token set {first `sinks` tokens} U {last `window` tokens}
+ * of each sequence (window = 0 means no window: the whole context; sinks = 0
+ * is the plain sliding window of Eq. 6). The set is gathered in increasing
+ * token order, each token once, then the same textbook softmax as above.
+ * pairs/out/lse as for oracle_paged_attention.
+ */
+int oracle_paged_attention_window(int kind, const void *k_pool, const void *v_pool,
+                                  const float *k_sz, const float *v_sz, int num_pages,
+                                  int page_size, int hkv, int d, const uint16_t *q, int B,
+                                  int hq, const int32_t *block_tables, int max_pages,
+                                  const int32_t *ctx, double scale, int sinks, int window,
+                                  const int32_t *pairs, int n_pairs, double *out,
+                                  double *lse) {
+  if (hkv <= 0 || hq % hkv != 0 || d <= 0 || page_size <= 0 || B < 0 || sinks < 0 ||
+      window < 0)
+    return ORC_BAD_ARG;
+  if (kind == 1 && (k_sz == NULL || v_sz == NULL)) return ORC_BAD_ARG;
+  const int G = hq / hkv;
+  const int n_items = pairs ? n_pairs : B * hq;
+  int status = ORC_OK;
+
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int it = 0; it < n_items; ++it) {
+    const int b = pairs ? pairs[2 * it] : it / hq;
+    const int qh = pairs ? pairs[2 * it + 1] : it % hq;
+    const int h = qh / G;
+    const int n_ctx = ctx[b];
+    double *o = out + (int64_t)it * d;
+    for (int j = 0; j < d; ++j) o[j] = 0.0;
+    if (lse) lse[it] = -INFINITY;
+    /* the token set, in increasing order */
+    int *tok = (int *)malloc(sizeof(int) * (size_t)(n_ctx > 0 ? n_ctx : 1));
+    int n = 0;
+    for (int t = 0; t < n_ctx; ++t) {
+      const int in_sinks = t < sinks;
+      const int in_window = window == 0 || t >= n_ctx - window;
+      if (in_sinks || in_window) tok[n++] = t;
+    }
+    if (n == 0) { free(tok); continue; }
+    double *Kc = (double *)malloc(sizeof(double) * (size_t)n * d);
+    double *Vc = (double *)malloc(sizeof(double) * (size_t)n * d);
+    double *s = (double *)malloc(sizeof(double) * (size_t)n);
+    int bad = 0;
+    for (int i = 0; i < n && !bad; ++i) {
+      const int t = tok[i];
+      const int lp = t / page_size;
+      if (lp >= max_pages) { bad = 1; break; }
+      const int32_t page = block_tables[(int64_t)b * max_pages + lp];
+      if (page < 0 || page >= num_pages) { bad = 1; break; }
+      const int64_t row = ((int64_t)page * hkv + h) * page_size + t % page_size;
+      for (int j = 0; j < d; ++j) {
+        Kc[(int64_t)i * d + j] = kv_elem(kind, k_pool, k_sz, row, d, j);
+        Vc[(int64_t)i * d + j] = kv_elem(kind, v_pool, v_sz, row, d, j);
+      }
+    }
+    if (!bad) {
+      const uint16_t *qv = q + ((int64_t)b * hq + qh) * d;
+      for (int i = 0; i < n; ++i) {
+        double acc = 0.0;
+        for (int j = 0; j < d; ++j) acc += bf16_bits_to_f64(qv[j]) * Kc[(int64_t)i * d + j];
+        s[i] = scale * acc;
+      }
+      double m = s[0];
+      for (int i = 1; i < n; ++i) if (s[i] > m) m = s[i];
+      double l = 0.0;
+      for (int i = 0; i < n; ++i) { s[i] = exp(s[i] - m); l += s[i]; }
+      for (int i = 0; i < n; ++i) {
+        const double w = s[i] / l;
+        for (int j = 0; j < d; ++j) o[j] += w * Vc[(int64_t)i * d + j];
+      }
+      if (lse) lse[it] = m + log(l);
+    } else {
+#pragma omp atomic write
+      status = ORC_BAD_TABLE;
+    }
+    free(Kc); free(Vc); free(s); free(tok);
+  }
+  return status;
+}

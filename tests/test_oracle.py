@@ -255,6 +255,56 @@ def test_scatter_follows_the_block_table_diagram(golden_dir):
     assert np.count_nonzero(pool.k) == len(pos) * 8
 
 
+# ------------------------------------------------------ Eq. 5 / Eq. 6 pins
+def test_window_covering_everything_is_full_attention():
+    """window >= ctx (or window = 0) keeps every token: identical to Eq. 1."""
+    q, K, V = _rand_case(20, B=3, T=64)
+    kp, vp, table = _contiguous_pool(K, V, 16)
+    pool = _pool("bf16", kp, vp, 16)
+    ctx = np.array([64, 41, 5], np.int32)
+    full, full_lse = oracle.paged_attention(pool, _bf16_bits(q), table, ctx, 0.125)
+    for sinks, window in [(0, 0), (0, 64), (3, 100), (4, 60)]:
+        out, lse = oracle.paged_attention_window(pool, _bf16_bits(q), table, ctx, 0.125,
+                                                 sinks, window)
+        np.testing.assert_array_equal(out, full)
+        np.testing.assert_array_equal(lse, full_lse)
+
+
+def test_window_of_one_returns_the_newest_value_row():
+    q, K, V = _rand_case(21, B=3, T=48)
+    kp, vp, table = _contiguous_pool(K, V, 16)
+    ctx = np.array([48, 17, 2], np.int32)
+    out, _ = oracle.paged_attention_window(_pool("bf16", kp, vp, 16), _bf16_bits(q), table,
+                                           ctx, 0.125, 0, 1)
+    for b in range(3):
+        for hq in range(8):
+            np.testing.assert_array_equal(out[b * 8 + hq], V[b, hq // 4, ctx[b] - 1].double().numpy())
+
+
+def test_sinks_and_window_equal_attention_over_the_kept_tokens():
+    """Eq. 5 as a token set: copy only the kept tokens (first s, last w) into
+    a fresh contiguous cache and run plain Eq. 1 on it; the results agree."""
+    q, K, V = _rand_case(22, B=3, Hq=8, Hkv=2, T=96)
+    kp, vp, table = _contiguous_pool(K, V, 16)
+    ctx = np.array([96, 70, 30], np.int32)
+    sinks, window = 4, 37
+    got, got_lse = oracle.paged_attention_window(_pool("bf16", kp, vp, 16), _bf16_bits(q),
+                                                 table, ctx, 0.125, sinks, window)
+    for b in range(3):
+        n = int(ctx[b])
+        keep = [t for t in range(n) if t < sinks or t >= n - window]
+        Kk = K[b:b + 1, :, keep, :]
+        Vk = V[b:b + 1, :, keep, :]
+        T2 = -(-len(keep) // 16) * 16
+        Kp = torch.zeros(1, 2, T2, 64, dtype=torch.bfloat16); Kp[:, :, :len(keep)] = Kk
+        Vp = torch.zeros(1, 2, T2, 64, dtype=torch.bfloat16); Vp[:, :, :len(keep)] = Vk
+        kp2, vp2, t2 = _contiguous_pool(Kp, Vp, 16)
+        ref, ref_lse = oracle.paged_attention(_pool("bf16", kp2, vp2, 16), _bf16_bits(q[b:b + 1]),
+                                              t2, np.array([len(keep)], np.int32), 0.125)
+        np.testing.assert_allclose(got[b * 8:(b + 1) * 8], ref, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(got_lse[b * 8:(b + 1) * 8], ref_lse, rtol=0, atol=1e-13)
+
+
 # ------------------------------------------------------------------ Eq. 3 pins
 def _row_bits(vals):
     t = torch.tensor(vals, dtype=torch.float32)
