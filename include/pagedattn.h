@@ -210,6 +210,33 @@ pa_status_t pa_decode_shared_prefix(const pa_kv_pool_t *pool, const void *q,
                                     int32_t *d_err, void *stream);
 
 /*
+ * pa_decode_window — decode over the StreamingLLM token set: the first `sinks`
+ * tokens (attention sinks) and the last `window` tokens of each sequence
+ * ("KV-Cache Optimization Techniques", section "Token Eviction Strategies",
+ * Eq. 5; sinks = 0 is the sliding-window cache of Eq. 6). Only the pages that
+ * hold kept tokens are read: the sink pages and the last ceil(window / P) + 1
+ * pages; table entries of evicted pages are never dereferenced, so a caller
+ * may free those pages and leave any value in their entries.
+ *   window : >= 0; 0 keeps every token (falls back to pa_decode)
+ *   sinks  : >= 0; tokens [0, min(sinks, ctx)) are always kept
+ *   workspace : >= pa_decode_window_workspace_bytes(...), zero-filled before
+ *               its first use, 256-byte aligned (NULL if that is 0)
+ * Other arguments and behaviour as for pa_decode (bf16 and INT8 pools).
+ */
+size_t pa_decode_window_workspace_bytes(const pa_kv_pool_t *pool,
+                                        int32_t num_seqs, int32_t num_q_heads,
+                                        int32_t max_pages, int32_t sinks,
+                                        int32_t window, int32_t num_splits);
+
+pa_status_t pa_decode_window(const pa_kv_pool_t *pool, const void *q,
+                             int32_t num_seqs, int32_t num_q_heads,
+                             const int32_t *block_tables, int32_t max_pages,
+                             const int32_t *context_lens, int32_t sinks,
+                             int32_t window, float scale, float *out,
+                             void *workspace, size_t workspace_bytes,
+                             int32_t num_splits, int32_t *d_err, void *stream);
+
+/*
  * pa_decode_noalloc — pa_decode for callers that cannot allocate device memory.
  * The pages have no counterpart to this entry point: it only changes where
  * pa_decode's split-KV scratch lives.

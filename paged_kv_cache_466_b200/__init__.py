@@ -16,6 +16,8 @@ Entry points (same names as the C ABI, see include/pagedattn.h):
 * ``pa_decode_shared_prefix`` — cascade decode for requests sharing a prefix:
                            the prefix as one tensor-core pass for all requests,
                            then the paged decode of each request's own tokens
+* ``pa_decode_window``   — decode over attention sinks + the last w tokens
+                           (StreamingLLM / sliding window); evicted pages unread
 * ``pa_decode_noalloc``  — pa_decode without a caller workspace, for callers
                            that cannot allocate device memory (the scratch is
                            a fixed-size array owned by the library)
@@ -36,6 +38,7 @@ from ._lib import (PA_DERR_BAD_CTX, PA_DERR_BAD_PAGE, PA_DERR_BAD_POS, PA_DERR_B
 
 __all__ = ["KVPool", "pa_kv_append", "pa_decode", "pa_decode_noalloc", "pa_splitkv_reduce",
            "pa_decode_shared_prefix", "pa_decode_shared_prefix_workspace_bytes",
+           "pa_decode_window", "pa_decode_window_workspace_bytes",
            "pa_validate_tables",
            "pa_decode_num_splits", "pa_decode_workspace_bytes", "PagedAttnError",
            "PA_KV_BF16", "PA_KV_U8_PER_TOKEN", "PA_DERR_BAD_PAGE", "PA_DERR_BAD_CTX",
@@ -206,6 +209,47 @@ def pa_decode_shared_prefix(pool: KVPool, q: torch.Tensor, prefix_pages: torch.T
         _ptr(block_tables), max_pages, _ptr(context_lens), float(scale), _ptr(out),
         _ptr(workspace), ws_bytes, num_splits, _ptr(d_err), _stream(stream))
     _lib.check(st, "pa_decode_shared_prefix")
+    return out
+
+
+def pa_decode_window_workspace_bytes(pool: KVPool, num_seqs: int, num_q_heads: int,
+                                     max_pages: int, sinks: int, window: int,
+                                     num_splits: int = 0) -> int:
+    return int(_lib.load().pa_decode_window_workspace_bytes(
+        ctypes.byref(pool.c), num_seqs, num_q_heads, max_pages, sinks, window, num_splits))
+
+
+def pa_decode_window(pool: KVPool, q: torch.Tensor, block_tables: torch.Tensor,
+                     context_lens: torch.Tensor, scale: float, sinks: int, window: int,
+                     out: Optional[torch.Tensor] = None,
+                     workspace: Optional[torch.Tensor] = None, num_splits: int = 0,
+                     d_err: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Decode over the first ``sinks`` and the last ``window`` tokens of each
+    sequence (StreamingLLM); ``window == 0`` keeps every token."""
+    dev = pool.device
+    _need(q, "q", torch.bfloat16, dev)
+    _need(block_tables, "block_tables", torch.int32, dev)
+    _need(context_lens, "context_lens", torch.int32, dev)
+    B, Hq, D = q.shape
+    if D != pool.head_dim or block_tables.shape[0] != B or context_lens.numel() != B:
+        raise ValueError("pa_decode_window: shape mismatch")
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    _need(out, "out", torch.float32, dev)
+    max_pages = block_tables.shape[1]
+    if workspace is None:
+        need = (pa_decode_window_workspace_bytes(pool, B, Hq, max_pages, sinks, window,
+                                                 num_splits) if window > 0 else
+                pa_decode_workspace_bytes(B, Hq, D,
+                                          pa_decode_num_splits(pool, B, max_pages, num_splits)))
+        if need > 0:
+            workspace = torch.zeros(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _lib.load().pa_decode_window(
+        ctypes.byref(pool.c), _ptr(q), B, Hq, _ptr(block_tables), max_pages, _ptr(context_lens),
+        int(sinks), int(window), float(scale), _ptr(out), _ptr(workspace), ws_bytes,
+        num_splits, _ptr(d_err), _stream(stream))
+    _lib.check(st, "pa_decode_window")
     return out
 
 

@@ -56,6 +56,9 @@ SIGNATURES = {
     "pa_decode_shared_prefix_workspace_bytes": (ctypes.c_size_t, [_POOL, _I, _I, _I, _I, _I]),
     "pa_decode_shared_prefix": (_I, [_POOL, _P, _I, _I, _P, _I, _P, _I, _P, ctypes.c_float, _P,
                                      _P, ctypes.c_size_t, _I, _P, _P]),
+    "pa_decode_window_workspace_bytes": (ctypes.c_size_t, [_POOL, _I, _I, _I, _I, _I, _I]),
+    "pa_decode_window": (_I, [_POOL, _P, _I, _I, _P, _I, _P, _I, _I, ctypes.c_float, _P, _P,
+                              ctypes.c_size_t, _I, _P, _P]),
     "pa_decode_noalloc": (_I, [_POOL, _P, _I, _I, _P, _I, _P, ctypes.c_float, _P, _I, _P, _P]),
     "pa_splitkv_reduce": (_I, [_P, _P, _I, _I, _I, _I, _P, _P]),
     "pa_validate_tables": (_I, [_P, _I, _I, _P, _I, _I, _P, _P]),

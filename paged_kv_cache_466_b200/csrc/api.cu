@@ -1,5 +1,6 @@
 // extern "C" boundary of libpagedattn.so: argument checks, split-KV planning
 // and kernel launches. See include/pagedattn.h for the contract of each call.
+#include <algorithm>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -253,7 +254,11 @@ pa_status_t pa_decode(const pa_kv_pool_t *pool, const void *q, int32_t num_seqs,
                                                    l_bytes)
                      : nullptr;
   a.S = S;
+  a.S_main = S;
   a.pages_per_split = chunk;
+  a.tbl_cap = chunk;
+  a.window = 0;
+  a.sinks = 0;
   a.tok_begin = 0;
   a.prior_o = nullptr;
   a.prior_lse = nullptr;
@@ -406,7 +411,11 @@ pa_status_t pa_decode_shared_prefix(const pa_kv_pool_t *pool, const void *q, int
   a.lse = reinterpret_cast<float *>(ws + pl.lse);
   a.counters = reinterpret_cast<int32_t *>(ws + pl.counters);
   a.S = pl.S;
+  a.S_main = pl.S;
   a.pages_per_split = pl.chunk;
+  a.tbl_cap = pl.chunk;
+  a.window = 0;
+  a.sinks = 0;
   a.tok_begin = prefix_len;
   a.prior_o = pa.o_pre;
   a.prior_lse = pa.lse_pre;
@@ -451,6 +460,124 @@ pa_status_t pa_validate_tables(const int32_t *block_tables, int32_t num_seqs, in
                                             num_pages, page_size, d_err,
                                             static_cast<cudaStream_t>(stream)),
                      "pa_validate_tables launch");
+}
+
+
+// ------------------------------------------------------------ sinks + window
+namespace {
+
+struct WindowPlan {
+  int S_main, S, chunk, tbl_cap;
+};
+
+bool plan_window(const pa_kv_pool_t *pool, int B, int max_pages, int sinks, int window,
+                 int num_splits, WindowPlan *pl) {
+  const int P = pool->page_size;
+  // the main range [max(ctx - window, min(sinks, ctx)), ctx) spans at most this many pages
+  long long wp = ((long long)window + P - 1) / P + 1;
+  if (wp > max_pages) wp = max_pages;
+  pl->S_main = pa_decode_num_splits(pool, B, (int)wp, num_splits);
+  if (pl->S_main <= 0) return false;
+  pl->chunk = ((int)wp + pl->S_main - 1) / pl->S_main;
+  pl->S = pl->S_main + (sinks > 0 ? 1 : 0);
+  // the sink split reads pages [0, ceil(min(sinks, ctx) / P)) at most
+  const long long sink_tok = std::min<long long>(sinks, (long long)max_pages * P);
+  const long long sink_pages = (sink_tok + P - 1) / P;
+  pl->tbl_cap = (int)std::max<long long>(pl->chunk, sink_pages);
+  return pl->tbl_cap <= kMaxPagesPerSplit;
+}
+
+}  // namespace
+
+size_t pa_decode_window_workspace_bytes(const pa_kv_pool_t *pool, int32_t num_seqs,
+                                        int32_t num_q_heads, int32_t max_pages, int32_t sinks,
+                                        int32_t window, int32_t num_splits) {
+  if (pool == nullptr || num_seqs <= 0 || num_q_heads <= 0 || max_pages <= 0 || sinks < 0 ||
+      window <= 0 || pool->page_size <= 0)
+    return 0;
+  WindowPlan pl;
+  if (!plan_window(pool, num_seqs, max_pages, sinks, window, num_splits, &pl)) return 0;
+  return pa_decode_workspace_bytes(num_seqs, num_q_heads, pool->head_dim, pl.S);
+}
+
+pa_status_t pa_decode_window(const pa_kv_pool_t *pool, const void *q, int32_t num_seqs,
+                             int32_t num_q_heads, const int32_t *block_tables, int32_t max_pages,
+                             const int32_t *context_lens, int32_t sinks, int32_t window,
+                             float scale, float *out, void *workspace, size_t workspace_bytes,
+                             int32_t num_splits, int32_t *d_err, void *stream) {
+  g_last_error.clear();
+  pa_status_t st = check_pool(pool);
+  if (st != PA_OK) return st;
+  if (window < 0 || sinks < 0)
+    return fail(PA_ERR_INVALID_ARG, "window=%d sinks=%d must be non-negative", window, sinks);
+  if (window == 0)  // no window: every token is kept
+    return pa_decode(pool, q, num_seqs, num_q_heads, block_tables, max_pages, context_lens, scale,
+                     out, workspace, workspace_bytes, num_splits, d_err, stream);
+  if (num_seqs < 0 || num_q_heads <= 0 || max_pages <= 0 || num_splits < 0)
+    return fail(PA_ERR_INVALID_ARG, "num_seqs=%d num_q_heads=%d max_pages=%d num_splits=%d",
+                num_seqs, num_q_heads, max_pages, num_splits);
+  if (num_q_heads % pool->num_kv_heads != 0)
+    return fail(PA_ERR_INVALID_ARG, "num_q_heads=%d is not a multiple of num_kv_heads=%d",
+                num_q_heads, pool->num_kv_heads);
+  const int G = num_q_heads / pool->num_kv_heads;
+  if (G > kMaxGroup)
+    return fail(PA_ERR_UNSUPPORTED, "GQA group %d > %d query heads per KV head", G, kMaxGroup);
+  if (num_seqs > 65535 || (long long)max_pages * pool->page_size > (1LL << 30))
+    return fail(PA_ERR_UNSUPPORTED, "too many sequences or pages");
+  if (!(scale == scale)) return fail(PA_ERR_INVALID_ARG, "scale is NaN");
+  if (num_seqs == 0) return PA_OK;
+  if (!q || !block_tables || !context_lens || !out)
+    return fail(PA_ERR_INVALID_ARG, "q, block_tables, context_lens and out are required");
+  if (!aligned(q, 16) || !aligned(out, 16))
+    return fail(PA_ERR_INVALID_ARG, "q and out must be 16-byte aligned");
+  WindowPlan pl;
+  if (!plan_window(pool, num_seqs, max_pages, sinks, window, num_splits, &pl))
+    return fail(PA_ERR_UNSUPPORTED, "windowed decode: at most %d sink pages are supported",
+                kMaxPagesPerSplit);
+  if (pl.S + 1 > kMaxSplits + 1) return fail(PA_ERR_UNSUPPORTED, "too many splits");
+  const size_t need = pa_decode_workspace_bytes(num_seqs, num_q_heads, pool->head_dim, pl.S);
+  if (need > 0) {
+    if (workspace == nullptr || workspace_bytes < need)
+      return fail(PA_ERR_WORKSPACE, "workspace: need %zu bytes for %d splits, got %zu", need,
+                  pl.S, workspace == nullptr ? (size_t)0 : workspace_bytes);
+    if (!aligned(workspace, 256)) return fail(PA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  }
+  const size_t rows = (size_t)num_seqs * num_q_heads;
+  const size_t o_bytes = align256(rows * pl.S * pool->head_dim * sizeof(float));
+  const size_t l_bytes = align256(rows * pl.S * sizeof(float));
+  DecodeArgs a;
+  a.k_pool = pool->k_pool;
+  a.v_pool = pool->v_pool;
+  a.k_sz = pool->k_sz;
+  a.v_sz = pool->v_sz;
+  a.num_pages = pool->num_pages;
+  a.hkv = pool->num_kv_heads;
+  a.q = q;
+  a.B = num_seqs;
+  a.hq = num_q_heads;
+  a.block_tables = block_tables;
+  a.max_pages = max_pages;
+  a.ctx = context_lens;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.out = out;
+  char *ws = static_cast<char *>(workspace);
+  a.o_part = pl.S > 1 ? reinterpret_cast<float *>(ws) : nullptr;
+  a.lse = pl.S > 1 ? reinterpret_cast<float *>(ws + o_bytes) : nullptr;
+  a.counters = pl.S > 1 ? reinterpret_cast<int32_t *>(ws + o_bytes + l_bytes) : nullptr;
+  a.S = pl.S;
+  a.S_main = pl.S_main;
+  a.pages_per_split = pl.chunk;
+  a.tbl_cap = pl.tbl_cap;
+  a.window = window;
+  a.sinks = sinks;
+  a.tok_begin = 0;
+  a.prior_o = nullptr;
+  a.prior_lse = nullptr;
+  a.n_prior = 0;
+  a.d_err = d_err;
+  return cuda_status(launch_decode(pool->head_dim, pool->page_size, pool->dtype, a,
+                                   static_cast<cudaStream_t>(stream)),
+                     "pa_decode_window launch");
 }
 
 }  // extern "C"

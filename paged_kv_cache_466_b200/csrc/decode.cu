@@ -215,8 +215,12 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
   int *tbl = reinterpret_cast<int *>(smem + SM::kRingBytes);
 
   // ---- this split's token range --------------------------------------------
-  // Tokens [tok_begin, ctx) are attended here (tok_begin > 0 when the caller
-  // supplies the shared-prefix part as prior partials); tok_begin is page aligned.
+  // Token ranges. The main range [mlo, ctx) is split over the first S_main
+  // splits: mlo = tok_begin (page aligned; > 0 when the caller supplies the
+  // shared-prefix part as prior partials) or, with a window, the start of the
+  // last `window` tokens. With attention sinks the extra split S_main covers
+  // [0, min(sinks, ctx)) ("Token Eviction Strategies", Eq. 5); the two ranges
+  // are disjoint and together hold exactly the kept tokens.
   int ctx = a.ctx[b];
   if (ctx < 0 || ctx > a.max_pages * P) {
     if (threadIdx.x == 0) flag_error(a.d_err, PA_DERR_BAD_CTX);
@@ -225,16 +229,42 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
     if (threadIdx.x == 0) flag_error(a.d_err, PA_DERR_BAD_CTX);
     ctx = a.tok_begin;
   }
+  int mlo = a.tok_begin;
+  int sink_hi = 0;
+  if (a.window > 0) {
+    sink_hi = min(a.sinks, ctx);
+    mlo = max(max(ctx - a.window, 0), sink_hi);
+  }
   const int n_pages = (ctx + P - 1) / P;
-  const int lpb = a.tok_begin / P;
-  const int lp0 = lpb + split * a.pages_per_split;
-  const int lp1 = min(lp0 + a.pages_per_split, n_pages);
-  const int tok0 = lp0 * P;
-  const int tok1 = min(lp1 * P, ctx);
-  const int nblk = tok1 > tok0 ? (tok1 - tok0 + 15) / 16 : 0;
+  const int lpb = mlo / P;
+  const int n_main_live = ctx > mlo ? (n_pages - lpb + a.pages_per_split - 1) / a.pages_per_split : 0;
+  const int n_live = n_main_live + (sink_hi > 0 ? 1 : 0);  // splits holding tokens
+  int lp0, lp1, tok_lo, tok_hi, slot;
+  if (split < a.S_main) {
+    lp0 = lpb + split * a.pages_per_split;
+    lp1 = min(lp0 + a.pages_per_split, n_pages);
+    tok_lo = max(lp0 * P, mlo);
+    tok_hi = min(lp1 * P, ctx);
+    slot = split;
+  } else {  // the attention-sink split
+    lp0 = 0;
+    lp1 = (sink_hi + P - 1) / P;
+    tok_lo = 0;
+    tok_hi = sink_hi;
+    slot = n_main_live;
+  }
+  if (lp1 - lp0 > a.tbl_cap) {
+    // Cannot happen with the host's plan (the table slot holds tbl_cap pages);
+    // kept so that no table read or write can leave the staged slot.
+    if (threadIdx.x == 0) flag_error(a.d_err, PA_DERR_BAD_CTX);
+    lp1 = lp0 + a.tbl_cap;
+    tok_hi = min(tok_hi, lp1 * P);
+  }
+  const int blk0 = tok_lo & ~15;  // blocks stay 16-aligned inside their page
+  const int nblk = tok_hi > tok_lo ? (tok_hi - blk0 + 15) / 16 : 0;
+  const int tok0 = blk0;
+  const int tok1 = tok_hi;
 
-  // splits [0, n_live) of this sequence hold tokens; the others have no work
-  const int n_live = (n_pages - lpb + a.pages_per_split - 1) / a.pages_per_split;
   if (nblk == 0) {
     if (split == 0 && n_live == 0) {
       if (a.n_prior > 0) {  // nothing of our own: the output is the priors' merge
@@ -319,7 +349,9 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
     const int lp = btok / P;
     const int page = tbl[lp - lp0];
     const int in_page = btok - lp * P;
-    const int nvalid = page >= 0 ? min(16, tok1 - btok) : 0;  // rows holding tokens
+    // rows [rlo, rhi) of the block hold tokens of this range
+    const int rlo = page >= 0 ? max(0, tok_lo - btok) : 16;
+    const int rhi = page >= 0 ? min(16, tok1 - btok) : 0;
     // rows of an invalid page are zero-filled; the address stays inside page 0
     const size_t row0 = ((size_t)(page >= 0 ? page : 0) * a.hkv + h) * P + in_page;
     const uint32_t dst = ring + st * T::kStageBytes;
@@ -327,16 +359,18 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
     const unsigned char *vsrc = vbase + row0 * T::kRowBytes + lane * 16;
 #pragma unroll
     for (int j = 0; j < T::kCopies; ++j) {
-      const uint32_t n = cp_row[j] < nvalid ? 16u : 0u;
+      const uint32_t n = (cp_row[j] >= rlo && cp_row[j] < rhi) ? 16u : 0u;
       cp_async16(dst + cp_soff[j], ksrc + j * 512, n);
       cp_async16(dst + T::kVOff + cp_soff[j], vsrc + j * 512, n);
     }
     if constexpr (T::kU8) {
       // lanes 0..7: K (scale, zero) of rows 2l, 2l+1; lanes 8..15: V
       if (lane < 16) {
+        // (a row outside [rlo, rhi) may come along with its neighbour; the
+        // consumer zeroes scale and zero of every masked token)
         const int l = lane & 7;
-        const uint32_t nbytes = 2 * l + 1 < nvalid ? 16u : (2 * l < nvalid ? 8u : 0u);
-        cp_async16(dst + sz_dst, sz_base + (row0 + 2 * l) * 2, nbytes);
+        const bool any = 2 * l + 1 >= rlo && 2 * l < rhi;
+        cp_async16(dst + sz_dst, sz_base + (row0 + 2 * l) * 2, any ? 16u : 0u);
       }
     }
   };
@@ -426,14 +460,18 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
 #pragma unroll
       for (int e = 0; e < 4; ++e) x[e] = fmaf(ks[e], x[e], kz[e] * qsum);
     }
-    if (pvalid && btok + 16 <= tok1) {  // warp-uniform: a full block needs no mask
+    if (pvalid && btok >= tok_lo && btok + 16 <= tok1) {  // warp-uniform: no mask needed
 #pragma unroll
       for (int e = 0; e < 4; ++e) x[e] *= a.scale_log2;
     } else {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int toff = (e & 1) + 2 * t + (e >> 1) * 8;
-        x[e] = (pvalid && btok + toff < tok1) ? x[e] * a.scale_log2 : -INFINITY;
+        const int tok = btok + (e & 1) + 2 * t + (e >> 1) * 8;
+        const bool ok = pvalid && tok >= tok_lo && tok < tok1;
+        x[e] = ok ? x[e] * a.scale_log2 : -INFINITY;
+        if constexpr (T::kU8) {
+          if (!ok) vs[e] = vz[e] = 0.f;
+        }
       }
     }
     float mb = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
@@ -582,8 +620,8 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
     if (n_live == 1 && a.n_prior == 0) {
       a.out[row * D + d] = val;
     } else {
-      a.o_part[(row * a.S + split) * D + d] = val;
-      if (d == 0) a.lse[row * a.S + split] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+      a.o_part[(row * a.S + slot) * D + d] = val;
+      if (d == 0) a.lse[row * a.S + slot] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
     }
   }
   if (n_live == 1) {
@@ -648,7 +686,7 @@ cudaError_t launch_t(const DecodeArgs &a, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.S, a.hkv, a.B);
   cfg.blockDim = dim3(C::W * 32);
-  cfg.dynamicSmemBytes = C::SM::bytes(a.pages_per_split);
+  cfg.dynamicSmemBytes = C::SM::bytes(a.tbl_cap);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -35,8 +35,12 @@ struct DecodeArgs {
   float *o_part;     // partials (S > 1)
   float *lse;        // partial log-sum-exps (S > 1)
   int32_t *counters; // per (sequence, KV head) split-arrival counters (S > 1)
-  int32_t S;
+  int32_t S;                // partial slots (= grid splits)
+  int32_t S_main;           // splits over the main range; S - S_main is the sink split
   int32_t pages_per_split;
+  int32_t tbl_cap;          // table entries staged per CTA (>= pages any split covers)
+  int32_t window;           // > 0: attend only the last `window` tokens (+ sinks)
+  int32_t sinks;            // attention sinks kept with a window
   int32_t tok_begin;        // first attended token (page aligned); 0 for plain decode
   const float *prior_o;     // [n_prior][B*Hq][D] partials merged into the output
   const float *prior_lse;   // [n_prior][B*Hq]
