@@ -13,6 +13,8 @@ Contents, each written from the pages ("KV-Cache Optimization Techniques",
   ``pos`` of a sequence lives in physical page ``table[pos // P]`` at slot
   ``pos % P`` (section "PagedAttention (vLLM)", "Architecture").
 * ``quantize_rows``        — Eq. 3 per-token INT8 quantiser (C, fp32 IEEE).
+* ``quantize_rows_fp8``    — per-token FP8 (E4M3) quantiser with an absmax scale
+  (the pages' FP8 KV cache; encoding written from the format definition).
 * ``paged_attention``      — Eq. 1 over gathered pages (C, fp64).
 * ``paged_attention_window`` — Eq. 1 over the StreamingLLM token set of Eq. 5
   (attention sinks + last w tokens) / the sliding window of Eq. 6 (C, fp64).
@@ -61,6 +63,13 @@ def lib() -> ctypes.CDLL:
             ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_int,
             ctypes.c_void_p, ctypes.c_double, ctypes.c_int, ctypes.c_int,
             ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+        L.oracle_quantize_rows_fp8.restype = None
+        L.oracle_quantize_rows_fp8.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+                                               ctypes.c_void_p, ctypes.c_void_p]
+        L.oracle_e4m3_value.restype = ctypes.c_double
+        L.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_encode.restype = ctypes.c_uint8
+        L.oracle_e4m3_encode.argtypes = [ctypes.c_float]
         L.oracle_quantize_rows.restype = None
         L.oracle_quantize_rows.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
                                            ctypes.c_void_p, ctypes.c_void_p]
@@ -94,6 +103,26 @@ def quantize_rows(x_bits: np.ndarray):
     return codes.reshape(x.shape), sz.reshape(x.shape[:-1] + (2,))
 
 
+def quantize_rows_fp8(x_bits: np.ndarray):
+    """Per-row FP8 (E4M3) quantisation with an absmax fp32 scale (s = max|x|/448);
+    returns codes (uint8 bit patterns) and sz [..., 2] = (s, 0)."""
+    x = _c(x_bits, np.uint16)
+    d = x.shape[-1]
+    rows = x.reshape(-1, d)
+    codes = np.empty(rows.shape, np.uint8)
+    sz = np.empty((rows.shape[0], 2), np.float32)
+    lib().oracle_quantize_rows_fp8(_ptr(rows), rows.shape[0], d, _ptr(codes), _ptr(sz))
+    return codes.reshape(x.shape), sz.reshape(x.shape[:-1] + (2,))
+
+
+def e4m3_value(code: int) -> float:
+    return float(lib().oracle_e4m3_value(int(code)))
+
+
+def e4m3_encode(r: float) -> int:
+    return int(lib().oracle_e4m3_encode(float(r)))
+
+
 def dequantize_rows(codes: np.ndarray, sz: np.ndarray) -> np.ndarray:
     """Right-hand side of Eq. 3 in fp64: s * code + z, per row."""
     return sz[..., 0:1].astype(np.float64) * codes.astype(np.float64) + \
@@ -106,7 +135,7 @@ def dequantize_rows(codes: np.ndarray, sz: np.ndarray) -> np.ndarray:
 @dataclass
 class HostPool:
     """A KV page pool in host memory: [num_pages][Hkv][P][D] per tensor."""
-    kind: str                      # "bf16" or "u8"
+    kind: str                      # "bf16", "u8" (INT8, Eq. 3) or "fp8" (E4M3)
     page_size: int
     k: np.ndarray                  # uint16 (bf16 bits) or uint8 codes
     v: np.ndarray
@@ -132,7 +161,7 @@ def empty_pool(kind: str, num_pages: int, hkv: int, page_size: int, d: int,
     if kind == "bf16":
         k = np.full((num_pages, hkv, page_size, d), fill_byte * 0x0101, np.uint16)
         return HostPool(kind, page_size, k, k.copy())
-    if kind == "u8":
+    if kind in ("u8", "fp8"):
         k = np.full((num_pages, hkv, page_size, d), fill_byte, np.uint8)
         sz = np.frombuffer(bytes([fill_byte]) * (num_pages * hkv * page_size * 8),
                            np.float32).reshape(num_pages, hkv, page_size, 2).copy()
@@ -159,8 +188,9 @@ def scatter_rows(pool: HostPool, block_tables: np.ndarray, seq_idx: np.ndarray,
         pool.k[pages, :, slots, :] = k_bits
         pool.v[pages, :, slots, :] = v_bits
     else:
-        kc, ks = quantize_rows(k_bits)
-        vc, vs = quantize_rows(v_bits)
+        qf = quantize_rows if pool.kind == "u8" else quantize_rows_fp8
+        kc, ks = qf(k_bits)
+        vc, vs = qf(v_bits)
         pool.k[pages, :, slots, :] = kc
         pool.v[pages, :, slots, :] = vc
         pool.k_sz[pages, :, slots, :] = ks
@@ -187,7 +217,7 @@ def paged_attention(pool: HostPool, q_bits: np.ndarray, block_tables: np.ndarray
     n = B * Hq if pr is None else pr.shape[0]
     out = np.zeros((n, D), np.float64)
     lse = np.zeros((n,), np.float64)
-    kind = 0 if pool.kind == "bf16" else 1
+    kind = {"bf16": 0, "u8": 1, "fp8": 2}[pool.kind]
     st = lib().oracle_paged_attention(
         kind, _ptr(_c(pool.k, pool.k.dtype)), _ptr(_c(pool.v, pool.v.dtype)),
         _ptr(None if pool.k_sz is None else _c(pool.k_sz, np.float32)),
@@ -214,7 +244,7 @@ def paged_attention_window(pool: HostPool, q_bits: np.ndarray, block_tables: np.
     n = B * Hq if pr is None else pr.shape[0]
     out = np.zeros((n, D), np.float64)
     lse = np.zeros((n,), np.float64)
-    kind = 0 if pool.kind == "bf16" else 1
+    kind = {"bf16": 0, "u8": 1, "fp8": 2}[pool.kind]
     st = lib().oracle_paged_attention_window(
         kind, _ptr(_c(pool.k, pool.k.dtype)), _ptr(_c(pool.v, pool.v.dtype)),
         _ptr(None if pool.k_sz is None else _c(pool.k_sz, np.float32)),

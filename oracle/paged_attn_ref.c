@@ -39,19 +39,22 @@ static double bf16_bits_to_f64(uint16_t b) {
   return (double)f;
 }
 
+double oracle_e4m3_value(uint8_t c); /* quant_ref.c: E4M3 code -> value */
+
 /* One element of a cached row, widened to fp64.  kind 0: bf16 bits;
- * kind 1: uint8 code with the row's fp32 (scale, zero). */
+ * kind 1: uint8 code with the row's fp32 (scale, zero), value s*code + z;
+ * kind 2: E4M3 code with the row's fp32 scale, value s*E4M3(code). */
 static double kv_elem(int kind, const void *pool, const float *sz, int64_t row,
                       int d, int j) {
   if (kind == 0) {
     const uint16_t *p = (const uint16_t *)pool;
     return bf16_bits_to_f64(p[row * d + j]);
-  } else {
-    const uint8_t *p = (const uint8_t *)pool;
-    double s = (double)sz[2 * row + 0];
-    double z = (double)sz[2 * row + 1];
-    return s * (double)p[row * d + j] + z;
   }
+  const uint8_t *p = (const uint8_t *)pool;
+  const double s = (double)sz[2 * row + 0];
+  const double z = (double)sz[2 * row + 1];
+  if (kind == 1) return s * (double)p[row * d + j] + z;
+  return s * oracle_e4m3_value(p[row * d + j]) + z;
 }
 
 /*
@@ -75,7 +78,7 @@ int oracle_paged_attention(int kind, const void *k_pool, const void *v_pool,
                            int n_pairs, double *out, double *lse) {
   if (hkv <= 0 || hq % hkv != 0 || d <= 0 || page_size <= 0 || B < 0)
     return ORC_BAD_ARG;
-  if (kind == 1 && (k_sz == NULL || v_sz == NULL)) return ORC_BAD_ARG;
+  if (kind != 0 && (k_sz == NULL || v_sz == NULL)) return ORC_BAD_ARG;
   const int G = hq / hkv;
   const int n_items = pairs ? n_pairs : B * hq;
   int status = ORC_OK;
@@ -160,7 +163,7 @@ int oracle_paged_attention_window(int kind, const void *k_pool, const void *v_po
   if (hkv <= 0 || hq % hkv != 0 || d <= 0 || page_size <= 0 || B < 0 || sinks < 0 ||
       window < 0)
     return ORC_BAD_ARG;
-  if (kind == 1 && (k_sz == NULL || v_sz == NULL)) return ORC_BAD_ARG;
+  if (kind != 0 && (k_sz == NULL || v_sz == NULL)) return ORC_BAD_ARG;
   const int G = hq / hkv;
   const int n_items = pairs ? n_pairs : B * hq;
   int status = ORC_OK;

@@ -188,6 +188,33 @@ def test_bad_table_entry_is_reported():
                                np.array([20], np.int32), 0.125)
 
 
+def test_fp8_dequantisation_uses_the_scale():
+    """E4M3 codes with s = 1/4: the FP8 pool must give the same fp64 output as
+    a bf16 pool holding s * value(code) (exact in bf16: 3 mantissa bits)."""
+    g = torch.Generator().manual_seed(32)
+    B, Hkv, T, D, P = 2, 2, 48, 64, 16
+    q = torch.randn(B, 4, D, generator=g).to(torch.bfloat16)
+    finite = [c for c in range(256) if c not in (0x7F, 0xFF)]
+    idx = torch.randint(0, len(finite), (2, B, Hkv, T, D), generator=g)
+    codes = torch.tensor(finite)[idx]
+    table = torch.tensor([oracle.e4m3_value(c) if c not in (0x7F, 0xFF) else 0.0
+                          for c in range(256)], dtype=torch.float64)
+    Kx, Vx = table[codes[0]] / 4, table[codes[1]] / 4
+    assert torch.equal(Kx.to(torch.bfloat16).double(), Kx)
+    kp, vp, table_ids = _contiguous_pool(Kx.float(), Vx.float(), P)
+    npg = T // P
+    def to_pool(C):
+        return C.reshape(B, Hkv, npg, P, D).permute(0, 2, 1, 3, 4).reshape(B * npg, Hkv, P, D) \
+            .numpy().astype(np.uint8)
+    sz = np.zeros((B * npg, Hkv, P, 2), np.float32)
+    sz[..., 0] = 0.25
+    ctx = np.array([48, 29], np.int32)
+    ref, _ = oracle.paged_attention(_pool("bf16", kp, vp, P), _bf16_bits(q), table_ids, ctx, 0.125)
+    out, _ = oracle.paged_attention(_pool("fp8", to_pool(codes[0]), to_pool(codes[1]), P, sz,
+                                          sz.copy()), _bf16_bits(q), table_ids, ctx, 0.125)
+    np.testing.assert_array_equal(out, ref)
+
+
 def test_int8_dequantisation_uses_scale_and_zero():
     """Eq. 3 right-hand side: with s = 1/8 and z = -16, s*code + z is an exact
     bf16 value, so the INT8 pool must give the same fp64 output as a bf16 pool
@@ -360,6 +387,59 @@ def test_quantiser_endpoints_and_round_trip_bound():
     assert np.all(np.abs(s - rel) <= rel * 2.0 ** -22)
     err = np.abs(xf - (s[:, None] * codes + z[:, None]))
     assert np.all(err <= s[:, None] * (0.5 + 255 * 2.0 ** -22) + 1e-30)
+
+
+# ------------------------------------------------------- FP8 (E4M3) pins
+def test_e4m3_code_table_from_the_format_definition():
+    """1 sign, 4 exponent bits (bias 7), 3 mantissa bits; no infinities;
+    S.1111.111 is NaN; subnormals have exponent 2^-6 and quantum 2^-9."""
+    assert oracle.e4m3_value(0x00) == 0.0 and oracle.e4m3_value(0x01) == 2.0 ** -9
+    assert oracle.e4m3_value(0x07) == 7 * 2.0 ** -9 and oracle.e4m3_value(0x08) == 2.0 ** -6
+    assert oracle.e4m3_value(0x38) == 1.0 and oracle.e4m3_value(0x7E) == 448.0
+    assert math.isnan(oracle.e4m3_value(0x7F)) and math.isnan(oracle.e4m3_value(0xFF))
+    vals = [oracle.e4m3_value(c) for c in range(0x7F)]
+    assert all(b > a for a, b in zip(vals, vals[1:]))             # strictly increasing
+    for c in range(0x7F):
+        assert oracle.e4m3_value(0x80 | c) == -vals[c] or (c == 0)
+        assert oracle.e4m3_encode(vals[c]) == c                     # exact values round trip
+        if c:
+            assert oracle.e4m3_encode(-vals[c]) == 0x80 | c
+
+
+def test_e4m3_rounding_matches_torch_float8_e4m3fn():
+    """Round to nearest, ties to even: agree with torch's float8_e4m3fn cast
+    (a library routine) on random values of every magnitude in range."""
+    g = torch.Generator().manual_seed(30)
+    mag = torch.exp2(torch.rand(200_000, generator=g) * 18 - 11)       # 2^-11 .. 2^7
+    x = (mag * torch.sign(torch.randn(200_000, generator=g))).float()
+    mids = torch.tensor([(oracle.e4m3_value(c) + oracle.e4m3_value(c + 1)) / 2
+                         for c in range(0x7E)], dtype=torch.float32)   # exact ties
+    x = torch.cat([x, mids, -mids, torch.tensor([448.0, 447.0, 460.0, -460.0])])
+    want = x.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.e4m3_encode(float(v)) for v in x.tolist()], np.uint8)
+    np.testing.assert_array_equal(got, want)
+
+
+def test_fp8_quantiser_scale_endpoints_and_bound():
+    """s = max|x| / 448 per row; the largest element maps to +-448 exactly; a
+    zero row stores s = 0; |x - s*E4M3(code)| <= s * half the code spacing."""
+    g = torch.Generator().manual_seed(31)
+    x = torch.randn(300, 128, generator=g) * torch.rand(300, 1, generator=g) * 5
+    x[3] = 0
+    xb = _bf16_bits(x)
+    codes, sz = oracle.quantize_rows_fp8(xb)
+    xf = _f64(xb)
+    amax = np.abs(xf).max(1)
+    np.testing.assert_array_equal(sz[:, 0], (amax.astype(np.float32) / np.float32(448)))
+    assert np.all(sz[:, 1] == 0) and sz[3, 0] == 0 and np.all(codes[3] == 0)
+    table = np.array([oracle.e4m3_value(c) for c in range(256)])
+    rows = np.arange(300)[amax > 0]
+    top = np.abs(xf[rows]).argmax(1)
+    assert np.all(np.isin(codes[rows, top], (0x7E, 0xFE)))
+    deq = sz[:, :1].astype(np.float64) * table[codes]
+    r = np.abs(xf) / np.where(sz[:, :1] > 0, sz[:, :1], 1)
+    spacing = np.where(r < 2.0 ** -6, 2.0 ** -9, 2.0 ** (np.floor(np.log2(np.maximum(r, 2.0 ** -6))) - 3))
+    assert np.all(np.abs(xf - deq) <= sz[:, :1] * (0.5 * spacing * (1 + 2.0 ** -20)) + 1e-30)
 
 
 # ---------------------------------------------- Eq. 2 and the memory formula
