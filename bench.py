@@ -43,7 +43,12 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="llama70b",
-                    choices=["llama70b", "llama8b", "int8", "prefix", "tiny"])
+                    choices=["llama70b", "llama8b", "int8", "fp8", "prefix", "tiny"])
+    ap.add_argument("--cascade", action="store_true",
+                    help="prefix workload: decode with pa_decode_shared_prefix")
+    ap.add_argument("--window", type=int, default=0,
+                    help="attend only the last W tokens (+ --sinks) via pa_decode_window")
+    ap.add_argument("--sinks", type=int, default=0)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--splits", type=int, default=0, help="split-KV count (0 = automatic)")
     ap.add_argument("--batch", type=int, default=0,
@@ -53,12 +58,20 @@ def parse():
 
 
 # ------------------------------------------------------------------ accounting
-def decode_bytes(w) -> int:
+def attended_tokens(w, sinks: int = 0, window: int = 0) -> int:
+    """Tokens one decode attends: the whole context, or sinks + the last window."""
+    ctx = w.context_lens.astype("int64")
+    if window <= 0:
+        return int(ctx.sum())
+    import numpy as np
+    return int(np.minimum(ctx, np.minimum(ctx, sinks) + window).sum())
+
+
+def decode_bytes(w, sinks: int = 0, window: int = 0) -> int:
     """Algorithmic bytes of one decode: every cached K/V element of every
     attended token once, plus q (Eq. 1 reads nothing else)."""
-    tok = int(w.context_lens.astype("int64").sum())
     per_tok = w.Hkv * 2 * (w.D * 2 if w.kv == "bf16" else w.D + 8)
-    return tok * per_tok + w.B * w.Hq * w.D * 2
+    return attended_tokens(w, sinks, window) * per_tok + w.B * w.Hq * w.D * 2
 
 
 def append_bytes(w) -> int:
@@ -216,14 +229,24 @@ def make_workload(name: str, seed: int, batch: int = 0):
     return getattr(W, name)(seed=seed, **kw)
 
 
+def workload_label(w, args) -> str:
+    extra = ""
+    if args.window > 0:
+        extra = f", sinks={args.sinks}, window={args.window}"
+    if args.cascade:
+        extra += f", cascade over the {w.notes.get('prefix_tokens', 0)}-token shared prefix"
+    return extra
+
+
 def config_of(w, args, n, S):
     c = {"workload": f"{w.name}: B={w.B}, ctx={'U' if len(set(w.context_lens.tolist())) > 1 else ''}"
                      f"{int(w.context_lens.min())}..{int(w.context_lens.max())}, Hq={w.Hq}, "
-                     f"Hkv={w.Hkv}, D={w.D}, P={w.P}, kv={w.kv}",
+                     f"Hkv={w.Hkv}, D={w.D}, P={w.P}, kv={w.kv}" + workload_label(w, args),
          "global_batch": w.B * n, "seq_len": int(w.context_lens.max()),
          "parallelism": f"dp{n} (independent sequences, no collective)",
          "num_splits": S, "pool_pages": w.num_pages,
-         "l2": "inputs larger than the 126 MB L2, not flushed" if decode_bytes(w) > 256e6
+         "l2": "inputs larger than the 126 MB L2, not flushed"
+               if decode_bytes(w, args.sinks, args.window) > 256e6
                else "L2 not flushed (working set may be L2-resident)"}
     return c
 
@@ -232,6 +255,9 @@ def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
     from paged_kv_cache_466_b200 import (KVPool, pa_decode, pa_decode_num_splits,
+                                         pa_decode_shared_prefix,
+                                         pa_decode_shared_prefix_workspace_bytes,
+                                         pa_decode_window, pa_decode_window_workspace_bytes,
                                          pa_decode_workspace_bytes, pa_kv_append)
 
     dev = torch.device("cuda", local_rank)
@@ -251,16 +277,35 @@ def run_ours(args, rank, world, local_rank):
     sseq = torch.from_numpy(w.step_seq).to(dev)
     spos = torch.from_numpy(w.step_pos).to(dev)
     S = pa_decode_num_splits(pool, w.B, w.max_pages, args.splits)
-    ws = torch.zeros(max(pa_decode_workspace_bytes(w.B, w.Hq, w.D, S), 256), dtype=torch.uint8,
-                     device=dev)
+    if args.cascade:
+        pre_len = int(w.notes["prefix_tokens"])
+        pre_pages = torch.from_numpy(w.notes["prefix_pages"].copy()).to(dev)
+        nbytes = pa_decode_shared_prefix_workspace_bytes(pool, w.B, w.Hq, w.max_pages, pre_len,
+                                                         args.splits)
+    elif args.window > 0:
+        nbytes = pa_decode_window_workspace_bytes(pool, w.B, w.Hq, w.max_pages, args.sinks,
+                                                  args.window, args.splits)
+    else:
+        nbytes = pa_decode_workspace_bytes(w.B, w.Hq, w.D, S)
+    ws = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=dev)
     out = torch.empty((w.B, w.Hq, w.D), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
+
+    def decode(qq, tt, cc):
+        if args.cascade:
+            pa_decode_shared_prefix(pool, qq, pre_pages, pre_len, tt, cc, w.scale, out=out,
+                                    workspace=ws, num_splits=args.splits)
+        elif args.window > 0:
+            pa_decode_window(pool, qq, tt, cc, w.scale, args.sinks, args.window, out=out,
+                             workspace=ws, num_splits=args.splits)
+        else:
+            pa_decode(pool, qq, tt, cc, w.scale, out=out, workspace=ws, num_splits=S)
 
     def step(ev0=None, ev1=None):
         pa_kv_append(pool, sk, sv, sseq, spos, bt)
         if ev0 is not None:
             ev0.record(stream)
-        pa_decode(pool, q, bt, ctx, w.scale, out=out, workspace=ws, num_splits=S)
+        decode(q, bt, ctx)
         if ev1 is not None:
             ev1.record(stream)
 
@@ -291,7 +336,8 @@ def run_ours(args, rank, world, local_rank):
     ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
     dec_ms = [a.elapsed_time(b) for a, b in evs]
     ms_step = ms / K
-    step_bytes = decode_bytes(w) + append_bytes(w)
+    dbytes = decode_bytes(w, args.sinks, args.window)
+    step_bytes = dbytes + append_bytes(w)
     value = whole_job_gbs(step_bytes, world, ms_step)
 
     # ---- end to end through the public API, host buffers in pinned memory
@@ -313,7 +359,7 @@ def run_ours(args, rank, world, local_rank):
                      (d_ctx, h_ctx), (d_bt, h_bt)):
             d.copy_(h, non_blocking=True)
         pa_kv_append(pool, d_k, d_v, d_seq, d_pos, d_bt)
-        pa_decode(pool, d_q, d_bt, d_ctx, w.scale, out=out, workspace=ws, num_splits=S)
+        decode(d_q, d_bt, d_ctx)
         h_out.copy_(out, non_blocking=True)
         stream.synchronize()   # the caller reads the result every step
 
@@ -334,9 +380,9 @@ def run_ours(args, rank, world, local_rank):
 
     peak, peak_kind = measured_peak()
     dec_avg_ms = statistics.mean(dec_ms)
-    achieved = decode_bytes(w) / (dec_avg_ms * 1e-3) / 1e9
-    traffic = recorded_traffic(w.name)
-    launches_per_step = 2 + (1 if S > 1 else 0)
+    achieved = dbytes / (dec_avg_ms * 1e-3) / 1e9
+    traffic = recorded_traffic(w.name) if not (args.cascade or args.window) else None
+    launches_per_step = 3 if args.cascade else 2
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
@@ -351,10 +397,13 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": Ke,
                 "ms_per_step": round(ems / Ke, 5)},
-        "roofline": {"bound": "hbm", "kernel": "pa_decode (decode kernel + split merge)",
+        "roofline": {"bound": "hbm",
+                     "kernel": ("pa_decode_shared_prefix (prefix pass + decode)" if args.cascade
+                                else "pa_decode_window" if args.window > 0
+                                else "pa_decode (one launch, split merge fused)"),
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "algorithmic_bytes": decode_bytes(w),
+                     "algorithmic_bytes": dbytes,
                      "avg_launch_ms": round(dec_avg_ms, 5)},
         "gpu_launches": K * launches_per_step,
         "clocks": clk,

@@ -62,17 +62,19 @@ typedef enum {
 #define PA_DERR_BAD_POS 8  /* append: pos < 0 or pos / page_size >= max_pages  */
 
 typedef enum {
-  PA_KV_BF16 = 0,         /* K/V stored as bf16                               */
-  PA_KV_U8_PER_TOKEN = 1  /* Eq. (3): uint8 codes + fp32 (scale, zero) per row */
+  PA_KV_BF16 = 0,          /* K/V stored as bf16                               */
+  PA_KV_U8_PER_TOKEN = 1,  /* Eq. (3): uint8 codes + fp32 (scale, zero) per row */
+  PA_KV_FP8_PER_TOKEN = 2  /* E4M3 codes + fp32 (scale, 0) per row; x = s * e4m3 */
 } pa_kv_dtype_t;
 
 /*
  * The physical page pool ("PagedAttention (vLLM)", "Architecture").
  * Layout of one tensor (K or V): [num_pages][num_kv_heads][page_size][head_dim],
  * row-major, so the page_size x head_dim block of one (page, KV head) is
- * contiguous. bf16 pools hold 2-byte elements, INT8 pools 1-byte codes plus
- * k_sz / v_sz = fp32 [num_pages][num_kv_heads][page_size][2] holding
- * (scale, zero) of each row. Every pointer must be 16-byte aligned.
+ * contiguous. bf16 pools hold 2-byte elements; INT8 and FP8 pools hold 1-byte
+ * codes plus k_sz / v_sz = fp32 [num_pages][num_kv_heads][page_size][2]
+ * holding (scale, zero) of each row (zero is 0 for FP8). Every pointer must be
+ * 16-byte aligned.
  * Supported: page_size in {16, 32}; head_dim in {64, 128}.
  */
 typedef struct {
@@ -94,6 +96,10 @@ typedef struct {
  * demand. For an INT8 pool each row is quantised on the way in by Eq. (3):
  * z = min of the row, s = (max - min) / 255, code = round-half-even((x - z)/s)
  * clamped to [0, 255], all in IEEE fp32; a constant row stores s = 0, codes 0.
+ * For an FP8 pool (the pages name FP8 KV caches without fixing the encoding;
+ * this library uses OCP E4M3 with a per-row absmax scale): s = max|x| / 448,
+ * code = E4M3(x / s) rounded to nearest even and saturated at +-448, zero 0;
+ * an all-zero row stores s = 0, codes 0.
  * Input rows must be finite; -0 is stored as +0.)
  *
  *   k_new, v_new : (device) bf16 [num_tokens][num_kv_heads][head_dim]

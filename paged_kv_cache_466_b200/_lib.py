@@ -25,6 +25,7 @@ PA_DERR_BAD_POS = 8
 
 PA_KV_BF16 = 0
 PA_KV_U8_PER_TOKEN = 1
+PA_KV_FP8_PER_TOKEN = 2
 
 PA_NOALLOC_SCRATCH_BYTES = 16 << 20
 

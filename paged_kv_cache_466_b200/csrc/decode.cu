@@ -36,10 +36,12 @@
 // Rows are stored with their 16-byte chunks XOR-permuted (staged_off) so that
 // both read patterns are free of shared-memory bank conflicts.
 //
-// INT8 cache (Eq. 3, "KV-Cache Quantization"): with x = s*c + z per row,
+// INT8 and FP8 caches (Eq. 3, "KV-Cache Quantization"; FP8 = E4M3 codes
+// with z = 0): with x = s*c + z per row,
 //   q.x = s (q.c) + z sum(q)          and    sum_t p_t x_t = sum_t (p_t s_t) c_t + sum_t p_t z_t,
-// so the codes go through the tensor cores as exact f16 integers and the scale
-// and zero are applied once per (token, head) instead of once per element.
+// so the codes go through the tensor cores as exact f16 values (INT8 codes as
+// integers, E4M3 codes converted exactly) and the scale and zero are applied
+// once per (token, head) instead of once per element.
 #include <atomic>
 #include <cfloat>
 #include <cmath>
@@ -76,7 +78,9 @@ constexpr float kRescaleLog2 = 8.0f;
 template <int D, int KVT>
 struct Tile {
   static_assert(D == 64 || D == 128, "head_dim");
-  static constexpr bool kU8 = KVT == PA_KV_U8_PER_TOKEN;
+  // INT8 and FP8 pools share the layout: 1-byte codes + (scale, zero) per row
+  static constexpr bool kU8 = KVT != PA_KV_BF16;
+  static constexpr bool kFp8 = KVT == PA_KV_FP8_PER_TOKEN;
   static constexpr int kElem = kU8 ? 1 : 2;
   static constexpr int kRowBytes = D * kElem;
   // one 16-token block of K (or V) is 16 contiguous rows of the page
@@ -123,7 +127,7 @@ struct Smem {
 // Row of O^T held in accumulator c0/c1 (row g) of m-tile j; c2/c3 hold d + 1.
 template <int D, int KVT>
 __device__ __forceinline__ int out_col(int j, int g) {
-  if constexpr (KVT == PA_KV_U8_PER_TOKEN) {
+  if constexpr (KVT != PA_KV_BF16) {
     return (D == 128 ? 16 * g : 8 * g) + 2 * j;
   } else {
     return 8 * (8 * (j / 4) + g) + 2 * (j % 4);
@@ -434,8 +438,10 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
           const uint32_t w4[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
           for (int w = 0; w < 4; ++w) {
-            mma_f16_16816(s[nt], qa[4 * i + w][0], 0u, qa[4 * i + w][1], 0u,
-                          u8x2_to_f16x2(w4[w], 0x4140), u8x2_to_f16x2(w4[w], 0x4342));
+            const uint32_t b0 = T::kFp8 ? e4m3x2_to_f16x2(w4[w]) : u8x2_to_f16x2(w4[w], 0x4140);
+            const uint32_t b1 =
+                T::kFp8 ? e4m3x2_to_f16x2(w4[w] >> 16) : u8x2_to_f16x2(w4[w], 0x4342);
+            mma_f16_16816(s[nt], qa[4 * i + w][0], 0u, qa[4 * i + w][1], 0u, b0, b1);
           }
         }
       }
@@ -552,10 +558,10 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
         const uint32_t w3 = D == 128 ? x3[j / 2] : ((g & 1) ? x3[2 + j / 2] : x3[j / 2]);
         const uint32_t xa = __byte_perm(w0, w1, sel);
         const uint32_t xb = __byte_perm(w2, w3, sel);
-        const uint32_t a0 = u8x2_to_f16x2(xa, 0x4140);
-        const uint32_t a1 = u8x2_to_f16x2(xa, 0x4342);
-        const uint32_t a2 = u8x2_to_f16x2(xb, 0x4140);
-        const uint32_t a3 = u8x2_to_f16x2(xb, 0x4342);
+        const uint32_t a0 = T::kFp8 ? e4m3x2_to_f16x2(xa) : u8x2_to_f16x2(xa, 0x4140);
+        const uint32_t a1 = T::kFp8 ? e4m3x2_to_f16x2(xa >> 16) : u8x2_to_f16x2(xa, 0x4342);
+        const uint32_t a2 = T::kFp8 ? e4m3x2_to_f16x2(xb) : u8x2_to_f16x2(xb, 0x4140);
+        const uint32_t a3 = T::kFp8 ? e4m3x2_to_f16x2(xb >> 16) : u8x2_to_f16x2(xb, 0x4342);
         mma_f16_16816(o[j], a0, a1, a2, a3, bh0, bh1);
         mma_f16_16816(o[j], a0, a1, a2, a3, bl0, bl1);
       }
@@ -652,8 +658,7 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
 template <int D, int P, int KVT>
 struct Config {
   static constexpr int W = PA_DECODE_WARPS;
-  static constexpr int NSTAGE =
-      KVT == PA_KV_U8_PER_TOKEN ? PA_DECODE_STAGES_U8 : PA_DECODE_STAGES_BF16;
+  static constexpr int NSTAGE = KVT != PA_KV_BF16 ? PA_DECODE_STAGES_U8 : PA_DECODE_STAGES_BF16;
   using SM = Smem<D, KVT, W, NSTAGE>;
   static void *fn() { return reinterpret_cast<void *>(&decode_kernel<D, P, KVT, W, NSTAGE>); }
 };
@@ -716,6 +721,7 @@ cudaError_t launch_decode(int D, int P, int kv_dtype, const DecodeArgs &a, cudaS
 #define PA_L(D_, P_, K_) PA_DISPATCH(D_, P_, K_, launch_t)(a, stream)
   PA_L(128, 16, 0); PA_L(128, 32, 0); PA_L(64, 16, 0); PA_L(64, 32, 0);
   PA_L(128, 16, 1); PA_L(128, 32, 1); PA_L(64, 16, 1); PA_L(64, 32, 1);
+  PA_L(128, 16, 2); PA_L(128, 32, 2); PA_L(64, 16, 2); PA_L(64, 32, 2);
 #undef PA_L
   return cudaErrorInvalidValue;
 }
@@ -724,6 +730,7 @@ int decode_ctas_per_sm(int D, int P, int kv_dtype) {
 #define PA_O(D_, P_, K_) PA_DISPATCH(D_, P_, K_, ctas_per_sm_t)()
   PA_O(128, 16, 0); PA_O(128, 32, 0); PA_O(64, 16, 0); PA_O(64, 32, 0);
   PA_O(128, 16, 1); PA_O(128, 32, 1); PA_O(64, 16, 1); PA_O(64, 32, 1);
+  PA_O(128, 16, 2); PA_O(128, 32, 2); PA_O(64, 16, 2); PA_O(64, 32, 2);
 #undef PA_O
   return 1;
 }

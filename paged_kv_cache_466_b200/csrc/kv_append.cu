@@ -4,7 +4,8 @@
 // "Architecture": each request's page table maps a logical KV position to a
 // physical page of P tokens; position pos lives in page table[pos / P], slot
 // pos % P. For an INT8 pool every (token, KV head) row is quantised on the way
-// in by Eq. 3 ("KV-Cache Quantization", per-token calibration):
+// in by Eq. 3 ("KV-Cache Quantization", per-token calibration; an FP8 pool
+// uses E4M3 codes with an absmax scale, see quantise_row_fp8):
 //   z = min(row), s = (max(row) - min(row)) / 255,
 //   code = clamp(round_half_even((x - z) / s), 0, 255)   (s == 0 -> code 0),
 // every step an IEEE fp32 operation in that order (explicit _rn intrinsics,
@@ -117,8 +118,40 @@ __device__ __forceinline__ void quantise_row(const unsigned char *src_row, unsig
   if (lane == 0) *reinterpret_cast<float2 *>(dst_sz) = make_float2(s, z);
 }
 
-// INT8: one warp per (token, head) row; K then V.
+// FP8 (E4M3) per-token quantiser: s = max|x| / 448 (IEEE fp32), code =
+// E4M3(x / s) rounded to nearest even and saturated; an all-zero row stores
+// s = 0 and codes 0. The zero point is stored as 0.
 template <int D>
+__device__ __forceinline__ void quantise_row_fp8(const unsigned char *src_row,
+                                                 unsigned char *dst_codes, float *dst_sz,
+                                                 int lane) {
+  constexpr int E = D / 32;  // elements per lane (even)
+  const __nv_bfloat16 *x16 = reinterpret_cast<const __nv_bfloat16 *>(src_row) + lane * E;
+  float x[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) x[e] = __fadd_rn(__bfloat162float(x16[e]), 0.0f);
+  float amax = 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(x[e]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float s = __fdiv_rn(amax, 448.0f);
+  uint32_t packed = 0;
+  if (s != 0.0f) {
+#pragma unroll
+    for (int e = 0; e < E; e += 2)
+      packed |= f32x2_to_e4m3x2(__fdiv_rn(x[e], s), __fdiv_rn(x[e + 1], s)) << (8 * e);
+  }
+  if constexpr (E == 4) {
+    *reinterpret_cast<uint32_t *>(dst_codes + lane * 4) = packed;
+  } else {
+    *reinterpret_cast<uint16_t *>(dst_codes + lane * 2) = static_cast<uint16_t>(packed);
+  }
+  if (lane == 0) *reinterpret_cast<float2 *>(dst_sz) = make_float2(s, 0.f);
+}
+
+// INT8 / FP8: one warp per (token, head) row; K then V.
+template <int D, bool kFp8>
 __global__ void append_u8_kernel(const AppendArgs a) {
   pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
@@ -133,8 +166,15 @@ __global__ void append_u8_kernel(const AppendArgs a) {
     row = __shfl_sync(0xffffffffu, row, 0);
     if (row < 0) continue;
     const size_t src = (size_t)r * D * 2;
-    quantise_row<D>(a.k_new + src, a.k_pool + (size_t)row * D, a.k_sz + (size_t)row * 2, lane);
-    quantise_row<D>(a.v_new + src, a.v_pool + (size_t)row * D, a.v_sz + (size_t)row * 2, lane);
+    if constexpr (kFp8) {
+      quantise_row_fp8<D>(a.k_new + src, a.k_pool + (size_t)row * D, a.k_sz + (size_t)row * 2,
+                          lane);
+      quantise_row_fp8<D>(a.v_new + src, a.v_pool + (size_t)row * D, a.v_sz + (size_t)row * 2,
+                          lane);
+    } else {
+      quantise_row<D>(a.k_new + src, a.k_pool + (size_t)row * D, a.k_sz + (size_t)row * 2, lane);
+      quantise_row<D>(a.v_new + src, a.v_pool + (size_t)row * D, a.v_sz + (size_t)row * 2, lane);
+    }
   }
 }
 
@@ -172,10 +212,15 @@ cudaError_t launch_kv_append(const pa_kv_pool_t &pool, const void *k_new, const 
     const long long rows = (long long)n * a.hkv;
     long long blocks = (rows + 7) / 8;
     blocks = blocks < 1 ? 1 : (blocks > 16LL * sms ? 16LL * sms : blocks);
-    if (a.D == 128)
-      append_u8_kernel<128><<<(unsigned)blocks, 256, 0, stream>>>(a);
+    const bool fp8 = pool.dtype == PA_KV_FP8_PER_TOKEN;
+    if (a.D == 128 && !fp8)
+      append_u8_kernel<128, false><<<(unsigned)blocks, 256, 0, stream>>>(a);
+    else if (a.D == 64 && !fp8)
+      append_u8_kernel<64, false><<<(unsigned)blocks, 256, 0, stream>>>(a);
+    else if (a.D == 128)
+      append_u8_kernel<128, true><<<(unsigned)blocks, 256, 0, stream>>>(a);
     else
-      append_u8_kernel<64><<<(unsigned)blocks, 256, 0, stream>>>(a);
+      append_u8_kernel<64, true><<<(unsigned)blocks, 256, 0, stream>>>(a);
   }
   return cudaGetLastError();
 }

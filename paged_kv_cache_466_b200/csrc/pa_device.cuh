@@ -148,6 +148,26 @@ __device__ __forceinline__ uint32_t u8x2_to_f16x2(uint32_t word, uint32_t sel) {
   return r;
 }
 
+// Two E4M3 codes (bits 0..7 and 8..15 of `pair`) -> f16x2 with the first code in
+// the low half. Exact: every E4M3 value is an f16 value.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t pair) {
+  uint32_t r;
+  asm("{\n .reg .b16 lo, hi;\n mov.b32 {lo, hi}, %1;\n cvt.rn.f16x2.e4m3x2 %0, lo;\n}\n"
+      : "=r"(r)
+      : "r"(pair));
+  return r;
+}
+
+// Two fp32 -> two E4M3 codes (round to nearest even, saturate to +-448), the
+// code of `lo` in bits 0..7.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+  uint32_t r;
+  asm("{\n .reg .b16 c;\n cvt.rn.satfinite.e4m3x2.f32 c, %1, %2;\n cvt.u32.u16 %0, c;\n}\n"
+      : "=r"(r)
+      : "f"(hi), "f"(lo));
+  return r;
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));

@@ -41,7 +41,7 @@ class Workload:
     Hkv: int
     D: int
     P: int
-    kv: str                         # "bf16" or "u8"
+    kv: str                         # "bf16", "u8" (INT8) or "fp8" (E4M3)
     num_pages: int
     max_pages: int
     scale: float
@@ -184,7 +184,7 @@ def tiny(seed: int = 0) -> Workload:
 def llama8b(B: int = 64, ctx_range=(128, 4096), seed: int = 0, kv: str = "bf16",
             outlier_frac: float = 0.0) -> Workload:
     """Llama-3-8B-shaped layer: Hq=32, Hkv=8, D=128, P=16, pool = 1.1 x need."""
-    return paged("llama8b" if kv == "bf16" else "int8", B=B, Hq=32, Hkv=8, D=128, P=16,
+    return paged({"bf16": "llama8b", "u8": "int8", "fp8": "fp8"}[kv], B=B, Hq=32, Hkv=8, D=128, P=16,
                  ctx_range=ctx_range, pool_slack=0.10, max_pages=-(-ctx_range[1] // 16),
                  kv=kv, outlier_frac=outlier_frac, seed=seed)
 
@@ -194,6 +194,13 @@ def llama70b(B: int = 32, ctx: int = 8192, seed: int = 0) -> Workload:
     every context 8192 tokens, pool exactly the 8192 pages needed (B=32)."""
     return paged("llama70b", B=B, Hq=64, Hkv=8, D=128, P=32, context_lens=[ctx] * B,
                  seed=seed)
+
+
+def fp8(B: int = 64, ctx_range=(128, 4096), seed: int = 0) -> Workload:
+    """``llama8b`` draws plus 1 % outliers ~ N(0, 8^2), cached as per-token FP8 (E4M3)."""
+    w = llama8b(B=B, ctx_range=ctx_range, seed=seed, kv="fp8", outlier_frac=0.01)
+    w.name = "fp8"
+    return w
 
 
 def int8(B: int = 64, ctx_range=(128, 4096), seed: int = 0) -> Workload:
@@ -268,10 +275,12 @@ def by_name(name: str, **kw):
         return llama70b(**kw)
     if name == "int8":
         return int8(**kw)
+    if name == "fp8":
+        return fp8(**kw)
     if name == "prefix":
         return prefix(**kw)[0]
     raise KeyError(name)
 
 
-__all__ = ["Workload", "bits", "paged", "tiny", "llama8b", "llama70b", "int8", "prefix",
+__all__ = ["Workload", "bits", "paged", "tiny", "llama8b", "llama70b", "int8", "fp8", "prefix",
            "by_name"]

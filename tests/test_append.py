@@ -20,7 +20,11 @@ pytestmark = pytest.mark.gpu
     lambda: W.paged("u8d64", B=5, Hq=4, Hkv=2, D=64, P=16, ctx_range=(1, 300), kv="u8",
                     outlier_frac=0.02),
     lambda: W.paged("u8p32", B=3, Hq=16, Hkv=2, D=128, P=32, ctx_range=(1, 200), kv="u8"),
-], ids=["tiny", "llama8b-small", "p32-d64", "int8-small", "int8-d64", "int8-p32"])
+    lambda: W.fp8(B=6, ctx_range=(1, 700)),
+    lambda: W.paged("fp8d64", B=5, Hq=4, Hkv=2, D=64, P=32, ctx_range=(1, 300), kv="fp8",
+                    outlier_frac=0.05),
+], ids=["tiny", "llama8b-small", "p32-d64", "int8-small", "int8-d64", "int8-p32", "fp8-small",
+        "fp8-d64-p32"])
 def test_append_matches_oracle_scatter_bit_exact(make):
     w = make()
     pool, bt, _, _ = device_inputs(w, fill_byte=0xA5)
@@ -38,6 +42,40 @@ def test_append_int8_full_pool_bit_exact():
     device_append(pool, w, bt)
     torch.cuda.synchronize()
     ok, msg = pool_bytes_equal(pool, oracle_pool(w, fill_byte=0x00))
+    assert ok, msg
+
+
+def test_append_fp8_full_pool_bit_exact():
+    """All pages of the FP8 workload: every E4M3 code and fp32 scale equals the
+    oracle's (round to nearest even, saturating, per-row absmax scale)."""
+    w = W.fp8()
+    pool, bt, _, _ = device_inputs(w, fill_byte=0x00)
+    device_append(pool, w, bt)
+    torch.cuda.synchronize()
+    ok, msg = pool_bytes_equal(pool, oracle_pool(w, fill_byte=0x00))
+    assert ok, msg
+
+
+@pytest.mark.parametrize("kind", ["u8", "fp8"])
+def test_append_quantiser_edge_rows_both_formats(kind):
+    D, Hkv = 128, 2
+    rows = []
+    rows.append(np.full(D, 3.25, np.float32))
+    r = np.zeros(D, np.float32); r[::2] = -0.0; r[5] = 2.0; rows.append(r)
+    r = np.arange(D, dtype=np.float32) + 0.5; r[0] = 0.0; r[1] = 255.0; rows.append(r)
+    r = np.linspace(-3e4, 3e4, D).astype(np.float32); rows.append(r)
+    r = np.linspace(-1e-30, 1e-30, D).astype(np.float32); rows.append(r)
+    r = np.zeros(D, np.float32); rows.append(r)
+    x = torch.from_numpy(np.stack(rows)).to(torch.bfloat16)
+    n = x.shape[0] // Hkv
+    k = x[:n * Hkv].reshape(n, Hkv, D)
+    w = W.paged("edge", B=1, Hq=2, Hkv=Hkv, D=D, P=16, context_lens=[n], kv=kind)
+    w.prefill_k, w.prefill_v = k[:-1].contiguous(), k.flip(0)[:-1].contiguous()
+    w.step_k, w.step_v = k[-1:].contiguous(), k.flip(0)[-1:].contiguous()
+    pool, bt, _, _ = device_inputs(w)
+    device_append(pool, w, bt)
+    torch.cuda.synchronize()
+    ok, msg = pool_bytes_equal(pool, oracle_pool(w))
     assert ok, msg
 
 

@@ -53,6 +53,9 @@ SMALL = {
     "u8-p32-g8": lambda: W.paged("u8p32", B=3, Hq=16, Hkv=2, D=128, P=32,
                                  ctx_range=(1, 400), kv="u8"),
     "g3": lambda: W.paged("g3", B=3, Hq=6, Hkv=2, D=128, P=16, ctx_range=(1, 100)),
+    "fp8-small": lambda: W.fp8(B=6, ctx_range=(1, 700)),
+    "fp8-d64-p32-g8": lambda: W.paged("fp8b", B=3, Hq=16, Hkv=2, D=64, P=32,
+                                      ctx_range=(1, 400), kv="fp8", outlier_frac=0.02),
 }
 
 
@@ -203,7 +206,7 @@ def _sample_pairs(w, n, seed=0):
     return sorted(set(pairs))
 
 
-@pytest.mark.parametrize("name", ["tiny", "llama8b", "llama70b", "int8"])
+@pytest.mark.parametrize("name", ["tiny", "llama8b", "llama70b", "int8", "fp8"])
 def test_full_size_sampled_outputs(name):
     """The full workloads, in the launch configuration the benchmark times
     (automatic split count), checked on sampled (sequence, head) rows."""

@@ -46,6 +46,7 @@ CASES = {
     "bf16-p32-g8": lambda: W.paged("p32", B=4, Hq=32, Hkv=4, D=128, P=32, ctx_range=(1, 1200)),
     "int8": lambda: W.int8(B=6, ctx_range=(1, 900)),
     "d64": lambda: W.paged("d64", B=5, Hq=8, Hkv=2, D=64, P=16, ctx_range=(1, 400)),
+    "fp8": lambda: W.fp8(B=6, ctx_range=(1, 900)),
 }
 
 
