@@ -13,6 +13,8 @@ Contents, each written from the pages ("KV-Cache Optimization Techniques",
   ``pos`` of a sequence lives in physical page ``table[pos // P]`` at slot
   ``pos % P`` (section "PagedAttention (vLLM)", "Architecture").
 * ``quantize_rows``        — Eq. 3 per-token INT8 quantiser (C, fp32 IEEE).
+* ``quantize_rows_int4``   — per-token INT4 quantiser (Eq. 3 with 16 levels,
+  two codes per byte).
 * ``quantize_rows_fp8``    — per-token FP8 (E4M3) quantiser with an absmax scale
   (the pages' FP8 KV cache; encoding written from the format definition).
 * ``paged_attention``      — Eq. 1 over gathered pages (C, fp64).
@@ -70,6 +72,9 @@ def lib() -> ctypes.CDLL:
         L.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
         L.oracle_e4m3_encode.restype = ctypes.c_uint8
         L.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        L.oracle_quantize_rows_int4.restype = None
+        L.oracle_quantize_rows_int4.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+                                                ctypes.c_void_p, ctypes.c_void_p]
         L.oracle_quantize_rows.restype = None
         L.oracle_quantize_rows.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
                                            ctypes.c_void_p, ctypes.c_void_p]
@@ -115,6 +120,25 @@ def quantize_rows_fp8(x_bits: np.ndarray):
     return codes.reshape(x.shape), sz.reshape(x.shape[:-1] + (2,))
 
 
+def quantize_rows_int4(x_bits: np.ndarray):
+    """Per-row INT4 quantisation (Eq. 3 with 16 levels); returns packed codes
+    [..., D/2] (element 2i in the low nibble of byte i) and sz [..., 2]."""
+    x = _c(x_bits, np.uint16)
+    d = x.shape[-1]
+    rows = x.reshape(-1, d)
+    packed = np.empty((rows.shape[0], d // 2), np.uint8)
+    sz = np.empty((rows.shape[0], 2), np.float32)
+    lib().oracle_quantize_rows_int4(_ptr(rows), rows.shape[0], d, _ptr(packed), _ptr(sz))
+    return packed.reshape(x.shape[:-1] + (d // 2,)), sz.reshape(x.shape[:-1] + (2,))
+
+
+def unpack_int4(packed: np.ndarray) -> np.ndarray:
+    """[..., D/2] bytes -> [..., D] codes (low nibble first)."""
+    lo = packed & 15
+    hi = packed >> 4
+    return np.stack([lo, hi], -1).reshape(packed.shape[:-1] + (packed.shape[-1] * 2,))
+
+
 def e4m3_value(code: int) -> float:
     return float(lib().oracle_e4m3_value(int(code)))
 
@@ -135,7 +159,7 @@ def dequantize_rows(codes: np.ndarray, sz: np.ndarray) -> np.ndarray:
 @dataclass
 class HostPool:
     """A KV page pool in host memory: [num_pages][Hkv][P][D] per tensor."""
-    kind: str                      # "bf16", "u8" (INT8, Eq. 3) or "fp8" (E4M3)
+    kind: str                      # "bf16", "u8" (INT8, Eq. 3), "fp8" (E4M3) or "u4" (INT4)
     page_size: int
     k: np.ndarray                  # uint16 (bf16 bits) or uint8 codes
     v: np.ndarray
@@ -152,7 +176,7 @@ class HostPool:
 
     @property
     def head_dim(self) -> int:
-        return self.k.shape[3]
+        return self.k.shape[3] * (2 if self.kind == "u4" else 1)
 
 
 def empty_pool(kind: str, num_pages: int, hkv: int, page_size: int, d: int,
@@ -161,8 +185,9 @@ def empty_pool(kind: str, num_pages: int, hkv: int, page_size: int, d: int,
     if kind == "bf16":
         k = np.full((num_pages, hkv, page_size, d), fill_byte * 0x0101, np.uint16)
         return HostPool(kind, page_size, k, k.copy())
-    if kind in ("u8", "fp8"):
-        k = np.full((num_pages, hkv, page_size, d), fill_byte, np.uint8)
+    if kind in ("u8", "fp8", "u4"):
+        k = np.full((num_pages, hkv, page_size, d // 2 if kind == "u4" else d), fill_byte,
+                    np.uint8)
         sz = np.frombuffer(bytes([fill_byte]) * (num_pages * hkv * page_size * 8),
                            np.float32).reshape(num_pages, hkv, page_size, 2).copy()
         return HostPool(kind, page_size, k, k.copy(), sz, sz.copy())
@@ -188,7 +213,7 @@ def scatter_rows(pool: HostPool, block_tables: np.ndarray, seq_idx: np.ndarray,
         pool.k[pages, :, slots, :] = k_bits
         pool.v[pages, :, slots, :] = v_bits
     else:
-        qf = quantize_rows if pool.kind == "u8" else quantize_rows_fp8
+        qf = {"u8": quantize_rows, "fp8": quantize_rows_fp8, "u4": quantize_rows_int4}[pool.kind]
         kc, ks = qf(k_bits)
         vc, vs = qf(v_bits)
         pool.k[pages, :, slots, :] = kc
@@ -211,13 +236,14 @@ def paged_attention(pool: HostPool, q_bits: np.ndarray, block_tables: np.ndarray
     """
     q = _c(q_bits, np.uint16)
     B, Hq, D = q.shape
+    assert D == pool.head_dim
     bt = _c(block_tables, np.int32)
     ctx = _c(context_lens, np.int32)
     pr = None if pairs is None else _c(np.asarray(pairs).reshape(-1, 2), np.int32)
     n = B * Hq if pr is None else pr.shape[0]
     out = np.zeros((n, D), np.float64)
     lse = np.zeros((n,), np.float64)
-    kind = {"bf16": 0, "u8": 1, "fp8": 2}[pool.kind]
+    kind = {"bf16": 0, "u8": 1, "fp8": 2, "u4": 3}[pool.kind]
     st = lib().oracle_paged_attention(
         kind, _ptr(_c(pool.k, pool.k.dtype)), _ptr(_c(pool.v, pool.v.dtype)),
         _ptr(None if pool.k_sz is None else _c(pool.k_sz, np.float32)),
@@ -244,7 +270,7 @@ def paged_attention_window(pool: HostPool, q_bits: np.ndarray, block_tables: np.
     n = B * Hq if pr is None else pr.shape[0]
     out = np.zeros((n, D), np.float64)
     lse = np.zeros((n,), np.float64)
-    kind = {"bf16": 0, "u8": 1, "fp8": 2}[pool.kind]
+    kind = {"bf16": 0, "u8": 1, "fp8": 2, "u4": 3}[pool.kind]
     st = lib().oracle_paged_attention_window(
         kind, _ptr(_c(pool.k, pool.k.dtype)), _ptr(_c(pool.v, pool.v.dtype)),
         _ptr(None if pool.k_sz is None else _c(pool.k_sz, np.float32)),

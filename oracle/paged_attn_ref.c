@@ -43,7 +43,9 @@ double oracle_e4m3_value(uint8_t c); /* quant_ref.c: E4M3 code -> value */
 
 /* One element of a cached row, widened to fp64.  kind 0: bf16 bits;
  * kind 1: uint8 code with the row's fp32 (scale, zero), value s*code + z;
- * kind 2: E4M3 code with the row's fp32 scale, value s*E4M3(code). */
+ * kind 2: E4M3 code with the row's fp32 scale, value s*E4M3(code);
+ * kind 3: 4-bit code (two per byte, element 2i in the low nibble of byte i)
+ *         with the row's fp32 (scale, zero), value s*code + z. */
 static double kv_elem(int kind, const void *pool, const float *sz, int64_t row,
                       int d, int j) {
   if (kind == 0) {
@@ -54,7 +56,10 @@ static double kv_elem(int kind, const void *pool, const float *sz, int64_t row,
   const double s = (double)sz[2 * row + 0];
   const double z = (double)sz[2 * row + 1];
   if (kind == 1) return s * (double)p[row * d + j] + z;
-  return s * oracle_e4m3_value(p[row * d + j]) + z;
+  if (kind == 2) return s * oracle_e4m3_value(p[row * d + j]) + z;
+  const uint8_t byte = p[row * (d / 2) + j / 2];
+  const int code = (j % 2 == 0) ? (byte & 15) : (byte >> 4);
+  return s * (double)code + z;
 }
 
 /*

@@ -144,3 +144,43 @@ void oracle_quantize_rows_fp8(const uint16_t *x, int64_t n_rows, int d, uint8_t 
     sz[2 * r + 1] = 0.0f;
   }
 }
+
+/*
+ * INT4 per-token quantiser: Eq. 3 with 16 levels ("KV-Cache Quantization",
+ * "FP16 -> INT4: 4x reduction"): z = min, s = (max - min) / 15, code =
+ * clamp(round_half_even((x - z) / s), 0, 15), every step in IEEE fp32 as for
+ * INT8; a constant row stores s = 0 and codes 0. Two codes per byte: element
+ * 2i in the low nibble of byte i, element 2i + 1 in the high nibble.
+ */
+void oracle_quantize_rows_int4(const uint16_t *x, int64_t n_rows, int d, uint8_t *packed,
+                               float *sz) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < n_rows; ++r) {
+    const uint16_t *row = x + r * d;
+    float mn = bf16_bits_to_f32(row[0]);
+    float mx = mn;
+    for (int j = 1; j < d; ++j) {
+      const float v = bf16_bits_to_f32(row[j]);
+      if (v < mn) mn = v;
+      if (v > mx) mx = v;
+    }
+    const float range = mx - mn;
+    const float s = range / 15.0f;
+    const float z = mn;
+    for (int j = 0; j < d; j += 2) {
+      uint8_t c[2] = {0, 0};
+      for (int k = 0; k < 2; ++k) {
+        if (s != 0.0f) {
+          const float diff = bf16_bits_to_f32(row[j + k]) - z;
+          float rq = nearbyintf(diff / s);
+          if (rq < 0.0f) rq = 0.0f;
+          if (rq > 15.0f) rq = 15.0f;
+          c[k] = (uint8_t)rq;
+        }
+      }
+      packed[r * (d / 2) + j / 2] = (uint8_t)(c[0] | (c[1] << 4));
+    }
+    sz[2 * r + 0] = s;
+    sz[2 * r + 1] = z;
+  }
+}

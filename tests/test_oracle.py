@@ -389,6 +389,60 @@ def test_quantiser_endpoints_and_round_trip_bound():
     assert np.all(err <= s[:, None] * (0.5 + 255 * 2.0 ** -22) + 1e-30)
 
 
+# ----------------------------------------------------------- INT4 pins
+def test_int4_quantiser_half_even_and_nibble_order():
+    """min 0, max 15 -> s = 1: codes are Python's round-half-even of x; element
+    2i sits in the low nibble of byte i, element 2i + 1 in the high nibble."""
+    vals = [0.0, 15.0, 1.0, 2.0, 0.5, 1.5, 2.5, 7.5, 14.5, 3.25, 9.75, 12.0]
+    packed, sz = oracle.quantize_rows_int4(_row_bits(vals))
+    assert sz[0, 0] == 1.0 and sz[0, 1] == 0.0
+    assert packed[0, 0] == 0xF0 and packed[0, 1] == 0x21
+    codes = oracle.unpack_int4(packed)[0].tolist()
+    assert codes == [round(v) for v in vals]
+
+
+def test_int4_quantiser_endpoints_constant_row_and_bound():
+    g = torch.Generator().manual_seed(40)
+    x = torch.randn(400, 64, generator=g) * torch.rand(400, 1, generator=g) * 3
+    x[5] = 1.5
+    xb = _bf16_bits(x)
+    packed, sz = oracle.quantize_rows_int4(xb)
+    codes = oracle.unpack_int4(packed)
+    xf = _f64(xb)
+    assert sz[5, 0] == 0 and sz[5, 1] == 1.5 and np.all(codes[5] == 0)
+    rows = np.flatnonzero(sz[:, 0] > 0)
+    assert np.all(codes[rows, xf[rows].argmin(1)] == 0)
+    assert np.all(codes[rows, xf[rows].argmax(1)] == 15)
+    s = sz[:, 0:1].astype(np.float64)
+    err = np.abs(xf - (s * codes + sz[:, 1:2]))
+    assert np.all(err <= s * (0.5 + 15 * 2.0 ** -22) + 1e-30)
+
+
+def test_int4_dequantisation_uses_scale_zero_and_nibbles():
+    """s = 1, z = -8: s*code + z is exact in bf16, so an INT4 pool must give the
+    same fp64 attention as a bf16 pool of those values (a nibble or order
+    mix-up, or a swapped s and z, fails)."""
+    g = torch.Generator().manual_seed(41)
+    B, Hkv, T, D, P = 2, 2, 48, 64, 16
+    q = torch.randn(B, 4, D, generator=g).to(torch.bfloat16)
+    ck = torch.randint(0, 16, (B, Hkv, T, D), generator=g)
+    cv = torch.randint(0, 16, (B, Hkv, T, D), generator=g)
+    kp, vp, table = _contiguous_pool((ck - 8).float(), (cv - 8).float(), P)
+    npg = T // P
+    def to_pool(C):
+        C = C.reshape(B, Hkv, npg, P, D).permute(0, 2, 1, 3, 4).reshape(B * npg, Hkv, P, D)
+        C = C.numpy().astype(np.uint8)
+        return (C[..., 0::2] | (C[..., 1::2] << 4)).astype(np.uint8)
+    sz = np.zeros((B * npg, Hkv, P, 2), np.float32)
+    sz[..., 0] = 1.0
+    sz[..., 1] = -8.0
+    ctx = np.array([48, 29], np.int32)
+    ref, _ = oracle.paged_attention(_pool("bf16", kp, vp, P), _bf16_bits(q), table, ctx, 0.125)
+    out, _ = oracle.paged_attention(_pool("u4", to_pool(ck), to_pool(cv), P, sz, sz.copy()),
+                                    _bf16_bits(q), table, ctx, 0.125)
+    np.testing.assert_array_equal(out, ref)
+
+
 # ------------------------------------------------------- FP8 (E4M3) pins
 def test_e4m3_code_table_from_the_format_definition():
     """1 sign, 4 exponent bits (bias 7), 3 mantissa bits; no infinities;
