@@ -43,7 +43,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="llama70b",
-                    choices=["llama70b", "llama8b", "int8", "fp8", "prefix", "tiny"])
+                    choices=["llama70b", "llama8b", "int8", "fp8", "int4", "prefix", "tiny"])
     ap.add_argument("--cascade", action="store_true",
                     help="prefix workload: decode with pa_decode_shared_prefix")
     ap.add_argument("--window", type=int, default=0,
@@ -70,13 +70,13 @@ def attended_tokens(w, sinks: int = 0, window: int = 0) -> int:
 def decode_bytes(w, sinks: int = 0, window: int = 0) -> int:
     """Algorithmic bytes of one decode: every cached K/V element of every
     attended token once, plus q (Eq. 1 reads nothing else)."""
-    per_tok = w.Hkv * 2 * (w.D * 2 if w.kv == "bf16" else w.D + 8)
-    return attended_tokens(w, sinks, window) * per_tok + w.B * w.Hq * w.D * 2
+    row = {"bf16": w.D * 2, "u8": w.D + 8, "fp8": w.D + 8, "u4": w.D // 2 + 8}[w.kv]
+    return attended_tokens(w, sinks, window) * w.Hkv * 2 * row + w.B * w.Hq * w.D * 2
 
 
 def append_bytes(w) -> int:
     n = len(w.step_seq)
-    row = w.D * 2 if w.kv == "bf16" else w.D + 8
+    row = {"bf16": w.D * 2, "u8": w.D + 8, "fp8": w.D + 8, "u4": w.D // 2 + 8}[w.kv]
     return n * w.Hkv * 2 * (w.D * 2 + row)
 
 
@@ -386,8 +386,9 @@ def run_ours(args, rank, world, local_rank):
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16"
-        if w.kv == "bf16" else "u8 codes, fp32 scale/zero; fp32 accumulate",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": {"bf16": "bf16", "u8": "u8 codes, fp32 scale/zero; fp32 accumulate",
+                   "fp8": "e4m3 codes, fp32 scale; fp32 accumulate",
+                   "u4": "u4 codes, fp32 scale/zero; fp32 accumulate"}[w.kv],
         "data": "synthetic (seeded N(0,1) bf16 K/V/q; no weights needed)",
         "config": config_of(w, args, world, S),
         "pct_of_peak": round(100.0 * value / world / peak, 2),
@@ -439,7 +440,7 @@ def run_reference(args, rank, world):
     n = int(min(len(pairs_all), max(1, budget / per_pair)))
     sample = pairs_all[:n]
     tok = sum(int(w.context_lens[b]) for b, _ in sample)
-    per_tok = 2 * (w.D * 2 if w.kv == "bf16" else w.D + 8)
+    per_tok = 2 * {"bf16": w.D * 2, "u8": w.D + 8, "fp8": w.D + 8, "u4": w.D // 2 + 8}[w.kv]
     sample_bytes = tok * per_tok // w.G + n * w.D * 2     # K/V rows are shared by G heads
     for _ in range(args.warmup):
         oracle.paged_attention(hp, qb, w.block_tables, w.context_lens, w.scale, pairs=sample)

@@ -60,11 +60,21 @@ typedef enum {
 #define PA_DERR_BAD_CTX 2  /* context_len < 0 or > max_pages * page_size       */
 #define PA_DERR_BAD_SEQ 4  /* append: seq_idx outside [0, num_seqs)            */
 #define PA_DERR_BAD_POS 8  /* append: pos < 0 or pos / page_size >= max_pages  */
+#define PA_DERR_BIG_SCALE 16 /* append: a quantised row's scale is not below
+                                PA_MAX_KV_SCALE (the row is still written)     */
+
+/* Quantised pools: pa_decode* feed s * (softmax weight) to the tensor cores
+ * as f16, with weights kept <= 8, so every row scale must be below this bound
+ * (rows spanning less than 6.1e4 for INT4, 1.0e6 for INT8; FP8 rows with
+ * max |x| below 1.8e6). pa_kv_append flags rows that break it. */
+#define PA_MAX_KV_SCALE 4096
 
 typedef enum {
   PA_KV_BF16 = 0,          /* K/V stored as bf16                               */
   PA_KV_U8_PER_TOKEN = 1,  /* Eq. (3): uint8 codes + fp32 (scale, zero) per row */
-  PA_KV_FP8_PER_TOKEN = 2  /* E4M3 codes + fp32 (scale, 0) per row; x = s * e4m3 */
+  PA_KV_FP8_PER_TOKEN = 2, /* E4M3 codes + fp32 (scale, 0) per row; x = s * e4m3 */
+  PA_KV_U4_PER_TOKEN = 3   /* Eq. (3) with 16 levels: two 4-bit codes per byte
+                              (element 2i in the low nibble) + fp32 (scale, zero) */
 } pa_kv_dtype_t;
 
 /*
@@ -72,8 +82,9 @@ typedef enum {
  * Layout of one tensor (K or V): [num_pages][num_kv_heads][page_size][head_dim],
  * row-major, so the page_size x head_dim block of one (page, KV head) is
  * contiguous. bf16 pools hold 2-byte elements; INT8 and FP8 pools hold 1-byte
- * codes plus k_sz / v_sz = fp32 [num_pages][num_kv_heads][page_size][2]
- * holding (scale, zero) of each row (zero is 0 for FP8). Every pointer must be
+ * codes and INT4 pools half-byte codes (rows of head_dim / 2 bytes), all three
+ * plus k_sz / v_sz = fp32 [num_pages][num_kv_heads][page_size][2] holding
+ * (scale, zero) of each row (zero is 0 for FP8). Every pointer must be
  * 16-byte aligned.
  * Supported: page_size in {16, 32}; head_dim in {64, 128}.
  */
@@ -99,7 +110,8 @@ typedef struct {
  * For an FP8 pool (the pages name FP8 KV caches without fixing the encoding;
  * this library uses OCP E4M3 with a per-row absmax scale): s = max|x| / 448,
  * code = E4M3(x / s) rounded to nearest even and saturated at +-448, zero 0;
- * an all-zero row stores s = 0, codes 0.
+ * an all-zero row stores s = 0, codes 0. An INT4 pool uses Eq. (3) with
+ * s = (max - min) / 15 and codes in [0, 15], in the same fp32 order as INT8.
  * Input rows must be finite; -0 is stored as +0.)
  *
  *   k_new, v_new : (device) bf16 [num_tokens][num_kv_heads][head_dim]

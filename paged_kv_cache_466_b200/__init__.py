@@ -34,17 +34,20 @@ import torch
 
 from . import _lib
 from ._lib import (PA_DERR_BAD_CTX, PA_DERR_BAD_PAGE, PA_DERR_BAD_POS, PA_DERR_BAD_SEQ,
-                   PA_KV_BF16, PA_KV_FP8_PER_TOKEN, PA_KV_U8_PER_TOKEN, PagedAttnError,
-                   pa_kv_pool_t)
+                   PA_DERR_BIG_SCALE, PA_MAX_KV_SCALE,
+                   PA_KV_BF16, PA_KV_FP8_PER_TOKEN, PA_KV_U4_PER_TOKEN, PA_KV_U8_PER_TOKEN,
+                   PagedAttnError, pa_kv_pool_t)
 
 __all__ = ["KVPool", "pa_kv_append", "pa_decode", "pa_decode_noalloc", "pa_splitkv_reduce",
            "pa_decode_shared_prefix", "pa_decode_shared_prefix_workspace_bytes",
            "pa_decode_window", "pa_decode_window_workspace_bytes",
            "pa_validate_tables",
            "pa_decode_num_splits", "pa_decode_workspace_bytes", "PagedAttnError",
-           "PA_KV_BF16", "PA_KV_U8_PER_TOKEN", "PA_KV_FP8_PER_TOKEN", "PA_DERR_BAD_PAGE",
+           "PA_KV_BF16", "PA_KV_U8_PER_TOKEN", "PA_KV_FP8_PER_TOKEN", "PA_KV_U4_PER_TOKEN",
+           "PA_DERR_BAD_PAGE",
            "PA_DERR_BAD_CTX",
-           "PA_DERR_BAD_SEQ", "PA_DERR_BAD_POS", "load_library"]
+           "PA_DERR_BAD_SEQ", "PA_DERR_BAD_POS", "PA_DERR_BIG_SCALE", "PA_MAX_KV_SCALE",
+           "load_library"]
 
 
 def load_library() -> ctypes.CDLL:
@@ -72,20 +75,22 @@ def _need(t: torch.Tensor, name: str, dtype, device=None):
 
 class KVPool:
     """The physical page pool: K and V as [num_pages, Hkv, P, D] tensors:
-    ``dtype`` "bf16", "u8" (INT8 codes, Eq. 3) or "fp8" (E4M3 codes), the
-    last two with fp32 [num_pages, Hkv, P, 2] (scale, zero) per row."""
+    ``dtype`` "bf16", "u8" (INT8 codes, Eq. 3), "fp8" (E4M3 codes) or "u4"
+    (INT4 codes, two per byte: [num_pages, Hkv, P, D/2]); the quantised ones
+    with fp32 [num_pages, Hkv, P, 2] (scale, zero) per row."""
 
     def __init__(self, num_pages: int, num_kv_heads: int, page_size: int, head_dim: int,
                  dtype: str = "bf16", device="cuda", fill_byte: Optional[int] = None):
         self.num_pages, self.num_kv_heads = num_pages, num_kv_heads
         self.page_size, self.head_dim = page_size, head_dim
         self.kind = dtype
-        shape = (num_pages, num_kv_heads, page_size, head_dim)
-        tdt = {"bf16": torch.bfloat16, "u8": torch.uint8, "fp8": torch.uint8}[dtype]
+        shape = (num_pages, num_kv_heads, page_size, head_dim // 2 if dtype == "u4" else head_dim)
+        tdt = {"bf16": torch.bfloat16, "u8": torch.uint8, "fp8": torch.uint8,
+               "u4": torch.uint8}[dtype]
         self.k = torch.empty(shape, dtype=tdt, device=device)
         self.v = torch.empty(shape, dtype=tdt, device=device)
         self.k_sz = self.v_sz = None
-        if dtype in ("u8", "fp8"):
+        if dtype in ("u8", "fp8", "u4"):
             self.k_sz = torch.empty(shape[:3] + (2,), dtype=torch.float32, device=device)
             self.v_sz = torch.empty(shape[:3] + (2,), dtype=torch.float32, device=device)
         if fill_byte is not None:
@@ -93,7 +98,7 @@ class KVPool:
                 t.view(torch.uint8).fill_(fill_byte)
         self._c = pa_kv_pool_t(num_pages, page_size, num_kv_heads, head_dim,
                                {"bf16": PA_KV_BF16, "u8": PA_KV_U8_PER_TOKEN,
-                                "fp8": PA_KV_FP8_PER_TOKEN}[dtype],
+                                "fp8": PA_KV_FP8_PER_TOKEN, "u4": PA_KV_U4_PER_TOKEN}[dtype],
                                self.k.data_ptr(), self.v.data_ptr(),
                                None if self.k_sz is None else self.k_sz.data_ptr(),
                                None if self.v_sz is None else self.v_sz.data_ptr())

@@ -32,7 +32,7 @@ bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_sm_count[kMaxDevices];
-std::atomic<int> g_ctas[kMaxDevices][2][2][3];  // [dev][D==128][P==32][dtype]
+std::atomic<int> g_ctas[kMaxDevices][2][2][4];  // [dev][D==128][P==32][dtype]
 
 int current_device() {
   int dev = 0;
@@ -49,8 +49,7 @@ pa_status_t check_pool(const pa_kv_pool_t *pool) {
     return fail(PA_ERR_UNSUPPORTED, "pool: page_size=%d (supported: 16, 32)", pool->page_size);
   if (pool->head_dim != 64 && pool->head_dim != 128)
     return fail(PA_ERR_UNSUPPORTED, "pool: head_dim=%d (supported: 64, 128)", pool->head_dim);
-  if (pool->dtype != PA_KV_BF16 && pool->dtype != PA_KV_U8_PER_TOKEN &&
-      pool->dtype != PA_KV_FP8_PER_TOKEN)
+  if (pool->dtype < PA_KV_BF16 || pool->dtype > PA_KV_U4_PER_TOKEN)
     return fail(PA_ERR_UNSUPPORTED, "pool: dtype=%d", pool->dtype);
   if (pool->k_pool == nullptr || pool->v_pool == nullptr)
     return fail(PA_ERR_INVALID_ARG, "pool: k_pool/v_pool is NULL");
@@ -58,7 +57,7 @@ pa_status_t check_pool(const pa_kv_pool_t *pool) {
     return fail(PA_ERR_INVALID_ARG, "pool: k_pool/v_pool must be 16-byte aligned");
   if (pool->dtype != PA_KV_BF16) {
     if (pool->k_sz == nullptr || pool->v_sz == nullptr)
-      return fail(PA_ERR_INVALID_ARG, "pool: an INT8/FP8 pool needs k_sz and v_sz");
+      return fail(PA_ERR_INVALID_ARG, "pool: an INT8/FP8/INT4 pool needs k_sz and v_sz");
     if (!aligned(pool->k_sz, 16) || !aligned(pool->v_sz, 16))
       return fail(PA_ERR_INVALID_ARG, "pool: k_sz/v_sz must be 16-byte aligned");
   }
@@ -144,8 +143,7 @@ int32_t pa_decode_num_splits(const pa_kv_pool_t *pool, int32_t num_seqs, int32_t
   if (pool == nullptr || num_seqs < 0 || max_pages <= 0 || requested < 0) return -1;
   if ((pool->head_dim != 64 && pool->head_dim != 128) ||
       (pool->page_size != 16 && pool->page_size != 32) ||
-      (pool->dtype != PA_KV_BF16 && pool->dtype != PA_KV_U8_PER_TOKEN &&
-       pool->dtype != PA_KV_FP8_PER_TOKEN) ||
+      pool->dtype < PA_KV_BF16 || pool->dtype > PA_KV_U4_PER_TOKEN ||
       pool->num_kv_heads <= 0)
     return -1;
   const int P = pool->page_size;

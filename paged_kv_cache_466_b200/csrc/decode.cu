@@ -73,7 +73,11 @@ namespace {
 constexpr float kLn2 = 0.693147180559945309f;
 // Lazy rescaling: the running max is only raised when a block's max exceeds it
 // by more than this many powers of two, so weights stay <= 2^kRescaleLog2.
-constexpr float kRescaleLog2 = 8.0f;
+// Quantised pools scale the weights by the row scale s < 2^12 into f16
+// operands, so they keep weights <= 2^3 (p * s < 2^15 < f16 max).
+template <int KVT>
+constexpr float kRescaleLog2 = KVT == PA_KV_BF16 ? 8.0f : 3.0f;
+static_assert(PA_MAX_KV_SCALE == 4096, "p * s must stay below the f16 maximum");
 
 template <int D, int KVT>
 struct Tile {
@@ -81,8 +85,9 @@ struct Tile {
   // INT8 and FP8 pools share the layout: 1-byte codes + (scale, zero) per row
   static constexpr bool kU8 = KVT != PA_KV_BF16;
   static constexpr bool kFp8 = KVT == PA_KV_FP8_PER_TOKEN;
+  static constexpr bool kU4 = KVT == PA_KV_U4_PER_TOKEN;  // two codes per byte
   static constexpr int kElem = kU8 ? 1 : 2;
-  static constexpr int kRowBytes = D * kElem;
+  static constexpr int kRowBytes = kU4 ? D / 2 : D * kElem;
   // one 16-token block of K (or V) is 16 contiguous rows of the page
   static constexpr int kBlockBytes = 16 * kRowBytes;
   static constexpr int kCopies = kBlockBytes / 512;  // 16-byte copies per lane per tensor
@@ -92,13 +97,21 @@ struct Tile {
   static constexpr int kVSzOff = 2 * kBlockBytes + kSzBytes;
   static constexpr int kStageBytes = 2 * kBlockBytes + 2 * kSzBytes;
   // 16-byte K chunks a lane reads per 8-token half-block (fragment layout)
-  static constexpr int kKChunks = kU8 ? D / 64 : D / 32;
+  static constexpr int kKChunks = kU4 ? 1 : (kU8 ? D / 64 : D / 32);
   // 16-byte V chunks a lane reads per token
   static constexpr int kVChunks = kU8 ? 1 : D / 64;
   static constexpr int kMTiles = D / 16;  // m16 tiles of O^T
   // rows of at least 128 bytes are stored with their 16-byte chunks permuted
   // (chunk ^ swz(row)), which makes both fragment read patterns conflict free
   static constexpr bool kSwizzle = kRowBytes >= 128;
+  // INT4 rows (32 or 64 bytes) are permuted instead: rows 2t (and 2t + 1),
+  // t = 0..3, which the V fragment reads together, land in distinct bank
+  // quarters (D = 64) or halves (D = 128) of a 128-byte line.
+  static __device__ __forceinline__ int staged_row(int row) {
+    if constexpr (!kU4) return row;
+    else if constexpr (D == 128) return row ^ ((row >> 1) & 1);
+    else return row ^ ((row >> 2) & 1);
+  }
 };
 
 // Shared-memory byte offset of 16-byte chunk `chunk` of row `row` in a staged
@@ -108,7 +121,7 @@ struct Tile {
 template <class T>
 __device__ __forceinline__ int staged_off(int row, int chunk) {
   const int swz = T::kSwizzle ? ((2 * ((row >> 1) & 3)) ^ (4 * (row & 1))) : 0;
-  return row * T::kRowBytes + ((chunk ^ swz) << 4);
+  return T::staged_row(row) * T::kRowBytes + ((chunk ^ swz) << 4);
 }
 
 template <int D, int KVT, int W, int NSTAGE>
@@ -306,6 +319,25 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
       qa[2 * i + 1][0] = v.z;
       qa[2 * i + 1][1] = v.w;
     }
+  } else if constexpr (T::kU4) {
+    // lane t contracts d in [t*D/4, (t+1)*D/4); per group of 8 elements the
+    // k-steps take (e0,e2 | e4,e6) and (e1,e3 | e5,e7), as the 4-bit unpack does
+#pragma unroll
+    for (int w = 0; w < D / 32; ++w) {
+      const uint4 v = head_ok ? ldg_nc128(qp + t * (D / 4) + 8 * w) : make_uint4(0, 0, 0, 0);
+      const uint32_t f02 = pack_f16(bf16_lo(v.x), bf16_lo(v.y));
+      const uint32_t f46 = pack_f16(bf16_lo(v.z), bf16_lo(v.w));
+      const uint32_t f13 = pack_f16(bf16_hi(v.x), bf16_hi(v.y));
+      const uint32_t f57 = pack_f16(bf16_hi(v.z), bf16_hi(v.w));
+      qsum += (f16_lo(f02) + f16_hi(f02)) + (f16_lo(f46) + f16_hi(f46)) +
+              (f16_lo(f13) + f16_hi(f13)) + (f16_lo(f57) + f16_hi(f57));
+      qa[2 * w][0] = f02;
+      qa[2 * w][1] = f46;
+      qa[2 * w + 1][0] = f13;
+      qa[2 * w + 1][1] = f57;
+    }
+    qsum += __shfl_xor_sync(0xffffffffu, qsum, 1);
+    qsum += __shfl_xor_sync(0xffffffffu, qsum, 2);
   } else {
 #pragma unroll
     for (int i = 0; i < T::kKChunks; ++i) {
@@ -384,15 +416,21 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-    for (int i = 0; i < T::kKChunks; ++i) koff[nt][i] = staged_off<T>(nt * 8 + g, 4 * i + t);
+    for (int i = 0; i < T::kKChunks; ++i)
+      koff[nt][i] = T::kU4 ? T::staged_row(nt * 8 + g) * T::kRowBytes + t * (D / 8)
+                           : staged_off<T>(nt * 8 + g, 4 * i + t);
   int voff[4][T::kVChunks];
 #pragma unroll
   for (int tau = 0; tau < 4; ++tau)
 #pragma unroll
     for (int c = 0; c < T::kVChunks; ++c) {
       const int row = (tau & 1) + 2 * t + (tau >> 1) * 8;
-      const int chunk = T::kU8 ? (D == 128 ? g : (g >> 1)) : 8 * c + g;
-      voff[tau][c] = T::kVOff + staged_off<T>(row, chunk);
+      if constexpr (T::kU4) {
+        voff[tau][c] = T::kVOff + T::staged_row(row) * T::kRowBytes + g * (D / 16);
+      } else {
+        const int chunk = T::kU8 ? (D == 128 ? g : (g >> 1)) : 8 * c + g;
+        voff[tau][c] = T::kVOff + staged_off<T>(row, chunk);
+      }
     }
 
   float o[T::kMTiles][4];
@@ -428,20 +466,41 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
       s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-#pragma unroll
-      for (int i = 0; i < T::kKChunks; ++i) {
-        const uint4 kv = lds128(src + koff[nt][i]);
-        if constexpr (!T::kU8) {
-          mma_bf16_16816(s[nt], qa[2 * i][0], 0u, qa[2 * i][1], 0u, kv.x, kv.y);
-          mma_bf16_16816(s[nt], qa[2 * i + 1][0], 0u, qa[2 * i + 1][1], 0u, kv.z, kv.w);
+      if constexpr (T::kU4) {
+        uint32_t wk[D / 32];
+        if constexpr (D == 128) {
+          const uint4 v = lds128(src + koff[nt][0]);
+          wk[0] = v.x; wk[1] = v.y; wk[2] = v.z; wk[3] = v.w;
         } else {
-          const uint32_t w4[4] = {kv.x, kv.y, kv.z, kv.w};
+          const uint2 v = lds64(src + koff[nt][0]);
+          wk[0] = v.x; wk[1] = v.y;
+        }
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const uint32_t b0 = T::kFp8 ? e4m3x2_to_f16x2(w4[w]) : u8x2_to_f16x2(w4[w], 0x4140);
-            const uint32_t b1 =
-                T::kFp8 ? e4m3x2_to_f16x2(w4[w] >> 16) : u8x2_to_f16x2(w4[w], 0x4342);
-            mma_f16_16816(s[nt], qa[4 * i + w][0], 0u, qa[4 * i + w][1], 0u, b0, b1);
+        for (int w = 0; w < D / 32; ++w) {
+          // even elements (low nibbles), then odd ones, each as c * 2^-9
+          uint32_t b02, b46, b13, b57;
+          nib4_to_f16x2x2(wk[w] & 0x0F0F0F0Fu, b02, b46);
+          nib4_to_f16x2x2((wk[w] >> 4) & 0x0F0F0F0Fu, b13, b57);
+          mma_f16_16816(s[nt], qa[2 * w][0], 0u, qa[2 * w][1], 0u, b02, b46);
+          mma_f16_16816(s[nt], qa[2 * w + 1][0], 0u, qa[2 * w + 1][1], 0u, b13, b57);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < T::kKChunks; ++i) {
+          const uint4 kv = lds128(src + koff[nt][i]);
+          if constexpr (!T::kU8) {
+            mma_bf16_16816(s[nt], qa[2 * i][0], 0u, qa[2 * i][1], 0u, kv.x, kv.y);
+            mma_bf16_16816(s[nt], qa[2 * i + 1][0], 0u, qa[2 * i + 1][1], 0u, kv.z, kv.w);
+          } else {
+            const uint32_t w4[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const uint32_t b0 =
+                  T::kFp8 ? e4m3x2_to_f16x2(w4[w]) : u8x2_to_f16x2(w4[w], 0x4140);
+              const uint32_t b1 =
+                  T::kFp8 ? e4m3x2_to_f16x2(w4[w] >> 16) : u8x2_to_f16x2(w4[w], 0x4342);
+              mma_f16_16816(s[nt], qa[4 * i + w][0], 0u, qa[4 * i + w][1], 0u, b0, b1);
+            }
           }
         }
       }
@@ -463,8 +522,11 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
       vs[1] = __uint_as_float(v01.z); vz[1] = __uint_as_float(v01.w);
       vs[2] = __uint_as_float(v89.x); vz[2] = __uint_as_float(v89.y);
       vs[3] = __uint_as_float(v89.z); vz[3] = __uint_as_float(v89.w);
+      // INT4 codes reach the MMA as c * 2^-9: the exact power of two goes
+      // back into the K scale here and into O after the loop
+      constexpr float kCodeScale = T::kU4 ? 512.f : 1.f;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) x[e] = fmaf(ks[e], x[e], kz[e] * qsum);
+      for (int e = 0; e < 4; ++e) x[e] = fmaf(ks[e] * kCodeScale, x[e], kz[e] * qsum);
     }
     if (pvalid && btok >= tok_lo && btok + 16 <= tok1) {  // warp-uniform: no mask needed
 #pragma unroll
@@ -483,7 +545,7 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
     float mb = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
     mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
     mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
-    const bool need = mb > m_run + kRescaleLog2 || (m_run == -INFINITY && mb > -INFINITY);
+    const bool need = mb > m_run + kRescaleLog2<KVT> || (m_run == -INFINITY && mb > -INFINITY);
     if (__any_sync(0xffffffffu, need)) {
       const float m_new = fmaxf(m_run, mb);
       const float alpha = m_new == -INFINITY ? 1.f : fast_exp2(m_run - m_new);
@@ -540,6 +602,40 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
       }
       split_f16(pv[0], pv[1], bh0, bl0);
       split_f16(pv[2], pv[3], bh1, bl1);
+      if constexpr (T::kU4) {
+        // byte j of this lane's slice holds d = base + 2j (low nibble) and + 1
+        uint32_t xv[4][D / 64];
+#pragma unroll
+        for (int tau = 0; tau < 4; ++tau) {
+          if constexpr (D == 128) {
+            const uint2 v = lds64(src + voff[tau][0]);
+            xv[tau][0] = v.x;
+            xv[tau][1] = v.y;
+          } else {
+            xv[tau][0] = lds32(src + voff[tau][0]);
+          }
+        }
+        // m-tiles j, j+1 use bytes j & 3, (j & 3) + 1 of word j / 4: gather them
+        // for token pairs (2t, 2t+1) and (8+2t, 9+2t), then low nibbles give
+        // rows d (a0, a2), high nibbles rows d + 1 (a1, a3)
+#pragma unroll
+        for (int j = 0; j < T::kMTiles; j += 2) {
+          const uint32_t sel = (j & 2) ? 0x7362 : 0x5140;
+          const uint32_t ya = __byte_perm(xv[0][j / 4], xv[1][j / 4], sel);
+          const uint32_t yb = __byte_perm(xv[2][j / 4], xv[3][j / 4], sel);
+          uint32_t a0[2], a1[2], a2[2], a3[2];
+          nib4_to_f16x2x2(ya & 0x0F0F0F0Fu, a0[0], a0[1]);
+          nib4_to_f16x2x2((ya >> 4) & 0x0F0F0F0Fu, a1[0], a1[1]);
+          nib4_to_f16x2x2(yb & 0x0F0F0F0Fu, a2[0], a2[1]);
+          nib4_to_f16x2x2((yb >> 4) & 0x0F0F0F0Fu, a3[0], a3[1]);
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            mma_f16_16816(o[j + u], a0[u], a1[u], a2[u], a3[u], bh0, bh1);
+            mma_f16_16816(o[j + u], a0[u], a1[u], a2[u], a3[u], bl0, bl1);
+          }
+        }
+        continue;
+      }
       const uint4 v0 = lds128(src + voff[0][0]);
       const uint4 v1 = lds128(src + voff[1][0]);
       const uint4 v2 = lds128(src + voff[2][0]);
@@ -578,12 +674,13 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
     zacc += __shfl_xor_sync(0xffffffffu, zacc, 2);
     const float z0 = __shfl_sync(0xffffffffu, zacc, 8 * t);
     const float z1 = __shfl_sync(0xffffffffu, zacc, 8 * t + 4);
+    constexpr float kCodeScale = T::kU4 ? 512.f : 1.f;  // INT4 codes were c * 2^-9
 #pragma unroll
     for (int j = 0; j < T::kMTiles; ++j) {
-      o[j][0] += z0;
-      o[j][1] += z1;
-      o[j][2] += z0;
-      o[j][3] += z1;
+      o[j][0] = fmaf(o[j][0], kCodeScale, z0);
+      o[j][1] = fmaf(o[j][1], kCodeScale, z1);
+      o[j][2] = fmaf(o[j][2], kCodeScale, z0);
+      o[j][3] = fmaf(o[j][3], kCodeScale, z1);
     }
   }
 
@@ -722,6 +819,7 @@ cudaError_t launch_decode(int D, int P, int kv_dtype, const DecodeArgs &a, cudaS
   PA_L(128, 16, 0); PA_L(128, 32, 0); PA_L(64, 16, 0); PA_L(64, 32, 0);
   PA_L(128, 16, 1); PA_L(128, 32, 1); PA_L(64, 16, 1); PA_L(64, 32, 1);
   PA_L(128, 16, 2); PA_L(128, 32, 2); PA_L(64, 16, 2); PA_L(64, 32, 2);
+  PA_L(128, 16, 3); PA_L(128, 32, 3); PA_L(64, 16, 3); PA_L(64, 32, 3);
 #undef PA_L
   return cudaErrorInvalidValue;
 }
@@ -731,6 +829,7 @@ int decode_ctas_per_sm(int D, int P, int kv_dtype) {
   PA_O(128, 16, 0); PA_O(128, 32, 0); PA_O(64, 16, 0); PA_O(64, 32, 0);
   PA_O(128, 16, 1); PA_O(128, 32, 1); PA_O(64, 16, 1); PA_O(64, 32, 1);
   PA_O(128, 16, 2); PA_O(128, 32, 2); PA_O(64, 16, 2); PA_O(64, 32, 2);
+  PA_O(128, 16, 3); PA_O(128, 32, 3); PA_O(64, 16, 3); PA_O(64, 32, 3);
 #undef PA_O
   return 1;
 }

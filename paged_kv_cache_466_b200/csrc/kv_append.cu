@@ -79,7 +79,7 @@ __global__ void append_bf16_kernel(const AppendArgs a) {
 }
 
 template <int D>
-__device__ __forceinline__ void quantise_row(const unsigned char *src_row, unsigned char *dst_codes,
+__device__ __forceinline__ float quantise_row(const unsigned char *src_row, unsigned char *dst_codes,
                                              float *dst_sz, int lane) {
   constexpr int E = D / 32;  // elements per lane
   const __nv_bfloat16 *x16 = reinterpret_cast<const __nv_bfloat16 *>(src_row) + lane * E;
@@ -116,13 +116,14 @@ __device__ __forceinline__ void quantise_row(const unsigned char *src_row, unsig
     *reinterpret_cast<uint16_t *>(dst_codes + lane * 2) = static_cast<uint16_t>(packed);
   }
   if (lane == 0) *reinterpret_cast<float2 *>(dst_sz) = make_float2(s, z);
+  return s;
 }
 
 // FP8 (E4M3) per-token quantiser: s = max|x| / 448 (IEEE fp32), code =
 // E4M3(x / s) rounded to nearest even and saturated; an all-zero row stores
 // s = 0 and codes 0. The zero point is stored as 0.
 template <int D>
-__device__ __forceinline__ void quantise_row_fp8(const unsigned char *src_row,
+__device__ __forceinline__ float quantise_row_fp8(const unsigned char *src_row,
                                                  unsigned char *dst_codes, float *dst_sz,
                                                  int lane) {
   constexpr int E = D / 32;  // elements per lane (even)
@@ -148,10 +149,55 @@ __device__ __forceinline__ void quantise_row_fp8(const unsigned char *src_row,
     *reinterpret_cast<uint16_t *>(dst_codes + lane * 2) = static_cast<uint16_t>(packed);
   }
   if (lane == 0) *reinterpret_cast<float2 *>(dst_sz) = make_float2(s, 0.f);
+  return s;
 }
 
-// INT8 / FP8: one warp per (token, head) row; K then V.
-template <int D, bool kFp8>
+// INT4: Eq. 3 with 16 levels, the INT8 arithmetic with 15 in place of 255;
+// element 2i goes to the low nibble of byte i.
+template <int D>
+__device__ __forceinline__ float quantise_row_u4(const unsigned char *src_row,
+                                                unsigned char *dst_codes, float *dst_sz,
+                                                int lane) {
+  constexpr int E = D / 32;  // elements per lane (even)
+  const __nv_bfloat16 *x16 = reinterpret_cast<const __nv_bfloat16 *>(src_row) + lane * E;
+  float x[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) x[e] = __fadd_rn(__bfloat162float(x16[e]), 0.0f);
+  float mn = x[0], mx = x[0];
+#pragma unroll
+  for (int e = 1; e < E; ++e) {
+    mn = fminf(mn, x[e]);
+    mx = fmaxf(mx, x[e]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  const float s = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+  const float z = mn;
+  uint32_t packed = 0;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    uint32_t c = 0;
+    if (s != 0.0f) {
+      float r = rintf(__fdiv_rn(__fsub_rn(x[e], z), s));
+      r = fminf(fmaxf(r, 0.0f), 15.0f);
+      c = static_cast<uint32_t>(r);
+    }
+    packed |= c << (4 * e);
+  }
+  if constexpr (E == 4) {
+    *reinterpret_cast<uint16_t *>(dst_codes + lane * 2) = static_cast<uint16_t>(packed);
+  } else {
+    dst_codes[lane] = static_cast<unsigned char>(packed);
+  }
+  if (lane == 0) *reinterpret_cast<float2 *>(dst_sz) = make_float2(s, z);
+  return s;
+}
+
+// INT8 / FP8 / INT4: one warp per (token, head) row; K then V.
+template <int D, int kFmt>  // kFmt: the pool's pa_kv_dtype_t
 __global__ void append_u8_kernel(const AppendArgs a) {
   pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
@@ -166,15 +212,26 @@ __global__ void append_u8_kernel(const AppendArgs a) {
     row = __shfl_sync(0xffffffffu, row, 0);
     if (row < 0) continue;
     const size_t src = (size_t)r * D * 2;
-    if constexpr (kFp8) {
-      quantise_row_fp8<D>(a.k_new + src, a.k_pool + (size_t)row * D, a.k_sz + (size_t)row * 2,
-                          lane);
-      quantise_row_fp8<D>(a.v_new + src, a.v_pool + (size_t)row * D, a.v_sz + (size_t)row * 2,
-                          lane);
+    float sk, sv;
+    if constexpr (kFmt == PA_KV_U4_PER_TOKEN) {
+      sk = quantise_row_u4<D>(a.k_new + src, a.k_pool + (size_t)row * (D / 2),
+                              a.k_sz + (size_t)row * 2, lane);
+      sv = quantise_row_u4<D>(a.v_new + src, a.v_pool + (size_t)row * (D / 2),
+                              a.v_sz + (size_t)row * 2, lane);
+    } else if constexpr (kFmt == PA_KV_FP8_PER_TOKEN) {
+      sk = quantise_row_fp8<D>(a.k_new + src, a.k_pool + (size_t)row * D,
+                               a.k_sz + (size_t)row * 2, lane);
+      sv = quantise_row_fp8<D>(a.v_new + src, a.v_pool + (size_t)row * D,
+                               a.v_sz + (size_t)row * 2, lane);
     } else {
-      quantise_row<D>(a.k_new + src, a.k_pool + (size_t)row * D, a.k_sz + (size_t)row * 2, lane);
-      quantise_row<D>(a.v_new + src, a.v_pool + (size_t)row * D, a.v_sz + (size_t)row * 2, lane);
+      sk = quantise_row<D>(a.k_new + src, a.k_pool + (size_t)row * D, a.k_sz + (size_t)row * 2,
+                           lane);
+      sv = quantise_row<D>(a.v_new + src, a.v_pool + (size_t)row * D, a.v_sz + (size_t)row * 2,
+                           lane);
     }
+    // the row is stored either way; decode needs scales below PA_MAX_KV_SCALE
+    if (lane == 0 && !(fmaxf(sk, sv) < (float)PA_MAX_KV_SCALE))
+      flag_error(a.d_err, PA_DERR_BIG_SCALE);
   }
 }
 
@@ -212,15 +269,19 @@ cudaError_t launch_kv_append(const pa_kv_pool_t &pool, const void *k_new, const 
     const long long rows = (long long)n * a.hkv;
     long long blocks = (rows + 7) / 8;
     blocks = blocks < 1 ? 1 : (blocks > 16LL * sms ? 16LL * sms : blocks);
-    const bool fp8 = pool.dtype == PA_KV_FP8_PER_TOKEN;
-    if (a.D == 128 && !fp8)
-      append_u8_kernel<128, false><<<(unsigned)blocks, 256, 0, stream>>>(a);
-    else if (a.D == 64 && !fp8)
-      append_u8_kernel<64, false><<<(unsigned)blocks, 256, 0, stream>>>(a);
-    else if (a.D == 128)
-      append_u8_kernel<128, true><<<(unsigned)blocks, 256, 0, stream>>>(a);
-    else
-      append_u8_kernel<64, true><<<(unsigned)blocks, 256, 0, stream>>>(a);
+#define PA_APPEND(D_, F_)                                                  \
+  if (a.D == D_ && pool.dtype == F_) {                                     \
+    append_u8_kernel<D_, F_><<<(unsigned)blocks, 256, 0, stream>>>(a);     \
+    return cudaGetLastError();                                             \
+  }
+    PA_APPEND(128, PA_KV_U8_PER_TOKEN)
+    PA_APPEND(64, PA_KV_U8_PER_TOKEN)
+    PA_APPEND(128, PA_KV_FP8_PER_TOKEN)
+    PA_APPEND(64, PA_KV_FP8_PER_TOKEN)
+    PA_APPEND(128, PA_KV_U4_PER_TOKEN)
+    PA_APPEND(64, PA_KV_U4_PER_TOKEN)
+#undef PA_APPEND
+    return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
 }

@@ -41,7 +41,7 @@ class Workload:
     Hkv: int
     D: int
     P: int
-    kv: str                         # "bf16", "u8" (INT8) or "fp8" (E4M3)
+    kv: str                         # "bf16", "u8" (INT8), "fp8" (E4M3) or "u4" (INT4)
     num_pages: int
     max_pages: int
     scale: float
@@ -184,7 +184,8 @@ def tiny(seed: int = 0) -> Workload:
 def llama8b(B: int = 64, ctx_range=(128, 4096), seed: int = 0, kv: str = "bf16",
             outlier_frac: float = 0.0) -> Workload:
     """Llama-3-8B-shaped layer: Hq=32, Hkv=8, D=128, P=16, pool = 1.1 x need."""
-    return paged({"bf16": "llama8b", "u8": "int8", "fp8": "fp8"}[kv], B=B, Hq=32, Hkv=8, D=128, P=16,
+    return paged({"bf16": "llama8b", "u8": "int8", "fp8": "fp8", "u4": "int4"}[kv], B=B, Hq=32,
+                 Hkv=8, D=128, P=16,
                  ctx_range=ctx_range, pool_slack=0.10, max_pages=-(-ctx_range[1] // 16),
                  kv=kv, outlier_frac=outlier_frac, seed=seed)
 
@@ -201,6 +202,11 @@ def fp8(B: int = 64, ctx_range=(128, 4096), seed: int = 0) -> Workload:
     w = llama8b(B=B, ctx_range=ctx_range, seed=seed, kv="fp8", outlier_frac=0.01)
     w.name = "fp8"
     return w
+
+
+def int4(B: int = 64, ctx_range=(128, 4096), seed: int = 0) -> Workload:
+    """``llama8b`` draws plus 1 % outliers ~ N(0, 8^2), cached as per-token INT4."""
+    return llama8b(B=B, ctx_range=ctx_range, seed=seed, kv="u4", outlier_frac=0.01)
 
 
 def int8(B: int = 64, ctx_range=(128, 4096), seed: int = 0) -> Workload:
@@ -277,10 +283,13 @@ def by_name(name: str, **kw):
         return int8(**kw)
     if name == "fp8":
         return fp8(**kw)
+    if name == "int4":
+        return int4(**kw)
     if name == "prefix":
         return prefix(**kw)[0]
     raise KeyError(name)
 
 
-__all__ = ["Workload", "bits", "paged", "tiny", "llama8b", "llama70b", "int8", "fp8", "prefix",
+__all__ = ["Workload", "bits", "paged", "tiny", "llama8b", "llama70b", "int8", "fp8", "int4",
+           "prefix",
            "by_name"]

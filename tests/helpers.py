@@ -56,7 +56,7 @@ def oracle_decode(w: Workload, hp: oracle.HostPool, pairs=None):
 def pool_bytes_equal(pool: KVPool, hp: oracle.HostPool):
     """Byte-for-byte comparison of the device pool with the oracle's pool."""
     pairs = [(pool.k, hp.k), (pool.v, hp.v)]
-    if hp.kind == "u8":
+    if hp.kind in ("u8", "fp8", "u4"):
         pairs += [(pool.k_sz, hp.k_sz), (pool.v_sz, hp.v_sz)]
     for dt, ht in pairs:
         got = dt.view(torch.uint8).cpu().numpy().reshape(-1)

@@ -4,8 +4,8 @@ import numpy as np
 import pytest
 import torch
 
-from paged_kv_cache_466_b200 import (PA_DERR_BAD_PAGE, PA_DERR_BAD_POS, PA_DERR_BAD_SEQ, KVPool,
-                                     pa_kv_append)
+from paged_kv_cache_466_b200 import (PA_DERR_BAD_PAGE, PA_DERR_BAD_POS, PA_DERR_BAD_SEQ,
+                                     PA_DERR_BIG_SCALE, PA_MAX_KV_SCALE, KVPool, pa_kv_append)
 from paged_kv_cache_466_b200 import workloads as W
 from tests.helpers import DEV, device_append, device_inputs, oracle_pool, pool_bytes_equal
 
@@ -23,8 +23,11 @@ pytestmark = pytest.mark.gpu
     lambda: W.fp8(B=6, ctx_range=(1, 700)),
     lambda: W.paged("fp8d64", B=5, Hq=4, Hkv=2, D=64, P=32, ctx_range=(1, 300), kv="fp8",
                     outlier_frac=0.05),
+    lambda: W.int4(B=6, ctx_range=(1, 700)),
+    lambda: W.paged("u4d64", B=5, Hq=4, Hkv=2, D=64, P=32, ctx_range=(1, 300), kv="u4",
+                    outlier_frac=0.05),
 ], ids=["tiny", "llama8b-small", "p32-d64", "int8-small", "int8-d64", "int8-p32", "fp8-small",
-        "fp8-d64-p32"])
+        "fp8-d64-p32", "int4-small", "int4-d64-p32"])
 def test_append_matches_oracle_scatter_bit_exact(make):
     w = make()
     pool, bt, _, _ = device_inputs(w, fill_byte=0xA5)
@@ -56,9 +59,10 @@ def test_append_fp8_full_pool_bit_exact():
     assert ok, msg
 
 
-@pytest.mark.parametrize("kind", ["u8", "fp8"])
-def test_append_quantiser_edge_rows_both_formats(kind):
-    D, Hkv = 128, 2
+@pytest.mark.parametrize("kind", ["u8", "fp8", "u4"])
+@pytest.mark.parametrize("D", [128, 64])
+def test_append_quantiser_edge_rows_all_formats(kind, D):
+    Hkv = 2
     rows = []
     rows.append(np.full(D, 3.25, np.float32))
     r = np.zeros(D, np.float32); r[::2] = -0.0; r[5] = 2.0; rows.append(r)
@@ -76,6 +80,17 @@ def test_append_quantiser_edge_rows_both_formats(kind):
     device_append(pool, w, bt)
     torch.cuda.synchronize()
     ok, msg = pool_bytes_equal(pool, oracle_pool(w))
+    assert ok, msg
+
+
+def test_append_int4_full_pool_bit_exact():
+    """All pages of the INT4 workload: every packed code pair and fp32
+    scale/zero equals the oracle's (Eq. 3 with 16 levels)."""
+    w = W.int4()
+    pool, bt, _, _ = device_inputs(w, fill_byte=0x00)
+    device_append(pool, w, bt)
+    torch.cuda.synchronize()
+    ok, msg = pool_bytes_equal(pool, oracle_pool(w, fill_byte=0x00))
     assert ok, msg
 
 
@@ -134,3 +149,26 @@ def test_append_empty_is_noop():
     pa_kv_append(pool, e, e, i, i, bt)
     torch.cuda.synchronize()
     assert torch.all(pool.k.view(torch.uint8) == 0x22)
+
+
+@pytest.mark.parametrize("kind,span,flagged", [
+    ("u4", 8e4, True), ("u4", 6e4, False), ("u8", 8e4, False), ("fp8", 8e4, False),
+    ("u8", 1.2e6, True)])
+def test_append_flags_scales_the_decode_cannot_take(kind, span, flagged):
+    """A row whose scale is not below PA_MAX_KV_SCALE is still stored (bit-exact
+    with the oracle) and flagged with PA_DERR_BIG_SCALE; smaller ones are not."""
+    D, Hkv = 128, 2
+    x = torch.linspace(-span / 2, span / 2, D).to(torch.bfloat16)
+    k = torch.zeros(3, Hkv, D, dtype=torch.bfloat16)
+    k[1, 1] = x
+    w = W.paged("bigscale", B=1, Hq=2, Hkv=Hkv, D=D, P=16, context_lens=[3], kv=kind)
+    w.prefill_k, w.prefill_v = k[:2].contiguous(), k[:2].flip(1).contiguous()
+    w.step_k, w.step_v = k[2:].contiguous(), k[2:].contiguous()
+    pool, bt, _, _ = device_inputs(w)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    device_append(pool, w, bt, d_err=err)
+    torch.cuda.synchronize()
+    assert bool(int(err.item()) & PA_DERR_BIG_SCALE) == flagged
+    ok, msg = pool_bytes_equal(pool, oracle_pool(w))
+    assert ok, msg
+    assert PA_MAX_KV_SCALE == 4096

@@ -56,6 +56,11 @@ SMALL = {
     "fp8-small": lambda: W.fp8(B=6, ctx_range=(1, 700)),
     "fp8-d64-p32-g8": lambda: W.paged("fp8b", B=3, Hq=16, Hkv=2, D=64, P=32,
                                       ctx_range=(1, 400), kv="fp8", outlier_frac=0.02),
+    "int4-small": lambda: W.int4(B=6, ctx_range=(1, 700)),
+    "int4-d64-p32-g8": lambda: W.paged("u4b", B=3, Hq=16, Hkv=2, D=64, P=32,
+                                       ctx_range=(1, 400), kv="u4", outlier_frac=0.02),
+    "int4-g1": lambda: W.paged("u4g1", B=3, Hq=4, Hkv=4, D=128, P=16, ctx_range=(1, 300),
+                               kv="u4"),
 }
 
 
@@ -75,6 +80,26 @@ def test_one_token_context_is_exact():
         v0 = w.step_v.float().numpy()                   # [B, Hkv, D]: the only token
         want = np.repeat(v0, w.G, axis=1).reshape(-1, w.D)
         np.testing.assert_array_equal(got, want)
+
+
+@pytest.mark.parametrize("kind", ["u4", "u8", "fp8"])
+def test_quantised_scales_near_the_bound(kind):
+    """V rows spanning up to the largest allowed scale (just below
+    PA_MAX_KV_SCALE for INT4): the f16 operands must not overflow. The
+    tolerance is relative to the value range (fp32 accumulation of terms up
+    to ~1e5)."""
+    span = {"u4": 6.0e4, "u8": 1.0e6, "fp8": 1.6e6}[kind]
+    w = W.paged("bigv", B=3, Hq=8, Hkv=2, D=128, P=16, context_lens=[300, 37, 1], kv=kind)
+    g = torch.Generator().manual_seed(5)
+    big = lambda t: ((torch.rand(t.shape, generator=g) - 0.5) * span).to(torch.bfloat16)
+    w.prefill_v, w.step_v = big(w.prefill_v), big(w.step_v)
+    for S in (1, 3):
+        got, _ = _run(w, num_splits=S)
+        ref, _ = oracle_decode(w, oracle_pool(w))
+        assert np.all(np.isfinite(got))
+        err = np.abs(got.astype(np.float64) - ref).max()
+        print(f"{kind}: max |gpu - oracle| = {err:.3e} on outputs up to {np.abs(ref).max():.3e}")
+        assert err <= 2e-6 * span
 
 
 def test_empty_context_gives_zero():
@@ -206,7 +231,7 @@ def _sample_pairs(w, n, seed=0):
     return sorted(set(pairs))
 
 
-@pytest.mark.parametrize("name", ["tiny", "llama8b", "llama70b", "int8", "fp8"])
+@pytest.mark.parametrize("name", ["tiny", "llama8b", "llama70b", "int8", "fp8", "int4"])
 def test_full_size_sampled_outputs(name):
     """The full workloads, in the launch configuration the benchmark times
     (automatic split count), checked on sampled (sequence, head) rows."""

@@ -47,6 +47,7 @@ CASES = {
     "int8": lambda: W.int8(B=6, ctx_range=(1, 900)),
     "d64": lambda: W.paged("d64", B=5, Hq=8, Hkv=2, D=64, P=16, ctx_range=(1, 400)),
     "fp8": lambda: W.fp8(B=6, ctx_range=(1, 900)),
+    "int4": lambda: W.int4(B=6, ctx_range=(1, 900)),
 }
 
 
