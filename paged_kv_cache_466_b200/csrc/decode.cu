@@ -209,6 +209,395 @@ __device__ void merge_rows(const DecodeArgs &a, int b, int h, int G, int nl, flo
   }
 }
 
+// ---- per-block building blocks ---------------------------------------------------
+
+// Query fragments of the head of lane group g (A operand, rows = heads; rows
+// 8..15 stay zero). Returns the sum of q as the MMA sees it (quantised pools).
+template <int D, int KVT>
+__device__ __forceinline__ float load_q(const __nv_bfloat16 *qp, bool head_ok, int t,
+                                        uint32_t (&qa)[D / 16][2]) {
+  using T = Tile<D, KVT>;
+  float qsum = 0.f;        // sum of this head's q (as the MMA sees it), INT8 only
+  if constexpr (!T::kU8) {
+#pragma unroll
+    for (int i = 0; i < T::kKChunks; ++i) {
+      uint4 v = head_ok ? ldg_nc128(qp + (4 * i + t) * 8) : make_uint4(0, 0, 0, 0);
+      qa[2 * i][0] = v.x;
+      qa[2 * i][1] = v.y;
+      qa[2 * i + 1][0] = v.z;
+      qa[2 * i + 1][1] = v.w;
+    }
+  } else if constexpr (T::kU4) {
+    // lane t contracts d in [t*D/4, (t+1)*D/4); per group of 8 elements the
+    // k-steps take (e0,e2 | e4,e6) and (e1,e3 | e5,e7), as the 4-bit unpack does
+#pragma unroll
+    for (int w = 0; w < D / 32; ++w) {
+      const uint4 v = head_ok ? ldg_nc128(qp + t * (D / 4) + 8 * w) : make_uint4(0, 0, 0, 0);
+      const uint32_t f02 = pack_f16(bf16_lo(v.x), bf16_lo(v.y));
+      const uint32_t f46 = pack_f16(bf16_lo(v.z), bf16_lo(v.w));
+      const uint32_t f13 = pack_f16(bf16_hi(v.x), bf16_hi(v.y));
+      const uint32_t f57 = pack_f16(bf16_hi(v.z), bf16_hi(v.w));
+      qsum += (f16_lo(f02) + f16_hi(f02)) + (f16_lo(f46) + f16_hi(f46)) +
+              (f16_lo(f13) + f16_hi(f13)) + (f16_lo(f57) + f16_hi(f57));
+      qa[2 * w][0] = f02;
+      qa[2 * w][1] = f46;
+      qa[2 * w + 1][0] = f13;
+      qa[2 * w + 1][1] = f57;
+    }
+    qsum += __shfl_xor_sync(0xffffffffu, qsum, 1);
+    qsum += __shfl_xor_sync(0xffffffffu, qsum, 2);
+  } else {
+#pragma unroll
+    for (int i = 0; i < T::kKChunks; ++i) {
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        uint4 v = head_ok ? ldg_nc128(qp + (4 * i + t) * 16 + hf * 8) : make_uint4(0, 0, 0, 0);
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t f = pack_f16(bf16_lo(w4[k]), bf16_hi(w4[k]));
+          qsum += f16_lo(f) + f16_hi(f);
+          // words of this 16-d chunk: k-step 4i + (2hf + k/2), half k%2
+          qa[4 * i + 2 * hf + k / 2][k % 2] = f;
+        }
+      }
+    }
+    qsum += __shfl_xor_sync(0xffffffffu, qsum, 1);
+    qsum += __shfl_xor_sync(0xffffffffu, qsum, 2);
+  }
+  return qsum;
+}
+
+// Lane-constant offsets: where each 16-byte copy of a block lands in the stage
+// (row and swizzled place), and where the lane reads its K and V fragments.
+template <int D, int KVT>
+struct LaneMap {
+  using T = Tile<D, KVT>;
+  int cp_row[T::kCopies], cp_soff[T::kCopies];
+  int sz_dst;
+  int koff[2][T::kKChunks];
+  int voff[4][T::kVChunks];
+  __device__ __forceinline__ explicit LaneMap(int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int j = 0; j < T::kCopies; ++j) {
+      const int o = j * 512 + lane * 16;
+      cp_row[j] = o / T::kRowBytes;
+      cp_soff[j] = staged_off<T>(cp_row[j], (o % T::kRowBytes) >> 4);
+    }
+    sz_dst = (lane < 8 ? T::kKSzOff : T::kVSzOff) + (lane & 7) * 16;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int i = 0; i < T::kKChunks; ++i)
+        koff[nt][i] = T::kU4 ? T::staged_row(nt * 8 + g) * T::kRowBytes + t * (D / 8)
+                             : staged_off<T>(nt * 8 + g, 4 * i + t);
+#pragma unroll
+    for (int tau = 0; tau < 4; ++tau)
+#pragma unroll
+      for (int c = 0; c < T::kVChunks; ++c) {
+        const int row = (tau & 1) + 2 * t + (tau >> 1) * 8;
+        if constexpr (T::kU4) {
+          voff[tau][c] = T::kVOff + T::staged_row(row) * T::kRowBytes + g * (D / 16);
+        } else {
+          const int chunk = T::kU8 ? (D == 128 ? g : (g >> 1)) : 8 * c + g;
+          voff[tau][c] = T::kVOff + staged_off<T>(row, chunk);
+        }
+      }
+  }
+};
+
+// Issue the copies of one 16-token block: pool rows row0 .. row0 + 15 of K and
+// V (and their scale/zero) into the stage at `dst`; rows outside [rlo, rhi)
+// are zero-filled instead of read. sz_base is k_sz for lanes 0..7, else v_sz.
+template <int D, int KVT>
+__device__ __forceinline__ void issue_block(const LaneMap<D, KVT> &lm, uint32_t dst,
+                                            const unsigned char *kbase,
+                                            const unsigned char *vbase, const float *sz_base,
+                                            size_t row0, int rlo, int rhi, int lane) {
+  using T = Tile<D, KVT>;
+  const unsigned char *ksrc = kbase + row0 * T::kRowBytes + lane * 16;
+  const unsigned char *vsrc = vbase + row0 * T::kRowBytes + lane * 16;
+#pragma unroll
+  for (int j = 0; j < T::kCopies; ++j) {
+    const uint32_t n = (lm.cp_row[j] >= rlo && lm.cp_row[j] < rhi) ? 16u : 0u;
+    cp_async16(dst + lm.cp_soff[j], ksrc + j * 512, n);
+    cp_async16(dst + T::kVOff + lm.cp_soff[j], vsrc + j * 512, n);
+  }
+  if constexpr (T::kU8) {
+    // lanes 0..7: K (scale, zero) of rows 2l, 2l+1; lanes 8..15: V
+    if (lane < 16) {
+      // (a row outside [rlo, rhi) may come along with its neighbour; the
+      // consumer zeroes scale and zero of every masked token)
+      const int l = lane & 7;
+      const bool any = 2 * l + 1 >= rlo && 2 * l < rhi;
+      cp_async16(dst + lm.sz_dst, sz_base + (row0 + 2 * l) * 2, any ? 16u : 0u);
+    }
+  }
+}
+
+// One warp's online-softmax state for the G heads of a (sequence, KV head).
+template <int D, int KVT>
+struct WarpAcc {
+  float o[Tile<D, KVT>::kMTiles][4];
+  float m_run;  // running max of this head's scores (log2 units)
+  float l_run;  // this lane's share of the softmax denominator
+  float zacc;   // quantised pools: this lane's share of sum_t p_t z_t
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int j = 0; j < Tile<D, KVT>::kMTiles; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+    m_run = -INFINITY;
+    l_run = 0.f;
+    zacc = 0.f;
+  }
+};
+
+// Scores, online softmax and O^T update for the 16-token block staged at
+// `src`, whose first token is btok; tokens outside [tok_lo, tok1) and all
+// tokens of an invalid page (pvalid false) are masked.
+template <int D, int KVT>
+__device__ __forceinline__ void block_step(const LaneMap<D, KVT> &lm, uint32_t src, int btok,
+                                           int tok_lo, int tok1, bool pvalid, float scale_log2,
+                                           const uint32_t (&qa)[D / 16][2], float qsum, int g,
+                                           int t, WarpAcc<D, KVT> &acc) {
+  using T = Tile<D, KVT>;
+  float(&o)[T::kMTiles][4] = acc.o;
+  float &m_run = acc.m_run;
+  float &l_run = acc.l_run;
+  float &zacc = acc.zacc;
+  const auto &koff = lm.koff;
+  const auto &voff = lm.voff;
+  // ---- S = Q K^T -------------------------------------------------------------
+  float s[2][4];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+    if constexpr (T::kU4) {
+      uint32_t wk[D / 32];
+      if constexpr (D == 128) {
+        const uint4 v = lds128(src + koff[nt][0]);
+        wk[0] = v.x; wk[1] = v.y; wk[2] = v.z; wk[3] = v.w;
+      } else {
+        const uint2 v = lds64(src + koff[nt][0]);
+        wk[0] = v.x; wk[1] = v.y;
+      }
+#pragma unroll
+      for (int w = 0; w < D / 32; ++w) {
+        // even elements (low nibbles), then odd ones, each as c * 2^-9
+        uint32_t b02, b46, b13, b57;
+        nib4_to_f16x2x2(wk[w] & 0x0F0F0F0Fu, b02, b46);
+        nib4_to_f16x2x2((wk[w] >> 4) & 0x0F0F0F0Fu, b13, b57);
+        mma_f16_16816(s[nt], qa[2 * w][0], 0u, qa[2 * w][1], 0u, b02, b46);
+        mma_f16_16816(s[nt], qa[2 * w + 1][0], 0u, qa[2 * w + 1][1], 0u, b13, b57);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < T::kKChunks; ++i) {
+        const uint4 kv = lds128(src + koff[nt][i]);
+        if constexpr (!T::kU8) {
+          mma_bf16_16816(s[nt], qa[2 * i][0], 0u, qa[2 * i][1], 0u, kv.x, kv.y);
+          mma_bf16_16816(s[nt], qa[2 * i + 1][0], 0u, qa[2 * i + 1][1], 0u, kv.z, kv.w);
+        } else {
+          const uint32_t w4[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const uint32_t b0 =
+                T::kFp8 ? e4m3x2_to_f16x2(w4[w]) : u8x2_to_f16x2(w4[w], 0x4140);
+            const uint32_t b1 =
+                T::kFp8 ? e4m3x2_to_f16x2(w4[w] >> 16) : u8x2_to_f16x2(w4[w], 0x4342);
+            mma_f16_16816(s[nt], qa[4 * i + w][0], 0u, qa[4 * i + w][1], 0u, b0, b1);
+          }
+        }
+      }
+    }
+  }
+
+  // ---- online softmax (log2 domain) ---------------------------------------
+  float x[4] = {s[0][0], s[0][1], s[1][0], s[1][1]};  // tokens 2t, 2t+1, 8+2t, 9+2t
+  float vs[4], vz[4];
+  if constexpr (T::kU8) {
+    const uint4 k01 = lds128(src + T::kKSzOff + 16 * t);
+    const uint4 k89 = lds128(src + T::kKSzOff + 16 * (4 + t));
+    const uint4 v01 = lds128(src + T::kVSzOff + 16 * t);
+    const uint4 v89 = lds128(src + T::kVSzOff + 16 * (4 + t));
+    const float ks[4] = {__uint_as_float(k01.x), __uint_as_float(k01.z),
+                         __uint_as_float(k89.x), __uint_as_float(k89.z)};
+    const float kz[4] = {__uint_as_float(k01.y), __uint_as_float(k01.w),
+                         __uint_as_float(k89.y), __uint_as_float(k89.w)};
+    vs[0] = __uint_as_float(v01.x); vz[0] = __uint_as_float(v01.y);
+    vs[1] = __uint_as_float(v01.z); vz[1] = __uint_as_float(v01.w);
+    vs[2] = __uint_as_float(v89.x); vz[2] = __uint_as_float(v89.y);
+    vs[3] = __uint_as_float(v89.z); vz[3] = __uint_as_float(v89.w);
+    // INT4 codes reach the MMA as c * 2^-9: the exact power of two goes
+    // back into the K scale here and into O after the loop
+    constexpr float kCodeScale = T::kU4 ? 512.f : 1.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) x[e] = fmaf(ks[e] * kCodeScale, x[e], kz[e] * qsum);
+  }
+  if (pvalid && btok >= tok_lo && btok + 16 <= tok1) {  // warp-uniform: no mask needed
+#pragma unroll
+    for (int e = 0; e < 4; ++e) x[e] *= scale_log2;
+  } else {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int tok = btok + (e & 1) + 2 * t + (e >> 1) * 8;
+      const bool ok = pvalid && tok >= tok_lo && tok < tok1;
+      x[e] = ok ? x[e] * scale_log2 : -INFINITY;
+      if constexpr (T::kU8) {
+        if (!ok) vs[e] = vz[e] = 0.f;
+      }
+    }
+  }
+  float mb = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+  mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
+  mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
+  const bool need = mb > m_run + kRescaleLog2<KVT> || (m_run == -INFINITY && mb > -INFINITY);
+  if (__any_sync(0xffffffffu, need)) {
+    const float m_new = fmaxf(m_run, mb);
+    const float alpha = m_new == -INFINITY ? 1.f : fast_exp2(m_run - m_new);
+    m_run = m_new;
+    l_run *= alpha;
+    zacc *= alpha;
+    const float al0 = __shfl_sync(0xffffffffu, alpha, 8 * t);      // head 2t
+    const float al1 = __shfl_sync(0xffffffffu, alpha, 8 * t + 4);  // head 2t+1
+#pragma unroll
+    for (int j = 0; j < T::kMTiles; ++j) {
+      o[j][0] *= al0;
+      o[j][1] *= al1;
+      o[j][2] *= al0;
+      o[j][3] *= al1;
+    }
+  }
+  const float mref = m_run == -INFINITY ? 0.f : m_run;
+  float p[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) p[e] = fast_exp2(x[e] - mref);
+  l_run += (p[0] + p[1]) + (p[2] + p[3]);
+
+  // ---- O^T += V^T P^T -------------------------------------------------------
+  uint32_t bh0, bl0, bh1, bl1;
+  if constexpr (!T::kU8) {
+    split_bf16(p[0], p[1], bh0, bl0);
+    split_bf16(p[2], p[3], bh1, bl1);
+#pragma unroll
+    for (int c = 0; c < T::kVChunks; ++c) {
+      const uint4 v0 = lds128(src + voff[0][c]);
+      const uint4 v1 = lds128(src + voff[1][c]);
+      const uint4 v2 = lds128(src + voff[2][c]);
+      const uint4 v3 = lds128(src + voff[3][c]);
+      const uint32_t x0[4] = {v0.x, v0.y, v0.z, v0.w};
+      const uint32_t x1[4] = {v1.x, v1.y, v1.z, v1.w};
+      const uint32_t x2[4] = {v2.x, v2.y, v2.z, v2.w};
+      const uint32_t x3[4] = {v3.x, v3.y, v3.z, v3.w};
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const uint32_t a0 = __byte_perm(x0[w], x1[w], 0x5410);
+        const uint32_t a1 = __byte_perm(x0[w], x1[w], 0x7632);
+        const uint32_t a2 = __byte_perm(x2[w], x3[w], 0x5410);
+        const uint32_t a3 = __byte_perm(x2[w], x3[w], 0x7632);
+        mma_bf16_16816(o[4 * c + w], a0, a1, a2, a3, bh0, bh1);
+        mma_bf16_16816(o[4 * c + w], a0, a1, a2, a3, bl0, bl1);
+      }
+    }
+  } else {
+    float pv[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      pv[e] = p[e] * vs[e];
+      zacc = fmaf(p[e], vz[e], zacc);
+    }
+    split_f16(pv[0], pv[1], bh0, bl0);
+    split_f16(pv[2], pv[3], bh1, bl1);
+    if constexpr (T::kU4) {
+      // byte j of this lane's slice holds d = base + 2j (low nibble) and + 1
+      uint32_t xv[4][D / 64];
+#pragma unroll
+      for (int tau = 0; tau < 4; ++tau) {
+        if constexpr (D == 128) {
+          const uint2 v = lds64(src + voff[tau][0]);
+          xv[tau][0] = v.x;
+          xv[tau][1] = v.y;
+        } else {
+          xv[tau][0] = lds32(src + voff[tau][0]);
+        }
+      }
+      // m-tiles j, j+1 use bytes j & 3, (j & 3) + 1 of word j / 4: gather them
+      // for token pairs (2t, 2t+1) and (8+2t, 9+2t), then low nibbles give
+      // rows d (a0, a2), high nibbles rows d + 1 (a1, a3)
+#pragma unroll
+      for (int j = 0; j < T::kMTiles; j += 2) {
+        const uint32_t sel = (j & 2) ? 0x7362 : 0x5140;
+        const uint32_t ya = __byte_perm(xv[0][j / 4], xv[1][j / 4], sel);
+        const uint32_t yb = __byte_perm(xv[2][j / 4], xv[3][j / 4], sel);
+        uint32_t a0[2], a1[2], a2[2], a3[2];
+        nib4_to_f16x2x2(ya & 0x0F0F0F0Fu, a0[0], a0[1]);
+        nib4_to_f16x2x2((ya >> 4) & 0x0F0F0F0Fu, a1[0], a1[1]);
+        nib4_to_f16x2x2(yb & 0x0F0F0F0Fu, a2[0], a2[1]);
+        nib4_to_f16x2x2((yb >> 4) & 0x0F0F0F0Fu, a3[0], a3[1]);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          mma_f16_16816(o[j + u], a0[u], a1[u], a2[u], a3[u], bh0, bh1);
+          mma_f16_16816(o[j + u], a0[u], a1[u], a2[u], a3[u], bl0, bl1);
+        }
+      }
+      return;
+    }
+    const uint4 v0 = lds128(src + voff[0][0]);
+    const uint4 v1 = lds128(src + voff[1][0]);
+    const uint4 v2 = lds128(src + voff[2][0]);
+    const uint4 v3 = lds128(src + voff[3][0]);
+    const uint32_t x0[4] = {v0.x, v0.y, v0.z, v0.w};
+    const uint32_t x1[4] = {v1.x, v1.y, v1.z, v1.w};
+    const uint32_t x2[4] = {v2.x, v2.y, v2.z, v2.w};
+    const uint32_t x3[4] = {v3.x, v3.y, v3.z, v3.w};
+#pragma unroll
+    for (int j = 0; j < T::kMTiles; ++j) {
+      const uint32_t sel = (j & 1) ? 0x7362 : 0x5140;
+      // select with a runtime word offset only for D == 64
+      const uint32_t w0 = D == 128 ? x0[j / 2] : ((g & 1) ? x0[2 + j / 2] : x0[j / 2]);
+      const uint32_t w1 = D == 128 ? x1[j / 2] : ((g & 1) ? x1[2 + j / 2] : x1[j / 2]);
+      const uint32_t w2 = D == 128 ? x2[j / 2] : ((g & 1) ? x2[2 + j / 2] : x2[j / 2]);
+      const uint32_t w3 = D == 128 ? x3[j / 2] : ((g & 1) ? x3[2 + j / 2] : x3[j / 2]);
+      const uint32_t xa = __byte_perm(w0, w1, sel);
+      const uint32_t xb = __byte_perm(w2, w3, sel);
+      const uint32_t a0 = T::kFp8 ? e4m3x2_to_f16x2(xa) : u8x2_to_f16x2(xa, 0x4140);
+      const uint32_t a1 = T::kFp8 ? e4m3x2_to_f16x2(xa >> 16) : u8x2_to_f16x2(xa, 0x4342);
+      const uint32_t a2 = T::kFp8 ? e4m3x2_to_f16x2(xb) : u8x2_to_f16x2(xb, 0x4140);
+      const uint32_t a3 = T::kFp8 ? e4m3x2_to_f16x2(xb >> 16) : u8x2_to_f16x2(xb, 0x4342);
+      mma_f16_16816(o[j], a0, a1, a2, a3, bh0, bh1);
+      mma_f16_16816(o[j], a0, a1, a2, a3, bl0, bl1);
+    }
+  }
+}
+
+// Reduce the per-lane softmax sums over each head's 4 lanes and apply the
+// quantised zero-point term: afterwards o holds sum_t p_t v_t for heads 2t and
+// 2t + 1 and l_run the denominator of head g.
+template <int D, int KVT>
+__device__ __forceinline__ void finish_acc(WarpAcc<D, KVT> &acc, int t) {
+  using T = Tile<D, KVT>;
+  float(&o)[T::kMTiles][4] = acc.o;
+  float &l_run = acc.l_run;
+  float &zacc = acc.zacc;
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+  if constexpr (T::kU8) {
+    zacc += __shfl_xor_sync(0xffffffffu, zacc, 1);
+    zacc += __shfl_xor_sync(0xffffffffu, zacc, 2);
+    const float z0 = __shfl_sync(0xffffffffu, zacc, 8 * t);
+    const float z1 = __shfl_sync(0xffffffffu, zacc, 8 * t + 4);
+    constexpr float kCodeScale = T::kU4 ? 512.f : 1.f;  // INT4 codes were c * 2^-9
+#pragma unroll
+    for (int j = 0; j < T::kMTiles; ++j) {
+      o[j][0] = fmaf(o[j][0], kCodeScale, z0);
+      o[j][1] = fmaf(o[j][1], kCodeScale, z1);
+      o[j][2] = fmaf(o[j][2], kCodeScale, z0);
+      o[j][3] = fmaf(o[j][3], kCodeScale, z1);
+    }
+  }
+}
+
+
 template <int D, int P, int KVT, int W, int NSTAGE>
 __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(const DecodeArgs a) {
   using T = Tile<D, KVT>;
@@ -304,59 +693,12 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
     tbl[i] = pg;
   }
 
-  // ---- query fragments (A operand, rows = heads; rows 8..15 stay zero) -------
+  // ---- query fragments ---------------------------------------------------------
   const bool head_ok = g < G;
   const size_t q_row = ((size_t)b * a.hq + (size_t)h * G + (head_ok ? g : 0)) * D;
   const __nv_bfloat16 *qp = reinterpret_cast<const __nv_bfloat16 *>(a.q) + q_row;
   uint32_t qa[D / 16][2];  // per k-step: a0 (k 2t..2t+1), a2 (k 2t+8..2t+9)
-  float qsum = 0.f;        // sum of this head's q (as the MMA sees it), INT8 only
-  if constexpr (!T::kU8) {
-#pragma unroll
-    for (int i = 0; i < T::kKChunks; ++i) {
-      uint4 v = head_ok ? ldg_nc128(qp + (4 * i + t) * 8) : make_uint4(0, 0, 0, 0);
-      qa[2 * i][0] = v.x;
-      qa[2 * i][1] = v.y;
-      qa[2 * i + 1][0] = v.z;
-      qa[2 * i + 1][1] = v.w;
-    }
-  } else if constexpr (T::kU4) {
-    // lane t contracts d in [t*D/4, (t+1)*D/4); per group of 8 elements the
-    // k-steps take (e0,e2 | e4,e6) and (e1,e3 | e5,e7), as the 4-bit unpack does
-#pragma unroll
-    for (int w = 0; w < D / 32; ++w) {
-      const uint4 v = head_ok ? ldg_nc128(qp + t * (D / 4) + 8 * w) : make_uint4(0, 0, 0, 0);
-      const uint32_t f02 = pack_f16(bf16_lo(v.x), bf16_lo(v.y));
-      const uint32_t f46 = pack_f16(bf16_lo(v.z), bf16_lo(v.w));
-      const uint32_t f13 = pack_f16(bf16_hi(v.x), bf16_hi(v.y));
-      const uint32_t f57 = pack_f16(bf16_hi(v.z), bf16_hi(v.w));
-      qsum += (f16_lo(f02) + f16_hi(f02)) + (f16_lo(f46) + f16_hi(f46)) +
-              (f16_lo(f13) + f16_hi(f13)) + (f16_lo(f57) + f16_hi(f57));
-      qa[2 * w][0] = f02;
-      qa[2 * w][1] = f46;
-      qa[2 * w + 1][0] = f13;
-      qa[2 * w + 1][1] = f57;
-    }
-    qsum += __shfl_xor_sync(0xffffffffu, qsum, 1);
-    qsum += __shfl_xor_sync(0xffffffffu, qsum, 2);
-  } else {
-#pragma unroll
-    for (int i = 0; i < T::kKChunks; ++i) {
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        uint4 v = head_ok ? ldg_nc128(qp + (4 * i + t) * 16 + hf * 8) : make_uint4(0, 0, 0, 0);
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint32_t f = pack_f16(bf16_lo(w4[k]), bf16_hi(w4[k]));
-          qsum += f16_lo(f) + f16_hi(f);
-          // words of this 16-d chunk: k-step 4i + (2hf + k/2), half k%2
-          qa[4 * i + 2 * hf + k / 2][k % 2] = f;
-        }
-      }
-    }
-    qsum += __shfl_xor_sync(0xffffffffu, qsum, 1);
-    qsum += __shfl_xor_sync(0xffffffffu, qsum, 2);
-  }
+  const float qsum = load_q<D, KVT>(qp, head_ok, t, qa);
   __syncthreads();  // tbl visible
 
   // ---- per-warp pipeline ---------------------------------------------------------
@@ -367,19 +709,8 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
   const unsigned char *kbase = static_cast<const unsigned char *>(a.k_pool);
   const unsigned char *vbase = static_cast<const unsigned char *>(a.v_pool);
   const int nmine = nblk > warp ? (nblk - warp + W - 1) / W : 0;
-
-  // lane-constant parts of the copies: byte offset in the block, its row and
-  // its swizzled place in the stage
-  int cp_row[T::kCopies], cp_soff[T::kCopies];
-#pragma unroll
-  for (int j = 0; j < T::kCopies; ++j) {
-    const int o = j * 512 + lane * 16;
-    cp_row[j] = o / T::kRowBytes;
-    cp_soff[j] = staged_off<T>(cp_row[j], (o % T::kRowBytes) >> 4);
-  }
+  const LaneMap<D, KVT> lm(lane);
   const float *sz_base = lane < 8 ? a.k_sz : a.v_sz;
-  const int sz_dst = (lane < 8 ? T::kKSzOff : T::kVSzOff) + (lane & 7) * 16;
-
   auto issue = [&](int kb, int st) {
     const int btok = tok0 + kb * 16;
     const int lp = btok / P;
@@ -390,55 +721,12 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
     const int rhi = page >= 0 ? min(16, tok1 - btok) : 0;
     // rows of an invalid page are zero-filled; the address stays inside page 0
     const size_t row0 = ((size_t)(page >= 0 ? page : 0) * a.hkv + h) * P + in_page;
-    const uint32_t dst = ring + st * T::kStageBytes;
-    const unsigned char *ksrc = kbase + row0 * T::kRowBytes + lane * 16;
-    const unsigned char *vsrc = vbase + row0 * T::kRowBytes + lane * 16;
-#pragma unroll
-    for (int j = 0; j < T::kCopies; ++j) {
-      const uint32_t n = (cp_row[j] >= rlo && cp_row[j] < rhi) ? 16u : 0u;
-      cp_async16(dst + cp_soff[j], ksrc + j * 512, n);
-      cp_async16(dst + T::kVOff + cp_soff[j], vsrc + j * 512, n);
-    }
-    if constexpr (T::kU8) {
-      // lanes 0..7: K (scale, zero) of rows 2l, 2l+1; lanes 8..15: V
-      if (lane < 16) {
-        // (a row outside [rlo, rhi) may come along with its neighbour; the
-        // consumer zeroes scale and zero of every masked token)
-        const int l = lane & 7;
-        const bool any = 2 * l + 1 >= rlo && 2 * l < rhi;
-        cp_async16(dst + sz_dst, sz_base + (row0 + 2 * l) * 2, any ? 16u : 0u);
-      }
-    }
+    issue_block<D, KVT>(lm, ring + st * T::kStageBytes, kbase, vbase, sz_base, row0, rlo, rhi,
+                        lane);
   };
 
-  // per-lane offsets of the fragment reads within a stage
-  int koff[2][T::kKChunks];
-#pragma unroll
-  for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-    for (int i = 0; i < T::kKChunks; ++i)
-      koff[nt][i] = T::kU4 ? T::staged_row(nt * 8 + g) * T::kRowBytes + t * (D / 8)
-                           : staged_off<T>(nt * 8 + g, 4 * i + t);
-  int voff[4][T::kVChunks];
-#pragma unroll
-  for (int tau = 0; tau < 4; ++tau)
-#pragma unroll
-    for (int c = 0; c < T::kVChunks; ++c) {
-      const int row = (tau & 1) + 2 * t + (tau >> 1) * 8;
-      if constexpr (T::kU4) {
-        voff[tau][c] = T::kVOff + T::staged_row(row) * T::kRowBytes + g * (D / 16);
-      } else {
-        const int chunk = T::kU8 ? (D == 128 ? g : (g >> 1)) : 8 * c + g;
-        voff[tau][c] = T::kVOff + staged_off<T>(row, chunk);
-      }
-    }
-
-  float o[T::kMTiles][4];
-#pragma unroll
-  for (int j = 0; j < T::kMTiles; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-  float m_run = -INFINITY;  // running max of this head's scores (log2 units)
-  float l_run = 0.f;        // this lane's share of the softmax denominator
-  float zacc = 0.f;         // INT8: this lane's share of sum_t p_t z_t
+  WarpAcc<D, KVT> acc;
+  acc.reset();
 
 #pragma unroll
   for (int st = 0; st < NSTAGE - 1; ++st) {
@@ -460,229 +748,14 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
     const int btok = tok0 + kb * 16;
     const bool pvalid = tbl[btok / P - lp0] >= 0;
     const uint32_t src = ring + (k % NSTAGE) * T::kStageBytes;
-
-    // ---- S = Q K^T -------------------------------------------------------------
-    float s[2][4];
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-      if constexpr (T::kU4) {
-        uint32_t wk[D / 32];
-        if constexpr (D == 128) {
-          const uint4 v = lds128(src + koff[nt][0]);
-          wk[0] = v.x; wk[1] = v.y; wk[2] = v.z; wk[3] = v.w;
-        } else {
-          const uint2 v = lds64(src + koff[nt][0]);
-          wk[0] = v.x; wk[1] = v.y;
-        }
-#pragma unroll
-        for (int w = 0; w < D / 32; ++w) {
-          // even elements (low nibbles), then odd ones, each as c * 2^-9
-          uint32_t b02, b46, b13, b57;
-          nib4_to_f16x2x2(wk[w] & 0x0F0F0F0Fu, b02, b46);
-          nib4_to_f16x2x2((wk[w] >> 4) & 0x0F0F0F0Fu, b13, b57);
-          mma_f16_16816(s[nt], qa[2 * w][0], 0u, qa[2 * w][1], 0u, b02, b46);
-          mma_f16_16816(s[nt], qa[2 * w + 1][0], 0u, qa[2 * w + 1][1], 0u, b13, b57);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < T::kKChunks; ++i) {
-          const uint4 kv = lds128(src + koff[nt][i]);
-          if constexpr (!T::kU8) {
-            mma_bf16_16816(s[nt], qa[2 * i][0], 0u, qa[2 * i][1], 0u, kv.x, kv.y);
-            mma_bf16_16816(s[nt], qa[2 * i + 1][0], 0u, qa[2 * i + 1][1], 0u, kv.z, kv.w);
-          } else {
-            const uint32_t w4[4] = {kv.x, kv.y, kv.z, kv.w};
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-              const uint32_t b0 =
-                  T::kFp8 ? e4m3x2_to_f16x2(w4[w]) : u8x2_to_f16x2(w4[w], 0x4140);
-              const uint32_t b1 =
-                  T::kFp8 ? e4m3x2_to_f16x2(w4[w] >> 16) : u8x2_to_f16x2(w4[w], 0x4342);
-              mma_f16_16816(s[nt], qa[4 * i + w][0], 0u, qa[4 * i + w][1], 0u, b0, b1);
-            }
-          }
-        }
-      }
-    }
-
-    // ---- online softmax (log2 domain) ---------------------------------------
-    float x[4] = {s[0][0], s[0][1], s[1][0], s[1][1]};  // tokens 2t, 2t+1, 8+2t, 9+2t
-    float vs[4], vz[4];
-    if constexpr (T::kU8) {
-      const uint4 k01 = lds128(src + T::kKSzOff + 16 * t);
-      const uint4 k89 = lds128(src + T::kKSzOff + 16 * (4 + t));
-      const uint4 v01 = lds128(src + T::kVSzOff + 16 * t);
-      const uint4 v89 = lds128(src + T::kVSzOff + 16 * (4 + t));
-      const float ks[4] = {__uint_as_float(k01.x), __uint_as_float(k01.z),
-                           __uint_as_float(k89.x), __uint_as_float(k89.z)};
-      const float kz[4] = {__uint_as_float(k01.y), __uint_as_float(k01.w),
-                           __uint_as_float(k89.y), __uint_as_float(k89.w)};
-      vs[0] = __uint_as_float(v01.x); vz[0] = __uint_as_float(v01.y);
-      vs[1] = __uint_as_float(v01.z); vz[1] = __uint_as_float(v01.w);
-      vs[2] = __uint_as_float(v89.x); vz[2] = __uint_as_float(v89.y);
-      vs[3] = __uint_as_float(v89.z); vz[3] = __uint_as_float(v89.w);
-      // INT4 codes reach the MMA as c * 2^-9: the exact power of two goes
-      // back into the K scale here and into O after the loop
-      constexpr float kCodeScale = T::kU4 ? 512.f : 1.f;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) x[e] = fmaf(ks[e] * kCodeScale, x[e], kz[e] * qsum);
-    }
-    if (pvalid && btok >= tok_lo && btok + 16 <= tok1) {  // warp-uniform: no mask needed
-#pragma unroll
-      for (int e = 0; e < 4; ++e) x[e] *= a.scale_log2;
-    } else {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int tok = btok + (e & 1) + 2 * t + (e >> 1) * 8;
-        const bool ok = pvalid && tok >= tok_lo && tok < tok1;
-        x[e] = ok ? x[e] * a.scale_log2 : -INFINITY;
-        if constexpr (T::kU8) {
-          if (!ok) vs[e] = vz[e] = 0.f;
-        }
-      }
-    }
-    float mb = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-    mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
-    mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
-    const bool need = mb > m_run + kRescaleLog2<KVT> || (m_run == -INFINITY && mb > -INFINITY);
-    if (__any_sync(0xffffffffu, need)) {
-      const float m_new = fmaxf(m_run, mb);
-      const float alpha = m_new == -INFINITY ? 1.f : fast_exp2(m_run - m_new);
-      m_run = m_new;
-      l_run *= alpha;
-      zacc *= alpha;
-      const float al0 = __shfl_sync(0xffffffffu, alpha, 8 * t);      // head 2t
-      const float al1 = __shfl_sync(0xffffffffu, alpha, 8 * t + 4);  // head 2t+1
-#pragma unroll
-      for (int j = 0; j < T::kMTiles; ++j) {
-        o[j][0] *= al0;
-        o[j][1] *= al1;
-        o[j][2] *= al0;
-        o[j][3] *= al1;
-      }
-    }
-    const float mref = m_run == -INFINITY ? 0.f : m_run;
-    float p[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) p[e] = fast_exp2(x[e] - mref);
-    l_run += (p[0] + p[1]) + (p[2] + p[3]);
-
-    // ---- O^T += V^T P^T -------------------------------------------------------
-    uint32_t bh0, bl0, bh1, bl1;
-    if constexpr (!T::kU8) {
-      split_bf16(p[0], p[1], bh0, bl0);
-      split_bf16(p[2], p[3], bh1, bl1);
-#pragma unroll
-      for (int c = 0; c < T::kVChunks; ++c) {
-        const uint4 v0 = lds128(src + voff[0][c]);
-        const uint4 v1 = lds128(src + voff[1][c]);
-        const uint4 v2 = lds128(src + voff[2][c]);
-        const uint4 v3 = lds128(src + voff[3][c]);
-        const uint32_t x0[4] = {v0.x, v0.y, v0.z, v0.w};
-        const uint32_t x1[4] = {v1.x, v1.y, v1.z, v1.w};
-        const uint32_t x2[4] = {v2.x, v2.y, v2.z, v2.w};
-        const uint32_t x3[4] = {v3.x, v3.y, v3.z, v3.w};
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const uint32_t a0 = __byte_perm(x0[w], x1[w], 0x5410);
-          const uint32_t a1 = __byte_perm(x0[w], x1[w], 0x7632);
-          const uint32_t a2 = __byte_perm(x2[w], x3[w], 0x5410);
-          const uint32_t a3 = __byte_perm(x2[w], x3[w], 0x7632);
-          mma_bf16_16816(o[4 * c + w], a0, a1, a2, a3, bh0, bh1);
-          mma_bf16_16816(o[4 * c + w], a0, a1, a2, a3, bl0, bl1);
-        }
-      }
-    } else {
-      float pv[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        pv[e] = p[e] * vs[e];
-        zacc = fmaf(p[e], vz[e], zacc);
-      }
-      split_f16(pv[0], pv[1], bh0, bl0);
-      split_f16(pv[2], pv[3], bh1, bl1);
-      if constexpr (T::kU4) {
-        // byte j of this lane's slice holds d = base + 2j (low nibble) and + 1
-        uint32_t xv[4][D / 64];
-#pragma unroll
-        for (int tau = 0; tau < 4; ++tau) {
-          if constexpr (D == 128) {
-            const uint2 v = lds64(src + voff[tau][0]);
-            xv[tau][0] = v.x;
-            xv[tau][1] = v.y;
-          } else {
-            xv[tau][0] = lds32(src + voff[tau][0]);
-          }
-        }
-        // m-tiles j, j+1 use bytes j & 3, (j & 3) + 1 of word j / 4: gather them
-        // for token pairs (2t, 2t+1) and (8+2t, 9+2t), then low nibbles give
-        // rows d (a0, a2), high nibbles rows d + 1 (a1, a3)
-#pragma unroll
-        for (int j = 0; j < T::kMTiles; j += 2) {
-          const uint32_t sel = (j & 2) ? 0x7362 : 0x5140;
-          const uint32_t ya = __byte_perm(xv[0][j / 4], xv[1][j / 4], sel);
-          const uint32_t yb = __byte_perm(xv[2][j / 4], xv[3][j / 4], sel);
-          uint32_t a0[2], a1[2], a2[2], a3[2];
-          nib4_to_f16x2x2(ya & 0x0F0F0F0Fu, a0[0], a0[1]);
-          nib4_to_f16x2x2((ya >> 4) & 0x0F0F0F0Fu, a1[0], a1[1]);
-          nib4_to_f16x2x2(yb & 0x0F0F0F0Fu, a2[0], a2[1]);
-          nib4_to_f16x2x2((yb >> 4) & 0x0F0F0F0Fu, a3[0], a3[1]);
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            mma_f16_16816(o[j + u], a0[u], a1[u], a2[u], a3[u], bh0, bh1);
-            mma_f16_16816(o[j + u], a0[u], a1[u], a2[u], a3[u], bl0, bl1);
-          }
-        }
-        continue;
-      }
-      const uint4 v0 = lds128(src + voff[0][0]);
-      const uint4 v1 = lds128(src + voff[1][0]);
-      const uint4 v2 = lds128(src + voff[2][0]);
-      const uint4 v3 = lds128(src + voff[3][0]);
-      const uint32_t x0[4] = {v0.x, v0.y, v0.z, v0.w};
-      const uint32_t x1[4] = {v1.x, v1.y, v1.z, v1.w};
-      const uint32_t x2[4] = {v2.x, v2.y, v2.z, v2.w};
-      const uint32_t x3[4] = {v3.x, v3.y, v3.z, v3.w};
-#pragma unroll
-      for (int j = 0; j < T::kMTiles; ++j) {
-        const uint32_t sel = (j & 1) ? 0x7362 : 0x5140;
-        // select with a runtime word offset only for D == 64
-        const uint32_t w0 = D == 128 ? x0[j / 2] : ((g & 1) ? x0[2 + j / 2] : x0[j / 2]);
-        const uint32_t w1 = D == 128 ? x1[j / 2] : ((g & 1) ? x1[2 + j / 2] : x1[j / 2]);
-        const uint32_t w2 = D == 128 ? x2[j / 2] : ((g & 1) ? x2[2 + j / 2] : x2[j / 2]);
-        const uint32_t w3 = D == 128 ? x3[j / 2] : ((g & 1) ? x3[2 + j / 2] : x3[j / 2]);
-        const uint32_t xa = __byte_perm(w0, w1, sel);
-        const uint32_t xb = __byte_perm(w2, w3, sel);
-        const uint32_t a0 = T::kFp8 ? e4m3x2_to_f16x2(xa) : u8x2_to_f16x2(xa, 0x4140);
-        const uint32_t a1 = T::kFp8 ? e4m3x2_to_f16x2(xa >> 16) : u8x2_to_f16x2(xa, 0x4342);
-        const uint32_t a2 = T::kFp8 ? e4m3x2_to_f16x2(xb) : u8x2_to_f16x2(xb, 0x4140);
-        const uint32_t a3 = T::kFp8 ? e4m3x2_to_f16x2(xb >> 16) : u8x2_to_f16x2(xb, 0x4342);
-        mma_f16_16816(o[j], a0, a1, a2, a3, bh0, bh1);
-        mma_f16_16816(o[j], a0, a1, a2, a3, bl0, bl1);
-      }
-    }
+    block_step<D, KVT>(lm, src, btok, tok_lo, tok1, pvalid, a.scale_log2, qa, qsum, g, t, acc);
   }
   cp_async_wait<0>();
   __syncwarp();
-
-  // ---- finish this warp's state ---------------------------------------------------
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
-  if constexpr (T::kU8) {
-    zacc += __shfl_xor_sync(0xffffffffu, zacc, 1);
-    zacc += __shfl_xor_sync(0xffffffffu, zacc, 2);
-    const float z0 = __shfl_sync(0xffffffffu, zacc, 8 * t);
-    const float z1 = __shfl_sync(0xffffffffu, zacc, 8 * t + 4);
-    constexpr float kCodeScale = T::kU4 ? 512.f : 1.f;  // INT4 codes were c * 2^-9
-#pragma unroll
-    for (int j = 0; j < T::kMTiles; ++j) {
-      o[j][0] = fmaf(o[j][0], kCodeScale, z0);
-      o[j][1] = fmaf(o[j][1], kCodeScale, z1);
-      o[j][2] = fmaf(o[j][2], kCodeScale, z0);
-      o[j][3] = fmaf(o[j][3], kCodeScale, z1);
-    }
-  }
+  finish_acc<D, KVT>(acc, t);
+  const float(&o)[T::kMTiles][4] = acc.o;
+  const float m_run = acc.m_run;
+  const float l_run = acc.l_run;
 
   // ---- merge the CTA's warps (fixed order: deterministic) --------------------
   float *rec = reinterpret_cast<float *>(smem + warp * SM::kRingBytesPerWarp);

@@ -75,7 +75,7 @@ def test_decode_small_matches_oracle(name, num_splits):
 def test_one_token_context_is_exact():
     """ctx = 1: the softmax weight is exactly 1 and out equals v_0 bit for bit."""
     w = W.paged("ctx1", B=5, Hq=16, Hkv=2, D=128, P=16, context_lens=[1] * 5)
-    for S in (1, 4):
+    for S in (0, 1, 4):
         got, _ = _run(w, num_splits=S)
         v0 = w.step_v.float().numpy()                   # [B, Hkv, D]: the only token
         want = np.repeat(v0, w.G, axis=1).reshape(-1, w.D)
@@ -107,7 +107,7 @@ def test_empty_context_gives_zero():
     pool, bt, ctx, q = device_inputs(w)
     device_append(pool, w, bt)
     ctx[1] = 0
-    for S in (1, 2):
+    for S in (0, 1, 2):
         out = pa_decode(pool, q, bt, ctx, w.scale, num_splits=S)
         torch.cuda.synchronize()
         assert torch.all(out[1] == 0) and torch.all(torch.isfinite(out))
@@ -116,7 +116,7 @@ def test_empty_context_gives_zero():
 def test_splits_agree():
     """Any split count gives the same answer up to fp32 merge rounding (1e-5)."""
     w = W.llama8b(B=4, ctx_range=(500, 2000))
-    outs = [_run(w, num_splits=S)[0] for S in (1, 2, 4, 8, 32, 128)]
+    outs = [_run(w, num_splits=S)[0] for S in (1, 0, 2, 4, 8, 32, 128)]
     for o in outs[1:]:
         assert np.abs(o - outs[0]).max() <= 1e-5
 
@@ -150,6 +150,40 @@ def test_workspace_reuse_across_calls():
         reused = pa_decode(pool, q, bt, ctx, w.scale, num_splits=S, workspace=ws)
         torch.cuda.synchronize()
         assert torch.equal(fresh, reused)
+
+
+@pytest.mark.parametrize("kv", ["bf16", "u8", "u4"])
+def test_automatic_splits_on_ragged_and_empty_contexts(kv):
+    """Automatic splitting on a ragged batch: empty sequences between long
+    ones, one-token ones, and one long sequence over many splits compared
+    with a fixed split count."""
+    ctx = [0, 1, 5000, 17, 0, 3, 16, 32, 4096, 0, 2049, 15]
+    w = W.paged("ragged", B=len(ctx), Hq=16, Hkv=4, D=128, P=16, context_lens=ctx, kv=kv)
+    got, _ = _run(w, num_splits=0)
+    _check(w, got)
+    # one long sequence over many splits; the same data through 7 fixed splits
+    w1 = W.paged("long", B=1, Hq=8, Hkv=1, D=128, P=32, context_lens=[30000], kv=kv)
+    a, (pool, bt, ctx1, q) = _run(w1, num_splits=0)
+    b = pa_decode(pool, q, bt, ctx1, w1.scale, num_splits=7).cpu().numpy().reshape(-1, w1.D)
+    # different partitions: fp32 merge rounding, and for quantised pools the
+    # rescaling points of the online softmax differ too
+    assert np.abs(a - b).max() <= 5e-5
+    _check(w1, a, pairs=[(0, h) for h in range(w1.Hq)])
+
+
+def test_automatic_splits_workspace_reuse_and_determinism():
+    """Automatic splitting re-arms its counters: one zero-filled workspace
+    serves many calls, and results repeat bit for bit."""
+    ws = torch.zeros(1 << 24, dtype=torch.uint8, device=DEV)
+    for seed in range(3):
+        w = W.llama8b(B=9, ctx_range=(1, 3000), seed=seed)
+        pool, bt, ctx, q = device_inputs(w)
+        device_append(pool, w, bt)
+        fresh = pa_decode(pool, q, bt, ctx, w.scale)
+        r1 = pa_decode(pool, q, bt, ctx, w.scale, workspace=ws)
+        r2 = pa_decode(pool, q, bt, ctx, w.scale, workspace=ws)
+        torch.cuda.synchronize()
+        assert torch.equal(fresh, r1) and torch.equal(r1, r2)
 
 
 def test_shared_prefix_equals_unshared_copy_bitwise():
