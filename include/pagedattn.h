@@ -62,6 +62,8 @@ typedef enum {
 #define PA_DERR_BAD_POS 8  /* append: pos < 0 or pos / page_size >= max_pages  */
 #define PA_DERR_BIG_SCALE 16 /* append: a quantised row's scale is not below
                                 PA_MAX_KV_SCALE (the row is still written)     */
+#define PA_DERR_TIMEOUT 32 /* a bounded wait on the kernel's own tensor-core
+                              work ran out (not expected; outputs invalid)    */
 
 /* Quantised pools: pa_decode* feed s * (softmax weight) to the tensor cores
  * as f16, with weights kept <= 8, so every row scale must be below this bound

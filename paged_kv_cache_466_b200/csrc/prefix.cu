@@ -1,4 +1,5 @@
-// Shared-prefix attention: the prefix half of a cascade decode.
+// Shared-prefix attention: the prefix half of a cascade decode, on the
+// fifth-generation tensor cores (tcgen05, accumulators in tensor memory).
 //
 // "KV-Cache Optimization Techniques", section "Prefix Caching" (Eq. 2): when
 // many requests share a prompt prefix, its KV pages are stored once and every
@@ -7,16 +8,29 @@
 // tokens, merged by log-sum-exp. This kernel does the prefix part for all
 // requests at once: per KV head, the B*G query rows that read that head form
 // an [rows x D] x [D x prefix] contraction, so each prefix K/V row is read once
-// per CTA row-tile instead of once per request, and the work runs as dense
-// tensor-core tiles (FlashAttention-2-style online softmax).
+// per 128-row tile instead of once per request, and the products run as dense
+// tensor-core tiles with a FlashAttention-style online softmax.
 //
-// CTA: 4 warps x 16 query rows = 64 rows of one KV head; it walks a range of
-// 64-token prefix tiles (a prefix split) and writes, per row, the normalised
-// partial output and its natural-log log-sum-exp. K/V tiles are staged by all
-// threads with cp.async into a 2-stage ring (16-byte chunks XOR-swizzled by
-// row so ldmatrix reads are conflict free); per tile each warp computes
-// S = Q K^T (m16n8k16, K via ldmatrix), the online softmax, and O += P V with
-// P split into bf16 hi + lo halves (V via ldmatrix.trans).
+// CTA (4 warps, 128 threads) = 128 query rows of one KV head (row r of the
+// head is sequence r / G, query head h * G + r % G) over one prefix split of
+// 64-token tiles. Per tile:
+//   S[128 x 64]  = Q K^T  : tcgen05.mma kind::f16, A = Q and B = K tile, both
+//                           K-major 128-byte-swizzled in shared memory, S in
+//                           tensor memory (64 fp32 columns)
+//   softmax                : thread r owns row r (TMEM lane r): tcgen05.ld of
+//                           its 64 scores, online max / sum in fp32, P split
+//                           into bf16 hi + lo and stored back to tensor memory
+//                           (tcgen05.st, two bf16 per column)
+//   O[128 x D]  += P V     : A = P from tensor memory, B = V tile (MN-major in
+//                           shared memory, the page rows as they are), O in
+//                           tensor memory
+// Thread 0 issues the MMAs and commits them to an mbarrier; every wait on it
+// is bounded. K/V tiles are staged by all threads with 16-byte cp.async into
+// a 2-stage ring, the copy of tile k + 1 overlapping the softmax and PV of
+// tile k; 96 KB of shared memory and 256 TMEM columns let two CTAs share an
+// SM, so one CTA's softmax overlaps the other's MMAs. The output per row is
+// the normalised partial and its natural-log log-sum-exp, merged with the
+// suffix by the decode kernel.
 #include <cmath>
 
 #include "pa_device.cuh"
@@ -26,37 +40,139 @@ namespace pa {
 namespace {
 
 constexpr float kLn2 = 0.693147180559945309f;
-constexpr int kRowsPerCta = 64;
-constexpr int kTileTok = 64;
-constexpr int kWarps = 4;
+constexpr int kRowsPerCta = 128;  // the MMA's M
+constexpr int kTileTok = 64;      // N of S, K of PV
+constexpr int kThreads = 128;
+constexpr int kTmemCols = 256;    // S [0, 64), P hi [64, 96), P lo [96, 128), O [128, 128 + D)
+constexpr float kRescaleLog2 = 8.0f;
+constexpr int kMaxWaitPolls = 1 << 24;
 
-template <int D>
-struct PTile {
-  static constexpr int kRowBytes = D * 2;
-  static constexpr int kChunks = kRowBytes / 16;
-  static constexpr int kTileBytes = kTileTok * kRowBytes;  // one tensor
-  static constexpr int kStageBytes = 2 * kTileBytes;       // K and V
-  static constexpr int kKSteps = D / 16;
-  static constexpr int kNTilesD = D / 8;
-};
-
-__device__ __forceinline__ int swz_off(int row, int chunk, int row_bytes) {
-  return row * row_bytes + ((chunk ^ (row & 7)) << 4);
+// Byte offset of 16-byte chunk `chunk` of row r in a K-major,
+// 128-byte-swizzled tile of `rows` rows: 64-element K atoms of rows * 128
+// bytes, 8-row groups of 1024 bytes, chunks XOR-permuted by row % 8 (the
+// layout the tensor core's SWIZZLE_128B descriptor reads). The MN-major V
+// tile uses the same formula with (row, chunk) = (token, d / 8).
+__device__ __forceinline__ uint32_t sw128(int r, int chunk, int rows) {
+  return (chunk >> 3) * rows * 128 + (r >> 3) * 1024 + (r & 7) * 128 +
+         (((chunk & 7) ^ (r & 7)) << 4);
 }
 
+// Shared-memory matrix descriptor: start address, leading / stride byte
+// offsets, version 1, SWIZZLE_128B.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  const uint32_t lo = ((addr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
+  const uint32_t hi = ((sbo >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
+  return ((uint64_t)hi << 32) | lo;
+}
+
+// Instruction descriptor: bf16 x bf16 -> fp32, M = 128, N = n, A K-major,
+// B K-major or MN-major.
+__host__ __device__ constexpr uint32_t instr_desc(int n, bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kRowsPerCta >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                          int accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+
+// The same with A read from tensor memory (lane = row, two bf16 per column).
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                             uint32_t idesc, int accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+      bar));
+}
+
+// Wait until the mbarrier's phase with this parity has completed; false if
+// the bounded number of polls ran out.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  for (int i = 0; i < kMaxWaitPolls; ++i) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(done)
+        : "r"(bar), "r"(parity));
+    if (done) return true;
+  }
+  return false;
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// 32 lanes x 32 bits x 32 columns from tensor memory: thread i of the warp
+// gets lane (taddr lane + i), columns taddr .. taddr + 31.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31]));
+}
+
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+template <int D>
+struct PLayout {
+  static constexpr int kChunks = D / 8;                       // 16-byte chunks per row
+  static constexpr int kQBytes = kRowsPerCta * D * 2;         // Q tile
+  static constexpr int kKVBytes = kTileTok * D * 2;           // one K or V tile
+  static constexpr int kQOff = 0;
+  static constexpr int kStageOff = kQBytes;                   // 2 stages of K, V
+  static constexpr int kBarOff = kStageOff + 4 * kKVBytes;    // 2 mbarriers + TMEM address
+  static constexpr int kPagesOff = kBarOff + 64;
+  static constexpr int kKSteps = D / 16;                      // MMAs per S
+};
+
 template <int D, int P>
-__global__ void __launch_bounds__(kWarps * 32, 2) prefix_kernel(const PrefixArgs a) {
-  using T = PTile<D>;
-  extern __shared__ __align__(128) unsigned char smem[];
+__global__ void __launch_bounds__(kThreads, 2) prefix_kernel(const PrefixArgs a) {
+  using L = PLayout<D>;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // the swizzled tiles need 1024-byte aligned atoms
+  unsigned char *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   pdl_wait_primary();
 
   const int mt = blockIdx.x;
   const int h = blockIdx.y;
   const int ps = blockIdx.z;
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int g = lane >> 2;
-  const int t = lane & 3;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
   const int G = a.hq / a.hkv;
   const int rows = a.B * G;
 
@@ -65,12 +181,18 @@ __global__ void __launch_bounds__(kWarps * 32, 2) prefix_kernel(const PrefixArgs
   const int tile1 = min(tile0 + a.tiles_per_split, n_tiles);
   const int tok_lo = tile0 * kTileTok;
   const int tok_hi = min(tile1 * kTileTok, a.prefix_len);
+  const int ntl = tile1 - tile0;
+
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar_s = sbase + L::kBarOff;       // S of tile k done (and PV of k - 1)
+  const uint32_t bar_pv = sbase + L::kBarOff + 8;  // last PV done
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kBarOff + 16);
+  int *pages = reinterpret_cast<int *>(smem + L::kPagesOff);
 
   // prefix page ids of this split, bounds-checked
-  int *pages = reinterpret_cast<int *>(smem + 2 * T::kStageBytes);
   const int pg0 = tok_lo / P;
   const int npg = tok_hi > tok_lo ? (tok_hi - 1) / P - pg0 + 1 : 0;
-  for (int i = threadIdx.x; i < npg; i += kWarps * 32) {
+  for (int i = tid; i < npg; i += kThreads) {
     int pg = __ldg(a.prefix_pages + pg0 + i);
     if (pg < 0 || pg >= a.num_pages) {
       flag_error(a.d_err, PA_DERR_BAD_PAGE);
@@ -79,194 +201,239 @@ __global__ void __launch_bounds__(kWarps * 32, 2) prefix_kernel(const PrefixArgs
     pages[i] = pg;
   }
 
-  // query rows g and g + 8 of this warp -> (sequence, query head)
-  int qrow[2];
-  bool qok[2];
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const int r = mt * kRowsPerCta + warp * 16 + g + 8 * i;
-    qok[i] = r < rows;
-    const int rr = qok[i] ? r : 0;
-    qrow[i] = (rr / G) * a.hq + h * G + rr % G;
-  }
-  uint32_t qa[T::kKSteps][4];
+  // this thread's query row (TMEM lane tid)
+  const int r = mt * kRowsPerCta + tid;
+  const bool row_ok = r < rows;
+  const size_t qrow = (size_t)(row_ok ? r / G : 0) * a.hq + (size_t)h * G + (row_ok ? r % G : 0);
+
+  // Q tile: row tid, D / 8 chunks of 16 bytes, zero rows past the batch
   {
-    const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(a.q);
+    const unsigned char *qsrc = static_cast<const unsigned char *>(a.q) + qrow * D * 2;
 #pragma unroll
-    for (int j = 0; j < T::kKSteps; ++j) {
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const uint32_t *qr = reinterpret_cast<const uint32_t *>(qb + (size_t)qrow[i] * D);
-        qa[j][i] = qok[i] ? __ldg(qr + 8 * j + t) : 0u;          // k = 16j + 2t
-        qa[j][2 + i] = qok[i] ? __ldg(qr + 8 * j + 4 + t) : 0u;  // k = 16j + 8 + 2t
-      }
-    }
+    for (int c = 0; c < L::kChunks; ++c)
+      cp_async16(sbase + L::kQOff + sw128(tid, c, kRowsPerCta), qsrc + c * 16, row_ok ? 16u : 0u);
+    cp_async_commit();
   }
-  __syncthreads();  // page ids visible
+
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  if (tid == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar_s), "r"(1));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar_pv), "r"(1));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();  // page ids, barriers and the TMEM address are visible
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t t_s = tmem;                              // S columns
+  const uint32_t t_ph = tmem + kTileTok;                  // P hi: 2 bf16 per column
+  const uint32_t t_pl = t_ph + kTileTok / 2;              // P lo
+  const uint32_t t_o = tmem + 2 * kTileTok;               // O columns
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;  // this warp's TMEM lanes
 
   const unsigned char *kbase = static_cast<const unsigned char *>(a.k_pool);
   const unsigned char *vbase = static_cast<const unsigned char *>(a.v_pool);
-  const uint32_t sbase = smem_u32(smem);
-  const int ntl = tile1 - tile0;
-
-  // all threads copy one 64-token tile of K and V (each copy instruction of the
-  // CTA moves 2 KB: 8 whole rows)
+  // K and V tile k into stage st: 64 token rows x D / 8 chunks each; rows of
+  // tokens past the split or of invalid pages are zero-filled
   auto load_tile = [&](int k, int st) {
     const int ttok = tok_lo + k * kTileTok;
-    const uint32_t dst = sbase + st * T::kStageBytes;
-    constexpr int kCopies = T::kTileBytes / (kWarps * 32 * 16);
+    const uint32_t ks = sbase + L::kStageOff + st * 2 * L::kKVBytes;
+    constexpr int kPer = kTileTok * L::kChunks / kThreads;
 #pragma unroll
-    for (int i = 0; i < kCopies; ++i) {
-      const int c = threadIdx.x + i * kWarps * 32;
-      const int row = c / T::kChunks;
-      const int chunk = c % T::kChunks;
+    for (int i = 0; i < kPer; ++i) {
+      const int c = tid + i * kThreads;
+      const int row = c / L::kChunks;
+      const int chunk = c % L::kChunks;
       const int tok = ttok + row;
       int page = -1;
       if (tok < tok_hi) page = pages[tok / P - pg0];
       const bool ok = page >= 0;
       const size_t grow = ((size_t)(ok ? page : 0) * a.hkv + h) * P + (ok ? tok % P : 0);
-      const int so = swz_off(row, chunk, T::kRowBytes);
-      cp_async16(dst + so, kbase + grow * T::kRowBytes + chunk * 16, ok ? 16u : 0u);
-      cp_async16(dst + T::kTileBytes + so, vbase + grow * T::kRowBytes + chunk * 16,
-                 ok ? 16u : 0u);
+      const uint32_t so = sw128(row, chunk, kTileTok);
+      cp_async16(ks + so, kbase + grow * D * 2 + chunk * 16, ok ? 16u : 0u);
+      cp_async16(ks + L::kKVBytes + so, vbase + grow * D * 2 + chunk * 16, ok ? 16u : 0u);
     }
   };
 
-  float o[T::kNTilesD][4];
-#pragma unroll
-  for (int n = 0; n < T::kNTilesD; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-  float m_run[2] = {-INFINITY, -INFINITY};
-  float l_run[2] = {0.f, 0.f};
+  float m_run = -INFINITY;  // this row's running max (log2 units)
+  float l_run = 0.f;        // this row's softmax denominator
+  bool ok_waits = true;
 
   if (ntl > 0) load_tile(0, 0);
   cp_async_commit();
   for (int k = 0; k < ntl; ++k) {
-    if (k + 1 < ntl) load_tile(k + 1, (k + 1) & 1);
-    cp_async_commit();
-    cp_async_wait<1>();
+    const int st = k & 1;
+    cp_async_wait<0>();                                           // Q (first time) and tile k
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor core
+    tc_fence_before();
     __syncthreads();
-    const uint32_t ks = sbase + (k & 1) * T::kStageBytes;
-    const uint32_t vs = ks + T::kTileBytes;
-    const int ttok = tok_lo + k * kTileTok;
+    tc_fence_after();
 
-    // ---- S = Q K^T: 8 n-tiles of 8 tokens
-    float s[8][4];
+    // ---- S = Q K^T
+    if (tid == 0) {
+      const uint32_t q0 = sbase + L::kQOff;
+      const uint32_t k0 = sbase + L::kStageOff + st * 2 * L::kKVBytes;
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+      for (int kk = 0; kk < L::kKSteps; ++kk) {
+        const uint32_t off = (kk & 3) * 32;  // 16 elements along K inside a 128-byte atom
+        umma_bf16(t_s, smem_desc(q0 + (kk >> 2) * (kRowsPerCta * 128) + off, 16, 1024),
+                  smem_desc(k0 + (kk >> 2) * (kTileTok * 128) + off, 16, 1024),
+                  instr_desc(kTileTok, false), kk > 0);
+      }
+      umma_commit(bar_s);
+    }
+    // S of tile k is complete, and with it the PV of tile k - 1 (a commit
+    // tracks every earlier MMA of the issuing thread): stage st ^ 1, the P
+    // columns and O are free
+    ok_waits &= mbar_wait(bar_s, k & 1);
+    tc_fence_after();
+    if (k + 1 < ntl) load_tile(k + 1, st ^ 1);
+    cp_async_commit();
+
+    // ---- online softmax of row tid (log2 units)
+    const int ttok = tok_lo + k * kTileTok;
+    float s[kTileTok];
+    {
+      uint32_t u[32];
+      tmem_ld32(t_s + lane_off, u);
+      tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < T::kKSteps; j += 2) {
-        const int row = nt * 8 + (lane & 7);
-        const int chunk = 2 * j + (lane >> 3);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(ks + swz_off(row, chunk, T::kRowBytes), b0, b1, b2, b3);
-        mma_bf16_16816(s[nt], qa[j][0], qa[j][1], qa[j][2], qa[j][3], b0, b1);
-        mma_bf16_16816(s[nt], qa[j + 1][0], qa[j + 1][1], qa[j + 1][2], qa[j + 1][3], b2, b3);
+      for (int j = 0; j < 32; ++j) s[j] = __uint_as_float(u[j]);
+      tmem_ld32(t_s + lane_off + 32, u);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) s[32 + j] = __uint_as_float(u[j]);
+    }
+    // a whole tile of valid pages needs no mask (uniform over the CTA)
+    bool full = ttok + kTileTok <= tok_hi;
+#pragma unroll
+    for (int i = 0; i < kTileTok / P; ++i) full = full && pages[ttok / P + i - pg0] >= 0;
+    float mx = -INFINITY;
+    if (full) {
+#pragma unroll
+      for (int j = 0; j < kTileTok; ++j) {
+        s[j] *= a.scale_log2;
+        mx = fmaxf(mx, s[j]);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < kTileTok; ++j) {
+        const int tok = ttok + j;
+        const bool live = tok < tok_hi && pages[tok / P - pg0] >= 0;
+        s[j] = live ? s[j] * a.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, s[j]);
       }
     }
-    // ---- online softmax for rows g (c0, c1) and g + 8 (c2, c3)
-    const bool full = ttok + kTileTok <= tok_hi;
-    float mx[2] = {-INFINITY, -INFINITY};
+    const bool need = mx > m_run + kRescaleLog2 || (m_run == -INFINITY && mx > -INFINITY);
+    if (__any_sync(0xffffffffu, need)) {  // warp-uniform: tcgen05.ld/st are warp-wide
+      const float m_new = need ? fmaxf(m_run, mx) : m_run;
+      const float alpha = need && m_run != -INFINITY ? fast_exp2(m_run - m_new) : 1.f;
+      if (need) {
+        m_run = m_new;
+        l_run *= alpha;
+      }
+      if (k > 0) {  // O holds earlier tiles: scale it
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t u[32];
+          tmem_ld32(t_o + lane_off + c0, u);
+          tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int tok = ttok + nt * 8 + 2 * t + (c & 1);
-        float v = s[nt][c] * a.scale_log2;
-        if (!full && tok >= tok_hi) v = -INFINITY;
-        s[nt][c] = v;
-        mx[c >> 1] = fmaxf(mx[c >> 1], v);
+          for (int j = 0; j < 32; ++j) u[j] = __float_as_uint(__uint_as_float(u[j]) * alpha);
+          tmem_st32(t_o + lane_off + c0, u);
+        }
+        tmem_wait_st();
       }
     }
-    float alpha[2];
+    const float mref = m_run == -INFINITY ? 0.f : m_run;
+    // P = exp2(s - m), split into bf16 hi + lo; column j of each half holds
+    // tokens 2j (low 16 bits) and 2j + 1 of row tid
+    {
+      uint32_t wh[kTileTok / 2], wl[kTileTok / 2];
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 1));
-      mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 2));
-      const float m_new = fmaxf(m_run[i], mx[i]);
-      alpha[i] = m_new == -INFINITY ? 1.f : fast_exp2(m_run[i] - m_new);
-      m_run[i] = m_new;
-      l_run[i] *= alpha[i];
-    }
-#pragma unroll
-    for (int n = 0; n < T::kNTilesD; ++n) {
-      o[n][0] *= alpha[0];
-      o[n][1] *= alpha[0];
-      o[n][2] *= alpha[1];
-      o[n][3] *= alpha[1];
-    }
-    const float mref[2] = {m_run[0] == -INFINITY ? 0.f : m_run[0],
-                           m_run[1] == -INFINITY ? 0.f : m_run[1]};
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const float p = fast_exp2(s[nt][c] - mref[c >> 1]);
-        s[nt][c] = p;
-        l_run[c >> 1] += p;
+      for (int j = 0; j < kTileTok / 2; ++j) {
+        const float p0 = fast_exp2(s[2 * j] - mref);
+        const float p1 = fast_exp2(s[2 * j + 1] - mref);
+        l_run += p0 + p1;
+        split_bf16(p0, p1, wh[j], wl[j]);
       }
+      tmem_st32(t_ph + lane_off, wh);
+      tmem_st32(t_pl + lane_off, wl);
+      tmem_wait_st();
     }
-    // ---- O += P V: 4 k-steps of 16 tokens; P from the score fragments
+    tc_fence_before();
+    __syncthreads();  // P stored, O scaled
+    tc_fence_after();
+
+    // ---- O += P V (hi and lo halves of P, A from tensor memory: 8 columns
+    // per 16 tokens)
+    if (tid == 0) {
+      const uint32_t v0 = sbase + L::kStageOff + st * 2 * L::kKVBytes + L::kKVBytes;
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      uint32_t ah[4], al[4];
-      split_bf16(s[2 * kk][0], s[2 * kk][1], ah[0], al[0]);
-      split_bf16(s[2 * kk][2], s[2 * kk][3], ah[1], al[1]);
-      split_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1], ah[2], al[2]);
-      split_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3], ah[3], al[3]);
-#pragma unroll
-      for (int n = 0; n < T::kNTilesD; n += 2) {
-        const int mi = lane >> 3;
-        const int row = 16 * kk + (lane & 7) + 8 * (mi & 1);
-        const int chunk = n + (mi >> 1);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_trans(vs + swz_off(row, chunk, T::kRowBytes), b0, b1, b2, b3);
-        mma_bf16_16816(o[n], ah[0], ah[1], ah[2], ah[3], b0, b1);
-        mma_bf16_16816(o[n], al[0], al[1], al[2], al[3], b0, b1);
-        mma_bf16_16816(o[n + 1], ah[0], ah[1], ah[2], ah[3], b2, b3);
-        mma_bf16_16816(o[n + 1], al[0], al[1], al[2], al[3], b2, b3);
+      for (int kk = 0; kk < kTileTok / 16; ++kk) {
+        const uint64_t dv = smem_desc(v0 + kk * 2048, kTileTok * 128, 1024);
+        umma_bf16_ts(t_o, t_ph + kk * 8, dv, instr_desc(D, true), k > 0 || kk > 0);
+        umma_bf16_ts(t_o, t_pl + kk * 8, dv, instr_desc(D, true), 1);
       }
+      umma_commit(bar_pv);
     }
-    __syncthreads();  // stage (k & 1) is refilled next iteration
   }
   cp_async_wait<0>();
 
-  // ---- normalise and write this split's partial for rows g and g + 8
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    l_run[i] += __shfl_xor_sync(0xffffffffu, l_run[i], 1);
-    l_run[i] += __shfl_xor_sync(0xffffffffu, l_run[i], 2);
-  }
+  // ---- normalise and write this split's partial for row tid
+  if (ntl > 0) ok_waits &= mbar_wait(bar_pv, (ntl - 1) & 1);
+  tc_fence_after();
   const size_t R = (size_t)a.B * a.hq;
+  const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+  float *orow = a.o_pre + ((size_t)ps * R + qrow) * D;
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    if (!qok[i]) continue;
-    const float inv = l_run[i] > 0.f ? 1.f / l_run[i] : 0.f;
-    float *orow = a.o_pre + ((size_t)ps * R + qrow[i]) * D;
+  for (int c0 = 0; c0 < D; c0 += 32) {
+    uint32_t u[32];
+    if (ntl > 0) {
+      tmem_ld32(t_o + lane_off + c0, u);
+      tmem_wait_ld();
+    } else {
 #pragma unroll
-    for (int n = 0; n < T::kNTilesD; ++n)
-      *reinterpret_cast<float2 *>(orow + 8 * n + 2 * t) =
-          make_float2(o[n][2 * i] * inv, o[n][2 * i + 1] * inv);
-    if (t == 0)
-      a.lse_pre[(size_t)ps * R + qrow[i]] =
-          l_run[i] > 0.f ? (m_run[i] + log2f(l_run[i])) * kLn2 : -INFINITY;
+      for (int j = 0; j < 32; ++j) u[j] = 0u;
+    }
+    if (row_ok) {
+#pragma unroll
+      for (int j = 0; j < 32; j += 4)
+        *reinterpret_cast<float4 *>(orow + c0 + j) =
+            make_float4(__uint_as_float(u[j]) * inv, __uint_as_float(u[j + 1]) * inv,
+                        __uint_as_float(u[j + 2]) * inv, __uint_as_float(u[j + 3]) * inv);
+    }
   }
+  if (row_ok)
+    a.lse_pre[(size_t)ps * R + qrow] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+  if (!ok_waits) flag_error(a.d_err, PA_DERR_TIMEOUT);
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols));
 }
 
 template <int D, int P>
 cudaError_t launch_prefix_t(const PrefixArgs &a, cudaStream_t stream) {
-  using T = PTile<D>;
+  using L = PLayout<D>;
   const int max_pages_per_split = a.tiles_per_split * kTileTok / P + 2;
-  const size_t smem = 2 * T::kStageBytes + (size_t)max_pages_per_split * 4;
-  static_assert(2 * PTile<D>::kStageBytes + 4 * 4096 <= 227 * 1024, "shared memory");
   if (max_pages_per_split > 4096) return cudaErrorInvalidValue;
+  constexpr int kMaxSmem = L::kPagesOff + 4 * 4096 + 1024;  // + alignment slack
+  static_assert(kMaxSmem <= 227 * 1024, "shared memory");
+  const size_t smem = L::kPagesOff + (size_t)max_pages_per_split * 4 + 1024;
   cudaError_t e = cudaFuncSetAttribute(prefix_kernel<D, P>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)(2 * T::kStageBytes + 4 * 4096));
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((a.B * (a.hq / a.hkv) + kRowsPerCta - 1) / kRowsPerCta, a.hkv, a.n_psplits);
-  cfg.blockDim = dim3(kWarps * 32);
+  cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
