@@ -382,7 +382,7 @@ def run_ours(args, rank, world, local_rank):
     dec_avg_ms = statistics.mean(dec_ms)
     achieved = dbytes / (dec_avg_ms * 1e-3) / 1e9
     traffic = recorded_traffic(w.name) if not (args.cascade or args.window) else None
-    launches_per_step = 3 if args.cascade else 2
+    launches_per_step = 4 if args.cascade else 2  # append, [prefix pass,] decode[, merge]
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),

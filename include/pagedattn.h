@@ -194,11 +194,13 @@ pa_status_t pa_decode(const pa_kv_pool_t *pool, const void *q,
  * begin with the same prompt prefix stored once in shared pages
  * ("KV-Cache Optimization Techniques", section "Prefix Caching", Eq. 2).
  * Computes exactly what pa_decode computes when every request's logical pages
- * [0, prefix_len / P) are prefix_pages, in two passes: (1) attention of all
- * num_seqs * num_q_heads query rows over the prefix, as dense tensor-core tiles
- * that read each prefix K/V row once per 64 query rows instead of once per
- * request; (2) the paged decode over each request's own tokens
- * [prefix_len, context_lens[b]), which merges (1) into its log-sum-exp merge.
+ * [0, prefix_len / P) are prefix_pages, in three launches: (1) attention of
+ * all num_seqs * num_q_heads query rows over the prefix, as dense tcgen05
+ * tensor-core tiles (accumulators in tensor memory) that read each prefix
+ * K/V row once per 128 query rows instead of once per request; (2) the paged
+ * decode over each request's own tokens [prefix_len, context_lens[b]),
+ * writing its split partials; (3) the log-sum-exp merge of (2) and (1) per
+ * row, in that order (deterministic).
  *
  *   prefix_pages : (device) int32 [prefix_len / P] physical pages of the prefix
  *   prefix_len   : tokens in the prefix; a multiple of the page size (0 falls
@@ -209,7 +211,7 @@ pa_status_t pa_decode(const pa_kv_pool_t *pool, const void *q,
  *                  one is flagged PA_DERR_BAD_CTX and treated as prefix_len)
  *   workspace    : (device) >= pa_decode_shared_prefix_workspace_bytes(...)
  *                  bytes, 256-byte aligned, zero-filled before its first use
- * Other arguments as for pa_decode. bf16 pools only. Two kernel launches.
+ * Other arguments as for pa_decode. bf16 pools only. Three kernel launches.
  */
 size_t pa_decode_shared_prefix_workspace_bytes(const pa_kv_pool_t *pool,
                                                int32_t num_seqs,

@@ -263,6 +263,7 @@ pa_status_t pa_decode(const pa_kv_pool_t *pool, const void *q, int32_t num_seqs,
   a.prior_o = nullptr;
   a.prior_lse = nullptr;
   a.n_prior = 0;
+  a.keep_partials = 0;
   a.d_err = d_err;
   return cuda_status(launch_decode(pool->head_dim, pool->page_size, pool->dtype, a,
                                    static_cast<cudaStream_t>(stream)),
@@ -388,10 +389,6 @@ pa_status_t pa_decode_shared_prefix(const pa_kv_pool_t *pool, const void *q, int
   pa.o_pre = reinterpret_cast<float *>(ws + pl.o_pre);
   pa.lse_pre = reinterpret_cast<float *>(ws + pl.lse_pre);
   pa.d_err = d_err;
-  st = cuda_status(launch_prefix(pool->head_dim, pool->page_size, pa, s),
-                   "pa_decode_shared_prefix prefix launch");
-  if (st != PA_OK) return st;
-
   DecodeArgs a;
   a.k_pool = pool->k_pool;
   a.v_pool = pool->v_pool;
@@ -417,12 +414,26 @@ pa_status_t pa_decode_shared_prefix(const pa_kv_pool_t *pool, const void *q, int
   a.window = 0;
   a.sinks = 0;
   a.tok_begin = prefix_len;
-  a.prior_o = pa.o_pre;
-  a.prior_lse = pa.lse_pre;
-  a.n_prior = pl.n_psplits;
   a.d_err = d_err;
-  return cuda_status(launch_decode(pool->head_dim, pool->page_size, pool->dtype, a, s),
+  // Three launches on `stream`: the prefix pass; the suffix decode, which
+  // writes its split partials (an empty split writes lse = -inf) instead of
+  // merging; one merge of the suffix splits and the prefix splits per row,
+  // with its loads batched (a decode CTA merging prefix partials in its
+  // epilogue measured slower).
+  a.prior_o = nullptr;
+  a.prior_lse = nullptr;
+  a.n_prior = 0;
+  a.keep_partials = 1;
+  st = cuda_status(launch_prefix(pool->head_dim, pool->page_size, pa, true, s),
+                   "pa_decode_shared_prefix prefix launch");
+  if (st == PA_OK)
+    st = cuda_status(launch_decode(pool->head_dim, pool->page_size, pool->dtype, a, s),
                      "pa_decode_shared_prefix suffix launch");
+  if (st != PA_OK) return st;
+  return cuda_status(launch_splitkv_reduce(a.o_part, a.lse, num_seqs, num_q_heads, pl.S,
+                                           pool->head_dim, out, true, s, pa.o_pre, pa.lse_pre,
+                                           pl.n_psplits),
+                     "pa_decode_shared_prefix merge launch");
 }
 
 pa_status_t pa_splitkv_reduce(const float *o_part, const float *lse, int32_t num_seqs,
@@ -574,6 +585,7 @@ pa_status_t pa_decode_window(const pa_kv_pool_t *pool, const void *q, int32_t nu
   a.prior_o = nullptr;
   a.prior_lse = nullptr;
   a.n_prior = 0;
+  a.keep_partials = 0;
   a.d_err = d_err;
   return cuda_status(launch_decode(pool->head_dim, pool->page_size, pool->dtype, a,
                                    static_cast<cudaStream_t>(stream)),

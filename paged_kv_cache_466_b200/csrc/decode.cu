@@ -672,6 +672,11 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
   const int tok1 = tok_hi;
 
   if (nblk == 0) {
+    if (a.keep_partials) {  // an empty partial: weight 0 in the caller's merge
+      for (int hd = threadIdx.x; hd < G; hd += W * 32)
+        a.lse[((size_t)b * a.hq + (size_t)h * G + hd) * a.S + slot] = -INFINITY;
+      return;
+    }
     if (split == 0 && n_live == 0) {
       if (a.n_prior > 0) {  // nothing of our own: the output is the priors' merge
         merge_rows<D>(a, b, h, G, 0, reinterpret_cast<float *>(smem));
@@ -793,13 +798,14 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
     }
     const size_t row = (size_t)b * a.hq + (size_t)h * G + hd;
     const float val = L > 0.f ? num / L : 0.f;
-    if (n_live == 1 && a.n_prior == 0) {
+    if (n_live == 1 && a.n_prior == 0 && !a.keep_partials) {
       a.out[row * D + d] = val;
     } else {
       a.o_part[(row * a.S + slot) * D + d] = val;
       if (d == 0) a.lse[row * a.S + slot] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
     }
   }
+  if (a.keep_partials) return;  // the caller merges
   if (n_live == 1) {
     if (a.n_prior == 0) return;
     __syncthreads();  // our own partial is visible to the whole CTA

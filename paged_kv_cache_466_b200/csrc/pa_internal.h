@@ -45,6 +45,8 @@ struct DecodeArgs {
   const float *prior_o;     // [n_prior][B*Hq][D] partials merged into the output
   const float *prior_lse;   // [n_prior][B*Hq]
   int32_t n_prior;
+  int32_t keep_partials;    // 1: every split writes its partial (an empty one lse = -inf)
+                            //    to its slot and nothing is merged
   int32_t *d_err;
 };
 
@@ -66,7 +68,8 @@ struct PrefixArgs {
   int32_t *d_err;
 };
 
-cudaError_t launch_prefix(int D, int P, const PrefixArgs &a, cudaStream_t stream);
+cudaError_t launch_prefix(int D, int P, const PrefixArgs &a, bool programmatic,
+                          cudaStream_t stream);
 int prefix_rows_per_cta();
 int prefix_tile_tokens();
 
@@ -75,9 +78,13 @@ cudaError_t launch_decode(int D, int P, int kv_dtype, const DecodeArgs &a,
 // CTAs of the decode kernel for (D, P, kv_dtype) that fit on one SM.
 int decode_ctas_per_sm(int D, int P, int kv_dtype);
 
+// Merges, per (sequence, query head) row, the S partials o_part[row][S][D] /
+// lse[row][S] and then n_prior more prior_o[p][row][D] / prior_lse[p][row].
 cudaError_t launch_splitkv_reduce(const float *o_part, const float *lse, int B,
                                   int hq, int S, int D, float *out,
-                                  bool programmatic, cudaStream_t stream);
+                                  bool programmatic, cudaStream_t stream,
+                                  const float *prior_o = nullptr,
+                                  const float *prior_lse = nullptr, int n_prior = 0);
 
 cudaError_t launch_kv_append(const pa_kv_pool_t &pool, const void *k_new,
                              const void *v_new, const int32_t *seq_idx,

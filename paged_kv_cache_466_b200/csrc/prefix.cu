@@ -421,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 2) prefix_kernel(const PrefixArgs a)
 }
 
 template <int D, int P>
-cudaError_t launch_prefix_t(const PrefixArgs &a, cudaStream_t stream) {
+cudaError_t launch_prefix_t(const PrefixArgs &a, bool programmatic, cudaStream_t stream) {
   using L = PLayout<D>;
   const int max_pages_per_split = a.tiles_per_split * kTileTok / P + 2;
   if (max_pages_per_split > 4096) return cudaErrorInvalidValue;
@@ -440,7 +440,7 @@ cudaError_t launch_prefix_t(const PrefixArgs &a, cudaStream_t stream) {
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = programmatic ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, prefix_kernel<D, P>, a);
 }
 
@@ -449,11 +449,12 @@ cudaError_t launch_prefix_t(const PrefixArgs &a, cudaStream_t stream) {
 int prefix_rows_per_cta() { return kRowsPerCta; }
 int prefix_tile_tokens() { return kTileTok; }
 
-cudaError_t launch_prefix(int D, int P, const PrefixArgs &a, cudaStream_t stream) {
-  if (D == 128 && P == 16) return launch_prefix_t<128, 16>(a, stream);
-  if (D == 128 && P == 32) return launch_prefix_t<128, 32>(a, stream);
-  if (D == 64 && P == 16) return launch_prefix_t<64, 16>(a, stream);
-  if (D == 64 && P == 32) return launch_prefix_t<64, 32>(a, stream);
+cudaError_t launch_prefix(int D, int P, const PrefixArgs &a, bool programmatic,
+                          cudaStream_t stream) {
+  if (D == 128 && P == 16) return launch_prefix_t<128, 16>(a, programmatic, stream);
+  if (D == 128 && P == 32) return launch_prefix_t<128, 32>(a, programmatic, stream);
+  if (D == 64 && P == 16) return launch_prefix_t<64, 16>(a, programmatic, stream);
+  if (D == 64 && P == 32) return launch_prefix_t<64, 32>(a, programmatic, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -16,42 +16,58 @@ namespace {
 
 constexpr int kWarps = 4;
 
+// Partials i < S are the row's own (o_part[row][i], lse[row][i]); i >= S are
+// prior partials p = i - S (prior_o[p][row], prior_lse[p][row]).
 __global__ void __launch_bounds__(kWarps * 32) splitkv_reduce_kernel(
     const float *__restrict__ o_part, const float *__restrict__ lse, int rows, int S, int D,
-    float *__restrict__ out) {
+    float *__restrict__ out, const float *__restrict__ prior_o,
+    const float *__restrict__ prior_lse, int n_prior) {
   pdl_wait_primary();  // partials come from the kernel just before us
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * kWarps + warp;
   if (row >= rows) return;
+  const int n_all = S + n_prior;
   const float *ls = lse + (size_t)row * S;
+  auto lse_at = [&](int i) { return i < S ? ls[i] : prior_lse[(size_t)(i - S) * rows + row]; };
   float M = -INFINITY;
-  for (int s = lane; s < S; s += 32) M = fmaxf(M, ls[s]);
+  for (int s = lane; s < n_all; s += 32) M = fmaxf(M, lse_at(s));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  const float4 *op = reinterpret_cast<const float4 *>(o_part + (size_t)row * S * D);
-  float4 *dst = reinterpret_cast<float4 *>(out + (size_t)row * D);
   const int D4 = D / 4;
+  const float4 *op = reinterpret_cast<const float4 *>(o_part + (size_t)row * S * D);
+  auto o_at = [&](int i) {
+    return i < S ? op + (size_t)i * D4
+                 : reinterpret_cast<const float4 *>(prior_o + ((size_t)(i - S) * rows + row) * D);
+  };
+  float4 *dst = reinterpret_cast<float4 *>(out + (size_t)row * D);
   for (int i0 = 0; i0 < D4; i0 += 32) {
     const int i = i0 + lane;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float den = 0.f;
-    // splits in chunks of 32: lane s holds the weight of split s0 + s, and
-    // every lane then issues its loads for the whole chunk back to back
-    for (int s0 = 0; s0 < S; s0 += 32) {
-      const int n = min(32, S - s0);
+    // partials in chunks of 32: lane s holds the weight of partial s0 + s,
+    // and every lane then issues its loads for the whole chunk back to back
+    for (int s0 = 0; s0 < n_all; s0 += 32) {
+      const int n = min(32, n_all - s0);
       const float wl =
-          (lane < n && M != -INFINITY) ? expf(ls[s0 + lane] - M) : 0.f;  // -inf -> 0
+          (lane < n && M != -INFINITY) ? expf(lse_at(s0 + lane) - M) : 0.f;  // -inf -> 0
       den += wl;
-#pragma unroll 8
-      for (int s = 0; s < n; ++s) {
-        const float w = __shfl_sync(0xffffffffu, wl, s);
-        if (i < D4 && w != 0.f) {  // weight-0 (empty) splits are never read
-          const float4 v = op[(size_t)(s0 + s) * D4 + i];
-          acc.x = fmaf(w, v.x, acc.x);
-          acc.y = fmaf(w, v.y, acc.y);
-          acc.z = fmaf(w, v.z, acc.z);
-          acc.w = fmaf(w, v.w, acc.w);
+      // eight loads in flight per lane; a weight-0 (empty) partial is loaded
+      // but never used, so whatever its slot holds cannot reach the sum
+      for (int b0 = 0; b0 < n; b0 += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          if (b0 + k < n && i < D4) v[k] = o_at(s0 + b0 + k)[i];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const float w = __shfl_sync(0xffffffffu, wl, (b0 + k) & 31);
+          if (b0 + k < n && i < D4 && w != 0.f) {
+            acc.x = fmaf(w, v[k].x, acc.x);
+            acc.y = fmaf(w, v[k].y, acc.y);
+            acc.z = fmaf(w, v[k].z, acc.z);
+            acc.w = fmaf(w, v[k].w, acc.w);
+          }
         }
       }
     }
@@ -67,7 +83,8 @@ __global__ void __launch_bounds__(kWarps * 32) splitkv_reduce_kernel(
 }  // namespace
 
 cudaError_t launch_splitkv_reduce(const float *o_part, const float *lse, int B, int hq, int S,
-                                  int D, float *out, bool programmatic, cudaStream_t stream) {
+                                  int D, float *out, bool programmatic, cudaStream_t stream,
+                                  const float *prior_o, const float *prior_lse, int n_prior) {
   const int rows = B * hq;
   if (rows == 0) return cudaSuccess;
   cudaLaunchConfig_t cfg = {};
@@ -80,7 +97,8 @@ cudaError_t launch_splitkv_reduce(const float *o_part, const float *lse, int B, 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = programmatic ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, splitkv_reduce_kernel, o_part, lse, rows, S, D, out);
+  return cudaLaunchKernelEx(&cfg, splitkv_reduce_kernel, o_part, lse, rows, S, D, out, prior_o,
+                            prior_lse, n_prior);
 }
 
 }  // namespace pa
