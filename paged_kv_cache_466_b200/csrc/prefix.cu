@@ -26,8 +26,9 @@
 //                           tensor memory
 // Thread 0 issues the MMAs and commits them to an mbarrier; every wait on it
 // is bounded. K/V tiles are staged by all threads with 16-byte cp.async into
-// a 2-stage ring, the copy of tile k + 1 overlapping the softmax and PV of
-// tile k; 96 KB of shared memory and 256 TMEM columns let two CTAs share an
+// a 2-stage ring, the copy of tile k + 1 overlapping the softmax of tile k,
+// and PV(k) and S(k + 1) go to the tensor core back to back behind one CTA
+// barrier per tile; 96 KB of shared memory and 256 TMEM columns let two CTAs share an
 // SM, so one CTA's softmax overlaps the other's MMAs. The output per row is
 // the normalised partial and its natural-log log-sum-exp, merged with the
 // suffix by the decode kernel.
@@ -185,7 +186,7 @@ __global__ void __launch_bounds__(kThreads, 2) prefix_kernel(const PrefixArgs a)
 
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar_s = sbase + L::kBarOff;       // S of tile k done (and PV of k - 1)
-  const uint32_t bar_pv = sbase + L::kBarOff + 8;  // last PV done
+  const uint32_t bar_pv = sbase + L::kBarOff + 8;  // the last tile's PV done
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kBarOff + 16);
   int *pages = reinterpret_cast<int *>(smem + L::kPagesOff);
 
@@ -264,32 +265,50 @@ __global__ void __launch_bounds__(kThreads, 2) prefix_kernel(const PrefixArgs a)
   float l_run = 0.f;        // this row's softmax denominator
   bool ok_waits = true;
 
+  // S = Q K^T of the tile staged in stage st, into the S columns
+  auto issue_s = [&](int st) {
+    const uint32_t q0 = sbase + L::kQOff;
+    const uint32_t k0 = sbase + L::kStageOff + st * 2 * L::kKVBytes;
+#pragma unroll
+    for (int kk = 0; kk < L::kKSteps; ++kk) {
+      const uint32_t off = (kk & 3) * 32;  // 16 elements along K inside a 128-byte atom
+      umma_bf16(t_s, smem_desc(q0 + (kk >> 2) * (kRowsPerCta * 128) + off, 16, 1024),
+                smem_desc(k0 + (kk >> 2) * (kTileTok * 128) + off, 16, 1024),
+                instr_desc(kTileTok, false), kk > 0);
+    }
+  };
+  // O += P V for the tile in stage st (hi and lo halves of P, A from tensor
+  // memory: 8 columns per 16 tokens)
+  auto issue_pv = [&](int st, bool first) {
+    const uint32_t v0 = sbase + L::kStageOff + st * 2 * L::kKVBytes + L::kKVBytes;
+#pragma unroll
+    for (int kk = 0; kk < kTileTok / 16; ++kk) {
+      const uint64_t dv = smem_desc(v0 + kk * 2048, kTileTok * 128, 1024);
+      umma_bf16_ts(t_o, t_ph + kk * 8, dv, instr_desc(D, true), !first || kk > 0);
+      umma_bf16_ts(t_o, t_pl + kk * 8, dv, instr_desc(D, true), 1);
+    }
+  };
+
+  // Pipeline: one barrier per tile. After the softmax of tile k (and the
+  // arrival of tile k + 1's copies), thread 0 issues PV(k) and S(k + 1) back
+  // to back and commits them together; the wait on that commit at the top of
+  // the next iteration covers both, which frees stage k's V, the P columns
+  // and O for the next softmax.
   if (ntl > 0) load_tile(0, 0);
   cp_async_commit();
+  cp_async_wait<0>();                                           // Q and tile 0
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor core
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (tid == 0 && ntl > 0) {
+    issue_s(0);
+    umma_commit(bar_s);
+  }
   for (int k = 0; k < ntl; ++k) {
     const int st = k & 1;
-    cp_async_wait<0>();                                           // Q (first time) and tile k
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor core
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-
-    // ---- S = Q K^T
-    if (tid == 0) {
-      const uint32_t q0 = sbase + L::kQOff;
-      const uint32_t k0 = sbase + L::kStageOff + st * 2 * L::kKVBytes;
-#pragma unroll
-      for (int kk = 0; kk < L::kKSteps; ++kk) {
-        const uint32_t off = (kk & 3) * 32;  // 16 elements along K inside a 128-byte atom
-        umma_bf16(t_s, smem_desc(q0 + (kk >> 2) * (kRowsPerCta * 128) + off, 16, 1024),
-                  smem_desc(k0 + (kk >> 2) * (kTileTok * 128) + off, 16, 1024),
-                  instr_desc(kTileTok, false), kk > 0);
-      }
-      umma_commit(bar_s);
-    }
-    // S of tile k is complete, and with it the PV of tile k - 1 (a commit
-    // tracks every earlier MMA of the issuing thread): stage st ^ 1, the P
-    // columns and O are free
+    // S(k) is complete, and with it PV(k - 1): stage st ^ 1, the P columns
+    // and O are free
     ok_waits &= mbar_wait(bar_s, k & 1);
     tc_fence_after();
     if (k + 1 < ntl) load_tile(k + 1, st ^ 1);
@@ -366,27 +385,25 @@ __global__ void __launch_bounds__(kThreads, 2) prefix_kernel(const PrefixArgs a)
       tmem_st32(t_pl + lane_off, wl);
       tmem_wait_st();
     }
+    cp_async_wait<0>();                                           // tile k + 1
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor core
     tc_fence_before();
-    __syncthreads();  // P stored, O scaled
+    __syncthreads();  // P stored, O scaled, S(k) read by all, tile k + 1 staged
     tc_fence_after();
-
-    // ---- O += P V (hi and lo halves of P, A from tensor memory: 8 columns
-    // per 16 tokens)
     if (tid == 0) {
-      const uint32_t v0 = sbase + L::kStageOff + st * 2 * L::kKVBytes + L::kKVBytes;
-#pragma unroll
-      for (int kk = 0; kk < kTileTok / 16; ++kk) {
-        const uint64_t dv = smem_desc(v0 + kk * 2048, kTileTok * 128, 1024);
-        umma_bf16_ts(t_o, t_ph + kk * 8, dv, instr_desc(D, true), k > 0 || kk > 0);
-        umma_bf16_ts(t_o, t_pl + kk * 8, dv, instr_desc(D, true), 1);
+      issue_pv(st, k == 0);
+      if (k + 1 < ntl) {
+        issue_s(st ^ 1);
+        umma_commit(bar_s);
+      } else {
+        umma_commit(bar_pv);
       }
-      umma_commit(bar_pv);
     }
   }
   cp_async_wait<0>();
 
   // ---- normalise and write this split's partial for row tid
-  if (ntl > 0) ok_waits &= mbar_wait(bar_pv, (ntl - 1) & 1);
+  if (ntl > 0) ok_waits &= mbar_wait(bar_pv, 0);  // the one commit of the last PV
   tc_fence_after();
   const size_t R = (size_t)a.B * a.hq;
   const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
