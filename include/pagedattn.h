@@ -299,6 +299,62 @@ pa_status_t pa_decode_noalloc(const pa_kv_pool_t *pool, const void *q,
                               void *stream);
 
 /*
+ * pa_decode_range — Eq. (1) restricted to a token range, returned as a
+ * normalised partial and its log-sum-exp, for merging with other ranges
+ * (e.g. the context-parallel decode of a sequence whose pages are spread over
+ * several GPUs: each GPU decodes its range, the partials are all-gathered and
+ * merged with pa_merge_partials).
+ * Every sequence b attends tokens [tok_begin, min(context_lens[b], tok_end));
+ * a sequence with no token there gets o = 0, lse = -inf (not an error).
+ *   tok_begin, tok_end : tok_begin a multiple of the page size, tok_end >=
+ *                        tok_begin; table entries outside the range's pages
+ *                        are not read
+ *   o_out   : (device) fp32 [num_seqs][num_q_heads][head_dim], the range's
+ *             attention output normalised by the range's own softmax sum
+ *   lse_out : (device) fp32 [num_seqs][num_q_heads], natural log of the sum
+ *             of exp(scale * q.k) over the range
+ *   workspace : >= pa_decode_range_workspace_bytes(...) bytes, 256-byte
+ *               aligned, zero-filled before first use (NULL when that is 0)
+ * Other arguments as for pa_decode (fixed split partition over the range's
+ * pages); one launch, or two when the range is split.
+ */
+size_t pa_decode_range_workspace_bytes(const pa_kv_pool_t *pool, int32_t num_seqs,
+                                       int32_t num_q_heads, int32_t max_pages,
+                                       int32_t tok_begin, int32_t tok_end,
+                                       int32_t num_splits);
+
+pa_status_t pa_decode_range(const pa_kv_pool_t *pool, const void *q,
+                            int32_t num_seqs, int32_t num_q_heads,
+                            const int32_t *block_tables, int32_t max_pages,
+                            const int32_t *context_lens, int32_t tok_begin,
+                            int32_t tok_end, float scale, float *o_out,
+                            float *lse_out, void *workspace,
+                            size_t workspace_bytes, int32_t num_splits,
+                            int32_t *d_err, void *stream);
+
+/*
+ * pa_merge_partials — merge num_parts partial results of disjoint token
+ * ranges, laid out part-major (what an all-gather of pa_decode_range outputs
+ * produces), with the same weights as pa_splitkv_reduce, in part order.
+ *   o_parts   : (device) fp32; part p is [rows][head_dim] at
+ *               o_parts + p * o_part_stride, normalised
+ *   lse_parts : (device) fp32; part p is [rows] at
+ *               lse_parts + p * lse_part_stride, natural log
+ *   o_part_stride, lse_part_stride : floats between parts; 0 = dense
+ *               (rows * head_dim, rows). One all-gathered buffer holding
+ *               each rank's o and lse back to back is read in place with
+ *               both strides set to that buffer's per-rank size. Parts must
+ *               not overlap; o_part_stride a multiple of 4.
+ *   out       : (device) fp32 [rows][head_dim]
+ *   lse_out   : (device) fp32 [rows], the merged log-sum-exp, or NULL
+ * head_dim a multiple of 4 and at most 512. One launch.
+ */
+pa_status_t pa_merge_partials(const float *o_parts, const float *lse_parts,
+                              int32_t num_parts, int32_t rows, int32_t head_dim,
+                              int64_t o_part_stride, int64_t lse_part_stride,
+                              float *out, float *lse_out, void *stream);
+
+/*
  * pa_splitkv_reduce — merge split-KV partial results.
  * (Not on the pages: the exact identity for softmax over disjoint token
  * ranges. With M = max_s lse_s and w_s = exp(lse_s - M):

@@ -41,6 +41,7 @@ from ._lib import (PA_DERR_BAD_CTX, PA_DERR_BAD_PAGE, PA_DERR_BAD_POS, PA_DERR_B
 __all__ = ["KVPool", "pa_kv_append", "pa_decode", "pa_decode_noalloc", "pa_splitkv_reduce",
            "pa_decode_shared_prefix", "pa_decode_shared_prefix_workspace_bytes",
            "pa_decode_window", "pa_decode_window_workspace_bytes",
+           "pa_decode_range", "pa_decode_range_workspace_bytes", "pa_merge_partials",
            "pa_validate_tables",
            "pa_decode_num_splits", "pa_decode_workspace_bytes", "PagedAttnError",
            "PA_KV_BF16", "PA_KV_U8_PER_TOKEN", "PA_KV_FP8_PER_TOKEN", "PA_KV_U4_PER_TOKEN",
@@ -301,6 +302,82 @@ def pa_splitkv_reduce(o_part: torch.Tensor, lse: torch.Tensor,
                                        _stream(stream))
     _lib.check(st, "pa_splitkv_reduce")
     return out
+
+
+def pa_decode_range_workspace_bytes(pool: KVPool, num_seqs: int, num_q_heads: int,
+                                    max_pages: int, tok_begin: int, tok_end: int,
+                                    num_splits: int = 0) -> int:
+    return int(_lib.load().pa_decode_range_workspace_bytes(
+        ctypes.byref(pool.c), num_seqs, num_q_heads, max_pages, tok_begin, tok_end, num_splits))
+
+
+def pa_decode_range(pool: KVPool, q: torch.Tensor, block_tables: torch.Tensor,
+                    context_lens: torch.Tensor, scale: float, tok_begin: int, tok_end: int,
+                    o_out: Optional[torch.Tensor] = None, lse_out: Optional[torch.Tensor] = None,
+                    workspace: Optional[torch.Tensor] = None, num_splits: int = 0,
+                    d_err: Optional[torch.Tensor] = None, stream=None):
+    """Attention over tokens [tok_begin, min(ctx, tok_end)) of every sequence:
+    returns (o [B, Hq, D] normalised over the range, lse [B, Hq] natural log)."""
+    dev = pool.device
+    _need(q, "q", torch.bfloat16, dev)
+    _need(block_tables, "block_tables", torch.int32, dev)
+    _need(context_lens, "context_lens", torch.int32, dev)
+    B, Hq, D = q.shape
+    if D != pool.head_dim or block_tables.shape[0] != B or context_lens.numel() != B:
+        raise ValueError("pa_decode_range: shape mismatch")
+    if o_out is None:
+        o_out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    if lse_out is None:
+        lse_out = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    _need(o_out, "o_out", torch.float32, dev)
+    _need(lse_out, "lse_out", torch.float32, dev)
+    if tuple(o_out.shape) != (B, Hq, D) or tuple(lse_out.shape) != (B, Hq):
+        raise ValueError("pa_decode_range: o_out must be [B, Hq, D] and lse_out [B, Hq]")
+    max_pages = block_tables.shape[1]
+    if workspace is None:
+        need = pa_decode_range_workspace_bytes(pool, B, Hq, max_pages, tok_begin, tok_end,
+                                               num_splits)
+        if need > 0:
+            workspace = torch.zeros(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _lib.load().pa_decode_range(
+        ctypes.byref(pool.c), _ptr(q), B, Hq, _ptr(block_tables), max_pages, _ptr(context_lens),
+        int(tok_begin), int(tok_end), float(scale), _ptr(o_out), _ptr(lse_out), _ptr(workspace),
+        ws_bytes, num_splits, _ptr(d_err), _stream(stream))
+    _lib.check(st, "pa_decode_range")
+    return o_out, lse_out
+
+
+def pa_merge_partials(o_parts: torch.Tensor, lse_parts: torch.Tensor,
+                      out: Optional[torch.Tensor] = None,
+                      lse_out: Optional[torch.Tensor] = None, stream=None):
+    """Merge part-major partials o_parts [n, ..., D], lse_parts [n, ...] ->
+    (out [..., D], lse [...]) (log-sum-exp weights, in part order). Each part
+    must be contiguous; the parts themselves may sit at any stride (e.g.
+    views into one all-gathered buffer)."""
+    for t, name in ((o_parts, "o_parts"), (lse_parts, "lse_parts")):
+        if t.dtype != torch.float32:
+            raise TypeError(f"{name} must be torch.float32, got {t.dtype}")
+        if t.dim() < 2 or not t[0].is_contiguous() or t.stride(0) < t[0].numel():
+            raise ValueError(f"{name}: every part must be contiguous and the parts disjoint")
+    if lse_parts.device != o_parts.device:
+        raise ValueError("lse_parts must be on the device of o_parts")
+    n, D = o_parts.shape[0], o_parts.shape[-1]
+    rows = lse_parts[0].numel()
+    if lse_parts.shape[0] != n or o_parts[0].numel() != rows * D:
+        raise ValueError("pa_merge_partials: shape mismatch")
+    if out is None:
+        out = torch.empty(o_parts.shape[1:], dtype=torch.float32, device=o_parts.device)
+    if lse_out is None:
+        lse_out = torch.empty(lse_parts.shape[1:], dtype=torch.float32, device=o_parts.device)
+    _need(out, "out", torch.float32, o_parts.device)
+    _need(lse_out, "lse_out", torch.float32, o_parts.device)
+    st = _lib.load().pa_merge_partials(_ptr(o_parts), _ptr(lse_parts), n, rows, D,
+                                       o_parts.stride(0) if n > 1 else 0,
+                                       lse_parts.stride(0) if n > 1 else 0, _ptr(out),
+                                       _ptr(lse_out), _stream(stream))
+    _lib.check(st, "pa_merge_partials")
+    return out, lse_out
 
 
 def pa_validate_tables(block_tables: torch.Tensor, context_lens: torch.Tensor, num_pages: int,

@@ -65,6 +65,11 @@ SIGNATURES = {
     "pa_decode_window": (_I, [_POOL, _P, _I, _I, _P, _I, _P, _I, _I, ctypes.c_float, _P, _P,
                               ctypes.c_size_t, _I, _P, _P]),
     "pa_decode_noalloc": (_I, [_POOL, _P, _I, _I, _P, _I, _P, ctypes.c_float, _P, _I, _P, _P]),
+    "pa_decode_range_workspace_bytes": (ctypes.c_size_t, [_POOL, _I, _I, _I, _I, _I, _I]),
+    "pa_decode_range": (_I, [_POOL, _P, _I, _I, _P, _I, _P, _I, _I, ctypes.c_float, _P, _P, _P,
+                             ctypes.c_size_t, _I, _P, _P]),
+    "pa_merge_partials": (_I, [_P, _P, _I, _I, _I, ctypes.c_int64, ctypes.c_int64, _P, _P,
+                                _P]),
     "pa_splitkv_reduce": (_I, [_P, _P, _I, _I, _I, _I, _P, _P]),
     "pa_validate_tables": (_I, [_P, _I, _I, _P, _I, _I, _P, _P]),
     "pa_status_str": (ctypes.c_char_p, [_I]),

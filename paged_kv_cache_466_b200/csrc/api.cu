@@ -267,6 +267,8 @@ pa_status_t pa_decode(const pa_kv_pool_t *pool, const void *q, int32_t num_seqs,
   a.prior_lse = nullptr;
   a.n_prior = 0;
   a.keep_partials = 0;
+  a.tok_end = 0x7fffffff;
+  a.range_mode = 0;
   a.d_err = d_err;
   return cuda_status(launch_decode(pool->head_dim, pool->page_size, pool->dtype, a,
                                    static_cast<cudaStream_t>(stream)),
@@ -427,6 +429,8 @@ pa_status_t pa_decode_shared_prefix(const pa_kv_pool_t *pool, const void *q, int
   a.prior_lse = nullptr;
   a.n_prior = 0;
   a.keep_partials = 1;
+  a.tok_end = 0x7fffffff;
+  a.range_mode = 0;
   st = cuda_status(launch_prefix(pool->head_dim, pool->page_size, pa, true, s),
                    "pa_decode_shared_prefix prefix launch");
   if (st == PA_OK)
@@ -437,6 +441,152 @@ pa_status_t pa_decode_shared_prefix(const pa_kv_pool_t *pool, const void *q, int
                                            pool->head_dim, out, true, s, pa.o_pre, pa.lse_pre,
                                            pl.n_psplits),
                      "pa_decode_shared_prefix merge launch");
+}
+
+// ---------------------------------------------------------------- token ranges
+namespace {
+
+// Splits and partial slots of pa_decode_range: the range's logical pages
+// [tok_begin / P, ceil(min(tok_end, max_pages * P) / P)) split like a decode.
+int range_splits(const pa_kv_pool_t *pool, int B, int max_pages, int tok_begin, int tok_end,
+                 int num_splits) {
+  const int P = pool->page_size;
+  const long long end = std::min<long long>(tok_end, (long long)max_pages * P);
+  const int pages = (int)((end + P - 1) / P) - tok_begin / P;
+  return pa_decode_num_splits(pool, B, pages < 1 ? 1 : pages, num_splits);
+}
+
+}  // namespace
+
+size_t pa_decode_range_workspace_bytes(const pa_kv_pool_t *pool, int32_t num_seqs,
+                                       int32_t num_q_heads, int32_t max_pages, int32_t tok_begin,
+                                       int32_t tok_end, int32_t num_splits) {
+  if (pool == nullptr || num_seqs <= 0 || num_q_heads <= 0 || max_pages <= 0 || tok_begin < 0 ||
+      tok_end < tok_begin || num_splits < 0 || pool->page_size <= 0)
+    return 0;
+  const int S = range_splits(pool, num_seqs, max_pages, tok_begin, tok_end, num_splits);
+  return S > 1 ? pa_decode_workspace_bytes(num_seqs, num_q_heads, pool->head_dim, S) : 0;
+}
+
+pa_status_t pa_decode_range(const pa_kv_pool_t *pool, const void *q, int32_t num_seqs,
+                            int32_t num_q_heads, const int32_t *block_tables, int32_t max_pages,
+                            const int32_t *context_lens, int32_t tok_begin, int32_t tok_end,
+                            float scale, float *o_out, float *lse_out, void *workspace,
+                            size_t workspace_bytes, int32_t num_splits, int32_t *d_err,
+                            void *stream) {
+  g_last_error.clear();
+  pa_status_t st = check_pool(pool);
+  if (st != PA_OK) return st;
+  if (num_seqs < 0 || num_q_heads <= 0 || max_pages <= 0 || num_splits < 0)
+    return fail(PA_ERR_INVALID_ARG, "num_seqs=%d num_q_heads=%d max_pages=%d num_splits=%d",
+                num_seqs, num_q_heads, max_pages, num_splits);
+  if (tok_begin < 0 || tok_end < tok_begin || tok_begin % pool->page_size != 0)
+    return fail(PA_ERR_INVALID_ARG,
+                "token range [%d, %d) must start on a page boundary and not be reversed",
+                tok_begin, tok_end);
+  if (tok_begin >= max_pages * pool->page_size && tok_end > tok_begin)
+    return fail(PA_ERR_INVALID_ARG, "tok_begin=%d is past the tables' %d pages", tok_begin,
+                max_pages);
+  if (num_q_heads % pool->num_kv_heads != 0)
+    return fail(PA_ERR_INVALID_ARG, "num_q_heads=%d is not a multiple of num_kv_heads=%d",
+                num_q_heads, pool->num_kv_heads);
+  const int G = num_q_heads / pool->num_kv_heads;
+  if (G > kMaxGroup)
+    return fail(PA_ERR_UNSUPPORTED, "GQA group %d > %d query heads per KV head", G, kMaxGroup);
+  if (num_seqs > 65535 || (long long)max_pages * pool->page_size > (1LL << 30))
+    return fail(PA_ERR_UNSUPPORTED, "too many sequences or pages");
+  if (!(scale == scale)) return fail(PA_ERR_INVALID_ARG, "scale is NaN");
+  if (num_seqs == 0) return PA_OK;
+  if (!q || !block_tables || !context_lens || !o_out || !lse_out)
+    return fail(PA_ERR_INVALID_ARG, "q, block_tables, context_lens, o_out and lse_out are required");
+  if (!aligned(q, 16) || !aligned(o_out, 16) || !aligned(lse_out, 4))
+    return fail(PA_ERR_INVALID_ARG, "q and o_out must be 16-byte aligned");
+  if (tok_begin >= max_pages * pool->page_size) tok_begin = tok_end = 0;  // empty range
+  const int S = range_splits(pool, num_seqs, max_pages, tok_begin, tok_end, num_splits);
+  if (S <= 0) return fail(PA_ERR_INVALID_ARG, "could not plan splits");
+  const size_t need = S > 1 ? pa_decode_workspace_bytes(num_seqs, num_q_heads, pool->head_dim, S)
+                            : 0;
+  if (need > 0) {
+    if (workspace == nullptr || workspace_bytes < need)
+      return fail(PA_ERR_WORKSPACE, "workspace: need %zu bytes for %d splits, got %zu", need, S,
+                  workspace == nullptr ? (size_t)0 : workspace_bytes);
+    if (!aligned(workspace, 256)) return fail(PA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  }
+  const int P = pool->page_size;
+  const long long end = std::min<long long>(tok_end, (long long)max_pages * P);
+  const int pages = std::max(1, (int)((end + P - 1) / P) - tok_begin / P);
+  const size_t rows = (size_t)num_seqs * num_q_heads;
+  DecodeArgs a;
+  a.k_pool = pool->k_pool;
+  a.v_pool = pool->v_pool;
+  a.k_sz = pool->k_sz;
+  a.v_sz = pool->v_sz;
+  a.num_pages = pool->num_pages;
+  a.hkv = pool->num_kv_heads;
+  a.q = q;
+  a.B = num_seqs;
+  a.hq = num_q_heads;
+  a.block_tables = block_tables;
+  a.max_pages = max_pages;
+  a.ctx = context_lens;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.out = o_out;
+  // one split writes o_out / lse_out directly ([row][1][D] is [row][D])
+  const size_t o_bytes = align256(rows * S * pool->head_dim * sizeof(float));
+  const size_t l_bytes = align256(rows * S * sizeof(float));
+  a.o_part = S > 1 ? static_cast<float *>(workspace) : o_out;
+  a.lse = S > 1 ? reinterpret_cast<float *>(static_cast<char *>(workspace) + o_bytes) : lse_out;
+  a.counters = S > 1 ? reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + o_bytes +
+                                                   l_bytes)
+                     : nullptr;
+  a.S = S;
+  a.S_main = S;
+  a.pages_per_split = (pages + S - 1) / S;
+  a.tbl_cap = a.pages_per_split;
+  a.window = 0;
+  a.sinks = 0;
+  a.tok_begin = tok_begin;
+  a.prior_o = nullptr;
+  a.prior_lse = nullptr;
+  a.n_prior = 0;
+  a.keep_partials = 1;
+  a.tok_end = tok_end;
+  a.range_mode = 1;
+  a.d_err = d_err;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = cuda_status(launch_decode(pool->head_dim, P, pool->dtype, a, s), "pa_decode_range launch");
+  if (st != PA_OK || S == 1) return st;
+  return cuda_status(launch_splitkv_reduce(a.o_part, a.lse, num_seqs, num_q_heads, S,
+                                           pool->head_dim, o_out, true, s, nullptr, nullptr, 0,
+                                           lse_out),
+                     "pa_decode_range merge launch");
+}
+
+pa_status_t pa_merge_partials(const float *o_parts, const float *lse_parts, int32_t num_parts,
+                              int32_t rows, int32_t head_dim, int64_t o_part_stride,
+                              int64_t lse_part_stride, float *out, float *lse_out,
+                              void *stream) {
+  g_last_error.clear();
+  if (num_parts < 1 || rows < 0 || head_dim <= 0 || head_dim % 4 != 0 || head_dim > 512)
+    return fail(PA_ERR_INVALID_ARG, "num_parts=%d rows=%d head_dim=%d", num_parts, rows,
+                head_dim);
+  if (o_part_stride == 0) o_part_stride = (int64_t)rows * head_dim;
+  if (lse_part_stride == 0) lse_part_stride = rows;
+  if (num_parts > 1 && (o_part_stride < (int64_t)rows * head_dim || o_part_stride % 4 != 0 ||
+                        lse_part_stride < rows))
+    return fail(PA_ERR_INVALID_ARG,
+                "part strides %lld / %lld: parts overlap or break 16-byte alignment",
+                (long long)o_part_stride, (long long)lse_part_stride);
+  if (rows == 0) return PA_OK;
+  if (!o_parts || !lse_parts || !out)
+    return fail(PA_ERR_INVALID_ARG, "o_parts, lse_parts and out are required");
+  if (!aligned(o_parts, 16) || !aligned(out, 16))
+    return fail(PA_ERR_INVALID_ARG, "o_parts and out must be 16-byte aligned");
+  return cuda_status(launch_splitkv_reduce(nullptr, nullptr, rows, 1, 0, head_dim, out, true,
+                                           static_cast<cudaStream_t>(stream), o_parts, lse_parts,
+                                           num_parts, lse_out, (size_t)o_part_stride,
+                                           (size_t)lse_part_stride),
+                     "pa_merge_partials launch");
 }
 
 pa_status_t pa_splitkv_reduce(const float *o_part, const float *lse, int32_t num_seqs,
@@ -589,6 +739,8 @@ pa_status_t pa_decode_window(const pa_kv_pool_t *pool, const void *q, int32_t nu
   a.prior_lse = nullptr;
   a.n_prior = 0;
   a.keep_partials = 0;
+  a.tok_end = 0x7fffffff;
+  a.range_mode = 0;
   a.d_err = d_err;
   return cuda_status(launch_decode(pool->head_dim, pool->page_size, pool->dtype, a,
                                    static_cast<cudaStream_t>(stream)),

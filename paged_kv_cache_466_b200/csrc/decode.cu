@@ -632,9 +632,10 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
     if (threadIdx.x == 0) flag_error(a.d_err, PA_DERR_BAD_CTX);
     ctx = a.tok_begin;
   } else if (ctx < a.tok_begin) {
-    if (threadIdx.x == 0) flag_error(a.d_err, PA_DERR_BAD_CTX);
+    if (threadIdx.x == 0 && !a.range_mode) flag_error(a.d_err, PA_DERR_BAD_CTX);
     ctx = a.tok_begin;
   }
+  ctx = min(ctx, max(a.tok_end, a.tok_begin));
   int mlo = a.tok_begin;
   int sink_hi = 0;
   if (a.window > 0) {
@@ -672,9 +673,12 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
   const int tok1 = tok_hi;
 
   if (nblk == 0) {
-    if (a.keep_partials) {  // an empty partial: weight 0 in the caller's merge
-      for (int hd = threadIdx.x; hd < G; hd += W * 32)
-        a.lse[((size_t)b * a.hq + (size_t)h * G + hd) * a.S + slot] = -INFINITY;
+    if (a.keep_partials) {  // an empty partial: o = 0, lse = -inf (weight 0)
+      for (int e = threadIdx.x; e < G * D; e += W * 32) {
+        const size_t row = (size_t)b * a.hq + (size_t)h * G + e / D;
+        a.o_part[(row * a.S + slot) * D + e % D] = 0.f;
+        if (e % D == 0) a.lse[row * a.S + slot] = -INFINITY;
+      }
       return;
     }
     if (split == 0 && n_live == 0) {

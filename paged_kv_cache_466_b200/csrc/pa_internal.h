@@ -45,8 +45,11 @@ struct DecodeArgs {
   const float *prior_o;     // [n_prior][B*Hq][D] partials merged into the output
   const float *prior_lse;   // [n_prior][B*Hq]
   int32_t n_prior;
-  int32_t keep_partials;    // 1: every split writes its partial (an empty one lse = -inf)
-                            //    to its slot and nothing is merged
+  int32_t keep_partials;    // 1: every split writes its partial (an empty one o = 0,
+                            //    lse = -inf) to its slot and nothing is merged
+  int32_t tok_end;          // attend tokens below min(ctx, tok_end) only
+  int32_t range_mode;       // 1: a context shorter than tok_begin is an empty range,
+                            //    not an error
   int32_t *d_err;
 };
 
@@ -84,7 +87,9 @@ cudaError_t launch_splitkv_reduce(const float *o_part, const float *lse, int B,
                                   int hq, int S, int D, float *out,
                                   bool programmatic, cudaStream_t stream,
                                   const float *prior_o = nullptr,
-                                  const float *prior_lse = nullptr, int n_prior = 0);
+                                  const float *prior_lse = nullptr, int n_prior = 0,
+                                  float *lse_out = nullptr, size_t prior_o_stride = 0,
+                                  size_t prior_lse_stride = 0);
 
 cudaError_t launch_kv_append(const pa_kv_pool_t &pool, const void *k_new,
                              const void *v_new, const int32_t *seq_idx,

@@ -17,11 +17,13 @@ namespace {
 constexpr int kWarps = 4;
 
 // Partials i < S are the row's own (o_part[row][i], lse[row][i]); i >= S are
-// prior partials p = i - S (prior_o[p][row], prior_lse[p][row]).
+// prior partials p = i - S (prior_o + p * po_stride + row * D,
+// prior_lse[p * pl_stride + row]); the strides are in floats.
 __global__ void __launch_bounds__(kWarps * 32) splitkv_reduce_kernel(
     const float *__restrict__ o_part, const float *__restrict__ lse, int rows, int S, int D,
     float *__restrict__ out, const float *__restrict__ prior_o,
-    const float *__restrict__ prior_lse, int n_prior) {
+    const float *__restrict__ prior_lse, int n_prior, size_t po_stride, size_t pl_stride,
+    float *__restrict__ lse_out) {
   pdl_wait_primary();  // partials come from the kernel just before us
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -29,7 +31,7 @@ __global__ void __launch_bounds__(kWarps * 32) splitkv_reduce_kernel(
   if (row >= rows) return;
   const int n_all = S + n_prior;
   const float *ls = lse + (size_t)row * S;
-  auto lse_at = [&](int i) { return i < S ? ls[i] : prior_lse[(size_t)(i - S) * rows + row]; };
+  auto lse_at = [&](int i) { return i < S ? ls[i] : prior_lse[(size_t)(i - S) * pl_stride + row]; };
   float M = -INFINITY;
   for (int s = lane; s < n_all; s += 32) M = fmaxf(M, lse_at(s));
 #pragma unroll
@@ -38,7 +40,8 @@ __global__ void __launch_bounds__(kWarps * 32) splitkv_reduce_kernel(
   const float4 *op = reinterpret_cast<const float4 *>(o_part + (size_t)row * S * D);
   auto o_at = [&](int i) {
     return i < S ? op + (size_t)i * D4
-                 : reinterpret_cast<const float4 *>(prior_o + ((size_t)(i - S) * rows + row) * D);
+                 : reinterpret_cast<const float4 *>(prior_o + (size_t)(i - S) * po_stride +
+                                                    (size_t)row * D);
   };
   float4 *dst = reinterpret_cast<float4 *>(out + (size_t)row * D);
   for (int i0 = 0; i0 < D4; i0 += 32) {
@@ -77,6 +80,9 @@ __global__ void __launch_bounds__(kWarps * 32) splitkv_reduce_kernel(
       const float r = den > 0.f ? 1.f / den : 0.f;
       dst[i] = make_float4(acc.x * r, acc.y * r, acc.z * r, acc.w * r);
     }
+    // the merged log-sum-exp: M + ln(sum_s exp(lse_s - M))
+    if (lse_out != nullptr && i0 == 0 && lane == 0)
+      lse_out[row] = den > 0.f ? M + logf(den) : -INFINITY;
   }
 }
 
@@ -84,8 +90,12 @@ __global__ void __launch_bounds__(kWarps * 32) splitkv_reduce_kernel(
 
 cudaError_t launch_splitkv_reduce(const float *o_part, const float *lse, int B, int hq, int S,
                                   int D, float *out, bool programmatic, cudaStream_t stream,
-                                  const float *prior_o, const float *prior_lse, int n_prior) {
+                                  const float *prior_o, const float *prior_lse, int n_prior,
+                                  float *lse_out, size_t prior_o_stride,
+                                  size_t prior_lse_stride) {
   const int rows = B * hq;
+  if (prior_o_stride == 0) prior_o_stride = (size_t)rows * D;
+  if (prior_lse_stride == 0) prior_lse_stride = (size_t)rows;
   if (rows == 0) return cudaSuccess;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((rows + kWarps - 1) / kWarps);
@@ -98,7 +108,7 @@ cudaError_t launch_splitkv_reduce(const float *o_part, const float *lse, int B, 
   cfg.attrs = attr;
   cfg.numAttrs = programmatic ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, splitkv_reduce_kernel, o_part, lse, rows, S, D, out, prior_o,
-                            prior_lse, n_prior);
+                            prior_lse, n_prior, prior_o_stride, prior_lse_stride, lse_out);
 }
 
 }  // namespace pa

@@ -55,3 +55,86 @@ def test_two_rank_timing_and_shards():
 def test_single_rank_passthrough():
     assert bench.max_over_ranks(4.25, 1) == 4.25
     assert bench.whole_job_gbs(2_000_000_000, 1, 1.0) == pytest.approx(2000.0)
+
+
+def _cp_worker(rank, world, port, q):
+    """One rank of a context-parallel decode with the oracle standing in for
+    pa_decode_range: partial over this rank's token range, written into this
+    rank's block of the packed layout decode_context_parallel gathers, one
+    all-gather, merge of the strided views."""
+    import oracle
+    from paged_kv_cache_466_b200 import workloads as W
+    from paged_kv_cache_466_b200.context_parallel import (gathered_views, partial_block_floats,
+                                                           partial_views, rank_range)
+    from paged_kv_cache_466_b200.workloads import bits
+    from tests.helpers import oracle_pool
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = W.paged("cp", B=3, Hq=4, Hkv=2, D=64, P=16, context_lens=[5, 70, 200], kv="bf16")
+        hp = oracle_pool(w)
+        b, e = rank_range(rank, world, 64)
+        o, lse = oracle.paged_attention(hp, bits(w.q), w.block_tables, w.context_lens, w.scale,
+                                        t_begin=b, t_end=e if e < 0x7FFFFFFF else -1)
+        block = torch.full((partial_block_floats(w.B, w.Hq, w.D),), float("nan"))
+        ov, lv = partial_views(block, w.B, w.Hq, w.D)
+        ov.copy_(torch.from_numpy(o).view(w.B, w.Hq, w.D))
+        lv.copy_(torch.from_numpy(lse).view(w.B, w.Hq))
+        gathered = torch.empty(world * block.numel())
+        dist.all_gather_into_tensor(gathered, block)
+        o_parts, l_parts = gathered_views(gathered, world, w.B, w.Hq, w.D)
+        merged = oracle.lse_merge(o_parts.double().numpy().reshape(world, -1, w.D).transpose(1, 0, 2),
+                                  l_parts.double().numpy().reshape(world, -1).T)
+        full, _ = oracle.paged_attention(hp, bits(w.q), w.block_tables, w.context_lens, w.scale)
+        # fp32 partials: the merge of the rounded parts is within fp32 rounding of Eq. 1
+        q.put((rank, float(np.abs(merged - full).max())))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_context_parallel_ranges_merge_to_the_full_decode():
+    """Three gloo ranks, 64 tokens each (the last one open-ended): the merged
+    range partials equal Eq. 1 over the whole contexts, which shows that the
+    ranges cover every token once and that the part-major gather is merged
+    with the right weights."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_cp_worker, args=(r, 3, port, q)) for r in range(3)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=180) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for _, err in res:
+        assert err <= 1e-6
+
+
+def test_rank_ranges():
+    from paged_kv_cache_466_b200.context_parallel import rank_range
+    assert [rank_range(r, 3, 32) for r in range(3)] == [(0, 32), (32, 64), (64, 0x7FFFFFFF)]
+    assert rank_range(0, 1, 16) == (0, 0x7FFFFFFF)
+    with pytest.raises(ValueError):
+        rank_range(3, 3, 32)
+
+
+def test_packed_partial_layout():
+    """Each rank's block holds o then lse, 256-byte aligned; the gathered
+    views see rank r's values in part r."""
+    from paged_kv_cache_466_b200.context_parallel import (gathered_views, partial_block_floats,
+                                                           partial_views)
+    B, Hq, D, world = 3, 5, 12, 4
+    n = partial_block_floats(B, Hq, D)
+    assert n % 64 == 0 and n >= B * Hq * (D + 1)
+    gathered = torch.zeros(world * n)
+    for r in range(world):
+        o, lse = partial_views(gathered[r * n:(r + 1) * n], B, Hq, D)
+        o.copy_(torch.arange(B * Hq * D, dtype=torch.float32).view(B, Hq, D) + 1000 * r)
+        lse.copy_(torch.arange(B * Hq, dtype=torch.float32).view(B, Hq) - 1000 * r)
+    o_parts, l_parts = gathered_views(gathered, world, B, Hq, D)
+    assert o_parts.shape == (world, B, Hq, D) and l_parts.shape == (world, B, Hq)
+    assert o_parts.stride(0) == n and l_parts.stride(0) == n and o_parts[0].is_contiguous()
+    for r in range(world):
+        assert torch.equal(o_parts[r].flatten(), torch.arange(B * Hq * D, dtype=torch.float32) + 1000 * r)
+        assert torch.equal(l_parts[r].flatten(), torch.arange(B * Hq, dtype=torch.float32) - 1000 * r)
