@@ -258,7 +258,8 @@ def run_ours(args, rank, world, local_rank):
                                          pa_decode_shared_prefix,
                                          pa_decode_shared_prefix_workspace_bytes,
                                          pa_decode_window, pa_decode_window_workspace_bytes,
-                                         pa_decode_workspace_bytes, pa_kv_append)
+                                         pa_decode_workspace_bytes, pa_kv_append,
+                                         StepPacket, pa_decode_step_host)
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -348,20 +349,35 @@ def run_ours(args, rank, world, local_rank):
     h_ctx = torch.from_numpy(w.context_lens).pin_memory()
     h_bt = torch.from_numpy(w.block_tables).pin_memory()
     h_out = torch.empty((w.B, w.Hq, w.D), dtype=torch.float32).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_seq, h_pos, h_ctx, h_bt))
     d2h = h_out.numel() * h_out.element_size()
-    d_q, d_k, d_v = torch.empty_like(q), torch.empty_like(sk), torch.empty_like(sv)
-    d_seq, d_pos = torch.empty_like(sseq), torch.empty_like(spos)
-    d_ctx, d_bt = torch.empty_like(ctx), torch.empty_like(bt)
+    if not args.cascade and args.window == 0:
+        # the library's host-packet step: one H2D copy of the packed inputs,
+        # append, decode and one D2H copy of the output, in one C-ABI call
+        packet = StepPacket(pool, w.B, w.Hq, w.max_pages, len(w.step_seq))
+        for view, h in ((packet.q, h_q), (packet.k_new, h_k), (packet.v_new, h_v),
+                        (packet.seq_idx, h_seq), (packet.pos, h_pos),
+                        (packet.context_lens, h_ctx), (packet.block_tables, h_bt)):
+            view.copy_(h)
+        h2d = packet.nbytes
 
-    def e2e_step():
-        for d, h in ((d_q, h_q), (d_k, h_k), (d_v, h_v), (d_seq, h_seq), (d_pos, h_pos),
-                     (d_ctx, h_ctx), (d_bt, h_bt)):
-            d.copy_(h, non_blocking=True)
-        pa_kv_append(pool, d_k, d_v, d_seq, d_pos, d_bt)
-        decode(d_q, d_bt, d_ctx)
-        h_out.copy_(out, non_blocking=True)
-        stream.synchronize()   # the caller reads the result every step
+        def e2e_step():
+            pa_decode_step_host(pool, packet, w.scale, h_out, out_dev=out, workspace=ws,
+                                num_splits=S, stream=stream, synchronize=True)
+    else:
+        h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_seq, h_pos, h_ctx,
+                                                         h_bt))
+        d_q, d_k, d_v = torch.empty_like(q), torch.empty_like(sk), torch.empty_like(sv)
+        d_seq, d_pos = torch.empty_like(sseq), torch.empty_like(spos)
+        d_ctx, d_bt = torch.empty_like(ctx), torch.empty_like(bt)
+
+        def e2e_step():
+            for d, h in ((d_q, h_q), (d_k, h_k), (d_v, h_v), (d_seq, h_seq), (d_pos, h_pos),
+                         (d_ctx, h_ctx), (d_bt, h_bt)):
+                d.copy_(h, non_blocking=True)
+            pa_kv_append(pool, d_k, d_v, d_seq, d_pos, d_bt)
+            decode(d_q, d_bt, d_ctx)
+            h_out.copy_(out, non_blocking=True)
+            stream.synchronize()   # the caller reads the result every step
 
     for _ in range(max(args.warmup, 3)):
         e2e_step()

@@ -384,6 +384,57 @@ pa_status_t pa_validate_tables(const int32_t *block_tables, int32_t num_seqs,
                                int32_t num_pages, int32_t page_size,
                                int32_t *d_err, void *stream);
 
+/*
+ * One decode step end to end from host memory: the step's inputs cross to the
+ * device as ONE packet (one host-to-device copy), the new K/V rows are written
+ * (pa_kv_append), Eq. (1) is decoded (pa_decode) and the output comes back
+ * (one device-to-host copy), all in stream order on `stream`.
+ *
+ * Packet layout: seven sections in this order, each starting on a 256-byte
+ * boundary of the packet:
+ *   0 q            bf16  [num_seqs][num_q_heads][head_dim]
+ *   1 k_new        bf16  [num_new][num_kv_heads][head_dim]
+ *   2 v_new        bf16  [num_new][num_kv_heads][head_dim]
+ *   3 seq_idx      int32 [num_new]
+ *   4 pos          int32 [num_new]
+ *   5 block_tables int32 [num_seqs][max_pages]
+ *   6 context_lens int32 [num_seqs]
+ * (the same meaning as the arguments of pa_kv_append and pa_decode).
+ *
+ * pa_step_packet_layout — host only (no device access): writes the seven
+ * section offsets in bytes to offsets[0..6] (when offsets is not NULL) and
+ * returns the packet size in bytes, or 0 on invalid arguments.
+ */
+size_t pa_step_packet_layout(const pa_kv_pool_t *pool, int32_t num_seqs,
+                             int32_t num_q_heads, int32_t max_pages,
+                             int32_t num_new, size_t *offsets);
+
+/*
+ * pa_decode_step_host — the step itself.
+ *   packet_host : (host) packet_bytes bytes laid out as above; page-locked
+ *                 memory makes the copy asynchronous (pageable memory works,
+ *                 but the copy then blocks the calling thread)
+ *   packet_dev  : (device) >= packet_bytes bytes, 256-byte aligned; the
+ *                 library copies the packet here and reads every input from it
+ *   packet_bytes: pa_step_packet_layout(...) for the same shape
+ *   out_dev     : (device) fp32 [num_seqs][num_q_heads][head_dim]
+ *   out_host    : (host) fp32, same shape; receives out_dev
+ *   workspace, workspace_bytes, num_splits, d_err : as for pa_decode
+ *   synchronize : nonzero = wait for the stream before returning, so that
+ *                 out_host holds the result when the call returns
+ * Errors: those of pa_kv_append and pa_decode, PA_ERR_INVALID_ARG for a
+ * packet_bytes that does not match the shape, PA_ERR_CUDA for a failed copy.
+ * The packet buffers may be reused by the next step once this one has
+ * completed on the stream.
+ */
+pa_status_t pa_decode_step_host(const pa_kv_pool_t *pool, const void *packet_host,
+                                void *packet_dev, size_t packet_bytes,
+                                int32_t num_seqs, int32_t num_q_heads,
+                                int32_t max_pages, int32_t num_new, float scale,
+                                float *out_dev, float *out_host, void *workspace,
+                                size_t workspace_bytes, int32_t num_splits,
+                                int32_t *d_err, void *stream, int32_t synchronize);
+
 /* Static description of a status code. */
 const char *pa_status_str(pa_status_t status);
 

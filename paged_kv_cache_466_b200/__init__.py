@@ -42,7 +42,7 @@ __all__ = ["KVPool", "pa_kv_append", "pa_decode", "pa_decode_noalloc", "pa_split
            "pa_decode_shared_prefix", "pa_decode_shared_prefix_workspace_bytes",
            "pa_decode_window", "pa_decode_window_workspace_bytes",
            "pa_decode_range", "pa_decode_range_workspace_bytes", "pa_merge_partials",
-           "pa_validate_tables",
+           "pa_validate_tables", "StepPacket", "pa_decode_step_host",
            "pa_decode_num_splits", "pa_decode_workspace_bytes", "PagedAttnError",
            "PA_KV_BF16", "PA_KV_U8_PER_TOKEN", "PA_KV_FP8_PER_TOKEN", "PA_KV_U4_PER_TOKEN",
            "PA_DERR_BAD_PAGE",
@@ -261,6 +261,82 @@ def pa_decode_window(pool: KVPool, q: torch.Tensor, block_tables: torch.Tensor,
         num_splits, _ptr(d_err), _stream(stream))
     _lib.check(st, "pa_decode_window")
     return out
+
+
+class StepPacket:
+    """The host and device buffers of one ``pa_decode_step_host`` step.
+
+    ``host`` is one page-locked byte buffer laid out by ``pa_step_packet_layout``;
+    fill its views (``q``, ``k_new``, ``v_new``, ``seq_idx``, ``pos``,
+    ``block_tables``, ``context_lens``) in place and the whole step's input
+    crosses to the device in one copy. ``dev`` is the device copy the kernels
+    read from."""
+
+    def __init__(self, pool: KVPool, num_seqs: int, num_q_heads: int, max_pages: int,
+                 num_new: int, pin: bool = True):
+        off = (ctypes.c_size_t * 7)()
+        n = int(_lib.load().pa_step_packet_layout(ctypes.byref(pool.c), num_seqs, num_q_heads,
+                                                  max_pages, num_new, off))
+        if n == 0:
+            raise ValueError("StepPacket: invalid shape")
+        self.nbytes = n
+        self.offsets = [int(o) for o in off]
+        self.shape = (num_seqs, num_q_heads, max_pages, num_new)
+        host = torch.zeros(n, dtype=torch.uint8)
+        self.host = host.pin_memory() if pin else host
+        self.dev = (torch.empty(n, dtype=torch.uint8, device=pool.device)
+                    if pool.device.type == "cuda" else None)
+        B, Hq, D, Hkv = num_seqs, num_q_heads, pool.head_dim, pool.num_kv_heads
+
+        def view(i, dtype, shape):
+            count = 1
+            for e in shape:
+                count *= e
+            nb = count * torch.empty((), dtype=dtype).element_size()
+            return self.host[self.offsets[i]:self.offsets[i] + nb].view(dtype).view(shape)
+
+        self.q = view(0, torch.bfloat16, (B, Hq, D))
+        self.k_new = view(1, torch.bfloat16, (num_new, Hkv, D))
+        self.v_new = view(2, torch.bfloat16, (num_new, Hkv, D))
+        self.seq_idx = view(3, torch.int32, (num_new,))
+        self.pos = view(4, torch.int32, (num_new,))
+        self.block_tables = view(5, torch.int32, (B, max_pages))
+        self.context_lens = view(6, torch.int32, (B,))
+
+
+def pa_decode_step_host(pool: KVPool, packet: StepPacket, scale: float, out_host: torch.Tensor,
+                        out_dev: Optional[torch.Tensor] = None,
+                        workspace: Optional[torch.Tensor] = None, num_splits: int = 0,
+                        d_err: Optional[torch.Tensor] = None, stream=None,
+                        synchronize: bool = True) -> torch.Tensor:
+    """One decode step from host memory: the packet's inputs go to the device
+    in one copy, the new rows are appended, Eq. 1 is decoded and the output is
+    copied into ``out_host`` (fp32 [B, Hq, D], pinned for an asynchronous copy);
+    with ``synchronize`` the call returns once ``out_host`` holds the result."""
+    B, Hq, max_pages, num_new = packet.shape
+    D = pool.head_dim
+    dev = pool.device
+    if packet.dev is None:
+        raise ValueError("pa_decode_step_host: the packet has no device buffer")
+    if out_host.dtype != torch.float32 or out_host.device.type != "cpu" \
+            or not out_host.is_contiguous() or tuple(out_host.shape) != (B, Hq, D):
+        raise ValueError("pa_decode_step_host: out_host must be a contiguous host fp32 [B, Hq, D]")
+    if out_dev is None:
+        out_dev = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    _need(out_dev, "out_dev", torch.float32, dev)
+    if workspace is None:
+        need = pa_decode_workspace_bytes(B, Hq, D,
+                                         pa_decode_num_splits(pool, B, max_pages, num_splits))
+        if need > 0:
+            workspace = torch.zeros(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _lib.load().pa_decode_step_host(
+        ctypes.byref(pool.c), ctypes.c_void_p(packet.host.data_ptr()), _ptr(packet.dev),
+        packet.nbytes, B, Hq, max_pages, num_new, float(scale), _ptr(out_dev),
+        ctypes.c_void_p(out_host.data_ptr()), _ptr(workspace), ws_bytes, num_splits,
+        _ptr(d_err), _stream(stream), 1 if synchronize else 0)
+    _lib.check(st, "pa_decode_step_host")
+    return out_host
 
 
 def pa_decode_noalloc(pool: KVPool, q: torch.Tensor, block_tables: torch.Tensor,

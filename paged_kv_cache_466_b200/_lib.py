@@ -68,6 +68,9 @@ SIGNATURES = {
     "pa_decode_range_workspace_bytes": (ctypes.c_size_t, [_POOL, _I, _I, _I, _I, _I, _I]),
     "pa_decode_range": (_I, [_POOL, _P, _I, _I, _P, _I, _P, _I, _I, ctypes.c_float, _P, _P, _P,
                              ctypes.c_size_t, _I, _P, _P]),
+    "pa_step_packet_layout": (ctypes.c_size_t, [_POOL, _I, _I, _I, _I, _P]),
+    "pa_decode_step_host": (_I, [_POOL, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, ctypes.c_float,
+                                 _P, _P, _P, ctypes.c_size_t, _I, _P, _P, _I]),
     "pa_merge_partials": (_I, [_P, _P, _I, _I, _I, ctypes.c_int64, ctypes.c_int64, _P, _P,
                                 _P]),
     "pa_splitkv_reduce": (_I, [_P, _P, _I, _I, _I, _I, _P, _P]),

@@ -562,6 +562,71 @@ pa_status_t pa_decode_range(const pa_kv_pool_t *pool, const void *q, int32_t num
                      "pa_decode_range merge launch");
 }
 
+// ------------------------------------------------------------ host packet step
+size_t pa_step_packet_layout(const pa_kv_pool_t *pool, int32_t num_seqs, int32_t num_q_heads,
+                             int32_t max_pages, int32_t num_new, size_t *offsets) {
+  if (pool == nullptr || num_seqs < 0 || num_q_heads <= 0 || max_pages <= 0 || num_new < 0 ||
+      pool->num_kv_heads <= 0 || pool->head_dim <= 0)
+    return 0;
+  const size_t D = (size_t)pool->head_dim;
+  const size_t sizes[7] = {
+      (size_t)num_seqs * num_q_heads * D * 2,       // q
+      (size_t)num_new * pool->num_kv_heads * D * 2,  // k_new
+      (size_t)num_new * pool->num_kv_heads * D * 2,  // v_new
+      (size_t)num_new * 4,                           // seq_idx
+      (size_t)num_new * 4,                           // pos
+      (size_t)num_seqs * max_pages * 4,              // block_tables
+      (size_t)num_seqs * 4};                         // context_lens
+  size_t at = 0;
+  for (int i = 0; i < 7; ++i) {
+    if (offsets) offsets[i] = at;
+    at = align256(at + sizes[i]);
+  }
+  return at;
+}
+
+pa_status_t pa_decode_step_host(const pa_kv_pool_t *pool, const void *packet_host,
+                                void *packet_dev, size_t packet_bytes, int32_t num_seqs,
+                                int32_t num_q_heads, int32_t max_pages, int32_t num_new,
+                                float scale, float *out_dev, float *out_host, void *workspace,
+                                size_t workspace_bytes, int32_t num_splits, int32_t *d_err,
+                                void *stream, int32_t synchronize) {
+  g_last_error.clear();
+  pa_status_t st = check_pool(pool);
+  if (st != PA_OK) return st;
+  size_t off[7];
+  const size_t need = pa_step_packet_layout(pool, num_seqs, num_q_heads, max_pages, num_new, off);
+  if (need == 0)
+    return fail(PA_ERR_INVALID_ARG, "num_seqs=%d num_q_heads=%d max_pages=%d num_new=%d",
+                num_seqs, num_q_heads, max_pages, num_new);
+  if (packet_bytes != need)
+    return fail(PA_ERR_INVALID_ARG, "packet_bytes=%zu, the layout needs %zu", packet_bytes, need);
+  if (!packet_host || !packet_dev || (num_seqs > 0 && (!out_dev || !out_host)))
+    return fail(PA_ERR_INVALID_ARG, "packet_host, packet_dev, out_dev and out_host are required");
+  if (!aligned(packet_dev, 256))
+    return fail(PA_ERR_INVALID_ARG, "packet_dev must be 256-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = cuda_status(cudaMemcpyAsync(packet_dev, packet_host, packet_bytes, cudaMemcpyHostToDevice, s),
+                   "pa_decode_step_host packet copy");
+  if (st != PA_OK) return st;
+  char *pd = static_cast<char *>(packet_dev);
+  const int32_t *tables = reinterpret_cast<const int32_t *>(pd + off[5]);
+  st = pa_kv_append(pool, pd + off[1], pd + off[2], reinterpret_cast<const int32_t *>(pd + off[3]),
+                    reinterpret_cast<const int32_t *>(pd + off[4]), num_new, tables, num_seqs,
+                    max_pages, d_err, stream);
+  if (st != PA_OK) return st;
+  st = pa_decode(pool, pd + off[0], num_seqs, num_q_heads, tables, max_pages,
+                 reinterpret_cast<const int32_t *>(pd + off[6]), scale, out_dev, workspace,
+                 workspace_bytes, num_splits, d_err, stream);
+  if (st != PA_OK || num_seqs == 0) return st;
+  st = cuda_status(cudaMemcpyAsync(out_host, out_dev,
+                                   (size_t)num_seqs * num_q_heads * pool->head_dim * sizeof(float),
+                                   cudaMemcpyDeviceToHost, s),
+                   "pa_decode_step_host output copy");
+  if (st != PA_OK || !synchronize) return st;
+  return cuda_status(cudaStreamSynchronize(s), "pa_decode_step_host synchronize");
+}
+
 pa_status_t pa_merge_partials(const float *o_parts, const float *lse_parts, int32_t num_parts,
                               int32_t rows, int32_t head_dim, int64_t o_part_stride,
                               int64_t lse_part_stride, float *out, float *lse_out,
