@@ -52,7 +52,11 @@ typedef enum {
   PA_ERR_UNSUPPORTED = 2,  /* shape outside the compiled set (D, P, G, dtype)  */
   PA_ERR_WORKSPACE = 3,    /* workspace too small or misaligned                */
   PA_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed             */
-  PA_ERR_BAD_TABLE = 5     /* reserved for callers that read d_err back        */
+  PA_ERR_BAD_TABLE = 5,    /* a device error word reports bad tables, context
+                              lengths, sequence indices or positions
+                              (pa_derr_status)                                 */
+  PA_ERR_TIMEOUT = 6       /* a device error word reports an expired bounded
+                              wait (pa_derr_status)                            */
 } pa_status_t;
 
 /* Bits a kernel ORs into *d_err (device int32) when it skips bad input. */
@@ -64,6 +68,16 @@ typedef enum {
                                 PA_MAX_KV_SCALE (the row is still written)     */
 #define PA_DERR_TIMEOUT 32 /* a bounded wait on the kernel's own tensor-core
                               work ran out (not expected; outputs invalid)    */
+
+/*
+ * pa_derr_status — the status a device error word stands for, once the
+ * caller has read *d_err back to the host (host only, no device access):
+ * 0 -> PA_OK; PA_DERR_TIMEOUT set -> PA_ERR_TIMEOUT (it wins over the
+ * others: outputs are invalid); any of PA_DERR_BAD_PAGE, _BAD_CTX, _BAD_SEQ,
+ * _BAD_POS -> PA_ERR_BAD_TABLE; PA_DERR_BIG_SCALE alone ->
+ * PA_ERR_UNSUPPORTED; any other bit -> PA_ERR_INVALID_ARG.
+ */
+pa_status_t pa_derr_status(int32_t derr);
 
 /* Quantised pools: pa_decode* feed s * (softmax weight) to the tensor cores
  * as f16, with weights kept <= 8, so every row scale must be below this bound
@@ -145,6 +159,19 @@ pa_status_t pa_kv_append(const pa_kv_pool_t *pool, const void *k_new,
  */
 int32_t pa_decode_num_splits(const pa_kv_pool_t *pool, int32_t num_seqs,
                              int32_t max_pages, int32_t requested);
+
+/*
+ * pa_decode_auto_splits — the split count pa_decode picks with
+ * num_splits == 0 for a batch of num_seqs sequences whose longest context is
+ * max_ctx tokens, in a bf16 pool of head_dim 128 with num_kv_heads heads and
+ * pages of page_size tokens, on the current device: the same as
+ * pa_decode_num_splits with such a pool and ceil(max_ctx / page_size) table
+ * columns. (A shape-only form for planners that hold no pool yet; use
+ * pa_decode_num_splits for other dtypes and head sizes.) Returns <= 0 on
+ * invalid arguments.
+ */
+int32_t pa_decode_auto_splits(int32_t num_seqs, int32_t num_kv_heads, int32_t max_ctx,
+                              int32_t page_size);
 
 /*
  * pa_decode_workspace_bytes — device scratch pa_decode needs for

@@ -34,7 +34,7 @@ import torch
 
 from . import _lib
 from ._lib import (PA_DERR_BAD_CTX, PA_DERR_BAD_PAGE, PA_DERR_BAD_POS, PA_DERR_BAD_SEQ,
-                   PA_DERR_BIG_SCALE, PA_MAX_KV_SCALE,
+                   PA_DERR_BIG_SCALE, PA_DERR_TIMEOUT, PA_MAX_KV_SCALE,
                    PA_KV_BF16, PA_KV_FP8_PER_TOKEN, PA_KV_U4_PER_TOKEN, PA_KV_U8_PER_TOKEN,
                    PagedAttnError, pa_kv_pool_t)
 
@@ -42,7 +42,8 @@ __all__ = ["KVPool", "pa_kv_append", "pa_decode", "pa_decode_noalloc", "pa_split
            "pa_decode_shared_prefix", "pa_decode_shared_prefix_workspace_bytes",
            "pa_decode_window", "pa_decode_window_workspace_bytes",
            "pa_decode_range", "pa_decode_range_workspace_bytes", "pa_merge_partials",
-           "pa_validate_tables", "StepPacket", "pa_decode_step_host",
+           "pa_validate_tables", "StepPacket", "pa_decode_step_host", "pa_derr_status",
+           "pa_decode_auto_splits", "PA_DERR_TIMEOUT",
            "pa_decode_num_splits", "pa_decode_workspace_bytes", "PagedAttnError",
            "PA_KV_BF16", "PA_KV_U8_PER_TOKEN", "PA_KV_FP8_PER_TOKEN", "PA_KV_U4_PER_TOKEN",
            "PA_DERR_BAD_PAGE",
@@ -114,6 +115,20 @@ class KVPool:
     @property
     def device(self):
         return self.k.device
+
+
+def pa_derr_status(derr: int) -> int:
+    """The PA_* status a device error word (read back to the host) stands for."""
+    return int(_lib.load().pa_derr_status(int(derr)))
+
+
+def pa_decode_auto_splits(num_seqs: int, num_kv_heads: int, max_ctx: int, page_size: int) -> int:
+    """Split count pa_decode picks automatically for a bf16, head_dim-128 pool of
+    this shape and a batch whose longest context is ``max_ctx`` tokens."""
+    s = _lib.load().pa_decode_auto_splits(num_seqs, num_kv_heads, max_ctx, page_size)
+    if s <= 0:
+        raise ValueError("pa_decode_auto_splits: invalid arguments")
+    return s
 
 
 def pa_decode_num_splits(pool: KVPool, num_seqs: int, max_pages: int, requested: int = 0) -> int:

@@ -17,6 +17,7 @@ PA_ERR_UNSUPPORTED = 2
 PA_ERR_WORKSPACE = 3
 PA_ERR_CUDA = 4
 PA_ERR_BAD_TABLE = 5
+PA_ERR_TIMEOUT = 6
 
 PA_DERR_BAD_PAGE = 1
 PA_DERR_BAD_CTX = 2
@@ -54,6 +55,8 @@ _POOL = ctypes.POINTER(pa_kv_pool_t)
 
 SIGNATURES = {
     "pa_kv_append": (_I, [_POOL, _P, _P, _P, _P, _I, _P, _I, _I, _P, _P]),
+    "pa_derr_status": (_I, [_I]),
+    "pa_decode_auto_splits": (_I, [_I, _I, _I, _I]),
     "pa_decode_num_splits": (_I, [_POOL, _I, _I, _I]),
     "pa_decode_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "pa_decode": (_I, [_POOL, _P, _I, _I, _P, _I, _P, ctypes.c_float, _P, _P, ctypes.c_size_t,

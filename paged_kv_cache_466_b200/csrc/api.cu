@@ -108,9 +108,19 @@ const char *pa_status_str(pa_status_t s) {
     case PA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
     case PA_ERR_WORKSPACE: return "workspace too small or misaligned";
     case PA_ERR_CUDA: return "CUDA error";
-    case PA_ERR_BAD_TABLE: return "bad page table";
+    case PA_ERR_BAD_TABLE: return "bad page table, context length, sequence index or position";
+    case PA_ERR_TIMEOUT: return "a bounded device wait expired";
   }
   return "unknown status";
+}
+
+pa_status_t pa_derr_status(int32_t derr) {
+  if (derr == 0) return PA_OK;
+  if (derr & PA_DERR_TIMEOUT) return PA_ERR_TIMEOUT;
+  if (derr & (PA_DERR_BAD_PAGE | PA_DERR_BAD_CTX | PA_DERR_BAD_SEQ | PA_DERR_BAD_POS))
+    return PA_ERR_BAD_TABLE;
+  if (derr == PA_DERR_BIG_SCALE) return PA_ERR_UNSUPPORTED;
+  return PA_ERR_INVALID_ARG;
 }
 
 const char *pa_last_error(void) { return g_last_error.c_str(); }
@@ -185,6 +195,19 @@ int32_t pa_decode_num_splits(const pa_kv_pool_t *pool, int32_t num_seqs, int32_t
   if (S < 1) S = 1;
   const int chunk = (max_pages + S - 1) / S;
   return (max_pages + chunk - 1) / chunk;
+}
+
+int32_t pa_decode_auto_splits(int32_t num_seqs, int32_t num_kv_heads, int32_t max_ctx,
+                              int32_t page_size) {
+  if (num_seqs < 0 || num_kv_heads <= 0 || max_ctx < 0 || page_size <= 0) return -1;
+  pa_kv_pool_t shape = {};
+  shape.page_size = page_size;
+  shape.num_kv_heads = num_kv_heads;
+  shape.head_dim = 128;
+  shape.dtype = PA_KV_BF16;
+  const int32_t max_pages = max_ctx > 0 ? (int32_t)((max_ctx + (int64_t)page_size - 1) / page_size)
+                                        : 1;
+  return pa_decode_num_splits(&shape, num_seqs, max_pages, 0);
 }
 
 size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,

@@ -40,8 +40,8 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_version_and_status_strings(lib):
     assert lib.pa_abi_version() == 1
-    for s in range(6):
-        assert lib.pa_status_str(s)
+    for s in range(7):
+        assert lib.pa_status_str(s) and lib.pa_status_str(s) != b"unknown status"
     assert lib.pa_status_str(99) == b"unknown status"
 
 
@@ -114,3 +114,35 @@ def test_split_planning_and_workspace_size(lib):
     l = 32 * 64 * 8 * 4
     c = 32 * 64 * 4
     assert ws == -(-o // 256) * 256 + -(-l // 256) * 256 + -(-c // 256) * 256
+
+
+def test_device_error_words_map_to_statuses(lib):
+    from paged_kv_cache_466_b200._lib import (PA_DERR_BAD_CTX, PA_DERR_BAD_PAGE,
+                                              PA_DERR_BAD_POS, PA_DERR_BAD_SEQ,
+                                              PA_DERR_BIG_SCALE, PA_DERR_TIMEOUT,
+                                              PA_ERR_BAD_TABLE, PA_ERR_TIMEOUT)
+    assert lib.pa_derr_status(0) == PA_OK
+    for bit in (PA_DERR_BAD_PAGE, PA_DERR_BAD_CTX, PA_DERR_BAD_SEQ, PA_DERR_BAD_POS):
+        assert lib.pa_derr_status(bit) == PA_ERR_BAD_TABLE
+        assert lib.pa_derr_status(bit | PA_DERR_BIG_SCALE) == PA_ERR_BAD_TABLE
+        assert lib.pa_derr_status(bit | PA_DERR_TIMEOUT) == PA_ERR_TIMEOUT
+    assert lib.pa_derr_status(PA_DERR_BIG_SCALE) == PA_ERR_UNSUPPORTED
+    assert lib.pa_derr_status(PA_DERR_TIMEOUT) == PA_ERR_TIMEOUT
+    assert lib.pa_derr_status(64) == PA_ERR_INVALID_ARG
+
+
+def test_auto_splits_and_step_host_reject_bad_arguments(lib):
+    assert lib.pa_decode_auto_splits(-1, 8, 100, 16) <= 0
+    assert lib.pa_decode_auto_splits(4, 0, 100, 16) <= 0
+    assert lib.pa_decode_auto_splits(4, 8, -5, 16) <= 0
+    pool = _pool()
+    n = lib.pa_step_packet_layout(ctypes.byref(pool), 2, 4, 4, 3, None)
+    assert n > 0 and n % 256 == 0
+    assert lib.pa_step_packet_layout(ctypes.byref(pool), 2, 4, 0, 3, None) == 0
+
+    def step(nbytes=n, dev=0x20000, host=0x30000):
+        return lib.pa_decode_step_host(ctypes.byref(pool), host, dev, nbytes, 2, 4, 4, 3, 0.1,
+                                       0x40000, 0x50000, None, 0, 1, None, None, 1)
+    assert step(nbytes=n + 256) == PA_ERR_INVALID_ARG
+    assert step(dev=0x20010) == PA_ERR_INVALID_ARG
+    assert step(host=None) == PA_ERR_INVALID_ARG

@@ -8,8 +8,8 @@ import pytest
 import torch
 
 import oracle
-from paged_kv_cache_466_b200 import (KVPool, StepPacket, _lib, pa_decode,
-                                     pa_decode_step_host)
+from paged_kv_cache_466_b200 import (KVPool, StepPacket, _lib, pa_decode, pa_decode_auto_splits,
+                                     pa_decode_num_splits, pa_decode_step_host)
 from paged_kv_cache_466_b200 import workloads as W
 from paged_kv_cache_466_b200.workloads import bits
 from tests.helpers import DEV, device_append, device_inputs, oracle_pool, pool_bytes_equal
@@ -95,3 +95,11 @@ def test_step_host_without_new_rows_and_bad_packet_size():
         None, 0, 1, None, None, 1)
     assert st == _lib.PA_ERR_INVALID_ARG
     assert b"packet_bytes" in _lib.load().pa_last_error()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("B,Hkv,ctx,P", [(32, 8, 8192, 32), (64, 8, 4095, 16), (4, 2, 64, 16),
+                                          (1, 1, 30000, 32), (0, 8, 100, 16)])
+def test_auto_splits_is_the_planner_for_a_bf16_d128_pool(B, Hkv, ctx, P):
+    pool = KVPool(4, Hkv, P, 128, "bf16", DEV)
+    assert pa_decode_auto_splits(B, Hkv, ctx, P) == pa_decode_num_splits(pool, B, -(-ctx // P))
