@@ -34,6 +34,7 @@ sys.path.insert(0, ROOT)
 METRIC = "decode-attention achieved HBM GB/s and % of B200 peak; sequences/sec per layer"
 FALLBACK_HBM_GBS = 6650.0
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+NOMINAL_HBM_GBS = 7700.0   # B200 (HGX) specification figure, for context only
 DECODE_SRC = os.path.join(ROOT, "paged_kv_cache_466_b200", "csrc", "decode.cu")
 
 
@@ -54,6 +55,9 @@ def parse():
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's number of sequences (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--flush-l2", action="store_true",
+                    help="write a buffer of twice the L2 size between timed steps; the step "
+                         "time is then the sum of per-step CUDA events, flush excluded")
     return ap.parse_args()
 
 
@@ -200,6 +204,7 @@ def cpu_oracle_throughput(w, budget_s: float = 12.0, max_reps: int = 40):
     repeated until ~budget_s of work. Returns (GB/s, cores, sample text)."""
     cores = len(os.sched_getaffinity(0))
     os.environ.setdefault("OMP_NUM_THREADS", str(cores))
+    cores = int(os.environ["OMP_NUM_THREADS"])
     import oracle
     from paged_kv_cache_466_b200.workloads import bits
     hp = oracle.empty_pool(w.kv, w.num_pages, w.Hkv, w.P, w.D, 0)
@@ -245,7 +250,9 @@ def config_of(w, args, n, S):
          "global_batch": w.B * n, "seq_len": int(w.context_lens.max()),
          "parallelism": f"dp{n} (independent sequences, no collective)",
          "num_splits": S, "pool_pages": w.num_pages,
-         "l2": "inputs larger than the 126 MB L2, not flushed"
+         "l2": "flushed between steps (write of 2x the L2 size, outside the step events)"
+               if args.flush_l2 else
+               "inputs larger than the 126 MB L2, not flushed"
                if decode_bytes(w, args.sinks, args.window) > 256e6
                else "L2 not flushed (working set may be L2-resident)"}
     return c
@@ -326,15 +333,28 @@ def run_ours(args, rank, world, local_rank):
     clocks = ClockSampler(local_rank)
     barrier()
     torch.cuda.synchronize()
+    if args.flush_l2:
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        flush = torch.empty(2 * max(l2, 1 << 20), dtype=torch.uint8, device=dev)
+        sevs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(K)]
     clocks.start()
     t0.record(stream)
     for i in range(K):
+        if args.flush_l2:
+            flush.fill_(i & 0xFF)
+            sevs[i][0].record(stream)
         step(*evs[i])
+        if args.flush_l2:
+            sevs[i][1].record(stream)
     t1.record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
     barrier()
-    ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
+    if args.flush_l2:
+        ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in sevs), world, dev)
+    else:
+        ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
     dec_ms = [a.elapsed_time(b) for a, b in evs]
     ms_step = ms / K
     dbytes = decode_bytes(w, args.sinks, args.window)
@@ -408,6 +428,8 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic (seeded N(0,1) bf16 K/V/q; no weights needed)",
         "config": config_of(w, args, world, S),
         "pct_of_peak": round(100.0 * value / world / peak, 2),
+        "nominal_gbs": NOMINAL_HBM_GBS,
+        "pct_of_nominal": round(100.0 * value / world / NOMINAL_HBM_GBS, 2),
         "peak_gbs": peak, "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
         if peak_kind == "measured" else "fallback 6.65 TB/s",
         "seq_per_s_per_layer": round(w.B * world / (ms_step * 1e-3), 1),
@@ -440,6 +462,7 @@ def run_reference(args, rank, world):
         return None
     cores = len(os.sched_getaffinity(0))
     os.environ.setdefault("OMP_NUM_THREADS", str(cores))
+    cores = int(os.environ["OMP_NUM_THREADS"])
     import oracle
     from paged_kv_cache_466_b200.workloads import bits
     w = make_workload(args.workload, seed=0, batch=args.batch)
