@@ -462,6 +462,16 @@ pa_status_t pa_decode_step_host(const pa_kv_pool_t *pool, const void *packet_hos
                                 size_t workspace_bytes, int32_t num_splits,
                                 int32_t *d_err, void *stream, int32_t synchronize);
 
+/*
+ * pa_selftest_wait_timeout — exercises the failure path of the kernels'
+ * bounded waits (the tcgen05 prefix pass waits on mbarriers for its tensor-
+ * core work): one thread waits on an mbarrier that nothing arrives at, gives
+ * up after limit_us microseconds of wall time and ORs PA_DERR_TIMEOUT into
+ * *d_err (device int32, required). It neither faults nor hangs, and the
+ * context stays usable. limit_us in [1, 1000000]. One launch.
+ */
+pa_status_t pa_selftest_wait_timeout(int32_t limit_us, int32_t *d_err, void *stream);
+
 /* Static description of a status code. */
 const char *pa_status_str(pa_status_t status);
 

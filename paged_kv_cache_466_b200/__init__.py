@@ -43,7 +43,7 @@ __all__ = ["KVPool", "pa_kv_append", "pa_decode", "pa_decode_noalloc", "pa_split
            "pa_decode_window", "pa_decode_window_workspace_bytes",
            "pa_decode_range", "pa_decode_range_workspace_bytes", "pa_merge_partials",
            "pa_validate_tables", "StepPacket", "pa_decode_step_host", "pa_derr_status",
-           "pa_decode_auto_splits", "PA_DERR_TIMEOUT",
+           "pa_decode_auto_splits", "pa_selftest_wait_timeout", "PA_DERR_TIMEOUT",
            "pa_decode_num_splits", "pa_decode_workspace_bytes", "PagedAttnError",
            "PA_KV_BF16", "PA_KV_U8_PER_TOKEN", "PA_KV_FP8_PER_TOKEN", "PA_KV_U4_PER_TOKEN",
            "PA_DERR_BAD_PAGE",
@@ -120,6 +120,14 @@ class KVPool:
 def pa_derr_status(derr: int) -> int:
     """The PA_* status a device error word (read back to the host) stands for."""
     return int(_lib.load().pa_derr_status(int(derr)))
+
+
+def pa_selftest_wait_timeout(limit_us: int, d_err: torch.Tensor, stream=None) -> None:
+    """Run the bounded-wait failure path once: a wait that can never complete
+    gives up after ``limit_us`` and sets PA_DERR_TIMEOUT in ``d_err``."""
+    _need(d_err, "d_err", torch.int32)
+    _lib.check(_lib.load().pa_selftest_wait_timeout(int(limit_us), _ptr(d_err), _stream(stream)),
+               "pa_selftest_wait_timeout")
 
 
 def pa_decode_auto_splits(num_seqs: int, num_kv_heads: int, max_ctx: int, page_size: int) -> int:

@@ -56,6 +56,7 @@ _POOL = ctypes.POINTER(pa_kv_pool_t)
 SIGNATURES = {
     "pa_kv_append": (_I, [_POOL, _P, _P, _P, _P, _I, _P, _I, _I, _P, _P]),
     "pa_derr_status": (_I, [_I]),
+    "pa_selftest_wait_timeout": (_I, [_I, _P, _P]),
     "pa_decode_auto_splits": (_I, [_I, _I, _I, _I]),
     "pa_decode_num_splits": (_I, [_POOL, _I, _I, _I]),
     "pa_decode_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),

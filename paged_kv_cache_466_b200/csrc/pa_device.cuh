@@ -197,6 +197,33 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// ------------------------------------------------------------- bounded waits
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait until the phase of the mbarrier at shared address `bar` with this
+// parity has completed. Gives up and returns false once `limit_ns` of wall
+// time (the global timer) has passed, or after 2^26 polls, so that a wait
+// that can never be satisfied ends in an error status instead of a hang.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  uint64_t limit_ns) {
+  const uint64_t t0 = global_ns();
+  for (int i = 0; i < (1 << 26); ++i) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(done)
+        : "r"(bar), "r"(parity));
+    if (done) return true;
+    if ((i & 15) == 15 && global_ns() - t0 > limit_ns) return false;
+  }
+  return false;
+}
+
 // ------------------------------------------------- programmatic dependent launch
 __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");

@@ -46,7 +46,6 @@ constexpr int kTileTok = 64;      // N of S, K of PV
 constexpr int kThreads = 128;
 constexpr int kTmemCols = 256;    // S [0, 64), P hi [64, 96), P lo [96, 128), O [128, 128 + D)
 constexpr float kRescaleLog2 = 8.0f;
-constexpr int kMaxWaitPolls = 1 << 24;
 
 // Byte offset of 16-byte chunk `chunk` of row r in a K-major,
 // 128-byte-swizzled tile of `rows` rows: 64-element K atoms of rows * 128
@@ -95,19 +94,12 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
       bar));
 }
 
-// Wait until the mbarrier's phase with this parity has completed; false if
-// the bounded number of polls ran out.
+// A commit that has not arrived after this long will not arrive: the kernel
+// stops waiting, reports PA_DERR_TIMEOUT and still releases its tensor memory.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s (a tile takes microseconds)
+
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-  for (int i = 0; i < kMaxWaitPolls; ++i) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(done)
-        : "r"(bar), "r"(parity));
-    if (done) return true;
-  }
-  return false;
+  return mbar_wait_bounded(bar, parity, kWaitLimitNs);
 }
 
 __device__ __forceinline__ void tc_fence_before() {

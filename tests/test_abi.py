@@ -146,3 +146,9 @@ def test_auto_splits_and_step_host_reject_bad_arguments(lib):
     assert step(nbytes=n + 256) == PA_ERR_INVALID_ARG
     assert step(dev=0x20010) == PA_ERR_INVALID_ARG
     assert step(host=None) == PA_ERR_INVALID_ARG
+
+
+def test_selftest_wait_timeout_rejects_bad_limits(lib):
+    assert lib.pa_selftest_wait_timeout(0, 0x1000, None) == PA_ERR_INVALID_ARG
+    assert lib.pa_selftest_wait_timeout(2_000_000, 0x1000, None) == PA_ERR_INVALID_ARG
+    assert lib.pa_selftest_wait_timeout(100, None, None) == PA_ERR_INVALID_ARG
