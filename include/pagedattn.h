@@ -149,7 +149,9 @@ pa_status_t pa_kv_append(const pa_kv_pool_t *pool, const void *k_new,
  * pa_decode_num_splits — the split-KV partition count S pa_decode uses for
  * this pool shape, table width and request. requested == 0 picks S from the
  * number of (sequence, KV head) units, the table width and how many decode
- * CTAs fit on the current device; requested > 0 is honoured as far as the
+ * CTAs fit on the current device: with fewer units than resident CTA slots,
+ * the fewest splits that give about 1.7 CTAs per SM in one wave; otherwise a
+ * wave model of the CTAs' lengths. requested > 0 is honoured as far as the
  * limits allow. Either way S is then clamped to [1, min(max_pages, 256)],
  * raised to at least ceil(max_pages / 2048) (a split stages at most 2048
  * table entries), and reduced so no split is empty by construction:
@@ -175,12 +177,18 @@ int32_t pa_decode_auto_splits(int32_t num_seqs, int32_t num_kv_heads, int32_t ma
 
 /*
  * pa_decode_workspace_bytes — device scratch pa_decode needs for
- * num_splits (already resolved, >= 1): 0 when num_splits == 1, else the
- * partial outputs fp32 [num_seqs][num_q_heads][num_splits][head_dim], their
- * log-sum-exps fp32 [num_seqs][num_q_heads][num_splits] and one int32 split
- * counter per (sequence, KV head) (num_seqs * num_q_heads are reserved), each
- * part 256-byte aligned. The counters must be zero before a workspace's first
- * use (allocate it zero-filled); every completed pa_decode leaves them zero.
+ * num_splits (already resolved, >= 1): 0 when num_splits == 1, else room for
+ * the partial outputs fp32 [num_seqs][num_q_heads][num_splits][head_dim] and
+ * their log-sum-exps fp32 [num_seqs][num_q_heads][num_splits] (each 256-byte
+ * aligned) plus the split counters.
+ * Workspace layout, for every entry point that takes one: bytes
+ * [0, C) with C = 256 * floor(workspace_bytes / 32768) hold int32 split
+ * counters, one per (sequence, KV head); the partials follow from byte C.
+ * C depends on the workspace's size only, so calls of any shape and entry
+ * point that share a workspace use the same counters, and nothing else is
+ * ever written there. The counters must be zero before a workspace's first
+ * use (allocate it zero-filled); every completed call leaves them zero, so a
+ * workspace zero-filled once serves any later call it is large enough for.
  */
 size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
                                  int32_t head_dim, int32_t num_splits);

@@ -68,6 +68,37 @@ pa_status_t check_pool(const pa_kv_pool_t *pool) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Split counters. The CTA that finishes a (sequence, KV head) last is found
+// with one atomic counter per unit, which that CTA re-arms to zero. The
+// counters sit at the start of every workspace, in a region whose size
+// depends on the workspace's size alone (1/128 of it, in whole 256-byte
+// units), and partial results are written only after that region. Calls of
+// any shape and any entry point that share a workspace therefore use the same
+// counter region and never write anything else into it: a workspace
+// zero-filled once stays valid for every later call.
+size_t counter_region(size_t ws_bytes) { return (ws_bytes / 32768) * 256; }
+
+bool workspace_fits(size_t ws_bytes, size_t rest, size_t counter_bytes) {
+  const size_t c = counter_region(ws_bytes);
+  return c >= counter_bytes && ws_bytes - c >= rest;
+}
+
+// Smallest workspace size (a multiple of 256) for `rest` bytes of partials
+// and `counter_bytes` of counters, with 256 bytes to spare so that every
+// larger size fits too (ws - counter_region(ws) dips by at most 255 bytes).
+size_t workspace_for(size_t rest, size_t counter_bytes) {
+  const size_t want = align256(rest) + 256;
+  size_t ws = want + align256(counter_bytes);
+  while (!workspace_fits(ws, want, counter_bytes)) {
+    const size_t c = counter_region(ws);
+    const size_t short_c = counter_bytes > c ? counter_bytes - c : 0;
+    const size_t short_r = want > ws - c ? want - (ws - c) : 0;
+    ws += align256(std::max<size_t>(std::max<size_t>(short_c * 128, short_r + short_r / 127),
+                                    256));
+  }
+  return ws;
+}
+
 }  // namespace
 
 void set_last_error_message(const char *msg) { g_last_error = msg; }
@@ -160,15 +191,27 @@ int32_t pa_decode_num_splits(const pa_kv_pool_t *pool, int32_t num_seqs, int32_t
   const int hi = max_pages < kMaxSplits ? max_pages : kMaxSplits;
   int S = requested;
   if (S == 0) {
-    // Wave model: CTAs of equal length run in waves of R = SMs x CTAs/SM. A
-    // split count is worth its extra partial writes only if it shortens
-    // (#waves x tokens per CTA); ties go to fewer splits.
+    // R = SMs x CTAs/SM resident CTA slots; a unit is one (sequence, KV head).
     const long long units = (long long)num_seqs * pool->num_kv_heads;
+    const long long sms = device_sm_count();
+    const long long R = sms * cached_ctas_per_sm(pool->head_dim, P, pool->dtype);
+    // CTAs that stream at once and keep HBM saturated: measured on the
+    // Llama-3-70B shapes (B = 8, 16, 32 x 8192 tokens), one wave of ~1.7
+    // CTAs per SM read at 79-103 % of the copy peak, and it was the fastest
+    // split count each time; more splits only added partial writes and a merge
+    const long long kSaturate = (sms * 17 + 9) / 10;
     if (units == 0) {
       S = 1;
+    } else if (units < R) {
+      // one wave: the fewest splits that reach kSaturate CTAs, without
+      // spilling into a second wave
+      long long s1 = (kSaturate + units - 1) / units;
+      if (s1 * units > R) s1 = R / units;
+      S = (int)(s1 < 1 ? 1 : (s1 > hi ? hi : s1));
     } else {
-      const long long R =
-          (long long)device_sm_count() * cached_ctas_per_sm(pool->head_dim, P, pool->dtype);
+      // Several waves. Wave model: CTAs of equal length run in waves of R; a
+      // split count is worth its extra partial writes only if it shortens
+      // (#waves x tokens per CTA); ties go to fewer splits.
       // CTA start-up, table staging and epilogue, in tokens of streaming
       // (measured: ~2,400 warp instructions plus two dependent loads per CTA;
       // on ragged Llama-3-8B-shaped batches 4 splits beat 6 by 2-7 %)
@@ -214,8 +257,9 @@ size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t 
                                  int32_t num_splits) {
   if (num_splits <= 1 || num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0) return 0;
   const size_t rows = (size_t)num_seqs * num_q_heads;
-  return align256(rows * num_splits * head_dim * sizeof(float)) +
-         align256(rows * num_splits * sizeof(float)) + align256(rows * sizeof(int32_t));
+  return workspace_for(align256(rows * num_splits * head_dim * sizeof(float)) +
+                           align256(rows * num_splits * sizeof(float)),
+                       rows * sizeof(int32_t));
 }
 
 pa_status_t pa_decode(const pa_kv_pool_t *pool, const void *q, int32_t num_seqs,
@@ -247,16 +291,22 @@ pa_status_t pa_decode(const pa_kv_pool_t *pool, const void *q, int32_t num_seqs,
     return fail(PA_ERR_INVALID_ARG, "q and out must be 16-byte aligned");
   const int S = pa_decode_num_splits(pool, num_seqs, max_pages, num_splits);
   if (S <= 0) return fail(PA_ERR_INVALID_ARG, "could not plan splits");
-  const size_t need = pa_decode_workspace_bytes(num_seqs, num_q_heads, pool->head_dim, S);
-  if (need > 0) {
-    if (workspace == nullptr || workspace_bytes < need)
-      return fail(PA_ERR_WORKSPACE, "workspace: need %zu bytes for %d splits, got %zu", need, S,
+  const int chunk = (max_pages + S - 1) / S;
+  const size_t rows = (size_t)num_seqs * num_q_heads;
+  const size_t o_bytes = align256(rows * S * pool->head_dim * sizeof(float));
+  const size_t l_bytes = align256(rows * S * sizeof(float));
+  if (S > 1) {
+    if (workspace == nullptr ||
+        workspace_bytes < workspace_for(o_bytes + l_bytes, rows * sizeof(int32_t)) ||
+        !workspace_fits(workspace_bytes, o_bytes + l_bytes, rows * sizeof(int32_t)))
+      return fail(PA_ERR_WORKSPACE, "workspace: need %zu bytes for %d splits, got %zu",
+                  pa_decode_workspace_bytes(num_seqs, num_q_heads, pool->head_dim, S), S,
                   workspace == nullptr ? (size_t)0 : workspace_bytes);
     if (!aligned(workspace, 256))
       return fail(PA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   }
-  const int chunk = (max_pages + S - 1) / S;
-  const size_t rows = (size_t)num_seqs * num_q_heads;
+  char *part_base = S > 1 ? static_cast<char *>(workspace) + counter_region(workspace_bytes)
+                          : nullptr;
   DecodeArgs a;
   a.k_pool = pool->k_pool;
   a.v_pool = pool->v_pool;
@@ -272,13 +322,9 @@ pa_status_t pa_decode(const pa_kv_pool_t *pool, const void *q, int32_t num_seqs,
   a.ctx = context_lens;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.out = out;
-  a.o_part = S > 1 ? static_cast<float *>(workspace) : nullptr;
-  const size_t o_bytes = align256(rows * S * pool->head_dim * sizeof(float));
-  const size_t l_bytes = align256(rows * S * sizeof(float));
-  a.lse = S > 1 ? reinterpret_cast<float *>(static_cast<char *>(workspace) + o_bytes) : nullptr;
-  a.counters = S > 1 ? reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + o_bytes +
-                                                   l_bytes)
-                     : nullptr;
+  a.o_part = S > 1 ? reinterpret_cast<float *>(part_base) : nullptr;
+  a.lse = S > 1 ? reinterpret_cast<float *>(part_base + o_bytes) : nullptr;
+  a.counters = S > 1 ? static_cast<int32_t *>(workspace) : nullptr;
   a.S = S;
   a.S_main = S;
   a.pages_per_split = chunk;
@@ -304,7 +350,7 @@ namespace {
 struct PrefixPlan {
   int n_psplits, tiles_per_split;  // prefix kernel
   int S, chunk;                    // suffix decode
-  size_t o_pre, lse_pre, o_part, lse, counters, total;  // workspace offsets / size
+  size_t o_pre, lse_pre, o_part, lse, total;  // offsets / size after the counter region
 };
 
 bool plan_prefix(const pa_kv_pool_t *pool, int B, int Hq, int max_pages, int prefix_len,
@@ -334,7 +380,6 @@ bool plan_prefix(const pa_kv_pool_t *pool, int B, int Hq, int max_pages, int pre
   pl->lse_pre = off;  off += align256(pl->n_psplits * R * sizeof(float));
   pl->o_part = off;   off += align256(R * pl->S * D * sizeof(float));
   pl->lse = off;      off += align256(R * pl->S * sizeof(float));
-  pl->counters = off; off += align256(R * sizeof(int32_t));
   pl->total = off;
   return true;
 }
@@ -350,7 +395,7 @@ size_t pa_decode_shared_prefix_workspace_bytes(const pa_kv_pool_t *pool, int32_t
     return 0;
   PrefixPlan pl;
   if (!plan_prefix(pool, num_seqs, num_q_heads, max_pages, prefix_len, num_splits, &pl)) return 0;
-  return pl.total;
+  return workspace_for(pl.total, (size_t)num_seqs * num_q_heads * sizeof(int32_t));
 }
 
 pa_status_t pa_decode_shared_prefix(const pa_kv_pool_t *pool, const void *q, int32_t num_seqs,
@@ -394,11 +439,15 @@ pa_status_t pa_decode_shared_prefix(const pa_kv_pool_t *pool, const void *q, int
   PrefixPlan pl;
   if (!plan_prefix(pool, num_seqs, num_q_heads, max_pages, prefix_len, num_splits, &pl))
     return fail(PA_ERR_INVALID_ARG, "could not plan the shared-prefix decode");
-  if (workspace == nullptr || workspace_bytes < pl.total)
-    return fail(PA_ERR_WORKSPACE, "workspace: need %zu bytes, got %zu", pl.total,
+  const size_t counter_bytes = (size_t)num_seqs * num_q_heads * sizeof(int32_t);
+  if (workspace == nullptr || workspace_bytes < workspace_for(pl.total, counter_bytes) ||
+      !workspace_fits(workspace_bytes, pl.total, counter_bytes))
+    return fail(PA_ERR_WORKSPACE, "workspace: need %zu bytes, got %zu",
+                workspace_for(pl.total, counter_bytes),
                 workspace == nullptr ? (size_t)0 : workspace_bytes);
   if (!aligned(workspace, 256)) return fail(PA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
-  char *ws = static_cast<char *>(workspace);
+  // partials after the workspace's counter region (which this path leaves alone)
+  char *ws = static_cast<char *>(workspace) + counter_region(workspace_bytes);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   PrefixArgs pa;
@@ -434,7 +483,7 @@ pa_status_t pa_decode_shared_prefix(const pa_kv_pool_t *pool, const void *q, int
   a.out = out;
   a.o_part = reinterpret_cast<float *>(ws + pl.o_part);
   a.lse = reinterpret_cast<float *>(ws + pl.lse);
-  a.counters = reinterpret_cast<int32_t *>(ws + pl.counters);
+  a.counters = nullptr;  // keep_partials: the suffix CTAs merge nothing themselves
   a.S = pl.S;
   a.S_main = pl.S;
   a.pages_per_split = pl.chunk;
@@ -527,18 +576,23 @@ pa_status_t pa_decode_range(const pa_kv_pool_t *pool, const void *q, int32_t num
   if (tok_begin >= max_pages * pool->page_size) tok_begin = tok_end = 0;  // empty range
   const int S = range_splits(pool, num_seqs, max_pages, tok_begin, tok_end, num_splits);
   if (S <= 0) return fail(PA_ERR_INVALID_ARG, "could not plan splits");
-  const size_t need = S > 1 ? pa_decode_workspace_bytes(num_seqs, num_q_heads, pool->head_dim, S)
-                            : 0;
-  if (need > 0) {
-    if (workspace == nullptr || workspace_bytes < need)
-      return fail(PA_ERR_WORKSPACE, "workspace: need %zu bytes for %d splits, got %zu", need, S,
+  const size_t rows = (size_t)num_seqs * num_q_heads;
+  const size_t o_bytes = align256(rows * S * pool->head_dim * sizeof(float));
+  const size_t l_bytes = align256(rows * S * sizeof(float));
+  if (S > 1) {
+    if (workspace == nullptr ||
+        workspace_bytes < workspace_for(o_bytes + l_bytes, rows * sizeof(int32_t)) ||
+        !workspace_fits(workspace_bytes, o_bytes + l_bytes, rows * sizeof(int32_t)))
+      return fail(PA_ERR_WORKSPACE, "workspace: need %zu bytes for %d splits, got %zu",
+                  pa_decode_workspace_bytes(num_seqs, num_q_heads, pool->head_dim, S), S,
                   workspace == nullptr ? (size_t)0 : workspace_bytes);
     if (!aligned(workspace, 256)) return fail(PA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   }
+  char *part_base = S > 1 ? static_cast<char *>(workspace) + counter_region(workspace_bytes)
+                          : nullptr;
   const int P = pool->page_size;
   const long long end = std::min<long long>(tok_end, (long long)max_pages * P);
   const int pages = std::max(1, (int)((end + P - 1) / P) - tok_begin / P);
-  const size_t rows = (size_t)num_seqs * num_q_heads;
   DecodeArgs a;
   a.k_pool = pool->k_pool;
   a.v_pool = pool->v_pool;
@@ -554,14 +608,12 @@ pa_status_t pa_decode_range(const pa_kv_pool_t *pool, const void *q, int32_t num
   a.ctx = context_lens;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.out = o_out;
-  // one split writes o_out / lse_out directly ([row][1][D] is [row][D])
-  const size_t o_bytes = align256(rows * S * pool->head_dim * sizeof(float));
-  const size_t l_bytes = align256(rows * S * sizeof(float));
-  a.o_part = S > 1 ? static_cast<float *>(workspace) : o_out;
-  a.lse = S > 1 ? reinterpret_cast<float *>(static_cast<char *>(workspace) + o_bytes) : lse_out;
-  a.counters = S > 1 ? reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + o_bytes +
-                                                   l_bytes)
-                     : nullptr;
+  // one split writes o_out / lse_out directly ([row][1][D] is [row][D]); more
+  // write partials after the workspace's counter region, which keep_partials
+  // leaves alone
+  a.o_part = S > 1 ? reinterpret_cast<float *>(part_base) : o_out;
+  a.lse = S > 1 ? reinterpret_cast<float *>(part_base + o_bytes) : lse_out;
+  a.counters = nullptr;
   a.S = S;
   a.S_main = S;
   a.pages_per_split = (pages + S - 1) / S;
@@ -787,16 +839,18 @@ pa_status_t pa_decode_window(const pa_kv_pool_t *pool, const void *q, int32_t nu
     return fail(PA_ERR_UNSUPPORTED, "windowed decode: at most %d sink pages are supported",
                 kMaxPagesPerSplit);
   if (pl.S + 1 > kMaxSplits + 1) return fail(PA_ERR_UNSUPPORTED, "too many splits");
-  const size_t need = pa_decode_workspace_bytes(num_seqs, num_q_heads, pool->head_dim, pl.S);
-  if (need > 0) {
-    if (workspace == nullptr || workspace_bytes < need)
-      return fail(PA_ERR_WORKSPACE, "workspace: need %zu bytes for %d splits, got %zu", need,
-                  pl.S, workspace == nullptr ? (size_t)0 : workspace_bytes);
-    if (!aligned(workspace, 256)) return fail(PA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
-  }
   const size_t rows = (size_t)num_seqs * num_q_heads;
   const size_t o_bytes = align256(rows * pl.S * pool->head_dim * sizeof(float));
   const size_t l_bytes = align256(rows * pl.S * sizeof(float));
+  if (pl.S > 1) {
+    if (workspace == nullptr ||
+        workspace_bytes < workspace_for(o_bytes + l_bytes, rows * sizeof(int32_t)) ||
+        !workspace_fits(workspace_bytes, o_bytes + l_bytes, rows * sizeof(int32_t)))
+      return fail(PA_ERR_WORKSPACE, "workspace: need %zu bytes for %d splits, got %zu",
+                  pa_decode_workspace_bytes(num_seqs, num_q_heads, pool->head_dim, pl.S), pl.S,
+                  workspace == nullptr ? (size_t)0 : workspace_bytes);
+    if (!aligned(workspace, 256)) return fail(PA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  }
   DecodeArgs a;
   a.k_pool = pool->k_pool;
   a.v_pool = pool->v_pool;
@@ -812,10 +866,11 @@ pa_status_t pa_decode_window(const pa_kv_pool_t *pool, const void *q, int32_t nu
   a.ctx = context_lens;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.out = out;
-  char *ws = static_cast<char *>(workspace);
+  char *ws = pl.S > 1 ? static_cast<char *>(workspace) + counter_region(workspace_bytes)
+                      : nullptr;
   a.o_part = pl.S > 1 ? reinterpret_cast<float *>(ws) : nullptr;
   a.lse = pl.S > 1 ? reinterpret_cast<float *>(ws + o_bytes) : nullptr;
-  a.counters = pl.S > 1 ? reinterpret_cast<int32_t *>(ws + o_bytes + l_bytes) : nullptr;
+  a.counters = pl.S > 1 ? static_cast<int32_t *>(workspace) : nullptr;
   a.S = pl.S;
   a.S_main = pl.S_main;
   a.pages_per_split = pl.chunk;

@@ -109,11 +109,18 @@ def test_split_planning_and_workspace_size(lib):
     assert lib.pa_decode_num_splits(ctypes.byref(pool), 4, 4000, 1) == 2   # 2048-entry cap
     assert lib.pa_decode_num_splits(ctypes.byref(pool), 4, 0, 0) <= 0
     assert lib.pa_decode_workspace_bytes(32, 64, 128, 1) == 0
-    ws = lib.pa_decode_workspace_bytes(32, 64, 128, 8)
-    o = 32 * 64 * 8 * 128 * 4
-    l = 32 * 64 * 8 * 4
-    c = 32 * 64 * 4
-    assert ws == -(-o // 256) * 256 + -(-l // 256) * 256 + -(-c // 256) * 256
+    for B, Hq, D, S in [(32, 64, 128, 8), (1, 8, 64, 2), (4096, 64, 128, 2), (7, 12, 64, 3)]:
+        ws = lib.pa_decode_workspace_bytes(B, Hq, D, S)
+        rest = -(-B * Hq * S * D * 4 // 256) * 256 + -(-B * Hq * S * 4 // 256) * 256
+        c = B * Hq * 4
+        assert ws % 256 == 0
+        # the counter region is [0, 256 * (size // 32768)); the partials follow it,
+        # for the returned size and for every larger one
+        for size in (ws, ws + 1, ws + 255, ws + 32768 * 3 - ws % 32768, 2 * ws):
+            region = 256 * (size // 32768)
+            assert region >= c and size - region >= rest, (B, Hq, D, S, size)
+        # about 1/128 over the parts, the counter region at least 256 bytes (32 KB)
+        assert ws <= max(rest * 128 / 127, 128 * c) + 33280
 
 
 def test_device_error_words_map_to_statuses(lib):

@@ -281,3 +281,33 @@ def test_full_size_prefix_shared_equals_unshared():
     b, _ = _run(unshared)
     np.testing.assert_array_equal(a, b)
     _check(shared, a, pairs=_sample_pairs(shared, 48))
+
+
+def test_one_workspace_serves_calls_of_every_shape_and_entry_point():
+    """A workspace zero-filled once serves a sequence of calls whose shapes
+    grow and shrink and that mix entry points: the split counters sit in a
+    region sized by the workspace alone, which no call writes partials into."""
+    from paged_kv_cache_466_b200 import pa_decode_range, pa_decode_window
+    ws = torch.zeros(48 << 20, dtype=torch.uint8, device=DEV)
+    plan = [(W.llama8b(B=6, ctx_range=(1, 3000), seed=4), "decode", 8),
+            (W.int8(B=30, ctx_range=(1, 2000), seed=5), "decode", 3),
+            (W.llama8b(B=9, ctx_range=(200, 3000), seed=6), "range", 4),
+            (W.llama8b(B=40, ctx_range=(1, 1500), seed=7), "decode", 2),
+            (W.llama8b(B=7, ctx_range=(500, 3000), seed=8), "window", 3),
+            (W.llama8b(B=64, ctx_range=(1, 900), seed=9), "decode", 5)]
+    for w, kind, S in plan:
+        pool, bt, ctx, q = device_inputs(w)
+        device_append(pool, w, bt)
+        if kind == "decode":
+            got = pa_decode(pool, q, bt, ctx, w.scale, num_splits=S, workspace=ws)
+            want = pa_decode(pool, q, bt, ctx, w.scale, num_splits=S)
+        elif kind == "range":
+            got = pa_decode_range(pool, q, bt, ctx, w.scale, 64, 2500, num_splits=S,
+                                  workspace=ws)[0]
+            want = pa_decode_range(pool, q, bt, ctx, w.scale, 64, 2500, num_splits=S)[0]
+        else:
+            got = pa_decode_window(pool, q, bt, ctx, w.scale, 4, 1000, num_splits=S,
+                                   workspace=ws)
+            want = pa_decode_window(pool, q, bt, ctx, w.scale, 4, 1000, num_splits=S)
+        torch.cuda.synchronize()
+        assert torch.equal(got, want), (w.name, kind, S)
