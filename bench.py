@@ -55,6 +55,9 @@ def parse():
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's number of sequences (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--separate-append", action="store_true",
+                    help="time pa_kv_append + pa_decode as two calls instead of the fused "
+                         "pa_decode_append step")
     ap.add_argument("--flush-l2", action="store_true",
                     help="write a buffer of twice the L2 size between timed steps; the step "
                          "time is then the sum of per-step CUDA events, flush excluded")
@@ -266,7 +269,8 @@ def run_ours(args, rank, world, local_rank):
                                          pa_decode_shared_prefix_workspace_bytes,
                                          pa_decode_window, pa_decode_window_workspace_bytes,
                                          pa_decode_workspace_bytes, pa_kv_append,
-                                         StepPacket, pa_decode_step_host)
+                                         pa_decode_append, StepPacket, pa_decode_step_host,
+                                         PA_STEP_NEWEST_PER_SEQ)
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -309,11 +313,25 @@ def run_ours(args, rank, world, local_rank):
         else:
             pa_decode(pool, qq, tt, cc, w.scale, out=out, workspace=ws, num_splits=S)
 
+    # the usual decode step (one new token per sequence, at ctx - 1) runs as one
+    # launch, the cache write fused into the decode; other steps as two calls
+    per_seq = (w.step_rows_by_sequence()
+               if not (args.cascade or args.window > 0 or args.separate_append) else None)
+    fused = per_seq is not None
+    if fused:
+        kn, vn = per_seq[0].to(dev), per_seq[1].to(dev)
+
     def step(ev0=None, ev1=None):
-        pa_kv_append(pool, sk, sv, sseq, spos, bt)
-        if ev0 is not None:
-            ev0.record(stream)
-        decode(q, bt, ctx)
+        if fused:
+            if ev0 is not None:
+                ev0.record(stream)
+            pa_decode_append(pool, q, kn, vn, bt, ctx, w.scale, out=out, workspace=ws,
+                             num_splits=S)
+        else:
+            pa_kv_append(pool, sk, sv, sseq, spos, bt)
+            if ev0 is not None:
+                ev0.record(stream)
+            decode(q, bt, ctx)
         if ev1 is not None:
             ev1.record(stream)
 
@@ -373,10 +391,16 @@ def run_ours(args, rank, world, local_rank):
     if not args.cascade and args.window == 0:
         # the library's host-packet step: one H2D copy of the packed inputs,
         # append, decode and one D2H copy of the output, in one C-ABI call
-        packet = StepPacket(pool, w.B, w.Hq, w.max_pages, len(w.step_seq))
-        for view, h in ((packet.q, h_q), (packet.k_new, h_k), (packet.v_new, h_v),
-                        (packet.seq_idx, h_seq), (packet.pos, h_pos),
-                        (packet.context_lens, h_ctx), (packet.block_tables, h_bt)):
+        if fused:   # one row per sequence, the cache write fused into the decode
+            packet = StepPacket(pool, w.B, w.Hq, w.max_pages, PA_STEP_NEWEST_PER_SEQ)
+            h_k, h_v = per_seq[0].pin_memory(), per_seq[1].pin_memory()
+            fills = ((packet.k_new, h_k), (packet.v_new, h_v))
+        else:
+            packet = StepPacket(pool, w.B, w.Hq, w.max_pages, len(w.step_seq))
+            fills = ((packet.k_new, h_k), (packet.v_new, h_v), (packet.seq_idx, h_seq),
+                     (packet.pos, h_pos))
+        for view, h in ((packet.q, h_q), (packet.context_lens, h_ctx),
+                        (packet.block_tables, h_bt)) + fills:
             view.copy_(h)
         h2d = packet.nbytes
 
@@ -416,9 +440,12 @@ def run_ours(args, rank, world, local_rank):
 
     peak, peak_kind = measured_peak()
     dec_avg_ms = statistics.mean(dec_ms)
-    achieved = dbytes / (dec_avg_ms * 1e-3) / 1e9
+    # the timed kernel: the fused step also reads the new rows and writes them
+    kbytes = dbytes + (append_bytes(w) if fused else 0)
+    achieved = kbytes / (dec_avg_ms * 1e-3) / 1e9
     traffic = recorded_traffic(w.name) if not (args.cascade or args.window) else None
-    launches_per_step = 4 if args.cascade else 2  # append, [prefix pass,] decode[, merge]
+    # append, [prefix pass,] decode[, merge]; the fused step is one launch
+    launches_per_step = 1 if fused else 4 if args.cascade else 2
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
@@ -439,10 +466,11 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "hbm",
                      "kernel": ("pa_decode_shared_prefix (prefix pass + decode)" if args.cascade
                                 else "pa_decode_window" if args.window > 0
-                                else "pa_decode (one launch, split merge fused)"),
+                                else "pa_decode_append (cache write + decode, one launch)"
+                                if fused else "pa_decode (one launch, split merge fused)"),
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "algorithmic_bytes": dbytes,
+                     "algorithmic_bytes": kbytes,
                      "avg_launch_ms": round(dec_avg_ms, 5)},
         "gpu_launches": K * launches_per_step,
         "clocks": clk,

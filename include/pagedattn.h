@@ -225,6 +225,29 @@ pa_status_t pa_decode(const pa_kv_pool_t *pool, const void *q,
                       int32_t num_splits, int32_t *d_err, void *stream);
 
 /*
+ * pa_decode_append — one decode step in one launch: the cache write of
+ * pa_kv_append for each sequence's newest token, fused into pa_decode.
+ *   k_new, v_new : (device) bf16 [num_seqs][num_kv_heads][head_dim], 16-byte
+ *                  aligned: the K/V rows of token context_lens[b] - 1 of
+ *                  sequence b (its page must already be in the table)
+ * Every other argument is pa_decode's. The CTA whose split holds position
+ * context_lens[b] - 1 stores that row (quantised for INT8/FP8/INT4 pools by
+ * the same per-row quantiser as pa_kv_append, so the stored bits are
+ * identical, and PA_DERR_BIG_SCALE is flagged the same way) before it reads
+ * the page; then Eq. (1) runs over tokens 0 .. context_lens[b] - 1 as in
+ * pa_decode. The result equals pa_kv_append(seq_idx = b, pos =
+ * context_lens[b] - 1) followed by pa_decode, bit for bit, without the
+ * append's launch. A sequence with context length 0 stores nothing.
+ */
+pa_status_t pa_decode_append(const pa_kv_pool_t *pool, const void *q,
+                             const void *k_new, const void *v_new,
+                             int32_t num_seqs, int32_t num_q_heads,
+                             const int32_t *block_tables, int32_t max_pages,
+                             const int32_t *context_lens, float scale, float *out,
+                             void *workspace, size_t workspace_bytes,
+                             int32_t num_splits, int32_t *d_err, void *stream);
+
+/*
  * pa_decode_shared_prefix — cascade decode for a batch whose requests all
  * begin with the same prompt prefix stored once in shared pages
  * ("KV-Cache Optimization Techniques", section "Prefix Caching", Eq. 2).
@@ -436,10 +459,17 @@ pa_status_t pa_validate_tables(const int32_t *block_tables, int32_t num_seqs,
  *   6 context_lens int32 [num_seqs]
  * (the same meaning as the arguments of pa_kv_append and pa_decode).
  *
+ * num_new == PA_STEP_NEWEST_PER_SEQ instead means one row per sequence, its
+ * newest token (position context_lens[b] - 1): k_new and v_new are then
+ * [num_seqs][num_kv_heads][head_dim], sections 3 and 4 are empty, and the
+ * step runs pa_decode_append (cache write fused into the decode, one launch)
+ * instead of pa_kv_append + pa_decode.
+ *
  * pa_step_packet_layout — host only (no device access): writes the seven
  * section offsets in bytes to offsets[0..6] (when offsets is not NULL) and
  * returns the packet size in bytes, or 0 on invalid arguments.
  */
+#define PA_STEP_NEWEST_PER_SEQ (-1)
 size_t pa_step_packet_layout(const pa_kv_pool_t *pool, int32_t num_seqs,
                              int32_t num_q_heads, int32_t max_pages,
                              int32_t num_new, size_t *offsets);

@@ -34,16 +34,18 @@ import torch
 
 from . import _lib
 from ._lib import (PA_DERR_BAD_CTX, PA_DERR_BAD_PAGE, PA_DERR_BAD_POS, PA_DERR_BAD_SEQ,
+                   PA_STEP_NEWEST_PER_SEQ,
                    PA_DERR_BIG_SCALE, PA_DERR_TIMEOUT, PA_MAX_KV_SCALE,
                    PA_KV_BF16, PA_KV_FP8_PER_TOKEN, PA_KV_U4_PER_TOKEN, PA_KV_U8_PER_TOKEN,
                    PagedAttnError, pa_kv_pool_t)
 
-__all__ = ["KVPool", "pa_kv_append", "pa_decode", "pa_decode_noalloc", "pa_splitkv_reduce",
+__all__ = ["KVPool", "pa_kv_append", "pa_decode", "pa_decode_append", "pa_decode_noalloc", "pa_splitkv_reduce",
            "pa_decode_shared_prefix", "pa_decode_shared_prefix_workspace_bytes",
            "pa_decode_window", "pa_decode_window_workspace_bytes",
            "pa_decode_range", "pa_decode_range_workspace_bytes", "pa_merge_partials",
            "pa_validate_tables", "StepPacket", "pa_decode_step_host", "pa_derr_status",
            "pa_decode_auto_splits", "pa_selftest_wait_timeout", "PA_DERR_TIMEOUT",
+           "PA_STEP_NEWEST_PER_SEQ",
            "pa_decode_num_splits", "pa_decode_workspace_bytes", "PagedAttnError",
            "PA_KV_BF16", "PA_KV_U8_PER_TOKEN", "PA_KV_FP8_PER_TOKEN", "PA_KV_U4_PER_TOKEN",
            "PA_DERR_BAD_PAGE",
@@ -205,6 +207,43 @@ def pa_decode(pool: KVPool, q: torch.Tensor, block_tables: torch.Tensor,
     return out
 
 
+
+def pa_decode_append(pool: KVPool, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                     block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
+                     out: Optional[torch.Tensor] = None,
+                     workspace: Optional[torch.Tensor] = None, num_splits: int = 0,
+                     d_err: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One decode step in one launch: store k_new / v_new [B, Hkv, D] bf16 at
+    position context_lens[b] - 1 of each sequence (as pa_kv_append would),
+    then Eq. 1 over tokens 0 .. context_lens[b] - 1 (as pa_decode)."""
+    dev = pool.device
+    _need(q, "q", torch.bfloat16, dev)
+    _need(k_new, "k_new", torch.bfloat16, dev)
+    _need(v_new, "v_new", torch.bfloat16, dev)
+    _need(block_tables, "block_tables", torch.int32, dev)
+    _need(context_lens, "context_lens", torch.int32, dev)
+    B, Hq, D = q.shape
+    if D != pool.head_dim or block_tables.shape[0] != B or context_lens.numel() != B \
+            or tuple(k_new.shape) != (B, pool.num_kv_heads, D) or k_new.shape != v_new.shape:
+        raise ValueError("pa_decode_append: shape mismatch")
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    _need(out, "out", torch.float32, dev)
+    max_pages = block_tables.shape[1]
+    if workspace is None:
+        need = pa_decode_workspace_bytes(B, Hq, D,
+                                         pa_decode_num_splits(pool, B, max_pages, num_splits))
+        if need > 0:
+            workspace = torch.zeros(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _lib.load().pa_decode_append(ctypes.byref(pool.c), _ptr(q), _ptr(k_new), _ptr(v_new), B,
+                                      Hq, _ptr(block_tables), max_pages, _ptr(context_lens),
+                                      float(scale), _ptr(out), _ptr(workspace), ws_bytes,
+                                      num_splits, _ptr(d_err), _stream(stream))
+    _lib.check(st, "pa_decode_append")
+    return out
+
+
 def pa_decode_shared_prefix_workspace_bytes(pool: KVPool, num_seqs: int, num_q_heads: int,
                                             max_pages: int, prefix_len: int,
                                             num_splits: int = 0) -> int:
@@ -297,6 +336,9 @@ class StepPacket:
 
     def __init__(self, pool: KVPool, num_seqs: int, num_q_heads: int, max_pages: int,
                  num_new: int, pin: bool = True):
+        # num_new == PA_STEP_NEWEST_PER_SEQ: one row per sequence (its newest
+        # token), k_new / v_new are [B, Hkv, D] and the step fuses the cache
+        # write into the decode
         off = (ctypes.c_size_t * 7)()
         n = int(_lib.load().pa_step_packet_layout(ctypes.byref(pool.c), num_seqs, num_q_heads,
                                                   max_pages, num_new, off))
@@ -319,10 +361,12 @@ class StepPacket:
             return self.host[self.offsets[i]:self.offsets[i] + nb].view(dtype).view(shape)
 
         self.q = view(0, torch.bfloat16, (B, Hq, D))
-        self.k_new = view(1, torch.bfloat16, (num_new, Hkv, D))
-        self.v_new = view(2, torch.bfloat16, (num_new, Hkv, D))
-        self.seq_idx = view(3, torch.int32, (num_new,))
-        self.pos = view(4, torch.int32, (num_new,))
+        per_seq = num_new == _lib.PA_STEP_NEWEST_PER_SEQ
+        rows = B if per_seq else num_new
+        self.k_new = view(1, torch.bfloat16, (rows, Hkv, D))
+        self.v_new = view(2, torch.bfloat16, (rows, Hkv, D))
+        self.seq_idx = view(3, torch.int32, (0 if per_seq else num_new,))
+        self.pos = view(4, torch.int32, (0 if per_seq else num_new,))
         self.block_tables = view(5, torch.int32, (B, max_pages))
         self.context_lens = view(6, torch.int32, (B,))
 

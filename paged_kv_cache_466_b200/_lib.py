@@ -33,6 +33,7 @@ PA_KV_FP8_PER_TOKEN = 2
 PA_KV_U4_PER_TOKEN = 3
 
 PA_NOALLOC_SCRATCH_BYTES = 16 << 20
+PA_STEP_NEWEST_PER_SEQ = -1
 
 
 class pa_kv_pool_t(ctypes.Structure):
@@ -58,6 +59,8 @@ SIGNATURES = {
     "pa_derr_status": (_I, [_I]),
     "pa_selftest_wait_timeout": (_I, [_I, _P, _P]),
     "pa_decode_auto_splits": (_I, [_I, _I, _I, _I]),
+    "pa_decode_append": (_I, [_POOL, _P, _P, _P, _I, _I, _P, _I, _P, ctypes.c_float, _P, _P,
+                              ctypes.c_size_t, _I, _P, _P]),
     "pa_decode_num_splits": (_I, [_POOL, _I, _I, _I]),
     "pa_decode_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "pa_decode": (_I, [_POOL, _P, _I, _I, _P, _I, _P, ctypes.c_float, _P, _P, ctypes.c_size_t,

@@ -262,11 +262,15 @@ size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t 
                        rows * sizeof(int32_t));
 }
 
-pa_status_t pa_decode(const pa_kv_pool_t *pool, const void *q, int32_t num_seqs,
-                      int32_t num_q_heads, const int32_t *block_tables, int32_t max_pages,
-                      const int32_t *context_lens, float scale, float *out, void *workspace,
-                      size_t workspace_bytes, int32_t num_splits, int32_t *d_err,
-                      void *stream) {
+namespace {
+
+// pa_decode, optionally with the fused cache write of pa_decode_append
+// (k_new / v_new non-null).
+pa_status_t decode_impl(const pa_kv_pool_t *pool, const void *q, int32_t num_seqs,
+                        int32_t num_q_heads, const int32_t *block_tables, int32_t max_pages,
+                        const int32_t *context_lens, float scale, float *out, void *workspace,
+                        size_t workspace_bytes, int32_t num_splits, int32_t *d_err,
+                        void *stream, const void *k_new, const void *v_new) {
   g_last_error.clear();
   pa_status_t st = check_pool(pool);
   if (st != PA_OK) return st;
@@ -339,9 +343,39 @@ pa_status_t pa_decode(const pa_kv_pool_t *pool, const void *q, int32_t num_seqs,
   a.tok_end = 0x7fffffff;
   a.range_mode = 0;
   a.d_err = d_err;
+  a.k_new = static_cast<const unsigned char *>(k_new);
+  a.v_new = static_cast<const unsigned char *>(v_new);
   return cuda_status(launch_decode(pool->head_dim, pool->page_size, pool->dtype, a,
                                    static_cast<cudaStream_t>(stream)),
-                     "pa_decode launch");
+                     k_new ? "pa_decode_append launch" : "pa_decode launch");
+}
+
+}  // namespace
+
+pa_status_t pa_decode(const pa_kv_pool_t *pool, const void *q, int32_t num_seqs,
+                      int32_t num_q_heads, const int32_t *block_tables, int32_t max_pages,
+                      const int32_t *context_lens, float scale, float *out, void *workspace,
+                      size_t workspace_bytes, int32_t num_splits, int32_t *d_err,
+                      void *stream) {
+  return decode_impl(pool, q, num_seqs, num_q_heads, block_tables, max_pages, context_lens,
+                     scale, out, workspace, workspace_bytes, num_splits, d_err, stream, nullptr,
+                     nullptr);
+}
+
+pa_status_t pa_decode_append(const pa_kv_pool_t *pool, const void *q, const void *k_new,
+                             const void *v_new, int32_t num_seqs, int32_t num_q_heads,
+                             const int32_t *block_tables, int32_t max_pages,
+                             const int32_t *context_lens, float scale, float *out,
+                             void *workspace, size_t workspace_bytes, int32_t num_splits,
+                             int32_t *d_err, void *stream) {
+  g_last_error.clear();
+  if (num_seqs > 0 && (k_new == nullptr || v_new == nullptr))
+    return fail(PA_ERR_INVALID_ARG, "k_new and v_new are required");
+  if (!aligned(k_new, 16) || !aligned(v_new, 16))
+    return fail(PA_ERR_INVALID_ARG, "k_new/v_new must be 16-byte aligned");
+  return decode_impl(pool, q, num_seqs, num_q_heads, block_tables, max_pages, context_lens,
+                     scale, out, workspace, workspace_bytes, num_splits, d_err, stream,
+                     num_seqs > 0 ? k_new : nullptr, num_seqs > 0 ? v_new : nullptr);
 }
 
 // ---------------------------------------------------------------- shared prefix
@@ -640,16 +674,20 @@ pa_status_t pa_decode_range(const pa_kv_pool_t *pool, const void *q, int32_t num
 // ------------------------------------------------------------ host packet step
 size_t pa_step_packet_layout(const pa_kv_pool_t *pool, int32_t num_seqs, int32_t num_q_heads,
                              int32_t max_pages, int32_t num_new, size_t *offsets) {
-  if (pool == nullptr || num_seqs < 0 || num_q_heads <= 0 || max_pages <= 0 || num_new < 0 ||
-      pool->num_kv_heads <= 0 || pool->head_dim <= 0)
+  if (pool == nullptr || num_seqs < 0 || num_q_heads <= 0 || max_pages <= 0 ||
+      (num_new < 0 && num_new != PA_STEP_NEWEST_PER_SEQ) || pool->num_kv_heads <= 0 ||
+      pool->head_dim <= 0)
     return 0;
   const size_t D = (size_t)pool->head_dim;
+  // one row per sequence (its newest token): no index sections
+  const size_t rows = num_new == PA_STEP_NEWEST_PER_SEQ ? (size_t)num_seqs : (size_t)num_new;
+  const size_t idx = num_new == PA_STEP_NEWEST_PER_SEQ ? 0 : (size_t)num_new;
   const size_t sizes[7] = {
-      (size_t)num_seqs * num_q_heads * D * 2,       // q
-      (size_t)num_new * pool->num_kv_heads * D * 2,  // k_new
-      (size_t)num_new * pool->num_kv_heads * D * 2,  // v_new
-      (size_t)num_new * 4,                           // seq_idx
-      (size_t)num_new * 4,                           // pos
+      (size_t)num_seqs * num_q_heads * D * 2,    // q
+      rows * pool->num_kv_heads * D * 2,         // k_new
+      rows * pool->num_kv_heads * D * 2,         // v_new
+      idx * 4,                                   // seq_idx
+      idx * 4,                                   // pos
       (size_t)num_seqs * max_pages * 4,              // block_tables
       (size_t)num_seqs * 4};                         // context_lens
   size_t at = 0;
@@ -686,13 +724,20 @@ pa_status_t pa_decode_step_host(const pa_kv_pool_t *pool, const void *packet_hos
   if (st != PA_OK) return st;
   char *pd = static_cast<char *>(packet_dev);
   const int32_t *tables = reinterpret_cast<const int32_t *>(pd + off[5]);
-  st = pa_kv_append(pool, pd + off[1], pd + off[2], reinterpret_cast<const int32_t *>(pd + off[3]),
-                    reinterpret_cast<const int32_t *>(pd + off[4]), num_new, tables, num_seqs,
-                    max_pages, d_err, stream);
-  if (st != PA_OK) return st;
-  st = pa_decode(pool, pd + off[0], num_seqs, num_q_heads, tables, max_pages,
-                 reinterpret_cast<const int32_t *>(pd + off[6]), scale, out_dev, workspace,
-                 workspace_bytes, num_splits, d_err, stream);
+  const int32_t *ctx = reinterpret_cast<const int32_t *>(pd + off[6]);
+  if (num_new == PA_STEP_NEWEST_PER_SEQ) {  // cache write fused into the decode
+    st = pa_decode_append(pool, pd + off[0], pd + off[1], pd + off[2], num_seqs, num_q_heads,
+                          tables, max_pages, ctx, scale, out_dev, workspace, workspace_bytes,
+                          num_splits, d_err, stream);
+  } else {
+    st = pa_kv_append(pool, pd + off[1], pd + off[2],
+                      reinterpret_cast<const int32_t *>(pd + off[3]),
+                      reinterpret_cast<const int32_t *>(pd + off[4]), num_new, tables, num_seqs,
+                      max_pages, d_err, stream);
+    if (st == PA_OK)
+      st = pa_decode(pool, pd + off[0], num_seqs, num_q_heads, tables, max_pages, ctx, scale,
+                     out_dev, workspace, workspace_bytes, num_splits, d_err, stream);
+  }
   if (st != PA_OK || num_seqs == 0) return st;
   st = cuda_status(cudaMemcpyAsync(out_host, out_dev,
                                    (size_t)num_seqs * num_q_heads * pool->head_dim * sizeof(float),

@@ -48,6 +48,7 @@
 
 #include "pa_device.cuh"
 #include "pa_internal.h"
+#include "pa_quant.cuh"
 
 // Tile configuration (warps per CTA, pipeline depth per warp, CTAs per SM the
 // register allocation must allow); overridable at build time for tuning.
@@ -598,6 +599,42 @@ __device__ __forceinline__ void finish_acc(WarpAcc<D, KVT> &acc, int t) {
 }
 
 
+// Fused cache write: store the K/V row of KV head h of sequence b's newest
+// token (bf16 k_new / v_new [B][Hkv][D]) into pool row `row`, as pa_kv_append
+// does (quantised pools through the same per-row quantisers, so the stored
+// bits are identical). Called by every thread of the CTA.
+template <int D, int KVT>
+__device__ __forceinline__ void append_new_row(const DecodeArgs &a, int b, int h, size_t row) {
+  const size_t src = ((size_t)b * a.hkv + h) * D * 2;  // bytes
+  unsigned char *kp = static_cast<unsigned char *>(const_cast<void *>(a.k_pool));
+  unsigned char *vp = static_cast<unsigned char *>(const_cast<void *>(a.v_pool));
+  if constexpr (KVT == PA_KV_BF16) {
+    for (int c = threadIdx.x; c < D / 8; c += blockDim.x) {
+      *reinterpret_cast<uint4 *>(kp + row * D * 2 + c * 16) = ldg_nc128(a.k_new + src + c * 16);
+      *reinterpret_cast<uint4 *>(vp + row * D * 2 + c * 16) = ldg_nc128(a.v_new + src + c * 16);
+    }
+  } else {
+    if (threadIdx.x < 32) {
+      const int lane = threadIdx.x;
+      float *ksz = const_cast<float *>(a.k_sz) + row * 2;
+      float *vsz = const_cast<float *>(a.v_sz) + row * 2;
+      float sk, sv;
+      if constexpr (KVT == PA_KV_U4_PER_TOKEN) {
+        sk = quantise_row_u4<D>(a.k_new + src, kp + row * (D / 2), ksz, lane);
+        sv = quantise_row_u4<D>(a.v_new + src, vp + row * (D / 2), vsz, lane);
+      } else if constexpr (KVT == PA_KV_FP8_PER_TOKEN) {
+        sk = quantise_row_fp8<D>(a.k_new + src, kp + row * D, ksz, lane);
+        sv = quantise_row_fp8<D>(a.v_new + src, vp + row * D, vsz, lane);
+      } else {
+        sk = quantise_row<D>(a.k_new + src, kp + row * D, ksz, lane);
+        sv = quantise_row<D>(a.v_new + src, vp + row * D, vsz, lane);
+      }
+      if (lane == 0 && !(fmaxf(sk, sv) < (float)PA_MAX_KV_SCALE))
+        flag_error(a.d_err, PA_DERR_BIG_SCALE);
+    }
+  }
+}
+
 template <int D, int P, int KVT, int W, int NSTAGE>
 __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(const DecodeArgs a) {
   using T = Tile<D, KVT>;
@@ -709,6 +746,18 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
   uint32_t qa[D / 16][2];  // per k-step: a0 (k 2t..2t+1), a2 (k 2t+8..2t+9)
   const float qsum = load_q<D, KVT>(qp, head_ok, t, qa);
   __syncthreads();  // tbl visible
+
+  // ---- fused cache write: the split whose pages hold the newest token
+  // (position ctx - 1) stores its row before any of the page is read
+  if (a.k_new != nullptr && ctx > 0 && split < a.S_main) {
+    const int lp_new = (ctx - 1) / P;
+    if (lp_new >= lp0 && lp_new < lp1) {  // CTA-uniform
+      const int page = tbl[lp_new - lp0];
+      if (page >= 0)
+        append_new_row<D, KVT>(a, b, h, ((size_t)page * a.hkv + h) * P + (ctx - 1) % P);
+      __syncthreads();  // the row is stored before the page is copied in
+    }
+  }
 
   // ---- per-warp pipeline ---------------------------------------------------------
   // Each lane copies 16-byte pieces of a block so that every copy instruction

@@ -51,6 +51,10 @@ struct DecodeArgs {
   int32_t range_mode;       // 1: a context shorter than tok_begin is an empty range,
                             //    not an error
   int32_t *d_err;
+  // fused cache write (pa_decode_append): bf16 [B][Hkv][D] rows of each
+  // sequence's newest token, stored at position ctx - 1 before it is read
+  const unsigned char *k_new = nullptr;
+  const unsigned char *v_new = nullptr;
 };
 
 struct PrefixArgs {

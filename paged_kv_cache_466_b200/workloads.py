@@ -73,6 +73,26 @@ class Workload:
                 torch.cat([self.prefill_k, self.step_k]),
                 torch.cat([self.prefill_v, self.step_v]))
 
+    def step_rows_by_sequence(self):
+        """The step rows laid out per sequence, as pa_decode_append takes them:
+        (k_new, v_new) bf16 [B, Hkv, D] with row b = sequence b's step token
+        and zeros for a sequence without one; None unless every step row is
+        its sequence's newest position (ctx_b - 1) and every sequence with
+        ctx_b >= 1 has one."""
+        ctx = self.context_lens
+        if len(set(self.step_seq.tolist())) != len(self.step_seq):
+            return None
+        if not np.array_equal(np.sort(self.step_seq), np.flatnonzero(ctx >= 1)):
+            return None
+        if not np.array_equal(self.step_pos, ctx[self.step_seq] - 1):
+            return None
+        k = torch.zeros((self.B, self.Hkv, self.D), dtype=torch.bfloat16)
+        v = torch.zeros_like(k)
+        idx = torch.from_numpy(self.step_seq.astype(np.int64))
+        k[idx] = self.step_k
+        v[idx] = self.step_v
+        return k, v
+
 
 def bits(t: torch.Tensor) -> np.ndarray:
     """bf16 tensor -> numpy uint16 array of its bit patterns (no copy if possible)."""

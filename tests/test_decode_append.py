@@ -1,0 +1,85 @@
+"""pa_decode_append: the newest token's cache write fused into the decode. It
+must store exactly what pa_kv_append stores (the whole pool byte for byte
+against the oracle's scatter and quantiser) and return exactly what
+pa_kv_append followed by pa_decode returns, bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from paged_kv_cache_466_b200 import (PA_DERR_BIG_SCALE, pa_decode, pa_decode_append)
+from paged_kv_cache_466_b200 import workloads as W
+from paged_kv_cache_466_b200.workloads import bits
+from tests.helpers import DEV, device_append, device_inputs, oracle_pool, pool_bytes_equal
+
+pytestmark = pytest.mark.gpu
+RAGGED = [0, 1, 5000, 17, 0, 3, 16, 32, 4096, 0, 2049, 15]
+
+
+@pytest.mark.parametrize("make", [
+    lambda: W.tiny(),
+    lambda: W.llama8b(B=6, ctx_range=(1, 700)),
+    lambda: W.paged("ragged", B=len(RAGGED), Hq=16, Hkv=4, D=128, P=16, context_lens=RAGGED,
+                    kv="bf16"),
+    lambda: W.int8(B=6, ctx_range=(1, 700)),
+    lambda: W.paged("ragged-u8", B=len(RAGGED), Hq=16, Hkv=4, D=128, P=32,
+                    context_lens=RAGGED, kv="u8", outlier_frac=0.02),
+    lambda: W.fp8(B=5, ctx_range=(1, 600)),
+    lambda: W.paged("u4d64", B=5, Hq=4, Hkv=2, D=64, P=32, ctx_range=(1, 300), kv="u4",
+                    outlier_frac=0.05),
+    lambda: W.int4(B=4, ctx_range=(1, 900)),
+], ids=["tiny", "llama8b", "ragged", "int8", "ragged-u8", "fp8", "u4-d64", "int4"])
+@pytest.mark.parametrize("splits", [0, 1, 3])
+def test_fused_step_equals_append_then_decode(make, splits):
+    w = make()
+    k_new, v_new = w.step_rows_by_sequence()
+    # reference: separate append, then decode
+    pool_a, bt, ctx, q = device_inputs(w, fill_byte=0x5A)
+    device_append(pool_a, w, bt)
+    want = pa_decode(pool_a, q, bt, ctx, w.scale, num_splits=splits)
+    # fused: the prefill rows, then one call
+    pool_b, _, _, _ = device_inputs(w, fill_byte=0x5A)
+    device_append(pool_b, w, bt, rows="prefill")
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    got = pa_decode_append(pool_b, q, k_new.to(DEV), v_new.to(DEV), bt, ctx, w.scale,
+                           num_splits=splits, d_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert torch.equal(got, want)
+    ok, msg = pool_bytes_equal(pool_b, oracle_pool(w, fill_byte=0x5A))
+    assert ok, msg
+    ref, _ = oracle.paged_attention(oracle_pool(w), bits(w.q), w.block_tables, w.context_lens,
+                                    w.scale)
+    assert np.abs(got.cpu().numpy().reshape(-1, w.D) - ref).max() <= 2e-3
+
+
+def test_fused_step_full_size_llama70b():
+    """The bench's workload and launch configuration (automatic splits)."""
+    w = W.llama70b()
+    k_new, v_new = w.step_rows_by_sequence()
+    pool, bt, ctx, q = device_inputs(w)
+    device_append(pool, w, bt, rows="prefill")
+    got = pa_decode_append(pool, q, k_new.to(DEV), v_new.to(DEV), bt, ctx, w.scale)
+    want = pa_decode(pool, q, bt, ctx, w.scale)   # the rows are in place now
+    torch.cuda.synchronize()
+    assert torch.equal(got, want)
+    # the stored step rows are the inputs, bit for bit
+    P = w.P
+    for b in (0, w.B // 2, w.B - 1):
+        pos = int(w.context_lens[b]) - 1
+        page = int(w.block_tables[b, pos // P])
+        assert torch.equal(pool.k[page, :, pos % P].cpu(), k_new[b])
+        assert torch.equal(pool.v[page, :, pos % P].cpu(), v_new[b])
+
+
+def test_fused_step_flags_scales_the_decode_cannot_take():
+    D, Hkv = 128, 2
+    w = W.paged("bigscale", B=2, Hq=2, Hkv=Hkv, D=D, P=16, context_lens=[3, 5], kv="u4")
+    k_new, v_new = w.step_rows_by_sequence()
+    k_new[1, 1] = torch.linspace(-4e4, 4e4, D).to(torch.bfloat16)   # span 8e4 > 15 * 4096
+    pool, bt, ctx, q = device_inputs(w)
+    device_append(pool, w, bt, rows="prefill")
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    pa_decode_append(pool, q, k_new.to(DEV), v_new.to(DEV), bt, ctx, w.scale, d_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & PA_DERR_BIG_SCALE

@@ -30,6 +30,10 @@ def test_packet_layout_is_packed_in_order_and_256_aligned():
         assert end <= nxt < end + 256
     assert p.nbytes % 256 == 0
     assert p.q.shape == (B, Hq, 128) and p.block_tables.shape == (B, mp)
+    # one row per sequence: B rows of K/V, no index sections
+    p1 = StepPacket(pool, B, Hq, mp, -1, pin=False)
+    assert p1.k_new.shape == (B, 8, 128) and p1.seq_idx.numel() == 0 and p1.pos.numel() == 0
+    assert p1.offsets[3] == p1.offsets[4] == p1.offsets[5]
     assert p.k_new.shape == (n, 8, 128) and p.context_lens.shape == (B,)
     # the views alias the packet bytes
     p.context_lens[1] = 0x01020304
@@ -103,3 +107,29 @@ def test_step_host_without_new_rows_and_bad_packet_size():
 def test_auto_splits_is_the_planner_for_a_bf16_d128_pool(B, Hkv, ctx, P):
     pool = KVPool(4, Hkv, P, 128, "bf16", DEV)
     assert pa_decode_auto_splits(B, Hkv, ctx, P) == pa_decode_num_splits(pool, B, -(-ctx // P))
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("make", [lambda: W.llama8b(B=6, ctx_range=(1, 700)),
+                                  lambda: W.int8(B=5, ctx_range=(1, 500))], ids=["bf16", "int8"])
+def test_step_host_one_row_per_sequence_runs_the_fused_step(make):
+    from paged_kv_cache_466_b200 import PA_STEP_NEWEST_PER_SEQ
+    w = make()
+    k_new, v_new = w.step_rows_by_sequence()
+    pool_a, bt, ctx, q = device_inputs(w)
+    device_append(pool_a, w, bt)
+    want = pa_decode(pool_a, q, bt, ctx, w.scale)
+    pool_b, _, _, _ = device_inputs(w)
+    device_append(pool_b, w, bt, rows="prefill")
+    packet = StepPacket(pool_b, w.B, w.Hq, w.max_pages, PA_STEP_NEWEST_PER_SEQ)
+    assert packet.k_new.shape == (w.B, w.Hkv, w.D) and packet.seq_idx.numel() == 0
+    packet.q.copy_(w.q)
+    packet.k_new.copy_(k_new)
+    packet.v_new.copy_(v_new)
+    packet.block_tables.copy_(torch.from_numpy(w.block_tables))
+    packet.context_lens.copy_(torch.from_numpy(w.context_lens))
+    out_host = torch.full((w.B, w.Hq, w.D), float("nan")).pin_memory()
+    pa_decode_step_host(pool_b, packet, w.scale, out_host)
+    assert torch.equal(out_host, want.cpu())
+    ok, msg = pool_bytes_equal(pool_b, oracle_pool(w))
+    assert ok, msg
