@@ -269,7 +269,7 @@ def run_ours(args, rank, world, local_rank):
                                          pa_decode_shared_prefix_workspace_bytes,
                                          pa_decode_window, pa_decode_window_workspace_bytes,
                                          pa_decode_workspace_bytes, pa_kv_append,
-                                         pa_decode_append, StepPacket, pa_decode_step_host,
+                                         pa_decode_append, StepPacket, StepGraph,
                                          PA_STEP_NEWEST_PER_SEQ)
 
     dev = torch.device("cuda", local_rank)
@@ -388,6 +388,7 @@ def run_ours(args, rank, world, local_rank):
     h_bt = torch.from_numpy(w.block_tables).pin_memory()
     h_out = torch.empty((w.B, w.Hq, w.D), dtype=torch.float32).pin_memory()
     d2h = h_out.numel() * h_out.element_size()
+    graph = None
     if not args.cascade and args.window == 0:
         # the library's host-packet step: one H2D copy of the packed inputs,
         # append, decode and one D2H copy of the output, in one C-ABI call
@@ -403,10 +404,11 @@ def run_ours(args, rank, world, local_rank):
                         (packet.block_tables, h_bt)) + fills:
             view.copy_(h)
         h2d = packet.nbytes
+        # the step captured once into a CUDA graph: one graph launch per step
+        graph = StepGraph(pool, packet, w.scale, h_out, out_dev=out, workspace=ws, num_splits=S)
 
         def e2e_step():
-            pa_decode_step_host(pool, packet, w.scale, h_out, out_dev=out, workspace=ws,
-                                num_splits=S, stream=stream, synchronize=True)
+            graph.launch(stream=stream, synchronize=True)
     else:
         h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_seq, h_pos, h_ctx,
                                                          h_bt))
@@ -437,6 +439,8 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     ems = max_over_ranks(e0.elapsed_time(e1), world, dev)
     e2e_value = whole_job_gbs(step_bytes, world, ems / Ke)
+    if graph is not None:
+        graph.close()
 
     peak, peak_kind = measured_peak()
     dec_avg_ms = statistics.mean(dec_ms)

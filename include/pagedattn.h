@@ -501,6 +501,36 @@ pa_status_t pa_decode_step_host(const pa_kv_pool_t *pool, const void *packet_hos
                                 int32_t *d_err, void *stream, int32_t synchronize);
 
 /*
+ * A pa_decode_step_host step captured once into a CUDA graph and replayed:
+ * per step the host then makes one graph launch instead of one copy, one or
+ * two kernel launches and a second copy. Every pointer and size is fixed at
+ * creation; each launch copies whatever packet_host holds at that time, so
+ * the caller refills the packet (and reads out_host) between launches.
+ *
+ * pa_step_graph_create — arguments as for pa_decode_step_host (minus stream
+ *   and synchronize; packet_host and out_host must be page-locked, as graph
+ *   copies require); plans the step, captures it on a private stream and
+ *   instantiates the graph into *graph (caller-owned, released with
+ *   pa_step_graph_destroy). Errors: those of pa_decode_step_host, or
+ *   PA_ERR_CUDA when capture or instantiation fails; *graph is then NULL.
+ * pa_step_graph_launch — launches the step on `stream`; synchronize != 0
+ *   waits for it (out_host then holds the result).
+ * pa_step_graph_destroy — releases the graph (NULL is ignored); no launch of
+ *   it may still be pending.
+ */
+typedef struct pa_step_graph pa_step_graph_t;
+
+pa_status_t pa_step_graph_create(const pa_kv_pool_t *pool, const void *packet_host,
+                                 void *packet_dev, size_t packet_bytes,
+                                 int32_t num_seqs, int32_t num_q_heads,
+                                 int32_t max_pages, int32_t num_new, float scale,
+                                 float *out_dev, float *out_host, void *workspace,
+                                 size_t workspace_bytes, int32_t num_splits,
+                                 int32_t *d_err, pa_step_graph_t **graph);
+pa_status_t pa_step_graph_launch(pa_step_graph_t *graph, void *stream, int32_t synchronize);
+void pa_step_graph_destroy(pa_step_graph_t *graph);
+
+/*
  * pa_selftest_wait_timeout — exercises the failure path of the kernels'
  * bounded waits (the tcgen05 prefix pass waits on mbarriers for its tensor-
  * core work): one thread waits on an mbarrier that nothing arrives at, gives

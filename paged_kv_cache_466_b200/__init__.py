@@ -43,7 +43,7 @@ __all__ = ["KVPool", "pa_kv_append", "pa_decode", "pa_decode_append", "pa_decode
            "pa_decode_shared_prefix", "pa_decode_shared_prefix_workspace_bytes",
            "pa_decode_window", "pa_decode_window_workspace_bytes",
            "pa_decode_range", "pa_decode_range_workspace_bytes", "pa_merge_partials",
-           "pa_validate_tables", "StepPacket", "pa_decode_step_host", "pa_derr_status",
+           "pa_validate_tables", "StepPacket", "pa_decode_step_host", "StepGraph", "pa_derr_status",
            "pa_decode_auto_splits", "pa_selftest_wait_timeout", "PA_DERR_TIMEOUT",
            "PA_STEP_NEWEST_PER_SEQ",
            "pa_decode_num_splits", "pa_decode_workspace_bytes", "PagedAttnError",
@@ -404,6 +404,68 @@ def pa_decode_step_host(pool: KVPool, packet: StepPacket, scale: float, out_host
         _ptr(d_err), _stream(stream), 1 if synchronize else 0)
     _lib.check(st, "pa_decode_step_host")
     return out_host
+
+
+class StepGraph:
+    """A ``pa_decode_step_host`` step captured once into a CUDA graph: each
+    ``launch`` copies the packet's current contents to the device, runs the
+    step and copies the output into ``out_host`` with one graph launch. Refill
+    the packet's views between launches; every buffer is fixed at creation."""
+
+    def __init__(self, pool: KVPool, packet: StepPacket, scale: float, out_host: torch.Tensor,
+                 out_dev: Optional[torch.Tensor] = None,
+                 workspace: Optional[torch.Tensor] = None, num_splits: int = 0,
+                 d_err: Optional[torch.Tensor] = None):
+        B, Hq, max_pages, num_new = packet.shape
+        D = pool.head_dim
+        dev = pool.device
+        if packet.dev is None or not packet.host.is_pinned():
+            raise ValueError("StepGraph: the packet needs a page-locked host buffer and a "
+                             "device copy")
+        if out_host.dtype != torch.float32 or not out_host.is_pinned() \
+                or not out_host.is_contiguous() or tuple(out_host.shape) != (B, Hq, D):
+            raise ValueError("StepGraph: out_host must be a page-locked contiguous fp32 "
+                             "[B, Hq, D]")
+        if out_dev is None:
+            out_dev = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+        _need(out_dev, "out_dev", torch.float32, dev)
+        if workspace is None:
+            need = pa_decode_workspace_bytes(B, Hq, D,
+                                             pa_decode_num_splits(pool, B, max_pages, num_splits))
+            if need > 0:
+                workspace = torch.zeros(need, dtype=torch.uint8, device=dev)
+        ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        # keep every buffer the graph points at alive as long as the graph
+        self._keep = (pool, packet, out_host, out_dev, workspace, d_err)
+        self.out_host = out_host
+        handle = ctypes.c_void_p()
+        st = _lib.load().pa_step_graph_create(
+            ctypes.byref(pool.c), ctypes.c_void_p(packet.host.data_ptr()), _ptr(packet.dev),
+            packet.nbytes, B, Hq, max_pages, num_new, float(scale), _ptr(out_dev),
+            ctypes.c_void_p(out_host.data_ptr()), _ptr(workspace), ws_bytes, num_splits,
+            _ptr(d_err), ctypes.byref(handle))
+        _lib.check(st, "pa_step_graph_create")
+        self._handle = handle
+
+    def launch(self, stream=None, synchronize: bool = True) -> torch.Tensor:
+        if self._handle is None:
+            raise ValueError("StepGraph: already closed")
+        _lib.check(_lib.load().pa_step_graph_launch(self._handle, _stream(stream),
+                                                    1 if synchronize else 0),
+                   "pa_step_graph_launch")
+        return self.out_host
+
+    def close(self) -> None:
+        if getattr(self, "_handle", None) is not None:
+            torch.cuda.synchronize(self._keep[3].device)
+            _lib.load().pa_step_graph_destroy(self._handle)
+            self._handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def pa_decode_noalloc(pool: KVPool, q: torch.Tensor, block_tables: torch.Tensor,

@@ -78,6 +78,10 @@ SIGNATURES = {
     "pa_step_packet_layout": (ctypes.c_size_t, [_POOL, _I, _I, _I, _I, _P]),
     "pa_decode_step_host": (_I, [_POOL, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, ctypes.c_float,
                                  _P, _P, _P, ctypes.c_size_t, _I, _P, _P, _I]),
+    "pa_step_graph_create": (_I, [_POOL, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, ctypes.c_float,
+                                  _P, _P, _P, ctypes.c_size_t, _I, _P, _P]),
+    "pa_step_graph_launch": (_I, [_P, _P, _I]),
+    "pa_step_graph_destroy": (None, [_P]),
     "pa_merge_partials": (_I, [_P, _P, _I, _I, _I, ctypes.c_int64, ctypes.c_int64, _P, _P,
                                 _P]),
     "pa_splitkv_reduce": (_I, [_P, _P, _I, _I, _I, _I, _P, _P]),

@@ -4,6 +4,7 @@
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
+#include <new>
 #include <string>
 
 #include "pa_internal.h"
@@ -745,6 +746,86 @@ pa_status_t pa_decode_step_host(const pa_kv_pool_t *pool, const void *packet_hos
                    "pa_decode_step_host output copy");
   if (st != PA_OK || !synchronize) return st;
   return cuda_status(cudaStreamSynchronize(s), "pa_decode_step_host synchronize");
+}
+
+// ------------------------------------------------------------ captured step
+struct pa_step_graph {
+  cudaGraphExec_t exec;
+};
+
+pa_status_t pa_step_graph_create(const pa_kv_pool_t *pool, const void *packet_host,
+                                 void *packet_dev, size_t packet_bytes, int32_t num_seqs,
+                                 int32_t num_q_heads, int32_t max_pages, int32_t num_new,
+                                 float scale, float *out_dev, float *out_host, void *workspace,
+                                 size_t workspace_bytes, int32_t num_splits, int32_t *d_err,
+                                 pa_step_graph_t **graph) {
+  g_last_error.clear();
+  if (graph == nullptr) return fail(PA_ERR_INVALID_ARG, "graph is NULL");
+  *graph = nullptr;
+  pa_status_t st = check_pool(pool);
+  if (st != PA_OK) return st;
+  if (num_seqs <= 0 || num_q_heads <= 0 || max_pages <= 0)
+    return fail(PA_ERR_INVALID_ARG, "num_seqs=%d num_q_heads=%d max_pages=%d", num_seqs,
+                num_q_heads, max_pages);
+  // plan (and set the kernels' shared-memory limits) before capturing, so
+  // that capture records stream work only
+  if (pa_decode_num_splits(pool, num_seqs, max_pages, num_splits) <= 0)
+    return fail(PA_ERR_INVALID_ARG, "could not plan splits");
+  cudaStream_t cs = nullptr;
+  st = cuda_status(cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking),
+                   "pa_step_graph_create stream");
+  if (st != PA_OK) return st;
+  st = cuda_status(cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal),
+                   "pa_step_graph_create begin capture");
+  if (st != PA_OK) {
+    cudaStreamDestroy(cs);
+    return st;
+  }
+  const pa_status_t step = pa_decode_step_host(pool, packet_host, packet_dev, packet_bytes,
+                                               num_seqs, num_q_heads, max_pages, num_new, scale,
+                                               out_dev, out_host, workspace, workspace_bytes,
+                                               num_splits, d_err, cs, 0);
+  const std::string step_error = g_last_error;
+  cudaGraph_t g = nullptr;
+  const cudaError_t end = cudaStreamEndCapture(cs, &g);
+  cudaStreamDestroy(cs);
+  if (step != PA_OK) {
+    if (g) cudaGraphDestroy(g);
+    g_last_error = step_error;
+    return step;
+  }
+  if (end != cudaSuccess || g == nullptr) {
+    if (g) cudaGraphDestroy(g);
+    return cuda_status(end != cudaSuccess ? end : cudaErrorUnknown,
+                       "pa_step_graph_create end capture");
+  }
+  cudaGraphExec_t exec = nullptr;
+  const cudaError_t inst = cudaGraphInstantiate(&exec, g, 0);
+  cudaGraphDestroy(g);
+  if (inst != cudaSuccess) return cuda_status(inst, "pa_step_graph_create instantiate");
+  pa_step_graph *h = new (std::nothrow) pa_step_graph;
+  if (h == nullptr) {
+    cudaGraphExecDestroy(exec);
+    return fail(PA_ERR_INVALID_ARG, "out of host memory");
+  }
+  h->exec = exec;
+  *graph = h;
+  return PA_OK;
+}
+
+pa_status_t pa_step_graph_launch(pa_step_graph_t *graph, void *stream, int32_t synchronize) {
+  g_last_error.clear();
+  if (graph == nullptr) return fail(PA_ERR_INVALID_ARG, "graph is NULL");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  pa_status_t st = cuda_status(cudaGraphLaunch(graph->exec, s), "pa_step_graph_launch");
+  if (st != PA_OK || !synchronize) return st;
+  return cuda_status(cudaStreamSynchronize(s), "pa_step_graph_launch synchronize");
+}
+
+void pa_step_graph_destroy(pa_step_graph_t *graph) {
+  if (graph == nullptr) return;
+  cudaGraphExecDestroy(graph->exec);
+  delete graph;
 }
 
 pa_status_t pa_merge_partials(const float *o_parts, const float *lse_parts, int32_t num_parts,

@@ -159,3 +159,14 @@ def test_selftest_wait_timeout_rejects_bad_limits(lib):
     assert lib.pa_selftest_wait_timeout(0, 0x1000, None) == PA_ERR_INVALID_ARG
     assert lib.pa_selftest_wait_timeout(2_000_000, 0x1000, None) == PA_ERR_INVALID_ARG
     assert lib.pa_selftest_wait_timeout(100, None, None) == PA_ERR_INVALID_ARG
+
+
+def test_step_graph_rejects_bad_arguments(lib):
+    h = ctypes.c_void_p(1234)
+    st = lib.pa_step_graph_create(None, None, None, 0, 1, 1, 1, 1, 0.1, None, None, None, 0, 0,
+                                  None, ctypes.byref(h))
+    assert st == PA_ERR_INVALID_ARG and h.value is None
+    assert lib.pa_step_graph_create(ctypes.byref(_pool()), None, None, 0, 0, 1, 1, 1, 0.1, None,
+                                    None, None, 0, 0, None, ctypes.byref(h)) == PA_ERR_INVALID_ARG
+    assert lib.pa_step_graph_launch(None, None, 1) == PA_ERR_INVALID_ARG
+    lib.pa_step_graph_destroy(None)

@@ -133,3 +133,38 @@ def test_step_host_one_row_per_sequence_runs_the_fused_step(make):
     assert torch.equal(out_host, want.cpu())
     ok, msg = pool_bytes_equal(pool_b, oracle_pool(w))
     assert ok, msg
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("per_seq", [True, False], ids=["fused", "append+decode"])
+def test_step_graph_replays_the_step_with_new_packet_contents(per_seq):
+    from paged_kv_cache_466_b200 import PA_STEP_NEWEST_PER_SEQ, StepGraph
+    w = W.int8(B=5, ctx_range=(1, 500))
+    pool, bt, ctx, q = device_inputs(w)
+    device_append(pool, w, bt, rows="prefill")
+    n = PA_STEP_NEWEST_PER_SEQ if per_seq else len(w.step_seq)
+    packet = StepPacket(pool, w.B, w.Hq, w.max_pages, n)
+    if per_seq:
+        k_new, v_new = w.step_rows_by_sequence()
+        packet.k_new.copy_(k_new)
+        packet.v_new.copy_(v_new)
+    else:
+        packet.k_new.copy_(w.step_k)
+        packet.v_new.copy_(w.step_v)
+        packet.seq_idx.copy_(torch.from_numpy(w.step_seq))
+        packet.pos.copy_(torch.from_numpy(w.step_pos))
+    packet.block_tables.copy_(torch.from_numpy(w.block_tables))
+    packet.context_lens.copy_(torch.from_numpy(w.context_lens))
+    out_host = torch.full((w.B, w.Hq, w.D), float("nan")).pin_memory()
+    graph = StepGraph(pool, packet, w.scale, out_host)
+    try:
+        for scale_q in (1.0, -0.5):          # new query each step, same cache
+            qq = (w.q.float() * scale_q).to(torch.bfloat16)
+            packet.q.copy_(qq)
+            got = graph.launch().clone()
+            want = pa_decode(pool, qq.to(DEV), bt, ctx, w.scale).cpu()
+            assert torch.equal(got, want)
+        ok, msg = pool_bytes_equal(pool, oracle_pool(w))
+        assert ok, msg
+    finally:
+        graph.close()
