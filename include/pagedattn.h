@@ -64,8 +64,9 @@ typedef enum {
 #define PA_DERR_BAD_CTX 2  /* context_len < 0 or > max_pages * page_size       */
 #define PA_DERR_BAD_SEQ 4  /* append: seq_idx outside [0, num_seqs)            */
 #define PA_DERR_BAD_POS 8  /* append: pos < 0 or pos / page_size >= max_pages  */
-#define PA_DERR_BIG_SCALE 16 /* append: a quantised row's scale is not below
-                                PA_MAX_KV_SCALE (the row is still written)     */
+#define PA_DERR_BIG_SCALE 16 /* append (and the fused cache write of
+                                pa_decode_append): a quantised row's scale is
+                                not below PA_MAX_KV_SCALE (still written)      */
 #define PA_DERR_TIMEOUT 32 /* a bounded wait on the kernel's own tensor-core
                               work ran out (not expected; outputs invalid)    */
 
@@ -112,8 +113,8 @@ typedef struct {
   int32_t dtype;      /* pa_kv_dtype_t */
   void *k_pool;       /* (device) */
   void *v_pool;       /* (device) */
-  float *k_sz;        /* (device) INT8 only, else NULL */
-  float *v_sz;        /* (device) INT8 only, else NULL */
+  float *k_sz;        /* (device) INT8, FP8 and INT4 pools, else NULL */
+  float *v_sz;        /* (device) INT8, FP8 and INT4 pools, else NULL */
 } pa_kv_pool_t;
 
 /*
