@@ -164,6 +164,16 @@ int32_t pa_decode_num_splits(const pa_kv_pool_t *pool, int32_t num_seqs,
                              int32_t max_pages, int32_t requested);
 
 /*
+ * pa_decode_plan_splits — the planning rule of pa_decode_num_splits as a pure
+ * host function (no device access), for num_units (sequence, KV head) units,
+ * a table of max_pages pages of page_size tokens, and a device with num_sms
+ * SMs holding ctas_per_sm decode CTAs each. requested as for
+ * pa_decode_num_splits (0 = automatic). Returns <= 0 on invalid arguments.
+ */
+int32_t pa_decode_plan_splits(int64_t num_units, int32_t max_pages, int32_t page_size,
+                              int32_t num_sms, int32_t ctas_per_sm, int32_t requested);
+
+/*
  * pa_decode_auto_splits — the split count pa_decode picks with
  * num_splits == 0 for a batch of num_seqs sequences whose longest context is
  * max_ctx tokens, in a bf16 pool of head_dim 128 with num_kv_heads heads and

@@ -180,22 +180,19 @@ pa_status_t pa_kv_append(const pa_kv_pool_t *pool, const void *k_new, const void
                      "pa_kv_append launch");
 }
 
-int32_t pa_decode_num_splits(const pa_kv_pool_t *pool, int32_t num_seqs, int32_t max_pages,
-                             int32_t requested) {
-  if (pool == nullptr || num_seqs < 0 || max_pages <= 0 || requested < 0) return -1;
-  if ((pool->head_dim != 64 && pool->head_dim != 128) ||
-      (pool->page_size != 16 && pool->page_size != 32) ||
-      pool->dtype < PA_KV_BF16 || pool->dtype > PA_KV_U4_PER_TOKEN ||
-      pool->num_kv_heads <= 0)
+int32_t pa_decode_plan_splits(int64_t num_units, int32_t max_pages, int32_t page_size,
+                              int32_t num_sms, int32_t ctas_per_sm, int32_t requested) {
+  if (num_units < 0 || max_pages <= 0 || page_size <= 0 || num_sms <= 0 || ctas_per_sm <= 0 ||
+      requested < 0)
     return -1;
-  const int P = pool->page_size;
+  const int P = page_size;
   const int hi = max_pages < kMaxSplits ? max_pages : kMaxSplits;
   int S = requested;
   if (S == 0) {
-    // R = SMs x CTAs/SM resident CTA slots; a unit is one (sequence, KV head).
-    const long long units = (long long)num_seqs * pool->num_kv_heads;
-    const long long sms = device_sm_count();
-    const long long R = sms * cached_ctas_per_sm(pool->head_dim, P, pool->dtype);
+    // R resident CTA slots; a unit is one (sequence, KV head).
+    const long long units = num_units;
+    const long long sms = num_sms;
+    const long long R = sms * ctas_per_sm;
     // CTAs that stream at once and keep HBM saturated: measured on the
     // Llama-3-70B shapes (B = 8, 16, 32 x 8192 tokens), one wave of ~1.7
     // CTAs per SM read at 79-103 % of the copy peak, and it was the fastest
@@ -239,6 +236,22 @@ int32_t pa_decode_num_splits(const pa_kv_pool_t *pool, int32_t num_seqs, int32_t
   if (S < 1) S = 1;
   const int chunk = (max_pages + S - 1) / S;
   return (max_pages + chunk - 1) / chunk;
+}
+
+int32_t pa_decode_num_splits(const pa_kv_pool_t *pool, int32_t num_seqs, int32_t max_pages,
+                             int32_t requested) {
+  if (pool == nullptr || num_seqs < 0 || max_pages <= 0 || requested < 0) return -1;
+  if ((pool->head_dim != 64 && pool->head_dim != 128) ||
+      (pool->page_size != 16 && pool->page_size != 32) ||
+      pool->dtype < PA_KV_BF16 || pool->dtype > PA_KV_U4_PER_TOKEN ||
+      pool->num_kv_heads <= 0)
+    return -1;
+  const int64_t units = (int64_t)num_seqs * pool->num_kv_heads;
+  if (requested > 0)  // no device query needed
+    return pa_decode_plan_splits(units, max_pages, pool->page_size, 1, 1, requested);
+  return pa_decode_plan_splits(units, max_pages, pool->page_size, device_sm_count(),
+                               cached_ctas_per_sm(pool->head_dim, pool->page_size, pool->dtype),
+                               0);
 }
 
 int32_t pa_decode_auto_splits(int32_t num_seqs, int32_t num_kv_heads, int32_t max_ctx,

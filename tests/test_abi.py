@@ -170,3 +170,26 @@ def test_step_graph_rejects_bad_arguments(lib):
                                     None, None, 0, 0, None, ctypes.byref(h)) == PA_ERR_INVALID_ARG
     assert lib.pa_step_graph_launch(None, None, 1) == PA_ERR_INVALID_ARG
     lib.pa_step_graph_destroy(None)
+
+
+def test_split_plan_rules_on_a_b200(lib):
+    """The planner's two regimes with the B200's 148 SMs and 3 decode CTAs per
+    SM (R = 444 slots). One wave when the units fit: the fewest splits that
+    give ~1.7 CTAs per SM (252), never a second wave. Otherwise the wave model
+    (the split counts measured best on the Llama-3-shaped batches)."""
+    plan = lambda units, pages, P, req=0, sms=148, cps=3: lib.pa_decode_plan_splits(
+        units, pages, P, sms, cps, req)
+    assert plan(32 * 8, 256, 32) == 1          # Llama-3-70B B=32 x 8192: one CTA per unit
+    assert plan(16 * 8, 256, 32) == 2
+    assert plan(8 * 8, 256, 32) == 4
+    assert plan(250, 256, 32) == 1             # 2 splits would spill past 444 slots
+    assert plan(200, 256, 32) == 2
+    assert plan(32 * 8, 65, 32) == 1           # the 2048-token window + sink pages
+    assert plan(64 * 8, 256, 16) == 4          # ragged Llama-3-8B-shaped batch (wave model)
+    assert plan(64 * 8, 256, 32) == 6          # B=64 x 8192 (wave model)
+    assert plan(0, 10, 16) == 1
+    assert plan(8, 4, 16) == 4                 # no more splits than pages
+    assert plan(64, 256, 32, req=5) == 5
+    assert plan(4, 4000, 32, req=1) == 2       # a split stages at most 2048 table entries
+    assert plan(100, 256, 32, sms=132, cps=2) == 2   # another GPU: R = 264, target 225
+    assert plan(-1, 4, 16) <= 0 and plan(4, 0, 16) <= 0 and plan(4, 4, 16, sms=0) <= 0
