@@ -138,3 +138,68 @@ def test_packed_partial_layout():
     for r in range(world):
         assert torch.equal(o_parts[r].flatten(), torch.arange(B * Hq * D, dtype=torch.float32) + 1000 * r)
         assert torch.equal(l_parts[r].flatten(), torch.arange(B * Hq, dtype=torch.float32) - 1000 * r)
+
+
+def _cp_api_worker(rank, world, port, q):
+    """decode_context_parallel itself on gloo ranks, with the two library calls
+    replaced by the oracle (same signatures, same output buffers): checks the
+    packing, the single all-gather and the strided merge views end to end."""
+    import types
+    import oracle
+    from paged_kv_cache_466_b200 import context_parallel as cp
+    from paged_kv_cache_466_b200 import workloads as W
+    from paged_kv_cache_466_b200.workloads import bits
+    from tests.helpers import oracle_pool
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = W.paged("cpapi", B=4, Hq=8, Hkv=2, D=64, P=16, context_lens=[1, 40, 130, 300],
+                    kv="u8")
+        hp = oracle_pool(w)
+        calls = []
+
+        def fake_range(pool, qq, bt, ctx, scale, b, e, o_out=None, lse_out=None, **kw):
+            calls.append((b, e))
+            o, l = oracle.paged_attention(pool.hp, bits(qq), bt.numpy(), ctx.numpy(), scale,
+                                          t_begin=b, t_end=e if e < 0x7FFFFFFF else -1)
+            o_out.copy_(torch.from_numpy(o).view(o_out.shape))
+            lse_out.copy_(torch.from_numpy(l).view(lse_out.shape))
+            return o_out, lse_out
+
+        def fake_merge(o_parts, lse_parts, out=None, lse_out=None, stream=None):
+            n, D = o_parts.shape[0], o_parts.shape[-1]
+            m = oracle.lse_merge(o_parts.double().numpy().reshape(n, -1, D).transpose(1, 0, 2),
+                                 lse_parts.double().numpy().reshape(n, -1).T)
+            res = torch.from_numpy(m).float().view(o_parts.shape[1:])
+            if out is not None:
+                out.copy_(res)
+                res = out
+            return res, None
+
+        cp.pa_decode_range, cp.pa_merge_partials = fake_range, fake_merge
+        pool = types.SimpleNamespace(page_size=w.P, hp=hp)
+        out = cp.decode_context_parallel(pool, w.q, torch.from_numpy(w.block_tables),
+                                         torch.from_numpy(w.context_lens), w.scale,
+                                         tokens_per_rank=64)
+        full, _ = oracle.paged_attention(hp, bits(w.q), w.block_tables, w.context_lens, w.scale)
+        err = float(np.abs(out.double().numpy().reshape(-1, w.D) - full).max())
+        q.put((rank, calls, err))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_decode_context_parallel_orchestration_on_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    world = 3
+    procs = [ctx.Process(target=_cp_api_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=180) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [r[1] for r in res] == [[(0, 64)], [(64, 128)], [(128, 0x7FFFFFFF)]]
+    for _, _, err in res:
+        assert err <= 1e-6
