@@ -2,7 +2,7 @@
  * pagedattn — single-token decode attention over a paged KV cache, for
  * NVIDIA B200 (sm_100a).  C ABI of libpagedattn.so.
  *
- * The method (all citations are to the surveyed web pages):
+ * The method (citations name the web pages by title and section):
  *  - "KV-Cache Optimization Techniques", section "PagedAttention (vLLM)":
  *    the cache is kept in fixed-size pages of P tokens in one physical pool;
  *    each request has a page table mapping its logical KV positions to
