@@ -102,7 +102,10 @@ def recorded_traffic(workload: str):
         rec = json.load(open(TRAFFIC_FILE))
         src_sha = hashlib.sha256(open(DECODE_SRC, "rb").read()).hexdigest()
         r = rec.get(workload)
-        if r and r.get("decode_cu_sha256") == src_sha:
+        # a record stays valid for a later source only where it says why
+        # (changes confined to code the recorded kernel does not instantiate)
+        if r and (r.get("decode_cu_sha256") == src_sha or
+                  src_sha in r.get("also_valid_for_decode_cu_sha256", [])):
             return int(r["dram_bytes_per_launch"])
     except Exception:
         pass

@@ -40,8 +40,8 @@
 // with z = 0): with x = s*c + z per row,
 //   q.x = s (q.c) + z sum(q)          and    sum_t p_t x_t = sum_t (p_t s_t) c_t + sum_t p_t z_t,
 // so the codes go through the tensor cores as exact f16 values (INT8 codes as
-// integers, E4M3 codes converted exactly) and the scale and zero are applied
-// once per (token, head) instead of once per element.
+// the subnormals c * 2^-24, E4M3 codes converted exactly) and the scale and
+// zero are applied once per (token, head) instead of once per element.
 #include <atomic>
 #include <cfloat>
 #include <cmath>
@@ -87,6 +87,10 @@ struct Tile {
   static constexpr bool kU8 = KVT != PA_KV_BF16;
   static constexpr bool kFp8 = KVT == PA_KV_FP8_PER_TOKEN;
   static constexpr bool kU4 = KVT == PA_KV_U4_PER_TOKEN;  // two codes per byte
+  // Codes reach the MMA scaled by an exact power of two (INT8 c * 2^-24 as an
+  // f16 subnormal, INT4 c * 2^-9 through the E4M3 converter; FP8 codes as
+  // they are); the K scale and O after the loop take it back.
+  static constexpr float kCodeScale = kU4 ? 512.f : (kFp8 ? 1.f : 16777216.f);
   static constexpr int kElem = kU8 ? 1 : 2;
   static constexpr int kRowBytes = kU4 ? D / 2 : D * kElem;
   // one 16-token block of K (or V) is 16 contiguous rows of the page
@@ -429,11 +433,10 @@ __device__ __forceinline__ void block_step(const LaneMap<D, KVT> &lm, uint32_t s
     vs[1] = __uint_as_float(v01.z); vz[1] = __uint_as_float(v01.w);
     vs[2] = __uint_as_float(v89.x); vz[2] = __uint_as_float(v89.y);
     vs[3] = __uint_as_float(v89.z); vz[3] = __uint_as_float(v89.w);
-    // INT4 codes reach the MMA as c * 2^-9: the exact power of two goes
-    // back into the K scale here and into O after the loop
-    constexpr float kCodeScale = T::kU4 ? 512.f : 1.f;
+    // the codes' power-of-two scale goes back into the K scale here (and
+    // into O after the loop)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) x[e] = fmaf(ks[e] * kCodeScale, x[e], kz[e] * qsum);
+    for (int e = 0; e < 4; ++e) x[e] = fmaf(ks[e] * T::kCodeScale, x[e], kz[e] * qsum);
   }
   if (pvalid && btok >= tok_lo && btok + 16 <= tok1) {  // warp-uniform: no mask needed
 #pragma unroll
@@ -587,13 +590,12 @@ __device__ __forceinline__ void finish_acc(WarpAcc<D, KVT> &acc, int t) {
     zacc += __shfl_xor_sync(0xffffffffu, zacc, 2);
     const float z0 = __shfl_sync(0xffffffffu, zacc, 8 * t);
     const float z1 = __shfl_sync(0xffffffffu, zacc, 8 * t + 4);
-    constexpr float kCodeScale = T::kU4 ? 512.f : 1.f;  // INT4 codes were c * 2^-9
 #pragma unroll
-    for (int j = 0; j < T::kMTiles; ++j) {
-      o[j][0] = fmaf(o[j][0], kCodeScale, z0);
-      o[j][1] = fmaf(o[j][1], kCodeScale, z1);
-      o[j][2] = fmaf(o[j][2], kCodeScale, z0);
-      o[j][3] = fmaf(o[j][3], kCodeScale, z1);
+    for (int j = 0; j < T::kMTiles; ++j) {  // undo the codes' power-of-two scale
+      o[j][0] = fmaf(o[j][0], T::kCodeScale, z0);
+      o[j][1] = fmaf(o[j][1], T::kCodeScale, z1);
+      o[j][2] = fmaf(o[j][2], T::kCodeScale, z0);
+      o[j][3] = fmaf(o[j][3], T::kCodeScale, z1);
     }
   }
 }

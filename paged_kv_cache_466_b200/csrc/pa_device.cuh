@@ -150,14 +150,12 @@ __device__ __forceinline__ void split_f16(float p0, float p1, uint32_t &hi,
   lo = pack_f16(p0 - f16_lo(hi), p1 - f16_hi(hi));
 }
 
-// Two uint8 codes -> f16x2 holding exactly (code_a, code_b). The byte lands in
-// the low mantissa byte of 1024.0h (0x6400 | c == 1024 + c), then 1024 is
-// subtracted, which is exact.
+// Two uint8 codes -> f16x2 holding exactly (code_a * 2^-24, code_b * 2^-24):
+// a byte under a zero high byte is the f16 subnormal c * 2^-24, so one byte
+// permute builds the pair and nothing is added or subtracted. The caller
+// puts the exact 2^24 back into the row scale.
 __device__ __forceinline__ uint32_t u8x2_to_f16x2(uint32_t word, uint32_t sel) {
-  const uint32_t biased = __byte_perm(word, 0x64646464u, sel);
-  uint32_t r;
-  asm("sub.rn.f16x2 %0, %1, %2;\n" : "=r"(r) : "r"(biased), "r"(0x64006400u));
-  return r;
+  return __byte_perm(word, 0u, sel);
 }
 
 // Four bytes, each holding a 4-bit code c in its low nibble (high nibble 0),
