@@ -193,3 +193,23 @@ def test_split_plan_rules_on_a_b200(lib):
     assert plan(4, 4000, 32, req=1) == 2       # a split stages at most 2048 table entries
     assert plan(100, 256, 32, sms=132, cps=2) == 2   # another GPU: R = 264, target 225
     assert plan(-1, 4, 16) <= 0 and plan(4, 0, 16) <= 0 and plan(4, 4, 16, sms=0) <= 0
+
+
+def test_header_compiles_as_c99_and_host_calls_work(lib, tmp_path):
+    """The header is plain C: a C99 program built against it alone links the
+    library and runs every entry point that needs no GPU."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    libdir = os.path.dirname(_lib.LIB_PATH)
+    exe = str(tmp_path / "abi_host_calls")
+    src = os.path.join(ROOT, "tests", "c", "abi_host_calls.c")
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        src, "-o", exe, "-L", libdir, "-lpagedattn", "-Wl,-rpath," + libdir],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "ok" in r.stdout
