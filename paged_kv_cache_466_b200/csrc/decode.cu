@@ -36,12 +36,13 @@
 // Rows are stored with their 16-byte chunks XOR-permuted (staged_off) so that
 // both read patterns are free of shared-memory bank conflicts.
 //
-// INT8 and FP8 caches (Eq. 3, "KV-Cache Quantization"; FP8 = E4M3 codes
-// with z = 0): with x = s*c + z per row,
+// INT8, FP8 and INT4 caches (Eq. 3, "KV-Cache Quantization"; FP8 = E4M3
+// codes with z = 0): with x = s*c + z per row,
 //   q.x = s (q.c) + z sum(q)          and    sum_t p_t x_t = sum_t (p_t s_t) c_t + sum_t p_t z_t,
-// so the codes go through the tensor cores as exact f16 values (INT8 codes as
-// the subnormals c * 2^-24, E4M3 codes converted exactly) and the scale and
-// zero are applied once per (token, head) instead of once per element.
+// so the codes go through the tensor cores as exact f16 values (INT8 codes and
+// INT4 low nibbles as the subnormals c * 2^-24, INT4 high nibbles in place as
+// c * 2^-20, E4M3 codes converted exactly) and the scale and zero are applied
+// once per (token, head) instead of once per element.
 #include <atomic>
 #include <cfloat>
 #include <cmath>
@@ -87,10 +88,11 @@ struct Tile {
   static constexpr bool kU8 = KVT != PA_KV_BF16;
   static constexpr bool kFp8 = KVT == PA_KV_FP8_PER_TOKEN;
   static constexpr bool kU4 = KVT == PA_KV_U4_PER_TOKEN;  // two codes per byte
-  // Codes reach the MMA scaled by an exact power of two (INT8 c * 2^-24 as an
-  // f16 subnormal, INT4 c * 2^-9 through the E4M3 converter; FP8 codes as
-  // they are); the K scale and O after the loop take it back.
-  static constexpr float kCodeScale = kU4 ? 512.f : (kFp8 ? 1.f : 16777216.f);
+  // Codes reach the MMA scaled by an exact power of two: an INT8 byte, or an
+  // INT4 low nibble, under zero high bits is the f16 subnormal c * 2^-24; an
+  // INT4 high nibble left in place is c * 2^-20; FP8 codes go as they are.
+  // The K scale and O after the loop take the powers of two back.
+  static constexpr float kCodeScale = kFp8 ? 1.f : 16777216.f;
   static constexpr int kElem = kU8 ? 1 : 2;
   static constexpr int kRowBytes = kU4 ? D / 2 : D * kElem;
   // one 16-token block of K (or V) is 16 contiguous rows of the page
@@ -234,20 +236,21 @@ __device__ __forceinline__ float load_q(const __nv_bfloat16 *qp, bool head_ok, i
     }
   } else if constexpr (T::kU4) {
     // lane t contracts d in [t*D/4, (t+1)*D/4); per group of 8 elements the
-    // k-steps take (e0,e2 | e4,e6) and (e1,e3 | e5,e7), as the 4-bit unpack does
+    // k-steps take (e0,e4 | e2,e6) (low nibbles) and (e1,e5 | e3,e7) (high
+    // nibbles), as the 4-bit unpack does
 #pragma unroll
     for (int w = 0; w < D / 32; ++w) {
       const uint4 v = head_ok ? ldg_nc128(qp + t * (D / 4) + 8 * w) : make_uint4(0, 0, 0, 0);
-      const uint32_t f02 = pack_f16(bf16_lo(v.x), bf16_lo(v.y));
-      const uint32_t f46 = pack_f16(bf16_lo(v.z), bf16_lo(v.w));
-      const uint32_t f13 = pack_f16(bf16_hi(v.x), bf16_hi(v.y));
-      const uint32_t f57 = pack_f16(bf16_hi(v.z), bf16_hi(v.w));
-      qsum += (f16_lo(f02) + f16_hi(f02)) + (f16_lo(f46) + f16_hi(f46)) +
-              (f16_lo(f13) + f16_hi(f13)) + (f16_lo(f57) + f16_hi(f57));
-      qa[2 * w][0] = f02;
-      qa[2 * w][1] = f46;
-      qa[2 * w + 1][0] = f13;
-      qa[2 * w + 1][1] = f57;
+      const uint32_t f04 = pack_f16(bf16_lo(v.x), bf16_lo(v.z));
+      const uint32_t f26 = pack_f16(bf16_lo(v.y), bf16_lo(v.w));
+      const uint32_t f15 = pack_f16(bf16_hi(v.x), bf16_hi(v.z));
+      const uint32_t f37 = pack_f16(bf16_hi(v.y), bf16_hi(v.w));
+      qsum += (f16_lo(f04) + f16_hi(f04)) + (f16_lo(f26) + f16_hi(f26)) +
+              (f16_lo(f15) + f16_hi(f15)) + (f16_lo(f37) + f16_hi(f37));
+      qa[2 * w][0] = f04;
+      qa[2 * w][1] = f26;
+      qa[2 * w + 1][0] = f15;
+      qa[2 * w + 1][1] = f37;
     }
     qsum += __shfl_xor_sync(0xffffffffu, qsum, 1);
     qsum += __shfl_xor_sync(0xffffffffu, qsum, 2);
@@ -374,10 +377,12 @@ __device__ __forceinline__ void block_step(const LaneMap<D, KVT> &lm, uint32_t s
   const auto &voff = lm.voff;
   // ---- S = Q K^T -------------------------------------------------------------
   float s[2][4];
+  float s_hi[2][4];  // INT4: the high-nibble products (codes scaled 16x more)
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt) {
     s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
     if constexpr (T::kU4) {
+      s_hi[nt][0] = s_hi[nt][1] = s_hi[nt][2] = s_hi[nt][3] = 0.f;
       uint32_t wk[D / 32];
       if constexpr (D == 128) {
         const uint4 v = lds128(src + koff[nt][0]);
@@ -388,12 +393,15 @@ __device__ __forceinline__ void block_step(const LaneMap<D, KVT> &lm, uint32_t s
       }
 #pragma unroll
       for (int w = 0; w < D / 32; ++w) {
-        // even elements (low nibbles), then odd ones, each as c * 2^-9
-        uint32_t b02, b46, b13, b57;
-        nib4_to_f16x2x2(wk[w] & 0x0F0F0F0Fu, b02, b46);
-        nib4_to_f16x2x2((wk[w] >> 4) & 0x0F0F0F0Fu, b13, b57);
-        mma_f16_16816(s[nt], qa[2 * w][0], 0u, qa[2 * w][1], 0u, b02, b46);
-        mma_f16_16816(s[nt], qa[2 * w + 1][0], 0u, qa[2 * w + 1][1], 0u, b13, b57);
+        // elements e0..e7 of the word (e2i in the low nibble of byte i): low
+        // nibbles under zero bits are the f16 subnormals c * 2^-24, pairs
+        // (e0, e4) and (e2, e6); high nibbles in place are c * 2^-20, pairs
+        // (e1, e5) and (e3, e7)
+        const uint32_t w8 = wk[w] >> 8;
+        mma_f16_16816(s[nt], qa[2 * w][0], 0u, qa[2 * w][1], 0u, wk[w] & 0x000F000Fu,
+                      w8 & 0x000F000Fu);
+        mma_f16_16816(s_hi[nt], qa[2 * w + 1][0], 0u, qa[2 * w + 1][1], 0u,
+                      wk[w] & 0x00F000F0u, w8 & 0x00F000F0u);
       }
     } else {
 #pragma unroll
@@ -419,6 +427,12 @@ __device__ __forceinline__ void block_step(const LaneMap<D, KVT> &lm, uint32_t s
 
   // ---- online softmax (log2 domain) ---------------------------------------
   float x[4] = {s[0][0], s[0][1], s[1][0], s[1][1]};  // tokens 2t, 2t+1, 8+2t, 9+2t
+  if constexpr (T::kU4) {  // high-nibble products were scaled 16x more
+    x[0] = fmaf(s_hi[0][0], 0.0625f, x[0]);
+    x[1] = fmaf(s_hi[0][1], 0.0625f, x[1]);
+    x[2] = fmaf(s_hi[1][0], 0.0625f, x[2]);
+    x[3] = fmaf(s_hi[1][1], 0.0625f, x[3]);
+  }
   float vs[4], vz[4];
   if constexpr (T::kU8) {
     const uint4 k01 = lds128(src + T::kKSzOff + 16 * t);
@@ -526,18 +540,20 @@ __device__ __forceinline__ void block_step(const LaneMap<D, KVT> &lm, uint32_t s
         }
       }
       // m-tiles j, j+1 use bytes j & 3, (j & 3) + 1 of word j / 4: gather them
-      // for token pairs (2t, 2t+1) and (8+2t, 9+2t), then low nibbles give
-      // rows d (a0, a2), high nibbles rows d + 1 (a1, a3)
+      // per token pair as (token 2t: byte b, b + 1 | token 2t + 1: byte b,
+      // b + 1), so that each 16-bit half holds one token's bytes; low nibbles
+      // under zero bits (c * 2^-24) give rows d (a0, a2), high nibbles in
+      // place (c * 2^-20) rows d + 1 (a1, a3)
 #pragma unroll
       for (int j = 0; j < T::kMTiles; j += 2) {
-        const uint32_t sel = (j & 2) ? 0x7362 : 0x5140;
+        const uint32_t sel = (j & 2) ? 0x7632 : 0x5410;
         const uint32_t ya = __byte_perm(xv[0][j / 4], xv[1][j / 4], sel);
         const uint32_t yb = __byte_perm(xv[2][j / 4], xv[3][j / 4], sel);
-        uint32_t a0[2], a1[2], a2[2], a3[2];
-        nib4_to_f16x2x2(ya & 0x0F0F0F0Fu, a0[0], a0[1]);
-        nib4_to_f16x2x2((ya >> 4) & 0x0F0F0F0Fu, a1[0], a1[1]);
-        nib4_to_f16x2x2(yb & 0x0F0F0F0Fu, a2[0], a2[1]);
-        nib4_to_f16x2x2((yb >> 4) & 0x0F0F0F0Fu, a3[0], a3[1]);
+        const uint32_t ya8 = ya >> 8, yb8 = yb >> 8;
+        const uint32_t a0[2] = {ya & 0x000F000Fu, ya8 & 0x000F000Fu};
+        const uint32_t a1[2] = {ya & 0x00F000F0u, ya8 & 0x00F000F0u};
+        const uint32_t a2[2] = {yb & 0x000F000Fu, yb8 & 0x000F000Fu};
+        const uint32_t a3[2] = {yb & 0x00F000F0u, yb8 & 0x00F000F0u};
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           mma_f16_16816(o[j + u], a0[u], a1[u], a2[u], a3[u], bh0, bh1);
@@ -590,12 +606,15 @@ __device__ __forceinline__ void finish_acc(WarpAcc<D, KVT> &acc, int t) {
     zacc += __shfl_xor_sync(0xffffffffu, zacc, 2);
     const float z0 = __shfl_sync(0xffffffffu, zacc, 8 * t);
     const float z1 = __shfl_sync(0xffffffffu, zacc, 8 * t + 4);
+    // undo the codes' power-of-two scale; INT4 rows g + 8 hold the high
+    // nibbles (d + 1), which were scaled 16x more
+    constexpr float kRowHiScale = T::kU4 ? T::kCodeScale / 16.f : T::kCodeScale;
 #pragma unroll
-    for (int j = 0; j < T::kMTiles; ++j) {  // undo the codes' power-of-two scale
+    for (int j = 0; j < T::kMTiles; ++j) {
       o[j][0] = fmaf(o[j][0], T::kCodeScale, z0);
       o[j][1] = fmaf(o[j][1], T::kCodeScale, z1);
-      o[j][2] = fmaf(o[j][2], T::kCodeScale, z0);
-      o[j][3] = fmaf(o[j][3], T::kCodeScale, z1);
+      o[j][2] = fmaf(o[j][2], kRowHiScale, z0);
+      o[j][3] = fmaf(o[j][3], kRowHiScale, z1);
     }
   }
 }

@@ -158,17 +158,6 @@ __device__ __forceinline__ uint32_t u8x2_to_f16x2(uint32_t word, uint32_t sel) {
   return __byte_perm(word, 0u, sel);
 }
 
-// Four bytes, each holding a 4-bit code c in its low nibble (high nibble 0),
-// -> two f16x2 of c * 2^-9: read as an E4M3 byte, 0000_0mmm is the subnormal
-// m * 2^-9 and 0000_1mmm the normal (8 + m) * 2^-9, so codes 0..15 land
-// exactly on a uniform grid. lo gets bytes 0, 1; hi gets bytes 2, 3.
-__device__ __forceinline__ void nib4_to_f16x2x2(uint32_t v, uint32_t &lo, uint32_t &hi) {
-  asm("{\n .reg .b16 a, b;\n mov.b32 {a, b}, %2;\n cvt.rn.f16x2.e4m3x2 %0, a;\n"
-      " cvt.rn.f16x2.e4m3x2 %1, b;\n}\n"
-      : "=r"(lo), "=r"(hi)
-      : "r"(v));
-}
-
 // Two E4M3 codes (bits 0..7 and 8..15 of `pair`) -> f16x2 with the first code in
 // the low half. Exact: every E4M3 value is an f16 value.
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t pair) {
