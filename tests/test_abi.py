@@ -213,3 +213,45 @@ def test_header_compiles_as_c99_and_host_calls_work(lib, tmp_path):
     r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0, r.stdout + r.stderr
     assert "ok" in r.stdout
+
+
+def test_split_plan_invariants_for_any_shape(lib):
+    """For random shapes and device sizes the plan is a valid partition: S in
+    [1, min(max_pages, 256)], no empty split, at most 2048 pages per split, an
+    honoured request where the limits allow it, and a single wave whenever
+    the units fit in the resident slots."""
+    from hypothesis import given, settings, strategies as st
+
+    @settings(max_examples=400, deadline=None)
+    @given(units=st.integers(0, 70000), pages=st.integers(1, 20000), P=st.sampled_from([16, 32]),
+           sms=st.integers(1, 200), cps=st.integers(1, 8), req=st.integers(0, 300))
+    def check(units, pages, P, sms, cps, req):
+        S = lib.pa_decode_plan_splits(units, pages, P, sms, cps, req)
+        assert 1 <= S <= min(pages, 256)
+        C = -(-pages // S)
+        assert -(-pages // C) == S and C <= 2048
+        lo = -(-pages // 2048)
+        if req > 0 and lo <= req <= min(pages, 256) and -(-pages // -(-pages // req)) == req:
+            assert S == req
+        if req == 0 and 0 < units < sms * cps and lo == 1:
+            assert units * S <= sms * cps          # never a second wave
+
+    check()
+
+
+def test_workspace_sizes_fit_every_larger_buffer(lib):
+    """The advertised workspace size, and every larger size, holds the split
+    counters in the size-only region and the partials after it."""
+    from hypothesis import given, settings, strategies as st
+
+    @settings(max_examples=300, deadline=None)
+    @given(B=st.integers(1, 4096), Hq=st.sampled_from([4, 8, 16, 32, 64, 128]),
+           D=st.sampled_from([64, 128]), S=st.integers(2, 256), extra=st.integers(0, 1 << 22))
+    def check(B, Hq, D, S, extra):
+        ws = lib.pa_decode_workspace_bytes(B, Hq, D, S)
+        rest = -(-B * Hq * S * D * 4 // 256) * 256 + -(-B * Hq * S * 4 // 256) * 256
+        size = ws + extra
+        region = 256 * (size // 32768)
+        assert region >= B * Hq * 4 and size - region >= rest
+
+    check()
