@@ -81,6 +81,18 @@ def decode_bytes(w, sinks: int = 0, window: int = 0) -> int:
     return attended_tokens(w, sinks, window) * w.Hkv * 2 * row + w.B * w.Hq * w.D * 2
 
 
+def unique_bytes(w) -> int:
+    """Bytes the decode must bring from HBM at least once when prefix pages
+    are shared: the shared prefix once plus every request's own tokens, plus
+    q (the shared prefix workload); decode_bytes for every other workload."""
+    pre = int(w.notes.get("prefix_tokens", 0)) if "prefix_pages" in w.notes else 0
+    if pre == 0:
+        return decode_bytes(w)
+    row = {"bf16": w.D * 2, "u8": w.D + 8, "fp8": w.D + 8, "u4": w.D // 2 + 8}[w.kv]
+    own = int((w.context_lens.astype("int64") - pre).clip(min=0).sum())
+    return (pre + own) * w.Hkv * 2 * row + w.B * w.Hq * w.D * 2
+
+
 def append_bytes(w) -> int:
     n = len(w.step_seq)
     row = {"bf16": w.D * 2, "u8": w.D + 8, "fp8": w.D + 8, "u4": w.D // 2 + 8}[w.kv]
@@ -449,6 +461,11 @@ def run_ours(args, rank, world, local_rank):
     dec_avg_ms = statistics.mean(dec_ms)
     # the timed kernel: the fused step also reads the new rows and writes them
     kbytes = dbytes + (append_bytes(w) if fused else 0)
+    # with shared prefix pages the roofline counts each unique byte once (the
+    # logical bytes, every request's prefix included, are the metric's value)
+    shared_prefix = "prefix_pages" in w.notes and not args.window
+    if shared_prefix:
+        kbytes = unique_bytes(w) + (append_bytes(w) if fused else 0)
     achieved = kbytes / (dec_avg_ms * 1e-3) / 1e9
     traffic = recorded_traffic(w.name) if not (args.cascade or args.window) else None
     # append, [prefix pass,] decode[, merge]; the fused step is one launch
@@ -478,6 +495,10 @@ def run_ours(args, rank, world, local_rank):
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "algorithmic_bytes": kbytes,
+                     "bytes_counted": ("unique: the shared prefix once, each request's own "
+                                       "tokens, q" if shared_prefix else
+                                       "every attended token's K/V once, q"
+                                       + (", the new rows" if fused else "")),
                      "avg_launch_ms": round(dec_avg_ms, 5)},
         "gpu_launches": K * launches_per_step,
         "clocks": clk,
