@@ -248,7 +248,10 @@ pa_status_t pa_decode(const pa_kv_pool_t *pool, const void *q,
  * the page; then Eq. (1) runs over tokens 0 .. context_lens[b] - 1 as in
  * pa_decode. The result equals pa_kv_append(seq_idx = b, pos =
  * context_lens[b] - 1) followed by pa_decode, bit for bit, without the
- * append's launch. A sequence with context length 0 stores nothing.
+ * append's launch. A sequence with context length 0 stores nothing. As with
+ * pa_kv_append, the page receiving a sequence's new token must belong to
+ * that sequence alone (copy-on-write is the caller's job): here another
+ * sequence's CTAs could otherwise read that page while it is written.
  */
 pa_status_t pa_decode_append(const pa_kv_pool_t *pool, const void *q,
                              const void *k_new, const void *v_new,
