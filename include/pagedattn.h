@@ -353,7 +353,13 @@ pa_status_t pa_decode_window(const pa_kv_pool_t *pool, const void *q,
  *
  * Set-up: the first call on each device (with that device current) looks up
  * the array's device address with cudaGetSymbolAddress; make that first call
- * before any stream capture. Every call on a device shares the one array and
+ * before any stream capture. The address is cached per device under the id of
+ * the CUDA context it was found in: after cudaDeviceReset (or anything else
+ * that destroys and re-creates the context) the module is loaded anew, the
+ * cached address is no longer valid, and the next call looks it up again —
+ * that call is a first call again, with the same rule on stream capture.
+ * A planner failure (e.g. an unsupported pool) is reported as pa_decode
+ * reports it. Every call on a device shares the one array and
  * it keeps the last call's contents. The only part that must start at zero is
  * the split counters, which the array holds from load time and which every
  * completed call returns to zero. Calls that overlap on the GPU — on

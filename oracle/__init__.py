@@ -147,12 +147,6 @@ def e4m3_encode(r: float) -> int:
     return int(lib().oracle_e4m3_encode(float(r)))
 
 
-def dequantize_rows(codes: np.ndarray, sz: np.ndarray) -> np.ndarray:
-    """Right-hand side of Eq. 3 in fp64: s * code + z, per row."""
-    return sz[..., 0:1].astype(np.float64) * codes.astype(np.float64) + \
-        sz[..., 1:2].astype(np.float64)
-
-
 # --------------------------------------------------------------------------
 # Host pool and page-table resolution
 # --------------------------------------------------------------------------

@@ -2,8 +2,10 @@
 // device memory. Its scratch (partial outputs and their log-sum-exps) lives in
 // a library-owned device array instead of a caller-provided workspace; the
 // computation is pa_decode's, unchanged.
-#include <atomic>
+#include <cuda.h>
+
 #include <cstdio>
+#include <mutex>
 
 #include "pa_internal.h"
 
@@ -21,15 +23,67 @@ constexpr size_t kScratchBytes = PA_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
-std::atomic<void *> g_scratch_addr[kMaxDevices];
 
 pa_status_t noalloc_fail(pa_status_t st, const char *msg) {
   set_last_error_message(msg);
   return st;
 }
 
-// Device address of g_noalloc_scratch on the current device, looked up once per
-// device (with that device current) and cached.
+// The array's device address is a property of the CUDA context that loaded
+// the library's module, not of the device alone: after cudaDeviceReset (or
+// anything else that destroys and re-creates the primary context) the module
+// is loaded again and the array may sit elsewhere. The cache is therefore
+// keyed by the context's id, which CUDA never reuses within a process. The
+// two driver calls that read it come through the runtime's entry-point
+// lookup, so the library needs no link against the driver library.
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+struct CtxCalls {
+  CtxGetCurrentFn get_current = nullptr;
+  CtxGetIdFn get_id = nullptr;
+};
+
+const CtxCalls &ctx_calls() {
+  static const CtxCalls calls = [] {
+    CtxCalls c;
+    void *f1 = nullptr, *f2 = nullptr;
+    cudaDriverEntryPointQueryResult r1 = cudaDriverEntryPointSymbolNotFound;
+    cudaDriverEntryPointQueryResult r2 = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &r1) == cudaSuccess &&
+        r1 == cudaDriverEntryPointSuccess &&
+        cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &r2) == cudaSuccess &&
+        r2 == cudaDriverEntryPointSuccess && f1 != nullptr && f2 != nullptr) {
+      c.get_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+      c.get_id = reinterpret_cast<CtxGetIdFn>(f2);
+    }
+    return c;
+  }();
+  return calls;
+}
+
+// Id of the context current on the calling thread, 0 if there is none or it
+// cannot be read (then nothing is cached and every call looks the address up).
+unsigned long long current_ctx_id() {
+  const CtxCalls &c = ctx_calls();
+  if (c.get_current == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (c.get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  if (c.get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+struct ScratchSlot {
+  unsigned long long ctx_id = 0;
+  void *addr = nullptr;
+};
+std::mutex g_scratch_mu;
+ScratchSlot g_scratch_addr[kMaxDevices];
+
+// Device address of g_noalloc_scratch for the current device and context:
+// looked up with cudaGetSymbolAddress (with that device current) the first
+// time a context is seen, then cached under the context's id.
 pa_status_t scratch_address(void **out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -40,16 +94,29 @@ pa_status_t scratch_address(void **out) {
   }
   if (dev < 0 || dev >= kMaxDevices)
     return noalloc_fail(PA_ERR_UNSUPPORTED, "pa_decode_noalloc: device index out of range");
-  void *p = g_scratch_addr[dev].load(std::memory_order_acquire);
-  if (p == nullptr) {
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || p == nullptr) {
-      char buf[256];
-      snprintf(buf, sizeof buf, "pa_decode_noalloc: cudaGetSymbolAddress: %s",
-               cudaGetErrorString(e));
-      return noalloc_fail(PA_ERR_CUDA, buf);
+  unsigned long long id = current_ctx_id();
+  if (id != 0) {
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (g_scratch_addr[dev].ctx_id == id && g_scratch_addr[dev].addr != nullptr) {
+      *out = g_scratch_addr[dev].addr;
+      return PA_OK;
     }
-    g_scratch_addr[dev].store(p, std::memory_order_release);
+  }
+  void *p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess || p == nullptr) {
+    char buf[256];
+    snprintf(buf, sizeof buf, "pa_decode_noalloc: cudaGetSymbolAddress: %s",
+             cudaGetErrorString(e));
+    return noalloc_fail(PA_ERR_CUDA, buf);
+  }
+  // the lookup itself makes the device's primary context current if no
+  // context was yet, so read the id again before caching
+  id = current_ctx_id();
+  if (id != 0) {
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    g_scratch_addr[dev].ctx_id = id;
+    g_scratch_addr[dev].addr = p;
   }
   *out = p;
   return PA_OK;
@@ -67,7 +134,11 @@ extern "C" pa_status_t pa_decode_noalloc(const pa_kv_pool_t *pool, const void *q
   int32_t S = num_splits;
   if (pool != nullptr && num_seqs > 0 && num_q_heads > 0 && max_pages > 0 && num_splits >= 0) {
     S = pa_decode_num_splits(pool, num_seqs, max_pages, num_splits);
-    if (S > 0) {
+    // a pool or shape the planner rejects goes to pa_decode with the caller's
+    // own split count, so that its error message names the real problem
+    if (S <= 0) {
+      S = num_splits;
+    } else {
       size_t need = pa_decode_workspace_bytes(num_seqs, num_q_heads, pool->head_dim, S);
       if (need > kScratchBytes && num_splits == 0) {
         // automatic: take the largest split count whose partials fit

@@ -31,12 +31,20 @@ def kv_bytes(layers: int, kv_heads: int, head_dim: int, tokens: int,
 
 def pool_bytes(num_pages: int, kv_heads: int, page_size: int, head_dim: int,
                kind: str = "bf16") -> int:
-    """Device bytes of one layer's pool in this library's layout (K and V,
-    plus the fp32 scale/zero of each row for the INT8 cache)."""
+    """Device bytes of one layer's pool in this library's layout: K and V,
+    each row ``head_dim`` bf16 values, or for the quantised caches its codes
+    (one byte per element for INT8 and FP8, two elements per byte for INT4)
+    plus the row's fp32 (scale, zero)."""
     rows = num_pages * kv_heads * page_size
     if kind == "bf16":
         return 2 * rows * head_dim * 2
-    return 2 * rows * (head_dim + 8)
+    if kind in ("u8", "fp8"):
+        return 2 * rows * (head_dim + 8)
+    if kind == "u4":
+        if head_dim % 2:
+            raise ValueError("an INT4 row packs two elements per byte: head_dim must be even")
+        return 2 * rows * (head_dim // 2 + 8)
+    raise ValueError(f"unknown cache kind {kind!r}")
 
 
 class OutOfPages(RuntimeError):

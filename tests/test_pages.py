@@ -76,3 +76,18 @@ def test_memory_helpers_match_the_pages():
     # the 70B-shaped single-layer pool: 8192 pages of 32 tokens x 8 heads x 128
     assert pages.pool_bytes(8192, 8, 32, 128) == 1_073_741_824
     assert pages.pool_bytes(10, 8, 16, 128, "u8") == 2 * 10 * 8 * 16 * 136
+    assert pages.pool_bytes(10, 8, 16, 128, "fp8") == 2 * 10 * 8 * 16 * 136
+    assert pages.pool_bytes(10, 8, 16, 128, "u4") == 2 * 10 * 8 * 16 * 72
+    with pytest.raises(ValueError):
+        pages.pool_bytes(10, 8, 16, 128, "int3")
+
+
+@pytest.mark.parametrize("kind", ["bf16", "u8", "fp8", "u4"])
+@pytest.mark.parametrize("shape", [(7, 2, 16, 64), (3, 8, 32, 128)])
+def test_pool_bytes_is_what_a_pool_holds(kind, shape):
+    # the formula against the tensors the binding actually allocates (host
+    # memory here: nothing is launched)
+    from paged_kv_cache_466_b200 import KVPool
+    pool = KVPool(*shape, dtype=kind, device="cpu")
+    assert pages.pool_bytes(*shape, kind) == sum(t.numel() * t.element_size()
+                                                 for t in pool.tensors())
