@@ -35,7 +35,11 @@ METRIC = "decode-attention achieved HBM GB/s and % of B200 peak; sequences/sec p
 FALLBACK_HBM_GBS = 6650.0
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
 NOMINAL_HBM_GBS = 7700.0   # B200 (HGX) specification figure, for context only
-DECODE_SRC = os.path.join(ROOT, "paged_kv_cache_466_b200", "csrc", "decode.cu")
+# every source file the decode kernel is compiled from: a recorded ncu traffic
+# figure is used only for the exact sources it was captured from
+KERNEL_SRCS = [os.path.join(ROOT, "paged_kv_cache_466_b200", "csrc", f)
+               for f in ("decode.cu", "pa_device.cuh", "pa_quant.cuh", "pa_internal.h")] + \
+              [os.path.join(ROOT, "include", "pagedattn.h")]
 
 
 def parse():
@@ -58,6 +62,9 @@ def parse():
     ap.add_argument("--separate-append", action="store_true",
                     help="time pa_kv_append + pa_decode as two calls instead of the fused "
                          "pa_decode_append step")
+    ap.add_argument("--alternate-pools", action="store_true",
+                    help="keep two independent copies of the pool and alternate between them "
+                         "step by step, so no step reads pages the previous step left in L2")
     ap.add_argument("--flush-l2", action="store_true",
                     help="write a buffer of twice the L2 size between timed steps; the step "
                          "time is then the sum of per-step CUDA events, flush excluded")
@@ -108,17 +115,21 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def kernel_sources_sha256() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SRCS:
+        h.update(os.path.basename(p).encode())
+        h.update(open(p, "rb").read())
+    return h.hexdigest()
+
+
 def recorded_traffic(workload: str):
-    """ncu DRAM bytes per decode launch, if recorded for the current kernel source."""
+    """ncu DRAM bytes per decode launch, if captured from exactly the current
+    kernel sources (any change to them voids the record until it is re-captured)."""
     try:
-        rec = json.load(open(TRAFFIC_FILE))
-        src_sha = hashlib.sha256(open(DECODE_SRC, "rb").read()).hexdigest()
-        r = rec.get(workload)
-        # a record stays valid for a later source only where it says why
-        # (changes confined to code the recorded kernel does not instantiate)
-        if r and (r.get("decode_cu_sha256") == src_sha or
-                  src_sha in r.get("also_valid_for_decode_cu_sha256", [])):
-            return int(r["dram_bytes_per_launch"])
+        rec = json.load(open(TRAFFIC_FILE)).get(workload)
+        if rec and rec.get("kernel_sources_sha256") == kernel_sources_sha256():
+            return int(rec["dram_bytes_per_launch"])
     except Exception:
         pass
     return None
@@ -148,9 +159,10 @@ class ClockSampler:
              0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
              0x100: "display_clock_setting"}
 
-    def __init__(self, index: int, period_s: float = 0.01):
+    def __init__(self, index: int, period_s: float = 5e-5):
         self.ok = False
-        self.samples, self.reasons = [], 0
+        self.samples, self.reasons = [], 0       # (host time, MHz)
+        self.window = None
         self.period = period_s
         try:
             import pynvml
@@ -184,36 +196,58 @@ class ClockSampler:
             r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
         except Exception:
             r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
-        self.samples.append(mhz)
-        self.reasons |= int(r)
+        self.samples.append((time.perf_counter(), mhz, int(r)))
 
     def _loop(self):
+        # a read every ~0.1 ms at most (each NVML query releases the GIL): a timed
+        # region of a few milliseconds still gets tens of samples
         while not self._stop.is_set():
             try:
                 self._read()
             except Exception:
                 pass
-            self._stop.wait(self.period)
+            self._first.set()
+            time.sleep(self.period)
 
     def start(self):
         if not self.ok:
             return
+        # hand the interpreter lock over every 50 us instead of every 5 ms, so
+        # the sampler runs while the main thread launches the steps
+        self._switch = sys.getswitchinterval()
+        sys.setswitchinterval(5e-5)
         self._stop = threading.Event()
+        self._first = threading.Event()
         self._t = threading.Thread(target=self._loop, daemon=True)
         self._t.start()
+        self._first.wait(5.0)   # sampling has begun before the first step
+
+    def mark(self, begin: bool):
+        """Host time at the start (before the first launch) and end (after the
+        synchronise) of the timed region."""
+        t = time.perf_counter()
+        self.window = (t, None) if begin else (self.window[0], t)
 
     def stop(self):
         if not self.ok:
             return None
         self._stop.set()
         self._t.join()
-        try:
-            self._read()
-        except Exception:
-            pass
-        names = [n for b, n in self.NAMES.items() if self.reasons & b]
-        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
-                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+        sys.setswitchinterval(self._switch)
+        lo, hi = self.window if self.window and self.window[1] else (float("-inf"), float("inf"))
+        timed = [(m, r) for t, m, r in self.samples if lo <= t <= hi]
+        every = [(m, r) for _, m, r in self.samples]
+        use = timed if timed else every
+        reasons = 0
+        for _, r in use:
+            reasons |= r
+        names = [n for b, n in self.NAMES.items() if reasons & b]
+        return {"sm_mhz": statistics.median(m for m, _ in use) if use else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(timed),
+                "samples_with_warmup": len(every),
+                "sampled": "NVML SM clock and clock-event reasons, read back to back from "
+                           "the start of the warm-up to the end of the timed region; sm_mhz, "
+                           "reasons and samples cover the timed region"}
 
 
 # ------------------------------------------------------------------ CPU oracle leg
@@ -270,6 +304,8 @@ def config_of(w, args, n, S):
          "num_splits": S, "pool_pages": w.num_pages,
          "l2": "flushed between steps (write of 2x the L2 size, outside the step events)"
                if args.flush_l2 else
+               "two independent pools alternated step by step (no step finds the previous "
+               "step's pages in L2), not flushed" if args.alternate_pools else
                "inputs larger than the 126 MB L2, not flushed"
                if decode_bytes(w, args.sinks, args.window) > 256e6
                else "L2 not flushed (working set may be L2-resident)"}
@@ -318,15 +354,15 @@ def run_ours(args, rank, world, local_rank):
     out = torch.empty((w.B, w.Hq, w.D), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
-    def decode(qq, tt, cc):
+    def decode(pl, qq, tt, cc):
         if args.cascade:
-            pa_decode_shared_prefix(pool, qq, pre_pages, pre_len, tt, cc, w.scale, out=out,
+            pa_decode_shared_prefix(pl, qq, pre_pages, pre_len, tt, cc, w.scale, out=out,
                                     workspace=ws, num_splits=args.splits)
         elif args.window > 0:
-            pa_decode_window(pool, qq, tt, cc, w.scale, args.sinks, args.window, out=out,
+            pa_decode_window(pl, qq, tt, cc, w.scale, args.sinks, args.window, out=out,
                              workspace=ws, num_splits=args.splits)
         else:
-            pa_decode(pool, qq, tt, cc, w.scale, out=out, workspace=ws, num_splits=S)
+            pa_decode(pl, qq, tt, cc, w.scale, out=out, workspace=ws, num_splits=S)
 
     # the usual decode step (one new token per sequence, at ctx - 1) runs as one
     # launch, the cache write fused into the decode; other steps as two calls
@@ -336,17 +372,27 @@ def run_ours(args, rank, world, local_rank):
     if fused:
         kn, vn = per_seq[0].to(dev), per_seq[1].to(dev)
 
-    def step(ev0=None, ev1=None):
+    pools = [pool]
+    if args.alternate_pools:
+        # a second, independent copy of the pool: steps alternate between the
+        # two, so no step can find the previous step's pages in the L2
+        twin = KVPool(w.num_pages, w.Hkv, w.P, w.D, w.kv, dev)
+        for a_t, b_t in zip(twin.tensors(), pool.tensors()):
+            a_t.copy_(b_t)
+        pools.append(twin)
+
+    def step(i=0, ev0=None, ev1=None):
+        pl = pools[i % len(pools)]
         if fused:
             if ev0 is not None:
                 ev0.record(stream)
-            pa_decode_append(pool, q, kn, vn, bt, ctx, w.scale, out=out, workspace=ws,
+            pa_decode_append(pl, q, kn, vn, bt, ctx, w.scale, out=out, workspace=ws,
                              num_splits=S)
         else:
-            pa_kv_append(pool, sk, sv, sseq, spos, bt)
+            pa_kv_append(pl, sk, sv, sseq, spos, bt)
             if ev0 is not None:
                 ev0.record(stream)
-            decode(q, bt, ctx)
+            decode(pl, q, bt, ctx)
         if ev1 is not None:
             ev1.record(stream)
 
@@ -354,8 +400,10 @@ def run_ours(args, rank, world, local_rank):
         if world > 1:
             dist.barrier()
 
-    for _ in range(max(args.warmup, 0)):
-        step()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    for i in range(max(args.warmup, 0)):
+        step(i)
     torch.cuda.synchronize()
 
     # ---- device-resident timed region
@@ -363,7 +411,6 @@ def run_ours(args, rank, world, local_rank):
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(K)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(local_rank)
     barrier()
     torch.cuda.synchronize()
     if args.flush_l2:
@@ -371,17 +418,18 @@ def run_ours(args, rank, world, local_rank):
         flush = torch.empty(2 * max(l2, 1 << 20), dtype=torch.uint8, device=dev)
         sevs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                 for _ in range(K)]
-    clocks.start()
+    clocks.mark(True)
     t0.record(stream)
     for i in range(K):
         if args.flush_l2:
             flush.fill_(i & 0xFF)
             sevs[i][0].record(stream)
-        step(*evs[i])
+        step(i, *evs[i])
         if args.flush_l2:
             sevs[i][1].record(stream)
     t1.record(stream)
     torch.cuda.synchronize()
+    clocks.mark(False)
     clk = clocks.stop()
     barrier()
     if args.flush_l2:
@@ -436,7 +484,7 @@ def run_ours(args, rank, world, local_rank):
                          (d_ctx, h_ctx), (d_bt, h_bt)):
                 d.copy_(h, non_blocking=True)
             pa_kv_append(pool, d_k, d_v, d_seq, d_pos, d_bt)
-            decode(d_q, d_bt, d_ctx)
+            decode(pool, d_q, d_bt, d_ctx)
             h_out.copy_(out, non_blocking=True)
             stream.synchronize()   # the caller reads the result every step
 

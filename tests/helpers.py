@@ -2,6 +2,8 @@
 and build the oracle's own host pool from the same inputs."""
 from __future__ import annotations
 
+import functools
+
 import numpy as np
 import torch
 
@@ -65,3 +67,15 @@ def pool_bytes_equal(pool: KVPool, hp: oracle.HostPool):
             bad = np.flatnonzero(got != want)
             return False, f"{bad.size} bytes differ, first at byte {bad[0]}"
     return True, ""
+
+
+@functools.lru_cache(maxsize=8)
+def full_size_reference(name: str):
+    """The named full-size workload with the oracle's pool and its fp64 Eq. 1
+    output for every (sequence, query head) row, computed once per test
+    process (the larger workloads take seconds on the host)."""
+    from paged_kv_cache_466_b200 import workloads as W
+    w = W.by_name(name)
+    hp = oracle_pool(w)
+    ref, lse = oracle_decode(w, hp)
+    return w, ref, lse

@@ -15,7 +15,8 @@ from paged_kv_cache_466_b200 import (PA_DERR_BAD_CTX, PA_DERR_BAD_PAGE, pa_decod
 from paged_kv_cache_466_b200 import workloads as W
 from paged_kv_cache_466_b200.workloads import bits
 import oracle
-from tests.helpers import DEV, device_append, device_inputs, oracle_decode, oracle_pool
+from tests.helpers import (DEV, device_append, device_inputs, full_size_reference,
+                           oracle_decode, oracle_pool)
 
 pytestmark = pytest.mark.gpu
 TOL = 2e-3
@@ -254,25 +255,44 @@ def test_workspace_and_split_planning():
 
 
 # ------------------------------------------------------------------ full sizes
-def _sample_pairs(w, n, seed=0):
-    rng = np.random.default_rng(seed)
-    b = rng.integers(0, w.B, n)
-    h = rng.integers(0, w.Hq, n)
-    pairs = sorted(set(zip(b.tolist(), h.tolist())))
-    # every head of the longest and the shortest sequence too
-    for bb in (int(np.argmax(w.context_lens)), int(np.argmin(w.context_lens))):
-        pairs += [(bb, hh) for hh in range(w.Hq)]
-    return sorted(set(pairs))
+def _check_all_rows(w, ref, got, tol=TOL):
+    got = got.reshape(ref.shape)
+    assert np.all(np.isfinite(got))
+    err = np.abs(got.astype(np.float64) - ref).max()
+    worst = np.unravel_index(np.argmax(np.abs(got - ref)), ref.shape)
+    print(f"{w.name}: all {ref.shape[0]} rows, max |gpu - oracle| = {err:.3e} at row {worst[0]}")
+    assert err <= tol, (w.name, err, worst)
+    return err
 
 
 @pytest.mark.parametrize("name", ["tiny", "llama8b", "llama70b", "int8", "fp8", "int4"])
-def test_full_size_sampled_outputs(name):
+def test_full_size_outputs(name):
     """The full workloads, in the launch configuration the benchmark times
-    (automatic split count), checked on sampled (sequence, head) rows."""
-    w = W.by_name(name)
+    (automatic split count), every (sequence, query head) row against the
+    oracle."""
+    w, ref, _ = full_size_reference(name)
     got, _ = _run(w)
-    pairs = None if name == "tiny" else _sample_pairs(w, 64)
-    _check(w, got, pairs=pairs)
+    _check_all_rows(w, ref, got)
+
+
+@pytest.mark.parametrize("num_splits", [2, 5, 8])
+def test_full_size_llama70b_split_kv(num_splits):
+    """The Llama-3-70B-shaped batch (32 x 8192 tokens) with its split-KV path
+    forced: every row against the oracle (2e-3), and against the unsplit
+    decode of the same pool (1e-5: the log-sum-exp merge is exact up to
+    rounding)."""
+    w, ref, _ = full_size_reference("llama70b")
+    pool, bt, ctx, q = device_inputs(w)
+    device_append(pool, w, bt)
+    assert pa_decode_num_splits(pool, w.B, w.max_pages, num_splits) == num_splits
+    one = pa_decode(pool, q, bt, ctx, w.scale, num_splits=1)
+    got = pa_decode(pool, q, bt, ctx, w.scale, num_splits=num_splits)
+    torch.cuda.synchronize()
+    got_np = got.cpu().numpy().reshape(-1, w.D)
+    _check_all_rows(w, ref, got_np)
+    d = (got - one).abs().max().item()
+    print(f"llama70b S={num_splits} vs S=1: {d:.3e}")
+    assert d <= 1e-5
 
 
 def test_full_size_prefix_shared_equals_unshared():
@@ -280,7 +300,8 @@ def test_full_size_prefix_shared_equals_unshared():
     a, _ = _run(shared)
     b, _ = _run(unshared)
     np.testing.assert_array_equal(a, b)
-    _check(shared, a, pairs=_sample_pairs(shared, 48))
+    w, ref, _ = full_size_reference("prefix")
+    _check_all_rows(w, ref, a)
 
 
 def test_one_workspace_serves_calls_of_every_shape_and_entry_point():

@@ -10,7 +10,8 @@ import oracle
 from paged_kv_cache_466_b200 import (PA_DERR_BIG_SCALE, pa_decode, pa_decode_append)
 from paged_kv_cache_466_b200 import workloads as W
 from paged_kv_cache_466_b200.workloads import bits
-from tests.helpers import DEV, device_append, device_inputs, oracle_pool, pool_bytes_equal
+from tests.helpers import (DEV, device_append, device_inputs, full_size_reference, oracle_pool,
+                           pool_bytes_equal)
 
 pytestmark = pytest.mark.gpu
 RAGGED = [0, 1, 5000, 17, 0, 3, 16, 32, 4096, 0, 2049, 15]
@@ -63,6 +64,10 @@ def test_fused_step_full_size_llama70b():
     want = pa_decode(pool, q, bt, ctx, w.scale)   # the rows are in place now
     torch.cuda.synchronize()
     assert torch.equal(got, want)
+    _, ref, _ = full_size_reference("llama70b")
+    err = np.abs(got.cpu().numpy().reshape(ref.shape) - ref).max()
+    print(f"fused step llama70b: all rows, max |gpu - oracle| = {err:.3e}")
+    assert err <= 2e-3
     # the stored step rows are the inputs, bit for bit
     P = w.P
     for b in (0, w.B // 2, w.B - 1):

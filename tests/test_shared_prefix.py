@@ -7,7 +7,8 @@ import torch
 
 from paged_kv_cache_466_b200 import pa_decode, pa_decode_shared_prefix
 from paged_kv_cache_466_b200 import workloads as W
-from tests.helpers import DEV, device_append, device_inputs, oracle_decode, oracle_pool
+from tests.helpers import (DEV, device_append, device_inputs, full_size_reference,
+                           oracle_decode, oracle_pool)
 
 pytestmark = pytest.mark.gpu
 
@@ -56,12 +57,11 @@ def test_cascade_requests_without_own_tokens():
 
 
 def test_cascade_full_size_prefix_workload():
-    """128 requests x (2000-token shared prefix + U{1..512} own tokens)."""
-    w, _ = W.prefix()
+    """128 requests x (2000-token shared prefix + U{1..512} own tokens): every
+    row against the oracle and against the plain paged decode."""
+    w, ref, _ = full_size_reference("prefix")
     casc, plain = _both(w)
-    rng = np.random.default_rng(0)
-    pairs = sorted(set(zip(rng.integers(0, w.B, 64).tolist(), rng.integers(0, w.Hq, 64).tolist())))
-    ref, _ = oracle_decode(w, oracle_pool(w), pairs=pairs)
-    got = np.stack([casc[b * w.Hq + h] for b, h in pairs])
-    assert np.abs(got - ref).max() <= 2e-3
+    err = np.abs(casc - ref).max()
+    print(f"cascade full size: all {ref.shape[0]} rows, max |gpu - oracle| = {err:.3e}")
+    assert np.all(np.isfinite(casc)) and err <= 2e-3
     assert np.abs(casc - plain).max() <= 1e-4
