@@ -65,6 +65,10 @@ def parse():
     ap.add_argument("--alternate-pools", action="store_true",
                     help="keep two independent copies of the pool and alternate between them "
                          "step by step, so no step reads pages the previous step left in L2")
+    ap.add_argument("--context-parallel", action="store_true",
+                    help="every rank holds 1/N of each sequence's tokens of the same batch "
+                         "and decodes its range; one all-gather of (o, lse) and a merge per "
+                         "step (strong scaling over the token dimension)")
     ap.add_argument("--flush-l2", action="store_true",
                     help="write a buffer of twice the L2 size between timed steps; the step "
                          "time is then the sum of per-step CUDA events, flush excluded")
@@ -558,6 +562,139 @@ def run_ours(args, rank, world, local_rank):
     return res
 
 
+def cp_shard_rows(w, rank: int, world: int):
+    """Rank ``rank``'s share of the batch for the context-parallel mode: the
+    tokens per rank, its own tables and page count, and the (seq, pos, k, v)
+    rows of its token range, taken from the same seeded workload on every
+    rank."""
+    import numpy as np
+    from paged_kv_cache_466_b200.context_parallel import (rank_range, shard_tables,
+                                                           tokens_per_rank_for)
+    T = tokens_per_rank_for(int(w.context_lens.max()), world, w.P)
+    begin, end = rank_range(rank, world, T)
+    tables, n_pages = shard_tables(w.max_pages, w.context_lens, rank, world, T, w.P, seed=rank)
+    seq, pos, k, v = w.all_rows()
+    sel = np.flatnonzero((pos >= begin) & (pos < end))
+    idx = __import__("torch").from_numpy(sel)
+    return T, (begin, end), tables, max(n_pages, 1), (seq[sel], pos[sel], k[idx], v[idx])
+
+
+def run_context_parallel(args, rank, world, local_rank):
+    """The context-parallel decode of one batch over the ranks: rank r holds
+    tokens [r T, (r + 1) T) of every sequence in a pool of its own, decodes them
+    (pa_decode_range), all-gathers (o, lse) and merges (pa_merge_partials). A
+    step is the whole decode of the batch; value = the batch's bytes over the
+    slowest rank's step time."""
+    import torch
+    import torch.distributed as dist
+    from paged_kv_cache_466_b200 import KVPool, pa_kv_append
+    from paged_kv_cache_466_b200.context_parallel import decode_context_parallel
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = make_workload(args.workload, seed=0, batch=args.batch)   # the same batch everywhere
+    T, (begin, end), tables, n_pages, (seq, pos, k, v) = cp_shard_rows(w, rank, world)
+    pool = KVPool(n_pages, w.Hkv, w.P, w.D, w.kv, dev, fill_byte=0)
+    bt = torch.from_numpy(tables).to(dev)
+    ctx = torch.from_numpy(w.context_lens).to(dev)
+    q = w.q.to(dev)
+    chunk = 1 << 18
+    for a in range(0, len(seq), chunk):
+        b = min(a + chunk, len(seq))
+        pa_kv_append(pool, k[a:b].to(dev), v[a:b].to(dev), torch.from_numpy(seq[a:b]).to(dev),
+                     torch.from_numpy(pos[a:b]).to(dev), bt)
+    out = torch.empty((w.B, w.Hq, w.D), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(qq=q):
+        decode_context_parallel(pool, qq, bt, ctx, w.scale, T, out=out, num_splits=args.splits)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    K = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize()
+    clocks.mark(True)
+    for i in range(K):
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    clocks.mark(False)
+    clk = clocks.stop()
+    barrier()
+    per = [a.elapsed_time(b) for a, b in evs]
+    ms_step = max_over_ranks(sum(per) / K, world, dev)
+    batch_bytes = decode_bytes(w)
+    value = batch_bytes / (ms_step * 1e-3) / 1e9
+    rank_tok = int(sum(max(0, min(int(c), end) - begin) for c in w.context_lens))
+    rank_bytes = rank_tok * w.Hkv * 2 * {"bf16": w.D * 2, "u8": w.D + 8, "fp8": w.D + 8,
+                                         "u4": w.D // 2 + 8}[w.kv] + w.B * w.Hq * w.D * 2
+    # end to end: q from pinned host memory, the decode, the output back
+    h_q = w.q.pin_memory()
+    h_out = torch.empty((w.B, w.Hq, w.D), dtype=torch.float32).pin_memory()
+    d_q = torch.empty_like(q)
+
+    def e2e_step():
+        d_q.copy_(h_q, non_blocking=True)
+        step(d_q)
+        h_out.copy_(out, non_blocking=True)
+        stream.synchronize()
+
+    for _ in range(max(args.warmup, 3)):
+        e2e_step()
+    Ke = min(K, 500)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(Ke):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ems = max_over_ranks(e0.elapsed_time(e1) / Ke, world, dev)
+    peak, peak_kind = measured_peak()
+    achieved = rank_bytes / (statistics.mean(per) * 1e-3) / 1e9
+    cfg = config_of(w, args, world, 0)
+    cfg["global_batch"] = w.B
+    cfg["parallelism"] = (f"cp{world}: each rank holds {T} tokens of every sequence "
+                          f"(the last rank the rest); one all-gather of (o, lse) per step")
+    cfg["tokens_per_rank"] = T
+    return {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+        "dtype": "bf16" if w.kv == "bf16" else w.kv + " codes; fp32 accumulate",
+        "data": "synthetic (seeded N(0,1) bf16 K/V/q; no weights needed)",
+        "config": cfg,
+        "pct_of_peak": round(100.0 * value / world / peak, 2),
+        "peak_gbs": peak, "peak_kind": peak_kind,
+        "seq_per_s_per_layer": round(w.B / (ms_step * 1e-3), 1),
+        "e2e": {"value": round(batch_bytes / (ems * 1e-3) / 1e9, 1), "unit": "GB/s",
+                "h2d_bytes_per_step": h_q.numel() * h_q.element_size(),
+                "d2h_bytes_per_step": h_out.numel() * h_out.element_size(),
+                "steps": Ke, "ms_per_step": round(ems, 5)},
+        "roofline": {"bound": "hbm", "kernel": "context-parallel step on rank 0 (range "
+                     "decode + all-gather + merge), its own range's bytes",
+                     "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "algorithmic_bytes": rank_bytes,
+                     "avg_launch_ms": round(statistics.mean(per), 5)},
+        "gpu_launches": K * 2,
+        "clocks": clk,
+    }
+
+
 def run_reference(args, rank, world):
     """The CPU oracle as the reference arm: every step a bounded sample of the
     workload (a fixed set of (sequence, head) rows), timed on the host cores."""
@@ -620,7 +757,8 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=timedelta(seconds=180))
     try:
-        res = run_ours(args, rank, world, local_rank)
+        res = (run_context_parallel if args.context_parallel else run_ours)(
+            args, rank, world, local_rank)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

@@ -44,7 +44,7 @@
 extern "C" {
 #endif
 
-#define PA_ABI_VERSION 1
+#define PA_ABI_VERSION 2
 
 typedef enum {
   PA_OK = 0,
@@ -64,9 +64,6 @@ typedef enum {
 #define PA_DERR_BAD_CTX 2  /* context_len < 0 or > max_pages * page_size       */
 #define PA_DERR_BAD_SEQ 4  /* append: seq_idx outside [0, num_seqs)            */
 #define PA_DERR_BAD_POS 8  /* append: pos < 0 or pos / page_size >= max_pages  */
-#define PA_DERR_BIG_SCALE 16 /* append (and the fused cache write of
-                                pa_decode_append): a quantised row's scale is
-                                not below PA_MAX_KV_SCALE (still written)      */
 #define PA_DERR_TIMEOUT 32 /* a bounded wait on the kernel's own tensor-core
                               work ran out (not expected; outputs invalid)    */
 
@@ -75,16 +72,9 @@ typedef enum {
  * caller has read *d_err back to the host (host only, no device access):
  * 0 -> PA_OK; PA_DERR_TIMEOUT set -> PA_ERR_TIMEOUT (it wins over the
  * others: outputs are invalid); any of PA_DERR_BAD_PAGE, _BAD_CTX, _BAD_SEQ,
- * _BAD_POS -> PA_ERR_BAD_TABLE; PA_DERR_BIG_SCALE alone ->
- * PA_ERR_UNSUPPORTED; any other bit -> PA_ERR_INVALID_ARG.
+ * _BAD_POS -> PA_ERR_BAD_TABLE; any other bit -> PA_ERR_INVALID_ARG.
  */
 pa_status_t pa_derr_status(int32_t derr);
-
-/* Quantised pools: pa_decode* feed s * (softmax weight) to the tensor cores
- * as f16, with weights kept <= 8, so every row scale must be below this bound
- * (rows spanning less than 6.1e4 for INT4, 1.0e6 for INT8; FP8 rows with
- * max |x| below 1.8e6). pa_kv_append flags rows that break it. */
-#define PA_MAX_KV_SCALE 4096
 
 typedef enum {
   PA_KV_BF16 = 0,          /* K/V stored as bf16                               */
@@ -244,7 +234,7 @@ pa_status_t pa_decode(const pa_kv_pool_t *pool, const void *q,
  * Every other argument is pa_decode's. The CTA whose split holds position
  * context_lens[b] - 1 stores that row (quantised for INT8/FP8/INT4 pools by
  * the same per-row quantiser as pa_kv_append, so the stored bits are
- * identical, and PA_DERR_BIG_SCALE is flagged the same way) before it reads
+ * identical) before it reads
  * the page; then Eq. (1) runs over tokens 0 .. context_lens[b] - 1 as in
  * pa_decode. The result equals pa_kv_append(seq_idx = b, pos =
  * context_lens[b] - 1) followed by pa_decode, bit for bit, without the

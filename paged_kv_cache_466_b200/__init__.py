@@ -35,7 +35,7 @@ import torch
 from . import _lib
 from ._lib import (PA_DERR_BAD_CTX, PA_DERR_BAD_PAGE, PA_DERR_BAD_POS, PA_DERR_BAD_SEQ,
                    PA_STEP_NEWEST_PER_SEQ,
-                   PA_DERR_BIG_SCALE, PA_DERR_TIMEOUT, PA_MAX_KV_SCALE,
+                   PA_DERR_TIMEOUT,
                    PA_KV_BF16, PA_KV_FP8_PER_TOKEN, PA_KV_U4_PER_TOKEN, PA_KV_U8_PER_TOKEN,
                    PagedAttnError, pa_kv_pool_t)
 
@@ -50,7 +50,7 @@ __all__ = ["KVPool", "pa_kv_append", "pa_decode", "pa_decode_append", "pa_decode
            "PA_KV_BF16", "PA_KV_U8_PER_TOKEN", "PA_KV_FP8_PER_TOKEN", "PA_KV_U4_PER_TOKEN",
            "PA_DERR_BAD_PAGE",
            "PA_DERR_BAD_CTX",
-           "PA_DERR_BAD_SEQ", "PA_DERR_BAD_POS", "PA_DERR_BIG_SCALE", "PA_MAX_KV_SCALE",
+           "PA_DERR_BAD_SEQ", "PA_DERR_BAD_POS",
            "load_library"]
 
 

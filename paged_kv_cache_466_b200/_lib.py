@@ -23,9 +23,7 @@ PA_DERR_BAD_PAGE = 1
 PA_DERR_BAD_CTX = 2
 PA_DERR_BAD_SEQ = 4
 PA_DERR_BAD_POS = 8
-PA_DERR_BIG_SCALE = 16
 PA_DERR_TIMEOUT = 32
-PA_MAX_KV_SCALE = 4096
 
 PA_KV_BF16 = 0
 PA_KV_U8_PER_TOKEN = 1

@@ -21,6 +21,39 @@ from . import KVPool, pa_decode_range, pa_merge_partials
 _NO_END = 0x7FFFFFFF
 
 
+def tokens_per_rank_for(max_context: int, world: int, page_size: int) -> int:
+    """The even split of the longest context over ``world`` ranks, rounded up
+    to whole pages (every rank but the last holds exactly this many tokens of
+    a sequence that long)."""
+    if max_context < 0 or world <= 0 or page_size <= 0:
+        raise ValueError("bad max_context, world or page_size")
+    per = -(-max(max_context, 1) // world)
+    return -(-per // page_size) * page_size
+
+
+def shard_tables(block_tables_width: int, context_lens, rank: int, world: int,
+                 tokens_per_rank: int, page_size: int, seed: int = 0):
+    """Rank ``rank``'s own page tables for a context-parallel layout: the
+    logical pages of its token range get ids of a pool of its own (randomly
+    permuted with ``seed``), every other entry is -1 (never read by the range
+    decode). Returns (tables int32 [B, width], number of pages used)."""
+    import numpy as np
+    begin, end = rank_range(rank, world, tokens_per_rank)
+    ctx = np.asarray(context_lens, dtype=np.int64)
+    tables = np.full((len(ctx), block_tables_width), -1, np.int32)
+    lp_begin = begin // page_size
+    want = []
+    for b, c in enumerate(ctx.tolist()):
+        hi = -(-c // page_size)
+        if end != _NO_END:
+            hi = min(hi, end // page_size)
+        want += [(b, lp) for lp in range(lp_begin, hi)]
+    ids = np.random.default_rng(seed).permutation(len(want)).astype(np.int32)
+    for (b, lp), pid in zip(want, ids.tolist()):
+        tables[b, lp] = pid
+    return tables, len(want)
+
+
 def rank_range(rank: int, world: int, tokens_per_rank: int) -> Tuple[int, int]:
     """Token range [begin, end) rank ``rank`` of ``world`` decodes."""
     if tokens_per_rank <= 0 or not 0 <= rank < world:
@@ -69,9 +102,13 @@ def decode_context_parallel(pool: KVPool, q: torch.Tensor, block_tables: torch.T
 
     The range's o and lse are written straight into this rank's block of one
     fp32 buffer, so a single all-gather moves both, and the merge reads the
-    gathered buffer in place."""
-    rank = dist.get_rank(group)
-    world = dist.get_world_size(group)
+    gathered buffer in place. Without an initialised process group the call
+    is the one-rank case (the whole context on this GPU, no collective)."""
+    if dist.is_available() and dist.is_initialized():
+        rank = dist.get_rank(group)
+        world = dist.get_world_size(group)
+    else:
+        rank, world = 0, 1
     if tokens_per_rank % pool.page_size != 0:
         raise ValueError("tokens_per_rank must be a multiple of the page size")
     B, Hq, D = q.shape
@@ -80,12 +117,15 @@ def decode_context_parallel(pool: KVPool, q: torch.Tensor, block_tables: torch.T
     o, lse = partial_views(block, B, Hq, D)
     pa_decode_range(pool, q, block_tables, context_lens, scale, begin, end, o_out=o,
                     lse_out=lse, num_splits=num_splits, d_err=d_err)
-    gathered = torch.empty(world * block.numel(), dtype=torch.float32, device=q.device)
-    dist.all_gather_into_tensor(gathered, block, group=group)
+    if world == 1:
+        gathered = block
+    else:
+        gathered = torch.empty(world * block.numel(), dtype=torch.float32, device=q.device)
+        dist.all_gather_into_tensor(gathered, block, group=group)
     o_parts, lse_parts = gathered_views(gathered, world, B, Hq, D)
     merged, _ = pa_merge_partials(o_parts, lse_parts, out=out)
     return merged
 
 
-__all__ = ["rank_range", "partial_block_floats", "partial_views", "gathered_views",
+__all__ = ["rank_range", "tokens_per_rank_for", "shard_tables", "partial_block_floats", "partial_views", "gathered_views",
            "decode_context_parallel"]

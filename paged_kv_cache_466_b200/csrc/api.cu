@@ -151,7 +151,6 @@ pa_status_t pa_derr_status(int32_t derr) {
   if (derr & PA_DERR_TIMEOUT) return PA_ERR_TIMEOUT;
   if (derr & (PA_DERR_BAD_PAGE | PA_DERR_BAD_CTX | PA_DERR_BAD_SEQ | PA_DERR_BAD_POS))
     return PA_ERR_BAD_TABLE;
-  if (derr == PA_DERR_BIG_SCALE) return PA_ERR_UNSUPPORTED;
   return PA_ERR_INVALID_ARG;
 }
 

@@ -75,24 +75,27 @@ namespace {
 constexpr float kLn2 = 0.693147180559945309f;
 // Lazy rescaling: the running max is only raised when a block's max exceeds it
 // by more than this many powers of two, so weights stay <= 2^kRescaleLog2.
-// Quantised pools scale the weights by the row scale s < 2^12 into f16
-// operands, so they keep weights <= 2^3 (p * s < 2^15 < f16 max).
+// Quantised pools keep the weights <= 2^3, so that the power of two that
+// normalises the V weights (below) moves rarely.
 template <int KVT>
 constexpr float kRescaleLog2 = KVT == PA_KV_BF16 ? 8.0f : 3.0f;
-static_assert(PA_MAX_KV_SCALE == 4096, "p * s must stay below the f16 maximum");
+
+// FP8 pools (E4M3 codes, z = 0) share the INT8 layout.
+template <int KVT>
+constexpr bool kIsFp8 = KVT == PA_KV_FP8_PER_TOKEN;
+// Codes reach the MMA scaled by an exact power of two: an INT8 byte, or an
+// INT4 low nibble, under zero high bits is the f16 subnormal c * 2^-24; an
+// INT4 high nibble left in place is c * 2^-20; FP8 codes go as they are. The
+// K scale and O after the loop take the powers of two back.
+template <int KVT>
+constexpr float kCodeScale = kIsFp8<KVT> ? 1.f : 16777216.f;
 
 template <int D, int KVT>
 struct Tile {
   static_assert(D == 64 || D == 128, "head_dim");
   // INT8 and FP8 pools share the layout: 1-byte codes + (scale, zero) per row
   static constexpr bool kU8 = KVT != PA_KV_BF16;
-  static constexpr bool kFp8 = KVT == PA_KV_FP8_PER_TOKEN;
   static constexpr bool kU4 = KVT == PA_KV_U4_PER_TOKEN;  // two codes per byte
-  // Codes reach the MMA scaled by an exact power of two: an INT8 byte, or an
-  // INT4 low nibble, under zero high bits is the f16 subnormal c * 2^-24; an
-  // INT4 high nibble left in place is c * 2^-20; FP8 codes go as they are.
-  // The K scale and O after the loop take the powers of two back.
-  static constexpr float kCodeScale = kFp8 ? 1.f : 16777216.f;
   static constexpr int kElem = kU8 ? 1 : 2;
   static constexpr int kRowBytes = kU4 ? D / 2 : D * kElem;
   // one 16-token block of K (or V) is 16 contiguous rows of the page
@@ -344,114 +347,51 @@ __device__ __forceinline__ void issue_block(const LaneMap<D, KVT> &lm, uint32_t 
   }
 }
 
+// ---- bf16 pools ---------------------------------------------------------------
+//
 // One warp's online-softmax state for the G heads of a (sequence, KV head).
-template <int D, int KVT>
+template <int D>
 struct WarpAcc {
-  float o[Tile<D, KVT>::kMTiles][4];
+  float o[D / 16][4];
   float m_run;  // running max of this head's scores (log2 units)
   float l_run;  // this lane's share of the softmax denominator
-  float zacc;   // quantised pools: this lane's share of sum_t p_t z_t
   __device__ __forceinline__ void reset() {
 #pragma unroll
-    for (int j = 0; j < Tile<D, KVT>::kMTiles; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+    for (int j = 0; j < D / 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
     m_run = -INFINITY;
     l_run = 0.f;
-    zacc = 0.f;
   }
 };
 
-// Scores, online softmax and O^T update for the 16-token block staged at
+// Scores, online softmax and O^T update for the 16-token bf16 block staged at
 // `src`, whose first token is btok; tokens outside [tok_lo, tok1) and all
 // tokens of an invalid page (pvalid false) are masked.
-template <int D, int KVT>
-__device__ __forceinline__ void block_step(const LaneMap<D, KVT> &lm, uint32_t src, int btok,
-                                           int tok_lo, int tok1, bool pvalid, float scale_log2,
-                                           const uint32_t (&qa)[D / 16][2], float qsum, int g,
-                                           int t, WarpAcc<D, KVT> &acc) {
-  using T = Tile<D, KVT>;
+template <int D>
+__device__ __forceinline__ void block_step(const LaneMap<D, PA_KV_BF16> &lm, uint32_t src,
+                                           int btok, int tok_lo, int tok1, bool pvalid,
+                                           float scale_log2, const uint32_t (&qa)[D / 16][2],
+                                           int t, WarpAcc<D> &acc) {
+  using T = Tile<D, PA_KV_BF16>;
   float(&o)[T::kMTiles][4] = acc.o;
   float &m_run = acc.m_run;
   float &l_run = acc.l_run;
-  float &zacc = acc.zacc;
   const auto &koff = lm.koff;
   const auto &voff = lm.voff;
   // ---- S = Q K^T -------------------------------------------------------------
   float s[2][4];
-  float s_hi[2][4];  // INT4: the high-nibble products (codes scaled 16x more)
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt) {
     s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-    if constexpr (T::kU4) {
-      s_hi[nt][0] = s_hi[nt][1] = s_hi[nt][2] = s_hi[nt][3] = 0.f;
-      uint32_t wk[D / 32];
-      if constexpr (D == 128) {
-        const uint4 v = lds128(src + koff[nt][0]);
-        wk[0] = v.x; wk[1] = v.y; wk[2] = v.z; wk[3] = v.w;
-      } else {
-        const uint2 v = lds64(src + koff[nt][0]);
-        wk[0] = v.x; wk[1] = v.y;
-      }
 #pragma unroll
-      for (int w = 0; w < D / 32; ++w) {
-        // elements e0..e7 of the word (e2i in the low nibble of byte i): low
-        // nibbles under zero bits are the f16 subnormals c * 2^-24, pairs
-        // (e0, e4) and (e2, e6); high nibbles in place are c * 2^-20, pairs
-        // (e1, e5) and (e3, e7)
-        const uint32_t w8 = wk[w] >> 8;
-        mma_f16_16816(s[nt], qa[2 * w][0], 0u, qa[2 * w][1], 0u, wk[w] & 0x000F000Fu,
-                      w8 & 0x000F000Fu);
-        mma_f16_16816(s_hi[nt], qa[2 * w + 1][0], 0u, qa[2 * w + 1][1], 0u,
-                      wk[w] & 0x00F000F0u, w8 & 0x00F000F0u);
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < T::kKChunks; ++i) {
-        const uint4 kv = lds128(src + koff[nt][i]);
-        if constexpr (!T::kU8) {
-          mma_bf16_16816(s[nt], qa[2 * i][0], 0u, qa[2 * i][1], 0u, kv.x, kv.y);
-          mma_bf16_16816(s[nt], qa[2 * i + 1][0], 0u, qa[2 * i + 1][1], 0u, kv.z, kv.w);
-        } else {
-          const uint32_t w4[4] = {kv.x, kv.y, kv.z, kv.w};
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const uint32_t b0 =
-                T::kFp8 ? e4m3x2_to_f16x2(w4[w]) : u8x2_to_f16x2(w4[w], 0x4140);
-            const uint32_t b1 =
-                T::kFp8 ? e4m3x2_to_f16x2(w4[w] >> 16) : u8x2_to_f16x2(w4[w], 0x4342);
-            mma_f16_16816(s[nt], qa[4 * i + w][0], 0u, qa[4 * i + w][1], 0u, b0, b1);
-          }
-        }
-      }
+    for (int i = 0; i < T::kKChunks; ++i) {
+      const uint4 kv = lds128(src + koff[nt][i]);
+      mma_bf16_16816(s[nt], qa[2 * i][0], 0u, qa[2 * i][1], 0u, kv.x, kv.y);
+      mma_bf16_16816(s[nt], qa[2 * i + 1][0], 0u, qa[2 * i + 1][1], 0u, kv.z, kv.w);
     }
   }
 
   // ---- online softmax (log2 domain) ---------------------------------------
   float x[4] = {s[0][0], s[0][1], s[1][0], s[1][1]};  // tokens 2t, 2t+1, 8+2t, 9+2t
-  if constexpr (T::kU4) {  // high-nibble products were scaled 16x more
-    x[0] = fmaf(s_hi[0][0], 0.0625f, x[0]);
-    x[1] = fmaf(s_hi[0][1], 0.0625f, x[1]);
-    x[2] = fmaf(s_hi[1][0], 0.0625f, x[2]);
-    x[3] = fmaf(s_hi[1][1], 0.0625f, x[3]);
-  }
-  float vs[4], vz[4];
-  if constexpr (T::kU8) {
-    const uint4 k01 = lds128(src + T::kKSzOff + 16 * t);
-    const uint4 k89 = lds128(src + T::kKSzOff + 16 * (4 + t));
-    const uint4 v01 = lds128(src + T::kVSzOff + 16 * t);
-    const uint4 v89 = lds128(src + T::kVSzOff + 16 * (4 + t));
-    const float ks[4] = {__uint_as_float(k01.x), __uint_as_float(k01.z),
-                         __uint_as_float(k89.x), __uint_as_float(k89.z)};
-    const float kz[4] = {__uint_as_float(k01.y), __uint_as_float(k01.w),
-                         __uint_as_float(k89.y), __uint_as_float(k89.w)};
-    vs[0] = __uint_as_float(v01.x); vz[0] = __uint_as_float(v01.y);
-    vs[1] = __uint_as_float(v01.z); vz[1] = __uint_as_float(v01.w);
-    vs[2] = __uint_as_float(v89.x); vz[2] = __uint_as_float(v89.y);
-    vs[3] = __uint_as_float(v89.z); vz[3] = __uint_as_float(v89.w);
-    // the codes' power-of-two scale goes back into the K scale here (and
-    // into O after the loop)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) x[e] = fmaf(ks[e] * T::kCodeScale, x[e], kz[e] * qsum);
-  }
   if (pvalid && btok >= tok_lo && btok + 16 <= tok1) {  // warp-uniform: no mask needed
 #pragma unroll
     for (int e = 0; e < 4; ++e) x[e] *= scale_log2;
@@ -461,21 +401,17 @@ __device__ __forceinline__ void block_step(const LaneMap<D, KVT> &lm, uint32_t s
       const int tok = btok + (e & 1) + 2 * t + (e >> 1) * 8;
       const bool ok = pvalid && tok >= tok_lo && tok < tok1;
       x[e] = ok ? x[e] * scale_log2 : -INFINITY;
-      if constexpr (T::kU8) {
-        if (!ok) vs[e] = vz[e] = 0.f;
-      }
     }
   }
   float mb = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
   mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
   mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
-  const bool need = mb > m_run + kRescaleLog2<KVT> || (m_run == -INFINITY && mb > -INFINITY);
+  const bool need = mb > m_run + kRescaleLog2<PA_KV_BF16> || (m_run == -INFINITY && mb > -INFINITY);
   if (__any_sync(0xffffffffu, need)) {
     const float m_new = fmaxf(m_run, mb);
     const float alpha = m_new == -INFINITY ? 1.f : fast_exp2(m_run - m_new);
     m_run = m_new;
     l_run *= alpha;
-    zacc *= alpha;
     const float al0 = __shfl_sync(0xffffffffu, alpha, 8 * t);      // head 2t
     const float al1 = __shfl_sync(0xffffffffu, alpha, 8 * t + 4);  // head 2t+1
 #pragma unroll
@@ -494,74 +430,184 @@ __device__ __forceinline__ void block_step(const LaneMap<D, KVT> &lm, uint32_t s
 
   // ---- O^T += V^T P^T -------------------------------------------------------
   uint32_t bh0, bl0, bh1, bl1;
-  if constexpr (!T::kU8) {
-    split_bf16(p[0], p[1], bh0, bl0);
-    split_bf16(p[2], p[3], bh1, bl1);
+  split_bf16(p[0], p[1], bh0, bl0);
+  split_bf16(p[2], p[3], bh1, bl1);
 #pragma unroll
-    for (int c = 0; c < T::kVChunks; ++c) {
-      const uint4 v0 = lds128(src + voff[0][c]);
-      const uint4 v1 = lds128(src + voff[1][c]);
-      const uint4 v2 = lds128(src + voff[2][c]);
-      const uint4 v3 = lds128(src + voff[3][c]);
-      const uint32_t x0[4] = {v0.x, v0.y, v0.z, v0.w};
-      const uint32_t x1[4] = {v1.x, v1.y, v1.z, v1.w};
-      const uint32_t x2[4] = {v2.x, v2.y, v2.z, v2.w};
-      const uint32_t x3[4] = {v3.x, v3.y, v3.z, v3.w};
+  for (int c = 0; c < T::kVChunks; ++c) {
+    const uint4 v0 = lds128(src + voff[0][c]);
+    const uint4 v1 = lds128(src + voff[1][c]);
+    const uint4 v2 = lds128(src + voff[2][c]);
+    const uint4 v3 = lds128(src + voff[3][c]);
+    const uint32_t x0[4] = {v0.x, v0.y, v0.z, v0.w};
+    const uint32_t x1[4] = {v1.x, v1.y, v1.z, v1.w};
+    const uint32_t x2[4] = {v2.x, v2.y, v2.z, v2.w};
+    const uint32_t x3[4] = {v3.x, v3.y, v3.z, v3.w};
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const uint32_t a0 = __byte_perm(x0[w], x1[w], 0x5410);
+      const uint32_t a1 = __byte_perm(x0[w], x1[w], 0x7632);
+      const uint32_t a2 = __byte_perm(x2[w], x3[w], 0x5410);
+      const uint32_t a3 = __byte_perm(x2[w], x3[w], 0x7632);
+      mma_bf16_16816(o[4 * c + w], a0, a1, a2, a3, bh0, bh1);
+      mma_bf16_16816(o[4 * c + w], a0, a1, a2, a3, bl0, bl1);
+    }
+  }
+}
+
+// ---- quantised pools (INT8, FP8, INT4): tokens as the MMA's M dimension ---------
+//
+// A warp step covers two 16-token blocks (32 tokens), and per block
+//   S^T[16 tokens x 8 heads]  = K[tokens x D] . Q^T[D x heads]      (A = K, B = Q)
+//   O^T[D x 8 heads]         += V^T[D x tokens] . P^T[tokens x heads]
+// With the tokens as M every row of the score MMA is a real token (with the
+// heads as M, rows 8..15 would be zero): half the score MMAs of a head-major
+// product. The lane then holds the scores of tokens g and g + 8 for heads 2t
+// and 2t + 1, the same two heads whose columns of O^T it accumulates, so the
+// online-softmax state of those heads lives in the lane and the rescale of O
+// needs no shuffle; P^T, the B operand of the second product, is the score
+// fragment transposed, which movmatrix does in registers. The K fragments
+// (A operand) are the registers the head-major B operand used, so the staging,
+// its swizzle and the code unpack are shared with the bf16 path.
+//
+// The V weights p_t * s_t (s_t the row scale of Eq. 3) enter the f16 MMA
+// scaled by a per-head power of two 2^-E, kept like the running max: E is set
+// from the first nonzero weights so that the largest sits at 2^12 .. 2^13, and
+// raised whenever a later weight would pass 2^14, O then being multiplied by
+// the exact power of two. O is thus carried in units of 2^E (fp32) and every
+// weight keeps the f16 precision whatever the row scales are, with no limit
+// on the scale from the f16 range.
+constexpr float kWeightHi = 16384.f;  // largest scaled V weight fed to the MMA (2^14)
+constexpr int kWeightTopExp = 12;     // a new E puts the largest weight at 2^12 .. 2^13
+constexpr int kEMin = -120, kEMax = 120;
+
+// 2^n as a float for -126 <= n <= 127; 0 below.
+__device__ __forceinline__ float exp2i(int n) {
+  return n < -126 ? 0.f : __uint_as_float(static_cast<uint32_t>(n + 127) << 23);
+}
+// floor(log2(x)) of a positive normal float (subnormals give -127).
+__device__ __forceinline__ int ilog2f(float x) {
+  return static_cast<int>((__float_as_uint(x) >> 23) & 0xffu) - 127;
+}
+
+template <int D>
+struct QAcc {
+  float o[D / 16][4];
+  float m[2];  // running max of the scores of heads 2t, 2t + 1 (log2 units)
+  float l[2];  // this lane's share of their softmax denominators
+  float z[2];  // this lane's share of sum_t p_t z_t
+  float f[2];  // 2^-E of each head; 0 until the head's first nonzero weight
+  int e[2];    // E of each head
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int j = 0; j < D / 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      m[h] = -INFINITY;
+      l[h] = z[h] = f[h] = 0.f;
+      e[h] = 0;
+    }
+  }
+};
+
+// S^T of the 16-token quantised block staged at `src` (codes times the
+// Tile's power of two): s[0], s[1] = token g, heads 2t, 2t + 1; s[2], s[3] =
+// token g + 8.
+template <int D, int KVT>
+__device__ __forceinline__ void scores_t(const LaneMap<D, KVT> &lm, uint32_t src,
+                                         const uint32_t (&qa)[D / 16][2], float (&s)[4]) {
+  using T = Tile<D, KVT>;
+  s[0] = s[1] = s[2] = s[3] = 0.f;
+  if constexpr (T::kU4) {
+    // rows g and g + 8; per word (e2i in the low nibble of byte i) the low
+    // nibbles under zero bits are the f16 subnormals c * 2^-24 (pairs e0, e4
+    // and e2, e6), the high nibbles in place c * 2^-20 (pairs e1, e5 and e3, e7)
+    float sh[4] = {0.f, 0.f, 0.f, 0.f};
+    uint32_t r0[D / 32], r1[D / 32];
+    if constexpr (D == 128) {
+      const uint4 a = lds128(src + lm.koff[0][0]);
+      const uint4 b = lds128(src + lm.koff[1][0]);
+      r0[0] = a.x; r0[1] = a.y; r0[2] = a.z; r0[3] = a.w;
+      r1[0] = b.x; r1[1] = b.y; r1[2] = b.z; r1[3] = b.w;
+    } else {
+      const uint2 a = lds64(src + lm.koff[0][0]);
+      const uint2 b = lds64(src + lm.koff[1][0]);
+      r0[0] = a.x; r0[1] = a.y;
+      r1[0] = b.x; r1[1] = b.y;
+    }
+#pragma unroll
+    for (int w = 0; w < D / 32; ++w) {
+      const uint32_t u0 = r0[w] >> 8, u1 = r1[w] >> 8;
+      mma_f16_16816(s, r0[w] & 0x000F000Fu, r1[w] & 0x000F000Fu, u0 & 0x000F000Fu,
+                    u1 & 0x000F000Fu, qa[2 * w][0], qa[2 * w][1]);
+      mma_f16_16816(sh, r0[w] & 0x00F000F0u, r1[w] & 0x00F000F0u, u0 & 0x00F000F0u,
+                    u1 & 0x00F000F0u, qa[2 * w + 1][0], qa[2 * w + 1][1]);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s[e] = fmaf(sh[e], 0.0625f, s[e]);  // high nibbles: 16x
+  } else {
+#pragma unroll
+    for (int i = 0; i < T::kKChunks; ++i) {
+      const uint4 k0 = lds128(src + lm.koff[0][i]);  // token g
+      const uint4 k1 = lds128(src + lm.koff[1][i]);  // token g + 8
+      const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w};
+      const uint32_t w1[4] = {k1.x, k1.y, k1.z, k1.w};
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
-        const uint32_t a0 = __byte_perm(x0[w], x1[w], 0x5410);
-        const uint32_t a1 = __byte_perm(x0[w], x1[w], 0x7632);
-        const uint32_t a2 = __byte_perm(x2[w], x3[w], 0x5410);
-        const uint32_t a3 = __byte_perm(x2[w], x3[w], 0x7632);
-        mma_bf16_16816(o[4 * c + w], a0, a1, a2, a3, bh0, bh1);
-        mma_bf16_16816(o[4 * c + w], a0, a1, a2, a3, bl0, bl1);
+        const uint32_t a0 = kIsFp8<KVT> ? e4m3x2_to_f16x2(w0[w]) : u8x2_to_f16x2(w0[w], 0x4140);
+        const uint32_t a1 = kIsFp8<KVT> ? e4m3x2_to_f16x2(w1[w]) : u8x2_to_f16x2(w1[w], 0x4140);
+        const uint32_t a2 =
+            kIsFp8<KVT> ? e4m3x2_to_f16x2(w0[w] >> 16) : u8x2_to_f16x2(w0[w], 0x4342);
+        const uint32_t a3 =
+            kIsFp8<KVT> ? e4m3x2_to_f16x2(w1[w] >> 16) : u8x2_to_f16x2(w1[w], 0x4342);
+        mma_f16_16816(s, a0, a1, a2, a3, qa[4 * i + w][0], qa[4 * i + w][1]);
+      }
+    }
+  }
+}
+
+// O^T += V^T W^T for the quantised block staged at `src`, with the weights'
+// B fragments (hi and lo halves, tokens 0..7 in b?0 and 8..15 in b?1).
+template <int D, int KVT>
+__device__ __forceinline__ void pv_quant(const LaneMap<D, KVT> &lm, uint32_t src, int g,
+                                         uint32_t bh0, uint32_t bh1, uint32_t bl0,
+                                         uint32_t bl1, float (&o)[D / 16][4]) {
+  using T = Tile<D, KVT>;
+  const auto &voff = lm.voff;
+  if constexpr (T::kU4) {
+    // byte j of this lane's slice holds d = base + 2j (low nibble) and + 1
+    uint32_t xv[4][D / 64];
+#pragma unroll
+    for (int tau = 0; tau < 4; ++tau) {
+      if constexpr (D == 128) {
+        const uint2 v = lds64(src + voff[tau][0]);
+        xv[tau][0] = v.x;
+        xv[tau][1] = v.y;
+      } else {
+        xv[tau][0] = lds32(src + voff[tau][0]);
+      }
+    }
+    // m-tiles j, j+1 use bytes j & 3, (j & 3) + 1 of word j / 4: gather them
+    // per token pair as (token 2t: byte b, b + 1 | token 2t + 1: byte b,
+    // b + 1), so that each 16-bit half holds one token's bytes; low nibbles
+    // under zero bits (c * 2^-24) give rows d (a0, a2), high nibbles in
+    // place (c * 2^-20) rows d + 1 (a1, a3)
+#pragma unroll
+    for (int j = 0; j < T::kMTiles; j += 2) {
+      const uint32_t sel = (j & 2) ? 0x7632 : 0x5410;
+      const uint32_t ya = __byte_perm(xv[0][j / 4], xv[1][j / 4], sel);
+      const uint32_t yb = __byte_perm(xv[2][j / 4], xv[3][j / 4], sel);
+      const uint32_t ya8 = ya >> 8, yb8 = yb >> 8;
+      const uint32_t a0[2] = {ya & 0x000F000Fu, ya8 & 0x000F000Fu};
+      const uint32_t a1[2] = {ya & 0x00F000F0u, ya8 & 0x00F000F0u};
+      const uint32_t a2[2] = {yb & 0x000F000Fu, yb8 & 0x000F000Fu};
+      const uint32_t a3[2] = {yb & 0x00F000F0u, yb8 & 0x00F000F0u};
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        mma_f16_16816(o[j + u], a0[u], a1[u], a2[u], a3[u], bh0, bh1);
+        mma_f16_16816(o[j + u], a0[u], a1[u], a2[u], a3[u], bl0, bl1);
       }
     }
   } else {
-    float pv[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      pv[e] = p[e] * vs[e];
-      zacc = fmaf(p[e], vz[e], zacc);
-    }
-    split_f16(pv[0], pv[1], bh0, bl0);
-    split_f16(pv[2], pv[3], bh1, bl1);
-    if constexpr (T::kU4) {
-      // byte j of this lane's slice holds d = base + 2j (low nibble) and + 1
-      uint32_t xv[4][D / 64];
-#pragma unroll
-      for (int tau = 0; tau < 4; ++tau) {
-        if constexpr (D == 128) {
-          const uint2 v = lds64(src + voff[tau][0]);
-          xv[tau][0] = v.x;
-          xv[tau][1] = v.y;
-        } else {
-          xv[tau][0] = lds32(src + voff[tau][0]);
-        }
-      }
-      // m-tiles j, j+1 use bytes j & 3, (j & 3) + 1 of word j / 4: gather them
-      // per token pair as (token 2t: byte b, b + 1 | token 2t + 1: byte b,
-      // b + 1), so that each 16-bit half holds one token's bytes; low nibbles
-      // under zero bits (c * 2^-24) give rows d (a0, a2), high nibbles in
-      // place (c * 2^-20) rows d + 1 (a1, a3)
-#pragma unroll
-      for (int j = 0; j < T::kMTiles; j += 2) {
-        const uint32_t sel = (j & 2) ? 0x7632 : 0x5410;
-        const uint32_t ya = __byte_perm(xv[0][j / 4], xv[1][j / 4], sel);
-        const uint32_t yb = __byte_perm(xv[2][j / 4], xv[3][j / 4], sel);
-        const uint32_t ya8 = ya >> 8, yb8 = yb >> 8;
-        const uint32_t a0[2] = {ya & 0x000F000Fu, ya8 & 0x000F000Fu};
-        const uint32_t a1[2] = {ya & 0x00F000F0u, ya8 & 0x00F000F0u};
-        const uint32_t a2[2] = {yb & 0x000F000Fu, yb8 & 0x000F000Fu};
-        const uint32_t a3[2] = {yb & 0x00F000F0u, yb8 & 0x00F000F0u};
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          mma_f16_16816(o[j + u], a0[u], a1[u], a2[u], a3[u], bh0, bh1);
-          mma_f16_16816(o[j + u], a0[u], a1[u], a2[u], a3[u], bl0, bl1);
-        }
-      }
-      return;
-    }
     const uint4 v0 = lds128(src + voff[0][0]);
     const uint4 v1 = lds128(src + voff[1][0]);
     const uint4 v2 = lds128(src + voff[2][0]);
@@ -580,45 +626,155 @@ __device__ __forceinline__ void block_step(const LaneMap<D, KVT> &lm, uint32_t s
       const uint32_t w3 = D == 128 ? x3[j / 2] : ((g & 1) ? x3[2 + j / 2] : x3[j / 2]);
       const uint32_t xa = __byte_perm(w0, w1, sel);
       const uint32_t xb = __byte_perm(w2, w3, sel);
-      const uint32_t a0 = T::kFp8 ? e4m3x2_to_f16x2(xa) : u8x2_to_f16x2(xa, 0x4140);
-      const uint32_t a1 = T::kFp8 ? e4m3x2_to_f16x2(xa >> 16) : u8x2_to_f16x2(xa, 0x4342);
-      const uint32_t a2 = T::kFp8 ? e4m3x2_to_f16x2(xb) : u8x2_to_f16x2(xb, 0x4140);
-      const uint32_t a3 = T::kFp8 ? e4m3x2_to_f16x2(xb >> 16) : u8x2_to_f16x2(xb, 0x4342);
+      const uint32_t a0 = kIsFp8<KVT> ? e4m3x2_to_f16x2(xa) : u8x2_to_f16x2(xa, 0x4140);
+      const uint32_t a1 = kIsFp8<KVT> ? e4m3x2_to_f16x2(xa >> 16) : u8x2_to_f16x2(xa, 0x4342);
+      const uint32_t a2 = kIsFp8<KVT> ? e4m3x2_to_f16x2(xb) : u8x2_to_f16x2(xb, 0x4140);
+      const uint32_t a3 = kIsFp8<KVT> ? e4m3x2_to_f16x2(xb >> 16) : u8x2_to_f16x2(xb, 0x4342);
       mma_f16_16816(o[j], a0, a1, a2, a3, bh0, bh1);
       mma_f16_16816(o[j], a0, a1, a2, a3, bl0, bl1);
     }
   }
 }
 
-// Reduce the per-lane softmax sums over each head's 4 lanes and apply the
-// quantised zero-point term: afterwards o holds sum_t p_t v_t for heads 2t and
-// 2t + 1 and l_run the denominator of head g.
+// One warp step over two quantised 16-token blocks staged at src and src +
+// one block (first tokens btok[0], btok[1]; pvalid false = invalid page or no
+// block). kscale = the Tile's code scale times scale * log2(e); qz = the sums
+// of q of heads 2t, 2t + 1 times scale * log2(e).
 template <int D, int KVT>
-__device__ __forceinline__ void finish_acc(WarpAcc<D, KVT> &acc, int t) {
+__device__ __forceinline__ void pair_step(const LaneMap<D, KVT> &lm, uint32_t src,
+                                          const int (&btok)[2], const bool (&pvalid)[2],
+                                          int tok_lo, int tok1, float kscale,
+                                          const float (&qz)[2],
+                                          const uint32_t (&qa)[D / 16][2], int g,
+                                          QAcc<D> &acc) {
   using T = Tile<D, KVT>;
-  float(&o)[T::kMTiles][4] = acc.o;
-  float &l_run = acc.l_run;
-  float &zacc = acc.zacc;
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
-  if constexpr (T::kU8) {
-    zacc += __shfl_xor_sync(0xffffffffu, zacc, 1);
-    zacc += __shfl_xor_sync(0xffffffffu, zacc, 2);
-    const float z0 = __shfl_sync(0xffffffffu, zacc, 8 * t);
-    const float z1 = __shfl_sync(0xffffffffu, zacc, 8 * t + 4);
-    // undo the codes' power-of-two scale; INT4 rows g + 8 hold the high
-    // nibbles (d + 1), which were scaled 16x more
-    constexpr float kRowHiScale = T::kU4 ? T::kCodeScale / 16.f : T::kCodeScale;
+  float x[2][4];           // [block][token g: heads 2t, 2t+1 | token g + 8: same]
+  float vs[2][2], vz[2][2];  // [block][token g | g + 8]
 #pragma unroll
-    for (int j = 0; j < T::kMTiles; ++j) {
-      o[j][0] = fmaf(o[j][0], T::kCodeScale, z0);
-      o[j][1] = fmaf(o[j][1], T::kCodeScale, z1);
-      o[j][2] = fmaf(o[j][2], kRowHiScale, z0);
-      o[j][3] = fmaf(o[j][3], kRowHiScale, z1);
+  for (int u = 0; u < 2; ++u) {
+    const uint32_t sb = src + u * T::kStageBytes;
+    float s[4];
+    scores_t<D, KVT>(lm, sb, qa, s);
+    const uint2 k0 = lds64(sb + T::kKSzOff + 8 * g);
+    const uint2 k1 = lds64(sb + T::kKSzOff + 8 * (g + 8));
+    const uint2 v0 = lds64(sb + T::kVSzOff + 8 * g);
+    const uint2 v1 = lds64(sb + T::kVSzOff + 8 * (g + 8));
+    // q.x = s (q.c) + z sum(q), per token
+    const float ka = __uint_as_float(k0.x) * kscale, kb = __uint_as_float(k1.x) * kscale;
+    const float za = __uint_as_float(k0.y), zb = __uint_as_float(k1.y);
+    x[u][0] = fmaf(ka, s[0], za * qz[0]);
+    x[u][1] = fmaf(ka, s[1], za * qz[1]);
+    x[u][2] = fmaf(kb, s[2], zb * qz[0]);
+    x[u][3] = fmaf(kb, s[3], zb * qz[1]);
+    vs[u][0] = __uint_as_float(v0.x);
+    vz[u][0] = __uint_as_float(v0.y);
+    vs[u][1] = __uint_as_float(v1.x);
+    vz[u][1] = __uint_as_float(v1.y);
+    if (!(pvalid[u] && btok[u] >= tok_lo && btok[u] + 16 <= tok1)) {  // warp-uniform
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int tok = btok[u] + g + 8 * r;
+        if (!(pvalid[u] && tok >= tok_lo && tok < tok1)) {
+          x[u][2 * r] = x[u][2 * r + 1] = -INFINITY;
+          vs[u][r] = vz[u][r] = 0.f;
+        }
+      }
     }
   }
-}
 
+  // ---- online softmax of heads 2t, 2t + 1 over the 32 tokens ----------------
+  float mb[2] = {fmaxf(fmaxf(x[0][0], x[0][2]), fmaxf(x[1][0], x[1][2])),
+                 fmaxf(fmaxf(x[0][1], x[0][3]), fmaxf(x[1][1], x[1][3]))};
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    mb[0] = fmaxf(mb[0], __shfl_xor_sync(0xffffffffu, mb[0], off));
+    mb[1] = fmaxf(mb[1], __shfl_xor_sync(0xffffffffu, mb[1], off));
+  }
+  bool need = false;
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+    need |= mb[h] > acc.m[h] + kRescaleLog2<KVT> || (acc.m[h] == -INFINITY && mb[h] > -INFINITY);
+  if (__any_sync(0xffffffffu, need)) {
+    float al[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float m_new = fmaxf(acc.m[h], mb[h]);
+      al[h] = m_new == -INFINITY ? 1.f : fast_exp2(acc.m[h] - m_new);
+      acc.m[h] = m_new;
+      acc.l[h] *= al[h];
+      acc.z[h] *= al[h];
+    }
+#pragma unroll
+    for (int j = 0; j < T::kMTiles; ++j) {
+      acc.o[j][0] *= al[0];
+      acc.o[j][1] *= al[1];
+      acc.o[j][2] *= al[0];
+      acc.o[j][3] *= al[1];
+    }
+  }
+  const float mr[2] = {acc.m[0] == -INFINITY ? 0.f : acc.m[0],
+                       acc.m[1] == -INFINITY ? 0.f : acc.m[1]};
+  float p[2][4], w[2][4];  // softmax weights, raw V weights p_t s_t
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      p[u][e] = fast_exp2(x[u][e] - mr[e & 1]);
+      w[u][e] = p[u][e] * vs[u][e >> 1];
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    acc.l[h] += (p[0][h] + p[0][2 + h]) + (p[1][h] + p[1][2 + h]);
+    acc.z[h] += fmaf(p[0][h], vz[0][0], p[0][2 + h] * vz[0][1]) +
+                fmaf(p[1][h], vz[1][0], p[1][2 + h] * vz[1][1]);
+  }
+
+  // ---- the weights' power of two -------------------------------------------
+  float wm[2] = {fmaxf(fmaxf(w[0][0], w[0][2]), fmaxf(w[1][0], w[1][2])),
+                 fmaxf(fmaxf(w[0][1], w[0][3]), fmaxf(w[1][1], w[1][3]))};
+  bool big = false;
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+    big |= wm[h] * acc.f[h] > kWeightHi || (acc.f[h] == 0.f && wm[h] > 0.f);
+  if (__any_sync(0xffffffffu, big)) {
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      wm[0] = fmaxf(wm[0], __shfl_xor_sync(0xffffffffu, wm[0], off));
+      wm[1] = fmaxf(wm[1], __shfl_xor_sync(0xffffffffu, wm[1], off));
+    }
+    float sc[2] = {1.f, 1.f};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      if (wm[h] > 0.f) {
+        const int en = min(max(ilog2f(wm[h]) - kWeightTopExp, kEMin), kEMax);
+        if (acc.f[h] == 0.f || en > acc.e[h]) {
+          // a head without weights so far has O = 0: nothing to rescale
+          if (acc.f[h] != 0.f) sc[h] = exp2i(acc.e[h] - en);
+          acc.e[h] = en;
+          acc.f[h] = exp2i(-en);
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < T::kMTiles; ++j) {
+      acc.o[j][0] *= sc[0];
+      acc.o[j][1] *= sc[1];
+      acc.o[j][2] *= sc[0];
+      acc.o[j][3] *= sc[1];
+    }
+  }
+
+  // ---- O^T += V^T W^T, W^T = the scaled weights transposed -------------------
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    uint32_t h0, l0, h1, l1;
+    split_f16(w[u][0] * acc.f[0], w[u][1] * acc.f[1], h0, l0);  // token g
+    split_f16(w[u][2] * acc.f[0], w[u][3] * acc.f[1], h1, l1);  // token g + 8
+    pv_quant<D, KVT>(lm, src + u * T::kStageBytes, g, movmatrix_trans(h0),
+                     movmatrix_trans(h1), movmatrix_trans(l0), movmatrix_trans(l1), acc.o);
+  }
+}
 
 // Fused cache write: store the K/V row of KV head h of sequence b's newest
 // token (bf16 k_new / v_new [B][Hkv][D]) into pool row `row`, as pa_kv_append
@@ -639,19 +795,16 @@ __device__ __forceinline__ void append_new_row(const DecodeArgs &a, int b, int h
       const int lane = threadIdx.x;
       float *ksz = const_cast<float *>(a.k_sz) + row * 2;
       float *vsz = const_cast<float *>(a.v_sz) + row * 2;
-      float sk, sv;
       if constexpr (KVT == PA_KV_U4_PER_TOKEN) {
-        sk = quantise_row_u4<D>(a.k_new + src, kp + row * (D / 2), ksz, lane);
-        sv = quantise_row_u4<D>(a.v_new + src, vp + row * (D / 2), vsz, lane);
+        quantise_row_u4<D>(a.k_new + src, kp + row * (D / 2), ksz, lane);
+        quantise_row_u4<D>(a.v_new + src, vp + row * (D / 2), vsz, lane);
       } else if constexpr (KVT == PA_KV_FP8_PER_TOKEN) {
-        sk = quantise_row_fp8<D>(a.k_new + src, kp + row * D, ksz, lane);
-        sv = quantise_row_fp8<D>(a.v_new + src, vp + row * D, vsz, lane);
+        quantise_row_fp8<D>(a.k_new + src, kp + row * D, ksz, lane);
+        quantise_row_fp8<D>(a.v_new + src, vp + row * D, vsz, lane);
       } else {
-        sk = quantise_row<D>(a.k_new + src, kp + row * D, ksz, lane);
-        sv = quantise_row<D>(a.v_new + src, vp + row * D, vsz, lane);
+        quantise_row<D>(a.k_new + src, kp + row * D, ksz, lane);
+        quantise_row<D>(a.v_new + src, vp + row * D, vsz, lane);
       }
-      if (lane == 0 && !(fmaxf(sk, sv) < (float)PA_MAX_KV_SCALE))
-        flag_error(a.d_err, PA_DERR_BIG_SCALE);
     }
   }
 }
@@ -804,55 +957,144 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
                         lane);
   };
 
-  WarpAcc<D, KVT> acc;
-  acc.reset();
+  // Each warp leaves a record in its ring: the running max m and denominator
+  // l of every head, and O already divided by l; the CTA merges the records.
+  float *rec = reinterpret_cast<float *>(smem + warp * SM::kRingBytesPerWarp);
+  float *rec_o = rec + 16;
 
+  if constexpr (KVT == PA_KV_BF16) {
+    WarpAcc<D> acc;
+    acc.reset();
 #pragma unroll
-  for (int st = 0; st < NSTAGE - 1; ++st) {
-    if (st < nmine) issue(warp + st * W, st);
-    cp_async_commit();
-  }
-
-  for (int k = 0; k < nmine; ++k) {
-    __syncwarp();
-    {
-      const int kn = k + NSTAGE - 1;
-      if (kn < nmine) issue(warp + kn * W, kn % NSTAGE);
+    for (int st = 0; st < NSTAGE - 1; ++st) {
+      if (st < nmine) issue(warp + st * W, st);
       cp_async_commit();
     }
-    cp_async_wait<NSTAGE - 1>();
-    __syncwarp();  // every lane's pieces of this block are now visible to the warp
+    for (int k = 0; k < nmine; ++k) {
+      __syncwarp();
+      {
+        const int kn = k + NSTAGE - 1;
+        if (kn < nmine) issue(warp + kn * W, kn % NSTAGE);
+        cp_async_commit();
+      }
+      cp_async_wait<NSTAGE - 1>();
+      __syncwarp();  // every lane's pieces of this block are now visible to the warp
 
-    const int kb = warp + k * W;
-    const int btok = tok0 + kb * 16;
-    const bool pvalid = tbl[btok / P - lp0] >= 0;
-    const uint32_t src = ring + (k % NSTAGE) * T::kStageBytes;
-    block_step<D, KVT>(lm, src, btok, tok_lo, tok1, pvalid, a.scale_log2, qa, qsum, g, t, acc);
-  }
-  cp_async_wait<0>();
-  __syncwarp();
-  finish_acc<D, KVT>(acc, t);
-  const float(&o)[T::kMTiles][4] = acc.o;
-  const float m_run = acc.m_run;
-  const float l_run = acc.l_run;
-
-  // ---- merge the CTA's warps (fixed order: deterministic) --------------------
-  float *rec = reinterpret_cast<float *>(smem + warp * SM::kRingBytesPerWarp);
-  if (t == 0) {
-    rec[g] = m_run;
-    rec[8 + g] = l_run;
-  }
-  {
-    float *O = rec + 16;
+      const int kb = warp + k * W;
+      const int btok = tok0 + kb * 16;
+      const bool pvalid = tbl[btok / P - lp0] >= 0;
+      const uint32_t src = ring + (k % NSTAGE) * T::kStageBytes;
+      block_step<D>(lm, src, btok, tok_lo, tok1, pvalid, a.scale_log2, qa, t, acc);
+    }
+    cp_async_wait<0>();
+    __syncwarp();
+    // lane (g, t) ends with head g's max and its share of head g's
+    // denominator, and O^T columns of heads 2t, 2t + 1
+    float l_run = acc.l_run;
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+    const float inv0 = __shfl_sync(0xffffffffu, inv, 8 * t);      // head 2t
+    const float inv1 = __shfl_sync(0xffffffffu, inv, 8 * t + 4);  // head 2t + 1
+    if (t == 0) {
+      rec[g] = acc.m_run;
+      rec[8 + g] = l_run;
+    }
 #pragma unroll
     for (int j = 0; j < T::kMTiles; ++j) {
       const int d0 = out_col<D, KVT>(j, g);
-      *reinterpret_cast<float2 *>(O + (2 * t) * D + d0) = make_float2(o[j][0], o[j][2]);
-      *reinterpret_cast<float2 *>(O + (2 * t + 1) * D + d0) = make_float2(o[j][1], o[j][3]);
+      *reinterpret_cast<float2 *>(rec_o + (2 * t) * D + d0) =
+          make_float2(acc.o[j][0] * inv0, acc.o[j][2] * inv0);
+      *reinterpret_cast<float2 *>(rec_o + (2 * t + 1) * D + d0) =
+          make_float2(acc.o[j][1] * inv1, acc.o[j][3] * inv1);
+    }
+  } else {
+    // two 16-token blocks per step: pair k of this warp is blocks 2 kp and
+    // 2 kp + 1, kp = warp + k W; a ring stage holds one pair
+    constexpr int NPS = NSTAGE / 2;
+    static_assert(NSTAGE % 2 == 0 && NPS >= 2, "quantised pools stage pairs of blocks");
+    const int npair = (nblk + 1) / 2;
+    const int npmine = npair > warp ? (npair - warp + W - 1) / W : 0;
+    auto issue_pair = [&](int kp, int st) {
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int kb = 2 * kp + u;
+        if (kb < nblk) {
+          issue(kb, 2 * st + u);
+        } else {  // no such block: zero-fill the stage (codes and scales 0)
+          issue_block<D, KVT>(lm, ring + (2 * st + u) * T::kStageBytes, kbase, vbase, sz_base,
+                              (size_t)h * P, 16, 0, lane);
+        }
+      }
+    };
+    QAcc<D> acc;
+    acc.reset();
+    // sums of q of heads 2t, 2t + 1 (held by lanes 8t and 8t + 4)
+    const float qz[2] = {__shfl_sync(0xffffffffu, qsum, 8 * t) * a.scale_log2,
+                         __shfl_sync(0xffffffffu, qsum, 8 * t + 4) * a.scale_log2};
+    const float kscale = kCodeScale<KVT> * a.scale_log2;
+#pragma unroll
+    for (int st = 0; st < NPS - 1; ++st) {
+      if (st < npmine) issue_pair(warp + st * W, st);
+      cp_async_commit();
+    }
+    for (int k = 0; k < npmine; ++k) {
+      __syncwarp();
+      {
+        const int kn = k + NPS - 1;
+        if (kn < npmine) issue_pair(warp + kn * W, kn % NPS);
+        cp_async_commit();
+      }
+      cp_async_wait<NPS - 1>();
+      __syncwarp();
+
+      const int kb = 2 * (warp + k * W);
+      const int btok[2] = {tok0 + kb * 16, tok0 + kb * 16 + 16};
+      const bool pvalid[2] = {tbl[btok[0] / P - lp0] >= 0,
+                              kb + 1 < nblk && tbl[btok[1] / P - lp0] >= 0};
+      const uint32_t src = ring + (k % NPS) * 2 * T::kStageBytes;
+      pair_step<D, KVT>(lm, src, btok, pvalid, tok_lo, tok1, kscale, qz, qa, g, acc);
+    }
+    cp_async_wait<0>();
+    __syncwarp();
+    // reduce the two heads' denominators and zero-point sums over the lanes
+    // holding their tokens, then O = (code scale * 2^E * O + sum p z) / l
+    // (the code scale is applied to O first: code scale x 2^E alone may pass
+    // the fp32 range when E is large)
+    constexpr float kRowHiScale = T::kU4 ? kCodeScale<KVT> / 16.f : kCodeScale<KVT>;
+    float pe[2], zl[2];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        acc.l[hh] += __shfl_xor_sync(0xffffffffu, acc.l[hh], off);
+        acc.z[hh] += __shfl_xor_sync(0xffffffffu, acc.z[hh], off);
+      }
+      const float inv = acc.l[hh] > 0.f ? 1.f / acc.l[hh] : 0.f;
+      pe[hh] = acc.f[hh] == 0.f ? 0.f : exp2i(acc.e[hh]) * inv;
+      zl[hh] = acc.z[hh] * inv;
+    }
+    if (g == 0) {
+      rec[2 * t] = acc.m[0];
+      rec[2 * t + 1] = acc.m[1];
+      rec[8 + 2 * t] = acc.l[0];
+      rec[8 + 2 * t + 1] = acc.l[1];
+    }
+#pragma unroll
+    for (int j = 0; j < T::kMTiles; ++j) {
+      const int d0 = out_col<D, KVT>(j, g);
+      // rows d + 1 of INT4 tiles hold the high nibbles (16x the code scale)
+      *reinterpret_cast<float2 *>(rec_o + (2 * t) * D + d0) =
+          make_float2(fmaf(acc.o[j][0] * kCodeScale<KVT>, pe[0], zl[0]),
+                      fmaf(acc.o[j][2] * kRowHiScale, pe[0], zl[0]));
+      *reinterpret_cast<float2 *>(rec_o + (2 * t + 1) * D + d0) =
+          make_float2(fmaf(acc.o[j][1] * kCodeScale<KVT>, pe[1], zl[1]),
+                      fmaf(acc.o[j][3] * kRowHiScale, pe[1], zl[1]));
     }
   }
   __syncthreads();
 
+  // ---- merge the CTA's warps (fixed order: deterministic) --------------------
   for (int e = threadIdx.x; e < G * D; e += W * 32) {
     const int hd = e / D;
     const int d = e - hd * D;
@@ -865,9 +1107,9 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
 #pragma unroll
       for (int w = 0; w < W; ++w) {
         const float *r = reinterpret_cast<const float *>(smem + w * SM::kRingBytesPerWarp);
-        const float f = fast_exp2(r[hd] - M);  // exp2(-inf) = 0 for empty warps
-        num = fmaf(f, r[16 + hd * D + d], num);
-        L = fmaf(f, r[8 + hd], L);
+        const float fl = fast_exp2(r[hd] - M) * r[8 + hd];  // 0 for empty warps
+        num = fmaf(fl, r[16 + hd * D + d], num);
+        L += fl;
       }
     }
     const size_t row = (size_t)b * a.hq + (size_t)h * G + hd;

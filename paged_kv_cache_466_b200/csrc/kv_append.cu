@@ -95,26 +95,22 @@ __global__ void append_u8_kernel(const AppendArgs a) {
     row = __shfl_sync(0xffffffffu, row, 0);
     if (row < 0) continue;
     const size_t src = (size_t)r * D * 2;
-    float sk, sv;
     if constexpr (kFmt == PA_KV_U4_PER_TOKEN) {
-      sk = quantise_row_u4<D>(a.k_new + src, a.k_pool + (size_t)row * (D / 2),
+      quantise_row_u4<D>(a.k_new + src, a.k_pool + (size_t)row * (D / 2),
                               a.k_sz + (size_t)row * 2, lane);
-      sv = quantise_row_u4<D>(a.v_new + src, a.v_pool + (size_t)row * (D / 2),
+      quantise_row_u4<D>(a.v_new + src, a.v_pool + (size_t)row * (D / 2),
                               a.v_sz + (size_t)row * 2, lane);
     } else if constexpr (kFmt == PA_KV_FP8_PER_TOKEN) {
-      sk = quantise_row_fp8<D>(a.k_new + src, a.k_pool + (size_t)row * D,
+      quantise_row_fp8<D>(a.k_new + src, a.k_pool + (size_t)row * D,
                                a.k_sz + (size_t)row * 2, lane);
-      sv = quantise_row_fp8<D>(a.v_new + src, a.v_pool + (size_t)row * D,
+      quantise_row_fp8<D>(a.v_new + src, a.v_pool + (size_t)row * D,
                                a.v_sz + (size_t)row * 2, lane);
     } else {
-      sk = quantise_row<D>(a.k_new + src, a.k_pool + (size_t)row * D, a.k_sz + (size_t)row * 2,
+      quantise_row<D>(a.k_new + src, a.k_pool + (size_t)row * D, a.k_sz + (size_t)row * 2,
                            lane);
-      sv = quantise_row<D>(a.v_new + src, a.v_pool + (size_t)row * D, a.v_sz + (size_t)row * 2,
+      quantise_row<D>(a.v_new + src, a.v_pool + (size_t)row * D, a.v_sz + (size_t)row * 2,
                            lane);
     }
-    // the row is stored either way; decode needs scales below PA_MAX_KV_SCALE
-    if (lane == 0 && !(fmaxf(sk, sv) < (float)PA_MAX_KV_SCALE))
-      flag_error(a.d_err, PA_DERR_BIG_SCALE);
   }
 }
 

@@ -87,6 +87,15 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t &r0, uint3
                : "r"(addr));
 }
 
+// Transpose of an 8x8 matrix of 16-bit elements held in the mma fragment layout
+// (lane l holds row l / 4, columns 2 (l % 4) and 2 (l % 4) + 1): afterwards
+// lane l holds the same positions of the transposed matrix.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(d) : "r"(a));
+  return d;
+}
+
 // ------------------------------------------------------------ tensor cores
 // D = A(16x16, row) * B(16x8, col) + D, fp32 accumulators.
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0,

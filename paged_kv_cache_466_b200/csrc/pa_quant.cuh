@@ -3,8 +3,7 @@
 // variants). One warp quantises one (token, KV head) row of D bf16 values:
 // lane l holds elements [l * D / 32, (l + 1) * D / 32). Every step is an IEEE
 // fp32 operation in a fixed order (explicit _rn intrinsics, no contraction),
-// so every kernel that includes this header stores the same bits. Each
-// returns the row's scale s.
+// so every kernel that includes this header stores the same bits.
 #pragma once
 
 #include "pa_device.cuh"
@@ -13,7 +12,7 @@ namespace pa {
 namespace {
 
 template <int D>
-__device__ __forceinline__ float quantise_row(const unsigned char *src_row, unsigned char *dst_codes,
+__device__ __forceinline__ void quantise_row(const unsigned char *src_row, unsigned char *dst_codes,
                                              float *dst_sz, int lane) {
   constexpr int E = D / 32;  // elements per lane
   const __nv_bfloat16 *x16 = reinterpret_cast<const __nv_bfloat16 *>(src_row) + lane * E;
@@ -50,14 +49,13 @@ __device__ __forceinline__ float quantise_row(const unsigned char *src_row, unsi
     *reinterpret_cast<uint16_t *>(dst_codes + lane * 2) = static_cast<uint16_t>(packed);
   }
   if (lane == 0) *reinterpret_cast<float2 *>(dst_sz) = make_float2(s, z);
-  return s;
 }
 
 // FP8 (E4M3) per-token quantiser: s = max|x| / 448 (IEEE fp32), code =
 // E4M3(x / s) rounded to nearest even and saturated; an all-zero row stores
 // s = 0 and codes 0. The zero point is stored as 0.
 template <int D>
-__device__ __forceinline__ float quantise_row_fp8(const unsigned char *src_row,
+__device__ __forceinline__ void quantise_row_fp8(const unsigned char *src_row,
                                                  unsigned char *dst_codes, float *dst_sz,
                                                  int lane) {
   constexpr int E = D / 32;  // elements per lane (even)
@@ -83,13 +81,12 @@ __device__ __forceinline__ float quantise_row_fp8(const unsigned char *src_row,
     *reinterpret_cast<uint16_t *>(dst_codes + lane * 2) = static_cast<uint16_t>(packed);
   }
   if (lane == 0) *reinterpret_cast<float2 *>(dst_sz) = make_float2(s, 0.f);
-  return s;
 }
 
 // INT4: Eq. 3 with 16 levels, the INT8 arithmetic with 15 in place of 255;
 // element 2i goes to the low nibble of byte i.
 template <int D>
-__device__ __forceinline__ float quantise_row_u4(const unsigned char *src_row,
+__device__ __forceinline__ void quantise_row_u4(const unsigned char *src_row,
                                                 unsigned char *dst_codes, float *dst_sz,
                                                 int lane) {
   constexpr int E = D / 32;  // elements per lane (even)
@@ -127,7 +124,6 @@ __device__ __forceinline__ float quantise_row_u4(const unsigned char *src_row,
     dst_codes[lane] = static_cast<unsigned char>(packed);
   }
   if (lane == 0) *reinterpret_cast<float2 *>(dst_sz) = make_float2(s, z);
-  return s;
 }
 
 }  // namespace

@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.pa_abi_version() == 1
+    assert lib.pa_abi_version() == 2
     for s in range(7):
         assert lib.pa_status_str(s) and lib.pa_status_str(s) != b"unknown status"
     assert lib.pa_status_str(99) == b"unknown status"
@@ -126,16 +126,16 @@ def test_split_planning_and_workspace_size(lib):
 def test_device_error_words_map_to_statuses(lib):
     from paged_kv_cache_466_b200._lib import (PA_DERR_BAD_CTX, PA_DERR_BAD_PAGE,
                                               PA_DERR_BAD_POS, PA_DERR_BAD_SEQ,
-                                              PA_DERR_BIG_SCALE, PA_DERR_TIMEOUT,
-                                              PA_ERR_BAD_TABLE, PA_ERR_TIMEOUT)
+                                              PA_DERR_TIMEOUT, PA_ERR_BAD_TABLE,
+                                              PA_ERR_TIMEOUT)
     assert lib.pa_derr_status(0) == PA_OK
     for bit in (PA_DERR_BAD_PAGE, PA_DERR_BAD_CTX, PA_DERR_BAD_SEQ, PA_DERR_BAD_POS):
         assert lib.pa_derr_status(bit) == PA_ERR_BAD_TABLE
-        assert lib.pa_derr_status(bit | PA_DERR_BIG_SCALE) == PA_ERR_BAD_TABLE
+        assert lib.pa_derr_status(bit | 16) == PA_ERR_BAD_TABLE
         assert lib.pa_derr_status(bit | PA_DERR_TIMEOUT) == PA_ERR_TIMEOUT
-    assert lib.pa_derr_status(PA_DERR_BIG_SCALE) == PA_ERR_UNSUPPORTED
     assert lib.pa_derr_status(PA_DERR_TIMEOUT) == PA_ERR_TIMEOUT
-    assert lib.pa_derr_status(64) == PA_ERR_INVALID_ARG
+    for bit in (16, 64):      # bits no kernel sets
+        assert lib.pa_derr_status(bit) == PA_ERR_INVALID_ARG
 
 
 def test_auto_splits_and_step_host_reject_bad_arguments(lib):

@@ -5,7 +5,7 @@ import pytest
 import torch
 
 from paged_kv_cache_466_b200 import (PA_DERR_BAD_PAGE, PA_DERR_BAD_POS, PA_DERR_BAD_SEQ,
-                                     PA_DERR_BIG_SCALE, PA_MAX_KV_SCALE, KVPool, pa_kv_append)
+                                     KVPool, pa_kv_append)
 from paged_kv_cache_466_b200 import workloads as W
 from tests.helpers import DEV, device_append, device_inputs, oracle_pool, pool_bytes_equal
 
@@ -151,12 +151,12 @@ def test_append_empty_is_noop():
     assert torch.all(pool.k.view(torch.uint8) == 0x22)
 
 
-@pytest.mark.parametrize("kind,span,flagged", [
-    ("u4", 8e4, True), ("u4", 6e4, False), ("u8", 8e4, False), ("fp8", 8e4, False),
-    ("u8", 1.2e6, True)])
-def test_append_flags_scales_the_decode_cannot_take(kind, span, flagged):
-    """A row whose scale is not below PA_MAX_KV_SCALE is still stored (bit-exact
-    with the oracle) and flagged with PA_DERR_BIG_SCALE; smaller ones are not."""
+@pytest.mark.parametrize("kind", ["u4", "u8", "fp8"])
+@pytest.mark.parametrize("span", [8e4, 1.2e6, 1e30, 1e-30])
+def test_append_stores_rows_of_any_scale(kind, span):
+    """Rows with very large and very small spans are stored bit-exact with the
+    oracle's quantiser, and the error word stays clear (no row scale is out of
+    range for the decode)."""
     D, Hkv = 128, 2
     x = torch.linspace(-span / 2, span / 2, D).to(torch.bfloat16)
     k = torch.zeros(3, Hkv, D, dtype=torch.bfloat16)
@@ -168,7 +168,6 @@ def test_append_flags_scales_the_decode_cannot_take(kind, span, flagged):
     err = torch.zeros(1, dtype=torch.int32, device=DEV)
     device_append(pool, w, bt, d_err=err)
     torch.cuda.synchronize()
-    assert bool(int(err.item()) & PA_DERR_BIG_SCALE) == flagged
+    assert int(err.item()) == 0
     ok, msg = pool_bytes_equal(pool, oracle_pool(w))
     assert ok, msg
-    assert PA_MAX_KV_SCALE == 4096

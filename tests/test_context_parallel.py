@@ -107,3 +107,37 @@ def test_merge_partials_against_the_oracle_merge():
     fin = np.isfinite(m)
     wl = np.log(np.sum(np.exp(lse.double().numpy()[:, fin] - m[fin]), axis=0)) + m[fin]
     assert np.abs(lo.cpu().numpy()[fin] - wl).max() <= 1e-5
+
+
+@pytest.mark.parametrize("world", [1, 2, 3])
+def test_bench_shards_decoded_per_rank_merge_to_the_oracle(world):
+    """The bench's context-parallel layout on one GPU: every emulated rank
+    gets its own pool and tables from bench.cp_shard_rows, decodes its token
+    range, and the packed partials merge to Eq. 1 over the whole contexts.
+    With one rank decode_context_parallel itself runs (no process group)."""
+    import bench
+    from paged_kv_cache_466_b200 import KVPool, pa_kv_append
+    from paged_kv_cache_466_b200.context_parallel import decode_context_parallel
+    w = W.llama8b(B=5, ctx_range=(1, 1500), seed=11)
+    ref, _ = oracle.paged_attention(oracle_pool(w), bits(w.q), w.block_tables, w.context_lens,
+                                    w.scale)
+    q = w.q.to(DEV)
+    ctx = torch.from_numpy(w.context_lens).to(DEV)
+    n = partial_block_floats(w.B, w.Hq, w.D)
+    gathered = torch.full((world * n,), float("nan"), device=DEV)
+    for r in range(world):
+        T, (b, e), tables, n_pages, (seq, pos, k, v) = bench.cp_shard_rows(w, r, world)
+        pool = KVPool(n_pages, w.Hkv, w.P, w.D, w.kv, DEV, fill_byte=0xFF)
+        bt = torch.from_numpy(tables).to(DEV)
+        pa_kv_append(pool, k.to(DEV), v.to(DEV), torch.from_numpy(seq).to(DEV),
+                     torch.from_numpy(pos).to(DEV), bt)
+        if world == 1:
+            out = decode_context_parallel(pool, q, bt, ctx, w.scale, T)
+            break
+        o, lse = partial_views(gathered[r * n:(r + 1) * n], w.B, w.Hq, w.D)
+        pa_decode_range(pool, q, bt, ctx, w.scale, b, e, o_out=o, lse_out=lse)
+    if world > 1:
+        o_parts, l_parts = gathered_views(gathered, world, w.B, w.Hq, w.D)
+        out, _ = pa_merge_partials(o_parts, l_parts)
+    torch.cuda.synchronize()
+    assert np.abs(out.cpu().numpy().reshape(-1, w.D) - ref).max() <= TOL

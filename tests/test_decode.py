@@ -84,22 +84,27 @@ def test_one_token_context_is_exact():
 
 
 @pytest.mark.parametrize("kind", ["u4", "u8", "fp8"])
-def test_quantised_scales_near_the_bound(kind):
-    """V rows spanning up to the largest allowed scale (just below
-    PA_MAX_KV_SCALE for INT4): the f16 operands must not overflow. The
-    tolerance is relative to the value range (fp32 accumulation of terms up
-    to ~1e5)."""
-    span = {"u4": 6.0e4, "u8": 1.0e6, "fp8": 1.6e6}[kind]
+@pytest.mark.parametrize("span", [6.0e4, 1.0e6, 1e12, 1e30, 1e-12, 1e-30])
+@pytest.mark.parametrize("which", ["v", "kv"])
+def test_quantised_rows_of_any_span(kind, span, which):
+    """Eq. 3 puts no bound on a row's scale. V rows (and K rows) drawn
+    uniformly over a span from 1e-30 to 1e30: the weights' power-of-two
+    normalisation keeps every f16 operand in range and at full precision. The
+    tolerance is relative to the span (fp32 accumulation, weights carried to
+    ~2^-22); with large K spans the softmax is one-hot in both."""
     w = W.paged("bigv", B=3, Hq=8, Hkv=2, D=128, P=16, context_lens=[300, 37, 1], kv=kind)
     g = torch.Generator().manual_seed(5)
     big = lambda t: ((torch.rand(t.shape, generator=g) - 0.5) * span).to(torch.bfloat16)
     w.prefill_v, w.step_v = big(w.prefill_v), big(w.step_v)
+    if which == "kv":
+        w.prefill_k, w.step_k = big(w.prefill_k), big(w.step_k)
+    ref, _ = oracle_decode(w, oracle_pool(w))
     for S in (1, 3):
         got, _ = _run(w, num_splits=S)
-        ref, _ = oracle_decode(w, oracle_pool(w))
         assert np.all(np.isfinite(got))
         err = np.abs(got.astype(np.float64) - ref).max()
-        print(f"{kind}: max |gpu - oracle| = {err:.3e} on outputs up to {np.abs(ref).max():.3e}")
+        print(f"{kind} {which} span {span:.0e}: max |gpu - oracle| = {err:.3e} "
+              f"on outputs up to {np.abs(ref).max():.3e}")
         assert err <= 2e-6 * span
 
 

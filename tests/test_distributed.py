@@ -203,3 +203,74 @@ def test_decode_context_parallel_orchestration_on_gloo():
     assert [r[1] for r in res] == [[(0, 64)], [(64, 128)], [(128, 0x7FFFFFFF)]]
     for _, _, err in res:
         assert err <= 1e-6
+
+
+def _cp_bench_worker(rank, world, port, q):
+    """The bench's context-parallel mode on gloo ranks: each rank builds its
+    own pool from bench.cp_shard_rows (its token range of the same seeded
+    batch, its own page ids) and runs decode_context_parallel with the oracle
+    standing in for the two library calls."""
+    import types
+    import oracle
+    from paged_kv_cache_466_b200 import context_parallel as cp
+    from paged_kv_cache_466_b200 import workloads as W
+    from paged_kv_cache_466_b200.workloads import bits
+    from tests.helpers import oracle_pool
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = W.paged("cpbench", B=5, Hq=8, Hkv=2, D=64, P=16, ctx_range=(1, 300), kv="bf16",
+                    seed=3)
+        T, (begin, end), tables, n_pages, (seq, pos, k, v) = bench.cp_shard_rows(w, rank, world)
+        hp = oracle.empty_pool(w.kv, n_pages, w.Hkv, w.P, w.D, 0xFF)   # NaN-ish filler
+        oracle.scatter_rows(hp, tables, seq, pos, bits(k), bits(v))
+
+        def fake_range(pool, qq, bt, ctx, scale, b, e, o_out=None, lse_out=None, **kw):
+            o, l = oracle.paged_attention(pool.hp, bits(qq), bt.numpy(), ctx.numpy(), scale,
+                                          t_begin=b, t_end=e if e < 0x7FFFFFFF else -1)
+            o_out.copy_(torch.from_numpy(o).view(o_out.shape))
+            lse_out.copy_(torch.from_numpy(l).view(lse_out.shape))
+            return o_out, lse_out
+
+        def fake_merge(o_parts, lse_parts, out=None, lse_out=None, stream=None):
+            n, D = o_parts.shape[0], o_parts.shape[-1]
+            m = oracle.lse_merge(o_parts.double().numpy().reshape(n, -1, D).transpose(1, 0, 2),
+                                 lse_parts.double().numpy().reshape(n, -1).T)
+            res = torch.from_numpy(m).float().view(o_parts.shape[1:])
+            out.copy_(res)
+            return out, None
+
+        cp.pa_decode_range, cp.pa_merge_partials = fake_range, fake_merge
+        pool = types.SimpleNamespace(page_size=w.P, hp=hp)
+        out = torch.empty((w.B, w.Hq, w.D))
+        cp.decode_context_parallel(pool, w.q, torch.from_numpy(tables),
+                                   torch.from_numpy(w.context_lens), w.scale, T, out=out)
+        full, _ = oracle.paged_attention(oracle_pool(w), bits(w.q), w.block_tables,
+                                         w.context_lens, w.scale)
+        err = float(np.abs(out.double().numpy().reshape(-1, w.D) - full).max())
+        own = int(sum(max(0, min(int(c), end) - begin) for c in w.context_lens))
+        q.put((rank, T, len(seq), own, n_pages, err))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_bench_context_parallel_shards_merge_to_the_full_decode(world):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_cp_bench_worker, args=(r, world, port, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=180) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    from paged_kv_cache_466_b200 import workloads as W
+    w = W.paged("cpbench", B=5, Hq=8, Hkv=2, D=64, P=16, ctx_range=(1, 300), kv="bf16", seed=3)
+    assert sum(r[2] for r in res) == w.total_tokens       # every row on exactly one rank
+    for _, T, nrows, own, n_pages, err in res:
+        assert T % w.P == 0 and nrows == own
+        assert n_pages >= -(-own // w.P)
+        assert err <= 1e-6
