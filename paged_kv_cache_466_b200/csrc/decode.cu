@@ -329,6 +329,18 @@ __device__ __forceinline__ void issue_block(const LaneMap<D, KVT> &lm, uint32_t 
   using T = Tile<D, KVT>;
   const unsigned char *ksrc = kbase + row0 * T::kRowBytes + lane * 16;
   const unsigned char *vsrc = vbase + row0 * T::kRowBytes + lane * 16;
+  if (rlo == 0 && rhi == 16) {  // warp-uniform: the whole block is read
+#pragma unroll
+    for (int j = 0; j < T::kCopies; ++j) {
+      cp_async16(dst + lm.cp_soff[j], ksrc + j * 512, 16u);
+      cp_async16(dst + T::kVOff + lm.cp_soff[j], vsrc + j * 512, 16u);
+    }
+    if constexpr (T::kU8) {
+      // lanes 0..7: K (scale, zero) of rows 2l, 2l+1; lanes 8..15: V
+      if (lane < 16) cp_async16(dst + lm.sz_dst, sz_base + (row0 + 2 * (lane & 7)) * 2, 16u);
+    }
+    return;
+  }
 #pragma unroll
   for (int j = 0; j < T::kCopies; ++j) {
     const uint32_t n = (lm.cp_row[j] >= rlo && lm.cp_row[j] < rhi) ? 16u : 0u;
@@ -336,7 +348,6 @@ __device__ __forceinline__ void issue_block(const LaneMap<D, KVT> &lm, uint32_t 
     cp_async16(dst + T::kVOff + lm.cp_soff[j], vsrc + j * 512, n);
   }
   if constexpr (T::kU8) {
-    // lanes 0..7: K (scale, zero) of rows 2l, 2l+1; lanes 8..15: V
     if (lane < 16) {
       // (a row outside [rlo, rhi) may come along with its neighbour; the
       // consumer zeroes scale and zero of every masked token)
@@ -1094,31 +1105,39 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
   }
   __syncthreads();
 
-  // ---- merge the CTA's warps (fixed order: deterministic) --------------------
-  for (int e = threadIdx.x; e < G * D; e += W * 32) {
-    const int hd = e / D;
-    const int d = e - hd * D;
+  // ---- merge the CTA's warps (fixed order: deterministic); a thread takes
+  // four consecutive elements of one head
+  constexpr int D4 = D / 4;
+  for (int e = threadIdx.x; e < G * D4; e += W * 32) {
+    const int hd = e / D4;
+    const int d4 = e - hd * D4;
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < W; ++w)
       M = fmaxf(M, reinterpret_cast<const float *>(smem + w * SM::kRingBytesPerWarp)[hd]);
-    float num = 0.f, L = 0.f;
+    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+    float L = 0.f;
     if (M != -INFINITY) {
 #pragma unroll
       for (int w = 0; w < W; ++w) {
         const float *r = reinterpret_cast<const float *>(smem + w * SM::kRingBytesPerWarp);
         const float fl = fast_exp2(r[hd] - M) * r[8 + hd];  // 0 for empty warps
-        num = fmaf(fl, r[16 + hd * D + d], num);
+        const float4 v = reinterpret_cast<const float4 *>(r + 16 + hd * D)[d4];
+        num.x = fmaf(fl, v.x, num.x);
+        num.y = fmaf(fl, v.y, num.y);
+        num.z = fmaf(fl, v.z, num.z);
+        num.w = fmaf(fl, v.w, num.w);
         L += fl;
       }
     }
     const size_t row = (size_t)b * a.hq + (size_t)h * G + hd;
-    const float val = L > 0.f ? num / L : 0.f;
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    const float4 val = make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
     if (n_live == 1 && a.n_prior == 0 && !a.keep_partials) {
-      a.out[row * D + d] = val;
+      reinterpret_cast<float4 *>(a.out + row * D)[d4] = val;
     } else {
-      a.o_part[(row * a.S + slot) * D + d] = val;
-      if (d == 0) a.lse[row * a.S + slot] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+      reinterpret_cast<float4 *>(a.o_part + (row * a.S + slot) * D)[d4] = val;
+      if (d4 == 0) a.lse[row * a.S + slot] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
     }
   }
   if (a.keep_partials) return;  // the caller merges
