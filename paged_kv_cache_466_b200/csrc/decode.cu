@@ -481,13 +481,17 @@ __device__ __forceinline__ void block_step(const LaneMap<D, PA_KV_BF16> &lm, uin
 // its swizzle and the code unpack are shared with the bf16 path.
 //
 // The V weights p_t * s_t (s_t the row scale of Eq. 3) enter the f16 MMA
-// scaled by a per-head power of two 2^-E, kept like the running max: E is set
-// from the first nonzero weights so that the largest sits at 2^12 .. 2^13, and
-// raised whenever a later weight would pass 2^14, O then being multiplied by
-// the exact power of two. O is thus carried in units of 2^E (fp32) and every
-// weight keeps the f16 precision whatever the row scales are, with no limit
-// on the scale from the f16 range.
+// scaled by a power of two 2^-E kept like the running max: the softmax keeps
+// every p_t <= 2^kRescaleLog2, so the largest V scale seen so far bounds every
+// weight, and E is set from the first nonzero scale so that this bound sits
+// at 2^12 .. 2^13, and raised whenever a larger scale arrives, O then being
+// multiplied by the exact power of two. O is thus carried in units of 2^E
+// (fp32) and the weights stay inside the f16 range whatever the row scales
+// are: no limit on the scale from the f16 range.
 constexpr float kWeightHi = 16384.f;  // largest scaled V weight fed to the MMA (2^14)
+// the largest scaled V scale: weights p s with p <= 2^kRescaleLog2 stay below kWeightHi
+template <int KVT>
+constexpr float kScaleHi = kWeightHi / (1 << (int)kRescaleLog2<KVT>);
 constexpr int kWeightTopExp = 12;     // a new E puts the largest weight at 2^12 .. 2^13
 constexpr int kEMin = -120, kEMax = 120;
 
@@ -506,17 +510,18 @@ struct QAcc {
   float m[2];  // running max of the scores of heads 2t, 2t + 1 (log2 units)
   float l[2];  // this lane's share of their softmax denominators
   float z[2];  // this lane's share of sum_t p_t z_t
-  float f[2];  // 2^-E of each head; 0 until the head's first nonzero weight
-  int e[2];    // E of each head
+  float f;     // 2^-E; 0 until the first nonzero V scale
+  int e;       // E
   __device__ __forceinline__ void reset() {
 #pragma unroll
     for (int j = 0; j < D / 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       m[h] = -INFINITY;
-      l[h] = z[h] = f[h] = 0.f;
-      e[h] = 0;
+      l[h] = z[h] = 0.f;
     }
+    f = 0.f;
+    e = 0;
   }
 };
 
@@ -725,15 +730,11 @@ __device__ __forceinline__ void pair_step(const LaneMap<D, KVT> &lm, uint32_t sr
   }
   const float mr[2] = {acc.m[0] == -INFINITY ? 0.f : acc.m[0],
                        acc.m[1] == -INFINITY ? 0.f : acc.m[1]};
-  float p[2][4], w[2][4];  // softmax weights, raw V weights p_t s_t
+  float p[2][4];  // softmax weights
 #pragma unroll
-  for (int u = 0; u < 2; ++u) {
+  for (int u = 0; u < 2; ++u)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      p[u][e] = fast_exp2(x[u][e] - mr[e & 1]);
-      w[u][e] = p[u][e] * vs[u][e >> 1];
-    }
-  }
+    for (int e = 0; e < 4; ++e) p[u][e] = fast_exp2(x[u][e] - mr[e & 1]);
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     acc.l[h] += (p[0][h] + p[0][2 + h]) + (p[1][h] + p[1][2 + h]);
@@ -742,46 +743,44 @@ __device__ __forceinline__ void pair_step(const LaneMap<D, KVT> &lm, uint32_t sr
   }
 
   // ---- the weights' power of two -------------------------------------------
-  float wm[2] = {fmaxf(fmaxf(w[0][0], w[0][2]), fmaxf(w[1][0], w[1][2])),
-                 fmaxf(fmaxf(w[0][1], w[0][3]), fmaxf(w[1][1], w[1][3]))};
-  bool big = false;
-#pragma unroll
-  for (int h = 0; h < 2; ++h)
-    big |= wm[h] * acc.f[h] > kWeightHi || (acc.f[h] == 0.f && wm[h] > 0.f);
+  // A weight is p s with p <= 2^kRescaleLog2, so the largest V scale seen so
+  // far bounds every weight: E keeps that scale times 2^kRescaleLog2 at
+  // 2^12 .. 2^13 (one E for the warp; it only moves when a larger scale comes)
+  float vm = fmaxf(fmaxf(vs[0][0], vs[0][1]), fmaxf(vs[1][0], vs[1][1]));
+  const bool big = vm * acc.f > kScaleHi<KVT> || (acc.f == 0.f && vm > 0.f);
   if (__any_sync(0xffffffffu, big)) {
 #pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      wm[0] = fmaxf(wm[0], __shfl_xor_sync(0xffffffffu, wm[0], off));
-      wm[1] = fmaxf(wm[1], __shfl_xor_sync(0xffffffffu, wm[1], off));
-    }
-    float sc[2] = {1.f, 1.f};
+    for (int off = 4; off < 32; off <<= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, off));
+    if (vm > 0.f) {
+      const int en = min(max(ilog2f(vm) + (int)kRescaleLog2<KVT> - kWeightTopExp, kEMin), kEMax);
+      if (acc.f == 0.f || en > acc.e) {
+        // with no weight so far O = 0: nothing to rescale
+        const float sc = acc.f == 0.f ? 1.f : exp2i(acc.e - en);
+        acc.e = en;
+        acc.f = exp2i(-en);
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      if (wm[h] > 0.f) {
-        const int en = min(max(ilog2f(wm[h]) - kWeightTopExp, kEMin), kEMax);
-        if (acc.f[h] == 0.f || en > acc.e[h]) {
-          // a head without weights so far has O = 0: nothing to rescale
-          if (acc.f[h] != 0.f) sc[h] = exp2i(acc.e[h] - en);
-          acc.e[h] = en;
-          acc.f[h] = exp2i(-en);
+        for (int j = 0; j < T::kMTiles; ++j) {
+          acc.o[j][0] *= sc;
+          acc.o[j][1] *= sc;
+          acc.o[j][2] *= sc;
+          acc.o[j][3] *= sc;
         }
       }
     }
+  }
+  float vf[2][2];  // V scales times 2^-E
 #pragma unroll
-    for (int j = 0; j < T::kMTiles; ++j) {
-      acc.o[j][0] *= sc[0];
-      acc.o[j][1] *= sc[1];
-      acc.o[j][2] *= sc[0];
-      acc.o[j][3] *= sc[1];
-    }
+  for (int u = 0; u < 2; ++u) {
+    vf[u][0] = vs[u][0] * acc.f;
+    vf[u][1] = vs[u][1] * acc.f;
   }
 
   // ---- O^T += V^T W^T, W^T = the scaled weights transposed -------------------
 #pragma unroll
   for (int u = 0; u < 2; ++u) {
     uint32_t h0, l0, h1, l1;
-    split_f16(w[u][0] * acc.f[0], w[u][1] * acc.f[1], h0, l0);  // token g
-    split_f16(w[u][2] * acc.f[0], w[u][3] * acc.f[1], h1, l1);  // token g + 8
+    split_f16(p[u][0] * vf[u][0], p[u][1] * vf[u][0], h0, l0);  // token g
+    split_f16(p[u][2] * vf[u][1], p[u][3] * vf[u][1], h1, l1);  // token g + 8
     pv_quant<D, KVT>(lm, src + u * T::kStageBytes, g, movmatrix_trans(h0),
                      movmatrix_trans(h1), movmatrix_trans(l0), movmatrix_trans(l1), acc.o);
   }
@@ -849,7 +848,29 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
   // last `window` tokens. With attention sinks the extra split S_main covers
   // [0, min(sinks, ctx)) ("Token Eviction Strategies", Eq. 5); the two ranges
   // are disjoint and together hold exactly the kept tokens.
+  // Loads that do not depend on the context length go out with it: the
+  // query fragments and, where the split's page range does not depend on the
+  // context (no window, a main split), that range's table entries.
   int ctx = a.ctx[b];
+  constexpr int kPre = 2;  // table entries prefetched per thread
+  int pre[kPre];
+  const bool nominal = a.window == 0 && split < a.S_main;
+  {
+    const int lp0n = a.tok_begin / P + split * a.pages_per_split;
+#pragma unroll
+    for (int k = 0; k < kPre; ++k) {
+      const int i = threadIdx.x + k * W * 32;
+      pre[k] = (nominal && i < a.pages_per_split && lp0n + i < a.max_pages)
+                   ? __ldg(a.block_tables + (size_t)b * a.max_pages + lp0n + i)
+                   : -1;
+    }
+  }
+  const bool head_ok = g < G;
+  const size_t q_row = ((size_t)b * a.hq + (size_t)h * G + (head_ok ? g : 0)) * D;
+  const __nv_bfloat16 *qp = reinterpret_cast<const __nv_bfloat16 *>(a.q) + q_row;
+  uint32_t qa[D / 16][2];  // per k-step: a0 (k 2t..2t+1), a2 (k 2t+8..2t+9)
+  const float qsum = load_q<D, KVT>(qp, head_ok, t, qa);
+
   if (ctx < 0 || ctx > a.max_pages * P) {
     if (threadIdx.x == 0) flag_error(a.d_err, PA_DERR_BAD_CTX);
     ctx = a.tok_begin;
@@ -915,21 +936,29 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
   }
 
   // ---- stage this split's block-table entries (bounds-checked) --------------
-  for (int i = threadIdx.x; i < lp1 - lp0; i += W * 32) {
-    int pg = __ldg(a.block_tables + (size_t)b * a.max_pages + lp0 + i);
-    if (pg < 0 || pg >= a.num_pages) {
-      flag_error(a.d_err, PA_DERR_BAD_PAGE);
-      pg = -1;
+  if (nominal && lp1 - lp0 <= kPre * W * 32) {  // CTA-uniform: the prefetch covers them
+#pragma unroll
+    for (int k = 0; k < kPre; ++k) {
+      const int i = threadIdx.x + k * W * 32;
+      if (i < lp1 - lp0) {
+        int pg = pre[k];
+        if (pg < 0 || pg >= a.num_pages) {
+          flag_error(a.d_err, PA_DERR_BAD_PAGE);
+          pg = -1;
+        }
+        tbl[i] = pg;
+      }
     }
-    tbl[i] = pg;
+  } else {
+    for (int i = threadIdx.x; i < lp1 - lp0; i += W * 32) {
+      int pg = __ldg(a.block_tables + (size_t)b * a.max_pages + lp0 + i);
+      if (pg < 0 || pg >= a.num_pages) {
+        flag_error(a.d_err, PA_DERR_BAD_PAGE);
+        pg = -1;
+      }
+      tbl[i] = pg;
+    }
   }
-
-  // ---- query fragments ---------------------------------------------------------
-  const bool head_ok = g < G;
-  const size_t q_row = ((size_t)b * a.hq + (size_t)h * G + (head_ok ? g : 0)) * D;
-  const __nv_bfloat16 *qp = reinterpret_cast<const __nv_bfloat16 *>(a.q) + q_row;
-  uint32_t qa[D / 16][2];  // per k-step: a0 (k 2t..2t+1), a2 (k 2t+8..2t+9)
-  const float qsum = load_q<D, KVT>(qp, head_ok, t, qa);
   __syncthreads();  // tbl visible
 
   // ---- fused cache write: the split whose pages hold the newest token
@@ -1082,7 +1111,7 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
         acc.z[hh] += __shfl_xor_sync(0xffffffffu, acc.z[hh], off);
       }
       const float inv = acc.l[hh] > 0.f ? 1.f / acc.l[hh] : 0.f;
-      pe[hh] = acc.f[hh] == 0.f ? 0.f : exp2i(acc.e[hh]) * inv;
+      pe[hh] = acc.f == 0.f ? 0.f : exp2i(acc.e) * inv;
       zl[hh] = acc.z[hh] * inv;
     }
     if (g == 0) {
