@@ -249,7 +249,7 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(m for m, _ in use) if use else None,
                 "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(timed),
                 "samples_with_warmup": len(every),
-                "sampled": "NVML SM clock and clock-event reasons, read back to back from "
+                "sampled": "NVML SM clock and clock-event reasons, read every ~0.1 ms from "
                            "the start of the warm-up to the end of the timed region; sm_mhz, "
                            "reasons and samples cover the timed region"}
 
