@@ -5,7 +5,8 @@
 // exact identity that lets pa_decode spread one long context over several
 // CTAs; the pages do not describe it, it is the plain algebra of Eq. 1's
 // softmax. One warp merges one (sequence, query head) row; splits are visited
-// in index order, so the result is deterministic.
+// in index order, so the result is deterministic (the order of the sum is
+// fixed, whichever path a row takes).
 #include <cmath>
 
 #include "pa_device.cuh"
@@ -15,6 +16,7 @@ namespace pa {
 namespace {
 
 constexpr int kWarps = 4;
+constexpr int kFast = 16;  // rows of at most this many partials take the one-round path
 
 // Partials i < S are the row's own (o_part[row][i], lse[row][i]); i >= S are
 // prior partials p = i - S (prior_o + p * po_stride + row * D,
@@ -32,10 +34,6 @@ __global__ void __launch_bounds__(kWarps * 32) splitkv_reduce_kernel(
   const int n_all = S + n_prior;
   const float *ls = lse + (size_t)row * S;
   auto lse_at = [&](int i) { return i < S ? ls[i] : prior_lse[(size_t)(i - S) * pl_stride + row]; };
-  float M = -INFINITY;
-  for (int s = lane; s < n_all; s += 32) M = fmaxf(M, lse_at(s));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   const int D4 = D / 4;
   const float4 *op = reinterpret_cast<const float4 *>(o_part + (size_t)row * S * D);
   auto o_at = [&](int i) {
@@ -44,6 +42,47 @@ __global__ void __launch_bounds__(kWarps * 32) splitkv_reduce_kernel(
                                                     (size_t)row * D);
   };
   float4 *dst = reinterpret_cast<float4 *>(out + (size_t)row * D);
+  if (n_all <= kFast && D4 <= 32) {
+    // Every load of the row goes out at once — lane s's log-sum-exp and each
+    // lane's four outputs of every partial — so the merge waits for one round
+    // trip instead of one for the log-sum-exps and more for the partials.
+    const float lv = lane < n_all ? lse_at(lane) : -INFINITY;
+    // (partials past n_all re-read the last one, and lanes past D4 their
+    // row's first chunk: valid addresses whose values get weight 0 / no store)
+    const int li = lane < D4 ? lane : 0;
+    float4 v[kFast];
+#pragma unroll
+    for (int k = 0; k < kFast; ++k) v[k] = o_at(min(k, n_all - 1))[li];
+    float M = lv;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float wl = (lane < n_all && M != -INFINITY) ? expf(lv - M) : 0.f;  // -inf -> 0
+    float den = wl;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < kFast; ++k) {
+      const float w = __shfl_sync(0xffffffffu, wl, k);
+      // a weight-0 (empty) partial is loaded but never used
+      if (k < n_all && w != 0.f) {
+        acc.x = fmaf(w, v[k].x, acc.x);
+        acc.y = fmaf(w, v[k].y, acc.y);
+        acc.z = fmaf(w, v[k].z, acc.z);
+        acc.w = fmaf(w, v[k].w, acc.w);
+      }
+    }
+    if (lane < D4) {
+      const float r = den > 0.f ? 1.f / den : 0.f;
+      dst[lane] = make_float4(acc.x * r, acc.y * r, acc.z * r, acc.w * r);
+    }
+    if (lse_out != nullptr && lane == 0) lse_out[row] = den > 0.f ? M + logf(den) : -INFINITY;
+    return;
+  }
+  float M = -INFINITY;
+  for (int s = lane; s < n_all; s += 32) M = fmaxf(M, lse_at(s));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   for (int i0 = 0; i0 < D4; i0 += 32) {
     const int i = i0 + lane;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
