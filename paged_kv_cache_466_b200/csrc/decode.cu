@@ -46,6 +46,7 @@
 #include <atomic>
 #include <cfloat>
 #include <cmath>
+#include <type_traits>
 
 #include "pa_device.cuh"
 #include "pa_internal.h"
@@ -561,6 +562,8 @@ __device__ __forceinline__ void scores_t(const LaneMap<D, KVT> &lm, uint32_t src
 #pragma unroll
     for (int e = 0; e < 4; ++e) s[e] = fmaf(sh[e], 0.0625f, s[e]);  // high nibbles: 16x
   } else {
+    // two accumulators halve the dependent MMA chain
+    float s2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int i = 0; i < T::kKChunks; ++i) {
       const uint4 k0 = lds128(src + lm.koff[0][i]);  // token g
@@ -575,15 +578,17 @@ __device__ __forceinline__ void scores_t(const LaneMap<D, KVT> &lm, uint32_t src
             kIsFp8<KVT> ? e4m3x2_to_f16x2(w0[w] >> 16) : u8x2_to_f16x2(w0[w], 0x4342);
         const uint32_t a3 =
             kIsFp8<KVT> ? e4m3x2_to_f16x2(w1[w] >> 16) : u8x2_to_f16x2(w1[w], 0x4342);
-        mma_f16_16816(s, a0, a1, a2, a3, qa[4 * i + w][0], qa[4 * i + w][1]);
+        mma_f16_16816((w & 1) ? s2 : s, a0, a1, a2, a3, qa[4 * i + w][0], qa[4 * i + w][1]);
       }
     }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s[e] += s2[e];
   }
 }
 
 // O^T += V^T W^T for the quantised block staged at `src`, with the weights'
 // B fragments (hi and lo halves, tokens 0..7 in b?0 and 8..15 in b?1).
-template <int D, int KVT>
+template <int D, int KVT, bool kTwo = true>
 __device__ __forceinline__ void pv_quant(const LaneMap<D, KVT> &lm, uint32_t src, int g,
                                          uint32_t bh0, uint32_t bh1, uint32_t bl0,
                                          uint32_t bl1, float (&o)[D / 16][4]) {
@@ -620,7 +625,7 @@ __device__ __forceinline__ void pv_quant(const LaneMap<D, KVT> &lm, uint32_t src
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         mma_f16_16816(o[j + u], a0[u], a1[u], a2[u], a3[u], bh0, bh1);
-        mma_f16_16816(o[j + u], a0[u], a1[u], a2[u], a3[u], bl0, bl1);
+        if constexpr (kTwo) mma_f16_16816(o[j + u], a0[u], a1[u], a2[u], a3[u], bl0, bl1);
       }
     }
   } else {
@@ -647,7 +652,7 @@ __device__ __forceinline__ void pv_quant(const LaneMap<D, KVT> &lm, uint32_t src
       const uint32_t a2 = kIsFp8<KVT> ? e4m3x2_to_f16x2(xb) : u8x2_to_f16x2(xb, 0x4140);
       const uint32_t a3 = kIsFp8<KVT> ? e4m3x2_to_f16x2(xb >> 16) : u8x2_to_f16x2(xb, 0x4342);
       mma_f16_16816(o[j], a0, a1, a2, a3, bh0, bh1);
-      mma_f16_16816(o[j], a0, a1, a2, a3, bl0, bl1);
+      if constexpr (kTwo) mma_f16_16816(o[j], a0, a1, a2, a3, bl0, bl1);
     }
   }
 }
@@ -656,12 +661,12 @@ __device__ __forceinline__ void pv_quant(const LaneMap<D, KVT> &lm, uint32_t src
 // one block (first tokens btok[0], btok[1]; pvalid false = invalid page or no
 // block). kscale = the Tile's code scale times scale * log2(e); qz = the sums
 // of q of heads 2t, 2t + 1 times scale * log2(e).
-template <int D, int KVT>
+template <int D, int KVT, bool kPack>
 __device__ __forceinline__ void pair_step(const LaneMap<D, KVT> &lm, uint32_t src,
                                           const int (&btok)[2], const bool (&pvalid)[2],
                                           int tok_lo, int tok1, float kscale,
                                           const float (&qz)[2],
-                                          const uint32_t (&qa)[D / 16][2], int g,
+                                          const uint32_t (&qa)[D / 16][2], int g, int t,
                                           QAcc<D> &acc) {
   using T = Tile<D, KVT>;
   float x[2][4];           // [block][token g: heads 2t, 2t+1 | token g + 8: same]
@@ -719,6 +724,16 @@ __device__ __forceinline__ void pair_step(const LaneMap<D, KVT> &lm, uint32_t sr
       acc.m[h] = m_new;
       acc.l[h] *= al[h];
       acc.z[h] *= al[h];
+    }
+    if constexpr (kPack) {
+      // O^T columns 2t, 2t + 1 of lanes t >= 2 hold the low halves of heads
+      // 2t - 4, 2t - 3, whose factors lanes t - 2 hold
+      const float x0 = __shfl_xor_sync(0xffffffffu, al[0], 2);
+      const float x1 = __shfl_xor_sync(0xffffffffu, al[1], 2);
+      if (t >= 2) {
+        al[0] = x0;
+        al[1] = x1;
+      }
     }
 #pragma unroll
     for (int j = 0; j < T::kMTiles; ++j) {
@@ -781,8 +796,19 @@ __device__ __forceinline__ void pair_step(const LaneMap<D, KVT> &lm, uint32_t sr
     uint32_t h0, l0, h1, l1;
     split_f16(p[u][0] * vf[u][0], p[u][1] * vf[u][0], h0, l0);  // token g
     split_f16(p[u][2] * vf[u][1], p[u][3] * vf[u][1], h1, l1);  // token g + 8
-    pv_quant<D, KVT>(lm, src + u * T::kStageBytes, g, movmatrix_trans(h0),
-                     movmatrix_trans(h1), movmatrix_trans(l0), movmatrix_trans(l1), acc.o);
+    if constexpr (kPack) {
+      // at most four live heads: columns 0..3 of W^T take the high halves of
+      // heads 0..3, columns 4..7 their low halves (lanes t >= 2 take them from
+      // lanes t - 2), and one MMA per m-tile does both
+      const uint32_t x0 = __shfl_xor_sync(0xffffffffu, l0, 2);
+      const uint32_t x1 = __shfl_xor_sync(0xffffffffu, l1, 2);
+      pv_quant<D, KVT, false>(lm, src + u * T::kStageBytes, g,
+                              movmatrix_trans(t < 2 ? h0 : x0),
+                              movmatrix_trans(t < 2 ? h1 : x1), 0u, 0u, acc.o);
+    } else {
+      pv_quant<D, KVT>(lm, src + u * T::kStageBytes, g, movmatrix_trans(h0),
+                       movmatrix_trans(h1), movmatrix_trans(l0), movmatrix_trans(l1), acc.o);
+    }
   }
 }
 
@@ -1078,22 +1104,37 @@ __global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(cons
       if (st < npmine) issue_pair(warp + st * W, st);
       cp_async_commit();
     }
-    for (int k = 0; k < npmine; ++k) {
-      __syncwarp();
-      {
-        const int kn = k + NPS - 1;
-        if (kn < npmine) issue_pair(warp + kn * W, kn % NPS);
-        cp_async_commit();
-      }
-      cp_async_wait<NPS - 1>();
-      __syncwarp();
+    auto loop = [&](auto pack_c) {
+      constexpr bool kPack = decltype(pack_c)::value;
+      for (int k = 0; k < npmine; ++k) {
+        __syncwarp();
+        {
+          const int kn = k + NPS - 1;
+          if (kn < npmine) issue_pair(warp + kn * W, kn % NPS);
+          cp_async_commit();
+        }
+        cp_async_wait<NPS - 1>();
+        __syncwarp();
 
-      const int kb = 2 * (warp + k * W);
-      const int btok[2] = {tok0 + kb * 16, tok0 + kb * 16 + 16};
-      const bool pvalid[2] = {tbl[btok[0] / P - lp0] >= 0,
-                              kb + 1 < nblk && tbl[btok[1] / P - lp0] >= 0};
-      const uint32_t src = ring + (k % NPS) * 2 * T::kStageBytes;
-      pair_step<D, KVT>(lm, src, btok, pvalid, tok_lo, tok1, kscale, qz, qa, g, acc);
+        const int kb = 2 * (warp + k * W);
+        const int btok[2] = {tok0 + kb * 16, tok0 + kb * 16 + 16};
+        const bool pvalid[2] = {tbl[btok[0] / P - lp0] >= 0,
+                                kb + 1 < nblk && tbl[btok[1] / P - lp0] >= 0};
+        const uint32_t src = ring + (k % NPS) * 2 * T::kStageBytes;
+        pair_step<D, KVT, kPack>(lm, src, btok, pvalid, tok_lo, tok1, kscale, qz, qa, g, t, acc);
+      }
+      if constexpr (kPack) {
+        // high + low halves: lanes t < 2 end with the full O^T of heads 2t, 2t + 1
+#pragma unroll
+        for (int j = 0; j < T::kMTiles; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc.o[j][e] += __shfl_xor_sync(0xffffffffu, acc.o[j][e], 2);
+      }
+    };
+    if (G <= 4) {  // CTA-uniform
+      loop(std::true_type{});
+    } else {
+      loop(std::false_type{});
     }
     cp_async_wait<0>();
     __syncwarp();
