@@ -1,6 +1,7 @@
 // Host-side declarations shared by the pagedattn translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -73,6 +74,12 @@ struct PrefixArgs {
   float *o_pre;    // [n_psplits][B*Hq][D]
   float *lse_pre;  // [n_psplits][B*Hq]
   int32_t *d_err;
+  // o_pre as a 5-D tensor [n_psplits][B][Hkv][G][D] fp32, written in boxes of
+  // 32 elements x G heads x 128 / G sequences; tma_store = 0 (G does not
+  // divide 128, or no encoder) writes it with plain stores instead. Filled in
+  // by launch_prefix.
+  CUtensorMap tmo;
+  int32_t tma_store;
 };
 
 cudaError_t launch_prefix(int D, int P, const PrefixArgs &a, bool programmatic,

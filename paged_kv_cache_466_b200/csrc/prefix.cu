@@ -141,6 +141,24 @@ __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ void sts128(uint32_t addr, float4 v) {
+  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y),
+               "f"(v.z), "f"(v.w)
+               : "memory");
+}
+
+// Box of the 5-D tensor map at `tmap` (a kernel parameter) whose first
+// element is (x0 .. x4), from shared memory at `src`; completes as a bulk
+// group of the issuing thread.
+__device__ __forceinline__ void tma_store_5d(const CUtensorMap *tmap, uint32_t src, int x0, int x1,
+                                             int x2, int x3, int x4) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3, %4, %5}], "
+      "[%6];" ::"l"(tmap),
+      "r"(x0), "r"(x1), "r"(x2), "r"(x3), "r"(x4), "r"(src)
+      : "memory");
+}
+
 template <int D>
 struct PLayout {
   static constexpr int kChunks = D / 8;                       // 16-byte chunks per row
@@ -154,7 +172,8 @@ struct PLayout {
 };
 
 template <int D, int P>
-__global__ void __launch_bounds__(kThreads, 2) prefix_kernel(const PrefixArgs a) {
+__global__ void __launch_bounds__(kThreads, 2)
+    prefix_kernel(const __grid_constant__ PrefixArgs a) {
   using L = PLayout<D>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // the swizzled tiles need 1024-byte aligned atoms
@@ -399,23 +418,59 @@ __global__ void __launch_bounds__(kThreads, 2) prefix_kernel(const PrefixArgs a)
   tc_fence_after();
   const size_t R = (size_t)a.B * a.hq;
   const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-  float *orow = a.o_pre + ((size_t)ps * R + qrow) * D;
+  if (a.tma_store) {
+    // Every MMA and copy has completed, so the Q tile and the K/V stages are
+    // free: O / l goes there as 32-column boxes of 128 rows (128-byte rows,
+    // 16-byte pieces swizzled by row, conflict-free), and one thread writes
+    // them with the tensor memory accelerator in whole lines. (Plain stores
+    // put 16-byte pieces of 32 rows in every warp instruction.)
 #pragma unroll
-  for (int c0 = 0; c0 < D; c0 += 32) {
-    uint32_t u[32];
-    if (ntl > 0) {
-      tmem_ld32(t_o + lane_off + c0, u);
-      tmem_wait_ld();
-    } else {
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      uint32_t u[32];
+      if (ntl > 0) {
+        tmem_ld32(t_o + lane_off + c0, u);
+        tmem_wait_ld();
+      } else {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) u[j] = 0u;
+        for (int j = 0; j < 32; ++j) u[j] = 0u;
+      }
+      const uint32_t rowb = sbase + (c0 / 32) * (kRowsPerCta * 128) + tid * 128;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        sts128(rowb + ((j ^ (tid & 7)) << 4),
+               make_float4(__uint_as_float(u[4 * j]) * inv, __uint_as_float(u[4 * j + 1]) * inv,
+                           __uint_as_float(u[4 * j + 2]) * inv,
+                           __uint_as_float(u[4 * j + 3]) * inv));
     }
-    if (row_ok) {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the copy engine
+    __syncthreads();
+    const int seq0 = mt * kRowsPerCta / G;
+    if (tid == 0 && seq0 < a.B) {
 #pragma unroll
-      for (int j = 0; j < 32; j += 4)
-        *reinterpret_cast<float4 *>(orow + c0 + j) =
-            make_float4(__uint_as_float(u[j]) * inv, __uint_as_float(u[j + 1]) * inv,
-                        __uint_as_float(u[j + 2]) * inv, __uint_as_float(u[j + 3]) * inv);
+      for (int c0 = 0; c0 < D; c0 += 32)
+        tma_store_5d(&a.tmo, sbase + (c0 / 32) * (kRowsPerCta * 128), c0, 0, h, seq0, ps);
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // before the CTA exits
+    }
+  } else {
+    float *orow = a.o_pre + ((size_t)ps * R + qrow) * D;
+#pragma unroll
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      uint32_t u[32];
+      if (ntl > 0) {
+        tmem_ld32(t_o + lane_off + c0, u);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) u[j] = 0u;
+      }
+      if (row_ok) {
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+          *reinterpret_cast<float4 *>(orow + c0 + j) =
+              make_float4(__uint_as_float(u[j]) * inv, __uint_as_float(u[j + 1]) * inv,
+                          __uint_as_float(u[j + 2]) * inv, __uint_as_float(u[j + 3]) * inv);
+      }
     }
   }
   if (row_ok)
@@ -429,9 +484,52 @@ __global__ void __launch_bounds__(kThreads, 2) prefix_kernel(const PrefixArgs a)
                  "r"(kTmemCols));
 }
 
+// cuTensorMapEncodeTiled, looked up through the runtime (the library does not
+// link the driver library); null if the driver lacks it.
+using TmapEncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+TmapEncodeFn tmap_encoder() {
+  static const TmapEncodeFn fn = [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<TmapEncodeFn>(p);
+  }();
+  return fn;
+}
+
+// The prefix partials o_pre [n_psplits][B][Hq][D] as the 5-D tensor
+// [n_psplits][B][Hkv][G][D], written in boxes of 32 elements x G heads x
+// 128 / G sequences (one 128-row tile of a KV head, 32 columns) with the
+// 128-byte swizzle. False where G does not divide 128 or the driver cannot
+// encode it: the kernel then uses plain stores.
+bool encode_partials(PrefixArgs *a, int D) {
+  const int G = a->hq / a->hkv;
+  if (kRowsPerCta % G != 0) return false;
+  const TmapEncodeFn f = tmap_encoder();
+  if (f == nullptr) return false;
+  const cuuint64_t dims[5] = {(cuuint64_t)D, (cuuint64_t)G, (cuuint64_t)a->hkv, (cuuint64_t)a->B,
+                              (cuuint64_t)a->n_psplits};
+  const cuuint64_t strides[4] = {(cuuint64_t)D * 4, (cuuint64_t)G * D * 4,
+                                 (cuuint64_t)a->hq * D * 4, (cuuint64_t)a->B * a->hq * D * 4};
+  const cuuint32_t box[5] = {32, (cuuint32_t)G, 1, (cuuint32_t)(kRowsPerCta / G), 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return f(&a->tmo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 5, a->o_pre, dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D, int P>
-cudaError_t launch_prefix_t(const PrefixArgs &a, bool programmatic, cudaStream_t stream) {
+cudaError_t launch_prefix_t(const PrefixArgs &a_in, bool programmatic, cudaStream_t stream) {
   using L = PLayout<D>;
+  PrefixArgs a = a_in;
+  a.tma_store = encode_partials(&a, D) ? 1 : 0;
   const int max_pages_per_split = a.tiles_per_split * kTileTok / P + 2;
   if (max_pages_per_split > 4096) return cudaErrorInvalidValue;
   constexpr int kMaxSmem = L::kPagesOff + 4 * 4096 + 1024;  // + alignment slack
