@@ -262,7 +262,14 @@ pa_status_t pa_decode_append(const pa_kv_pool_t *pool, const void *q,
  * K/V row once per 128 query rows instead of once per request; (2) the paged
  * decode over each request's own tokens [prefix_len, context_lens[b]),
  * writing its split partials; (3) the log-sum-exp merge of (2) and (1) per
- * row, in that order (deterministic).
+ * row, in that order (deterministic). (1) runs on `stream` and (2) on a
+ * second stream the library keeps per device, forked from `stream` before
+ * (1) and joined back before (3), so the prefix pass (tensor-core and L2
+ * bound) overlaps the suffix decode (HBM bound); the split count of (1) is
+ * pa_prefix_plan_splits'. The call stays one unit of `stream` (all three
+ * complete before later work on it; it can be captured in a CUDA graph, the
+ * fork and join becoming graph edges). Calls from several host threads are
+ * serialised around the fork.
  *
  *   prefix_pages : (device) int32 [prefix_len / P] physical pages of the prefix
  *   prefix_len   : tokens in the prefix; a multiple of the page size (0 falls
@@ -292,6 +299,25 @@ pa_status_t pa_decode_shared_prefix(const pa_kv_pool_t *pool, const void *q,
                                     float *out, void *workspace,
                                     size_t workspace_bytes, int32_t num_splits,
                                     int32_t *d_err, void *stream);
+
+/*
+ * pa_prefix_plan_splits — host only (no device access): how many 64-token
+ * tiles of the shared prefix each CTA of pa_decode_shared_prefix's prefix pass
+ * takes, for `units` (128-row query tile, KV head) pairs, a prefix of `tiles`
+ * 64-token tiles, a device of num_sms SMs holding decode_ctas_per_sm suffix
+ * decode CTAs each, and an estimate of the bytes the suffix decode streams.
+ * The pass runs beside the suffix decode, so the rule picks the split count
+ * whose estimated finish, the later of the two, is earliest: the prefix pass
+ * takes 4 us plus 1.6 us per tile with one of its CTAs on an SM (2.2 us with
+ * two; more than two per SM run in waves), and the decode streams at 6.5 TB/s
+ * while it keeps at least 2 * num_sms CTAs resident, slower in proportion
+ * below that (an SM holding one prefix CTA keeps decode_ctas_per_sm - 2
+ * decode CTAs, one holding two keeps none). Ties go to fewer CTAs. The
+ * constants were measured on B200. The pass then has ceil(tiles / result)
+ * splits. Returns <= 0 on invalid arguments.
+ */
+int32_t pa_prefix_plan_splits(int64_t units, int32_t tiles, int32_t num_sms,
+                              int32_t decode_ctas_per_sm, double suffix_bytes);
 
 /*
  * pa_decode_window — decode over the StreamingLLM token set: the first `sinks`

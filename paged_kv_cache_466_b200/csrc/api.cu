@@ -4,6 +4,7 @@
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
+#include <mutex>
 #include <new>
 #include <string>
 
@@ -177,6 +178,55 @@ pa_status_t pa_kv_append(const pa_kv_pool_t *pool, const void *k_new, const void
                                       block_tables, num_seqs, max_pages, d_err,
                                       static_cast<cudaStream_t>(stream)),
                      "pa_kv_append launch");
+}
+
+int32_t pa_prefix_plan_splits(int64_t units, int32_t tiles, int32_t num_sms,
+                              int32_t decode_ctas_per_sm, double suffix_bytes) {
+  if (units <= 0 || tiles <= 0 || num_sms <= 0 || decode_ctas_per_sm <= 0 ||
+      !(suffix_bytes >= 0.0))
+    return -1;
+  // Measured on B200 (cascade steps of 32..256 requests, prefixes of 1024..8000
+  // tokens, suffixes of up to 64..1024 tokens): a prefix CTA's set-up and
+  // epilogue, one 64-token tile with one or two prefix CTAs on the SM, the
+  // copy bandwidth, and the decode CTAs that keep HBM streaming.
+  constexpr double kFixedUs = 4.0, kTile1Us = 1.6, kTile2Us = 2.2, kBytesPerUs = 6.5e6;
+  const long long sms = num_sms;
+  const long long need = 2 * sms;
+  const double td0 = suffix_bytes / kBytesPerUs;
+  const int with_prefix = decode_ctas_per_sm > 2 ? decode_ctas_per_sm - 2 : 0;
+  double best = 0.0;
+  bool have = false;
+  int best_tp = tiles;
+  int last_n = -1;
+  for (int ns = 1; ns <= tiles && ns <= kMaxSplits; ++ns) {
+    const int tp = (tiles + ns - 1) / ns;  // tiles per split
+    const int n = (tiles + tp - 1) / tp;   // splits
+    if (n == last_n) continue;
+    last_n = n;
+    const long long ctas = units * n;
+    double tprefix;
+    long long slots;
+    if (ctas <= sms) {
+      tprefix = kFixedUs + tp * kTile1Us;
+      slots = (sms - ctas) * decode_ctas_per_sm + ctas * with_prefix;
+    } else if (ctas <= 2 * sms) {
+      tprefix = kFixedUs + tp * kTile2Us;
+      slots = (2 * sms - ctas) * with_prefix;
+    } else {
+      const long long waves = (ctas + 2 * sms - 1) / (2 * sms);
+      tprefix = kFixedUs + (double)waves * tp * kTile2Us;
+      slots = 0;
+    }
+    const double tdecode =
+        td0 * (slots >= need ? 1.0 : (double)need / (double)(slots > 0 ? slots : 1));
+    const double cost = tprefix > tdecode ? tprefix : tdecode;
+    if (!have || cost < best) {  // strictly better: ties keep fewer CTAs
+      have = true;
+      best = cost;
+      best_tp = tp;
+    }
+  }
+  return best_tp;
 }
 
 int32_t pa_decode_plan_splits(int64_t num_units, int32_t max_pages, int32_t page_size,
@@ -394,6 +444,33 @@ pa_status_t pa_decode_append(const pa_kv_pool_t *pool, const void *q, const void
 // ---------------------------------------------------------------- shared prefix
 namespace {
 
+// The cascade's second stream and its fork and join events, per device,
+// created on first use (a device whose creation failed runs the three
+// launches on the caller's stream). g_fork_mu serialises the fork sequence.
+struct Fork {
+  cudaStream_t s2 = nullptr;
+  cudaEvent_t forked = nullptr, joined = nullptr;
+  bool failed = false;
+};
+std::mutex g_fork_mu;
+Fork g_fork[64];
+
+Fork *fork_for_device() {
+  const int dev = current_device();
+  if (dev < 0 || dev >= 64) return nullptr;
+  Fork &f = g_fork[dev];
+  if (f.s2 == nullptr && !f.failed) {
+    if (cudaStreamCreateWithFlags(&f.s2, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&f.forked, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&f.joined, cudaEventDisableTiming) != cudaSuccess) {
+      cudaGetLastError();
+      f.s2 = nullptr;
+      f.failed = true;
+    }
+  }
+  return f.s2 != nullptr ? &f : nullptr;
+}
+
 struct PrefixPlan {
   int n_psplits, tiles_per_split;  // prefix kernel
   int S, chunk;                    // suffix decode
@@ -407,16 +484,24 @@ bool plan_prefix(const pa_kv_pool_t *pool, int B, int Hq, int max_pages, int pre
   const int lpb = prefix_len / P;
   const int sfx_pages = max_pages - lpb;
   if (sfx_pages < 1) return false;
-  // prefix: enough CTAs to cover the GPU twice, splits of whole 64-token tiles
+  // prefix: splits of whole 64-token tiles, as many as pa_prefix_plan_splits
+  // finds best for a pass that runs beside the suffix decode; the suffix
+  // bytes are estimated from the table width (half of it attended on average)
   const int tiles = (prefix_len + prefix_tile_tokens() - 1) / prefix_tile_tokens();
   const int mtiles = (B * G + prefix_rows_per_cta() - 1) / prefix_rows_per_cta();
-  const long long base = (long long)mtiles * pool->num_kv_heads;
-  int ns = (int)((2LL * device_sm_count() + base - 1) / base);
-  if (ns > tiles) ns = tiles;
-  if (ns > kMaxSplits) ns = kMaxSplits;
-  if (ns < 1) ns = 1;
-  pl->tiles_per_split = tiles > 0 ? (tiles + ns - 1) / ns : 1;
-  pl->n_psplits = tiles > 0 ? (tiles + pl->tiles_per_split - 1) / pl->tiles_per_split : 0;
+  const long long units = (long long)mtiles * pool->num_kv_heads;
+  const int hd = pool->head_dim;
+  const int row = pool->dtype == PA_KV_BF16 ? 2 * hd
+                  : pool->dtype == PA_KV_U4_PER_TOKEN ? hd / 2 + 8 : hd + 8;
+  const double sfx_bytes =
+      (double)B * pool->num_kv_heads * 2.0 * row * ((double)sfx_pages * P) / 2.0;
+  int tp = tiles > 0 ? pa_prefix_plan_splits(units, tiles, device_sm_count(),
+                                             cached_ctas_per_sm(hd, P, pool->dtype), sfx_bytes)
+                     : 1;
+  if (tp < 1) tp = tiles > 0 ? tiles : 1;
+  if (tiles > 0 && (tiles + tp - 1) / tp > kMaxSplits) tp = (tiles + kMaxSplits - 1) / kMaxSplits;
+  pl->tiles_per_split = tp;
+  pl->n_psplits = tiles > 0 ? (tiles + tp - 1) / tp : 0;
   // suffix: the plain decode's split planning over the suffix pages
   pl->S = pa_decode_num_splits(pool, B, sfx_pages, num_splits);
   if (pl->S <= 0) return false;
@@ -539,22 +624,40 @@ pa_status_t pa_decode_shared_prefix(const pa_kv_pool_t *pool, const void *q, int
   a.sinks = 0;
   a.tok_begin = prefix_len;
   a.d_err = d_err;
-  // Three launches on `stream`: the prefix pass; the suffix decode, which
+  // Three launches: the prefix pass on `stream`; the suffix decode, which
   // writes its split partials (an empty split writes lse = -inf) instead of
-  // merging; one merge of the suffix splits and the prefix splits per row,
-  // with its loads batched (a decode CTA merging prefix partials in its
-  // epilogue measured slower).
+  // merging, on the second stream (forked after the work already on
+  // `stream`, the prefix pass launched first so that its CTAs are placed
+  // first); then, joined back on `stream`, one merge of the suffix splits and
+  // the prefix splits per row, with its loads batched (a decode CTA merging
+  // prefix partials in its epilogue measured slower).
   a.prior_o = nullptr;
   a.prior_lse = nullptr;
   a.n_prior = 0;
   a.keep_partials = 1;
   a.tok_end = 0x7fffffff;
   a.range_mode = 0;
-  st = cuda_status(launch_prefix(pool->head_dim, pool->page_size, pa, true, s),
-                   "pa_decode_shared_prefix prefix launch");
-  if (st == PA_OK)
-    st = cuda_status(launch_decode(pool->head_dim, pool->page_size, pool->dtype, a, s),
-                     "pa_decode_shared_prefix suffix launch");
+  {
+    std::lock_guard<std::mutex> lock(g_fork_mu);
+    Fork *f = fork_for_device();
+    if (f != nullptr) {
+      st = cuda_status(cudaEventRecord(f->forked, s), "pa_decode_shared_prefix fork");
+      if (st == PA_OK)
+        st = cuda_status(cudaStreamWaitEvent(f->s2, f->forked, 0), "pa_decode_shared_prefix fork");
+    }
+    if (st == PA_OK)
+      st = cuda_status(launch_prefix(pool->head_dim, pool->page_size, pa, true, s),
+                       "pa_decode_shared_prefix prefix launch");
+    if (st == PA_OK)
+      st = cuda_status(launch_decode(pool->head_dim, pool->page_size, pool->dtype, a,
+                                     f != nullptr ? f->s2 : s),
+                       "pa_decode_shared_prefix suffix launch");
+    if (st == PA_OK && f != nullptr) {
+      st = cuda_status(cudaEventRecord(f->joined, f->s2), "pa_decode_shared_prefix join");
+      if (st == PA_OK)
+        st = cuda_status(cudaStreamWaitEvent(s, f->joined, 0), "pa_decode_shared_prefix join");
+    }
+  }
   if (st != PA_OK) return st;
   return cuda_status(launch_splitkv_reduce(a.o_part, a.lse, num_seqs, num_q_heads, pl.S,
                                            pool->head_dim, out, true, s, pa.o_pre, pa.lse_pre,

@@ -31,6 +31,9 @@ int main(void) {
   CHECK(pa_decode_plan_splits(32 * 8, 256, 32, 148, 3, 0) == 1);
   CHECK(pa_decode_plan_splits(8 * 8, 256, 32, 148, 3, 0) == 4);
   CHECK(pa_decode_plan_splits(64 * 8, 256, 16, 148, 3, 0) == 4);
+  /* 128 requests x (2000-token prefix + up to 512 own tokens): 3 splits of 11 tiles */
+  CHECK(pa_prefix_plan_splits(32, 32, 148, 3, 128.0 * 8 * 2 * 256 * 512 / 2) == 11);
+  CHECK(pa_prefix_plan_splits(0, 32, 148, 3, 0.0) <= 0);
 
   memset(&pool, 0, sizeof pool);
   pool.num_pages = 16;

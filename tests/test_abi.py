@@ -195,6 +195,57 @@ def test_split_plan_rules_on_a_b200(lib):
     assert plan(-1, 4, 16) <= 0 and plan(4, 0, 16) <= 0 and plan(4, 4, 16, sms=0) <= 0
 
 
+def _prefix_shape(B, prefix, suffix_max, G=4, Hkv=8, D=128, P=16):
+    """(units, tiles, estimated suffix bytes) of a cascade batch, as the
+    library derives them: 128-row query tiles x KV heads, 64-token prefix
+    tiles, half of the table's suffix capacity in bf16 K and V rows."""
+    units = -(-(B * G) // 128) * Hkv
+    tiles = -(-prefix // 64)
+    capacity = -(-suffix_max // P) * P
+    return units, tiles, B * Hkv * 2 * (2 * D) * capacity / 2
+
+
+def test_prefix_plan_rules_on_a_b200(lib):
+    """The cascade's prefix split rule with the B200's 148 SMs and 3 decode
+    CTAs per SM. Each shape's answer is the split count measured fastest for
+    it (cascade step with the prefix pass beside the suffix decode, split
+    counts 1..32 swept): long suffixes leave the SMs to the decode, long
+    prefixes spread over all of them."""
+    plan = lambda B, pre, sfx, sms=148, cps=3: lib.pa_prefix_plan_splits(
+        *_prefix_shape(B, pre, sfx)[:2], sms, cps, _prefix_shape(B, pre, sfx)[2])
+    splits = lambda B, pre, sfx: -(-_prefix_shape(B, pre, sfx)[1] // plan(B, pre, sfx))
+    assert plan(128, 2000, 512) == 11 and splits(128, 2000, 512) == 3    # 96 CTAs (bench)
+    assert splits(32, 2000, 512) == 16                                  # 128 CTAs
+    assert splits(64, 4000, 256) == 9                                   # 144 CTAs
+    assert splits(128, 8000, 64) == 8                                   # 256 CTAs
+    assert splits(256, 1024, 1024) == 1                                 # 64 CTAs
+    # no suffix: the fastest prefix pass; equal estimates keep fewer CTAs
+    # (8 splits = 256 CTAs, 12.8 us, ties 16 splits in two waves)
+    assert lib.pa_prefix_plan_splits(32, 32, 148, 3, 0.0) == 4
+    assert lib.pa_prefix_plan_splits(0, 4, 148, 3, 0.0) <= 0
+    assert lib.pa_prefix_plan_splits(4, 0, 148, 3, 0.0) <= 0
+    assert lib.pa_prefix_plan_splits(4, 4, 0, 3, 0.0) <= 0
+    assert lib.pa_prefix_plan_splits(4, 4, 148, 0, 0.0) <= 0
+    assert lib.pa_prefix_plan_splits(4, 4, 148, 3, -1.0) <= 0
+
+
+def test_prefix_plan_invariants_for_any_shape(lib):
+    """Any shape gets a valid tile count per split (1..tiles, at most 256
+    splits), and a larger suffix never gives the prefix pass more CTAs."""
+    from hypothesis import given, settings, strategies as st
+
+    @settings(max_examples=300, deadline=None)
+    @given(units=st.integers(1, 512), tiles=st.integers(1, 2000), sms=st.integers(1, 200),
+           cps=st.integers(1, 8), mb=st.floats(0, 4000), more=st.floats(1, 10))
+    def check(units, tiles, sms, cps, mb, more):
+        tp = lib.pa_prefix_plan_splits(units, tiles, sms, cps, mb * 1e6)
+        assert 1 <= tp <= tiles and -(-tiles // tp) <= 256
+        tp2 = lib.pa_prefix_plan_splits(units, tiles, sms, cps, mb * 1e6 * more)
+        assert -(-tiles // tp2) <= -(-tiles // tp)
+
+    check()
+
+
 def test_header_compiles_as_c99_and_host_calls_work(lib, tmp_path):
     """The header is plain C: a C99 program built against it alone links the
     library and runs every entry point that needs no GPU."""

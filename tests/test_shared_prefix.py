@@ -5,7 +5,8 @@ import numpy as np
 import pytest
 import torch
 
-from paged_kv_cache_466_b200 import pa_decode, pa_decode_shared_prefix
+from paged_kv_cache_466_b200 import (pa_decode, pa_decode_shared_prefix,
+                                     pa_decode_shared_prefix_workspace_bytes)
 from paged_kv_cache_466_b200 import workloads as W
 from tests.helpers import (DEV, device_append, device_inputs, full_size_reference,
                            oracle_decode, oracle_pool)
@@ -65,3 +66,33 @@ def test_cascade_full_size_prefix_workload():
     print(f"cascade full size: all {ref.shape[0]} rows, max |gpu - oracle| = {err:.3e}")
     assert np.all(np.isfinite(casc)) and err <= 2e-3
     assert np.abs(casc - plain).max() <= 1e-4
+
+
+def test_cascade_captured_in_a_cuda_graph_replays_the_eager_bits():
+    """The prefix pass and the suffix decode run on two streams (forked from
+    and joined back to the caller's stream); captured in a CUDA graph, the
+    call replays to the eager call's bits, twice in a row."""
+    w, _ = W.prefix(B=33, prefix_tokens=1008, suffix_range=(1, 200))
+    pool, bt, ctx, q = device_inputs(w)
+    device_append(pool, w, bt)
+    pre = torch.from_numpy(np.ascontiguousarray(w.notes["prefix_pages"])).to(DEV)
+    eager = pa_decode_shared_prefix(pool, q, pre, w.notes["prefix_tokens"], bt, ctx, w.scale)
+    torch.cuda.synchronize()
+    out = torch.zeros_like(eager)
+    need = pa_decode_shared_prefix_workspace_bytes(pool, w.B, w.Hq, bt.shape[1],
+                                                   w.notes["prefix_tokens"], 0)
+    ws = torch.zeros(need, dtype=torch.uint8, device=DEV)
+    pa_decode_shared_prefix(pool, q, pre, w.notes["prefix_tokens"], bt, ctx, w.scale, out=out,
+                            workspace=ws)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        pa_decode_shared_prefix(pool, q, pre, w.notes["prefix_tokens"], bt, ctx, w.scale,
+                                out=out, workspace=ws)
+    for _ in range(2):
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, eager)
+    ref, _ = oracle_decode(w, oracle_pool(w))
+    assert np.abs(out.cpu().numpy().reshape(-1, w.D) - ref).max() <= 2e-3
