@@ -59,13 +59,22 @@ def load_library() -> ctypes.CDLL:
 
 
 def _ptr(t: Optional[torch.Tensor]):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    # ctypes converts a plain int for a c_void_p parameter
+    return None if t is None else t.data_ptr()
+
+
+try:  # the raw handle without building a Stream object (a few microseconds per call)
+    _raw_stream = torch._C._cuda_getCurrentRawStream
+except AttributeError:  # pragma: no cover
+    _raw_stream = None
 
 
 def _stream(stream=None):
-    if stream is None:
-        stream = torch.cuda.current_stream()
-    return ctypes.c_void_p(stream.cuda_stream)
+    if stream is not None:
+        return stream.cuda_stream
+    if _raw_stream is not None:
+        return _raw_stream(torch._C._cuda_getDevice())
+    return torch.cuda.current_stream().cuda_stream
 
 
 def _need(t: torch.Tensor, name: str, dtype, device=None):

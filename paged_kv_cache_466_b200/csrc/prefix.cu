@@ -32,7 +32,9 @@
 // SM, so one CTA's softmax overlaps the other's MMAs. The output per row is
 // the normalised partial and its natural-log log-sum-exp, merged with the
 // suffix by the decode kernel.
+#include <atomic>
 #include <cmath>
+#include <cstring>
 
 #include "pa_device.cuh"
 #include "pa_internal.h"
@@ -509,9 +511,24 @@ TmapEncodeFn tmap_encoder() {
 // 128 / G sequences (one 128-row tile of a KV head, 32 columns) with the
 // 128-byte swizzle. False where G does not divide 128 or the driver cannot
 // encode it: the kernel then uses plain stores.
+// The last map this thread encoded and what it was encoded for: a cascade
+// called step after step with the same workspace and shapes reuses it.
+struct PartialsMapCache {
+  const void *o_pre = nullptr;
+  int D = 0, B = 0, hq = 0, hkv = 0, n = 0;
+  bool ok = false;
+  CUtensorMap map;
+};
+
 bool encode_partials(PrefixArgs *a, int D) {
   const int G = a->hq / a->hkv;
   if (kRowsPerCta % G != 0) return false;
+  thread_local PartialsMapCache c;
+  if (c.o_pre == a->o_pre && c.D == D && c.B == a->B && c.hq == a->hq && c.hkv == a->hkv &&
+      c.n == a->n_psplits) {
+    if (c.ok) std::memcpy(&a->tmo, &c.map, sizeof(CUtensorMap));
+    return c.ok;
+  }
   const TmapEncodeFn f = tmap_encoder();
   if (f == nullptr) return false;
   const cuuint64_t dims[5] = {(cuuint64_t)D, (cuuint64_t)G, (cuuint64_t)a->hkv, (cuuint64_t)a->B,
@@ -520,9 +537,34 @@ bool encode_partials(PrefixArgs *a, int D) {
                                  (cuuint64_t)a->hq * D * 4, (cuuint64_t)a->B * a->hq * D * 4};
   const cuuint32_t box[5] = {32, (cuuint32_t)G, 1, (cuuint32_t)(kRowsPerCta / G), 1};
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  return f(&a->tmo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 5, a->o_pre, dims, strides, box, estr,
-           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-           CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  const bool ok =
+      f(&a->tmo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 5, a->o_pre, dims, strides, box, estr,
+        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+        CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  c.o_pre = a->o_pre;
+  c.D = D;
+  c.B = a->B;
+  c.hq = a->hq;
+  c.hkv = a->hkv;
+  c.n = a->n_psplits;
+  c.ok = ok;
+  if (ok) std::memcpy(&c.map, &a->tmo, sizeof(CUtensorMap));
+  return ok;
+}
+
+// Opt the kernel instance in to its shared memory once per device.
+template <int D, int P>
+cudaError_t ensure_prefix_smem(int max_smem) {
+  static std::atomic<uint64_t> done{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(prefix_kernel<D, P>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           max_smem);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
 }
 
 template <int D, int P>
@@ -535,8 +577,7 @@ cudaError_t launch_prefix_t(const PrefixArgs &a_in, bool programmatic, cudaStrea
   constexpr int kMaxSmem = L::kPagesOff + 4 * 4096 + 1024;  // + alignment slack
   static_assert(kMaxSmem <= 227 * 1024, "shared memory");
   const size_t smem = L::kPagesOff + (size_t)max_pages_per_split * 4 + 1024;
-  cudaError_t e = cudaFuncSetAttribute(prefix_kernel<D, P>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+  const cudaError_t e = ensure_prefix_smem<D, P>(kMaxSmem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((a.B * (a.hq / a.hkv) + kRowsPerCta - 1) / kRowsPerCta, a.hkv, a.n_psplits);
