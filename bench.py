@@ -346,6 +346,9 @@ def run_ours(args, rank, world, local_rank):
     S = pa_decode_num_splits(pool, w.B, w.max_pages, args.splits)
     if args.cascade:
         pre_len = int(w.notes["prefix_tokens"])
+        # the suffix decode's split count, planned over the suffix pages as the
+        # library plans it
+        S = pa_decode_num_splits(pool, w.B, w.max_pages - pre_len // w.P, args.splits)
         pre_pages = torch.from_numpy(w.notes["prefix_pages"].copy()).to(dev)
         nbytes = pa_decode_shared_prefix_workspace_bytes(pool, w.B, w.Hq, w.max_pages, pre_len,
                                                          args.splits)
