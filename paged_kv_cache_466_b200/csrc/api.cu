@@ -298,9 +298,14 @@ int32_t pa_decode_num_splits(const pa_kv_pool_t *pool, int32_t num_seqs, int32_t
   const int64_t units = (int64_t)num_seqs * pool->num_kv_heads;
   if (requested > 0)  // no device query needed
     return pa_decode_plan_splits(units, max_pages, pool->page_size, 1, 1, requested);
+  // The rule's regimes and constants were measured with three resident decode
+  // CTAs per SM; a kernel that fits a fourth (INT4) is planned as if it had
+  // three: with more slots the one-wave regime would hand a ragged batch one
+  // CTA per (sequence, KV head), whose longest member then sets the time
+  // (INT4, ragged Llama-3-8B shapes: 74.5 us at S = 1 vs 60.6 us at S = 4).
+  const int cps = cached_ctas_per_sm(pool->head_dim, pool->page_size, pool->dtype);
   return pa_decode_plan_splits(units, max_pages, pool->page_size, device_sm_count(),
-                               cached_ctas_per_sm(pool->head_dim, pool->page_size, pool->dtype),
-                               0);
+                               cps < 3 ? cps : 3, 0);
 }
 
 int32_t pa_decode_auto_splits(int32_t num_seqs, int32_t num_kv_heads, int32_t max_ctx,

@@ -66,6 +66,9 @@
 #ifndef PA_DECODE_MIN_CTAS
 #define PA_DECODE_MIN_CTAS 3
 #endif
+#ifndef PA_DECODE_MIN_CTAS_U4
+#define PA_DECODE_MIN_CTAS_U4 4
+#endif
 #ifndef PA_DECODE_PDL
 #define PA_DECODE_PDL 1
 #endif
@@ -845,8 +848,15 @@ __device__ __forceinline__ void append_new_row(const DecodeArgs &a, int b, int h
   }
 }
 
+// CTAs per SM the register allocation must allow. An INT4 CTA's ring (two
+// pair stages of 2.3 KB blocks per warp, 37 KB) leaves room for a fourth CTA,
+// which 128 registers allow (12 bytes of spill); measured on the ragged
+// Llama-3-8B-shaped INT4 step: 63.8 -> 60.6 us at S = 4.
+template <int KVT>
+constexpr int kMinCtas = KVT == PA_KV_U4_PER_TOKEN ? PA_DECODE_MIN_CTAS_U4 : PA_DECODE_MIN_CTAS;
+
 template <int D, int P, int KVT, int W, int NSTAGE>
-__global__ void __launch_bounds__(W * 32, PA_DECODE_MIN_CTAS) decode_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(W * 32, kMinCtas<KVT>) decode_kernel(const DecodeArgs a) {
   using T = Tile<D, KVT>;
   using SM = Smem<D, KVT, W, NSTAGE>;
   static_assert(P % 16 == 0, "a 16-token block must not straddle pages");
