@@ -1029,11 +1029,12 @@ bool plan_window(const pa_kv_pool_t *pool, int B, int max_pages, int sinks, int 
   pl->S_main = pa_decode_num_splits(pool, B, (int)wp, num_splits);
   if (pl->S_main <= 0) return false;
   pl->chunk = ((int)wp + pl->S_main - 1) / pl->S_main;
-  pl->S = pl->S_main + (sinks > 0 ? 1 : 0);
-  // the sink split reads pages [0, ceil(min(sinks, ctx) / P)) at most
+  // the sinks are a second range of split 0 (no split of their own): its
+  // table slice holds pages [0, ceil(min(sinks, ctx) / P)) and then a chunk
+  pl->S = pl->S_main;
   const long long sink_tok = std::min<long long>(sinks, (long long)max_pages * P);
   const long long sink_pages = (sink_tok + P - 1) / P;
-  pl->tbl_cap = (int)std::max<long long>(pl->chunk, sink_pages);
+  pl->tbl_cap = (int)(pl->chunk + sink_pages);
   return pl->tbl_cap <= kMaxPagesPerSplit;
 }
 

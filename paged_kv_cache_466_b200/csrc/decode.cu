@@ -881,9 +881,10 @@ __global__ void __launch_bounds__(W * 32, kMinCtas<KVT>) decode_kernel(const Dec
   // Token ranges. The main range [mlo, ctx) is split over the first S_main
   // splits: mlo = tok_begin (page aligned; > 0 when the caller supplies the
   // shared-prefix part as prior partials) or, with a window, the start of the
-  // last `window` tokens. With attention sinks the extra split S_main covers
-  // [0, min(sinks, ctx)) ("Token Eviction Strategies", Eq. 5); the two ranges
-  // are disjoint and together hold exactly the kept tokens.
+  // last `window` tokens. With attention sinks, split 0 also covers
+  // [0, min(sinks, ctx)) ("Token Eviction Strategies", Eq. 5) as a second
+  // range processed before its main one; the two ranges are disjoint and
+  // together hold exactly the kept tokens.
   // Loads that do not depend on the context length go out with it: the
   // query fragments and, where the split's page range does not depend on the
   // context (no window, a main split), that range's table entries.
@@ -924,26 +925,21 @@ __global__ void __launch_bounds__(W * 32, kMinCtas<KVT>) decode_kernel(const Dec
   const int n_pages = (ctx + P - 1) / P;
   const int lpb = mlo / P;
   const int n_main_live = ctx > mlo ? (n_pages - lpb + a.pages_per_split - 1) / a.pages_per_split : 0;
-  const int n_live = n_main_live + (sink_hi > 0 ? 1 : 0);  // splits holding tokens
-  int lp0, lp1, tok_lo, tok_hi, slot;
-  if (split < a.S_main) {
-    lp0 = lpb + split * a.pages_per_split;
-    lp1 = min(lp0 + a.pages_per_split, n_pages);
-    tok_lo = max(lp0 * P, mlo);
-    tok_hi = min(lp1 * P, ctx);
-    slot = split;
-  } else {  // the attention-sink split
-    lp0 = 0;
-    lp1 = (sink_hi + P - 1) / P;
-    tok_lo = 0;
-    tok_hi = sink_hi;
-    slot = n_main_live;
-  }
-  if (lp1 - lp0 > a.tbl_cap) {
+  // splits holding tokens (split 0 holds the sinks even when the main range is empty)
+  const int n_live = n_main_live > 0 ? n_main_live : (sink_hi > 0 ? 1 : 0);
+  const int slot = split;
+  // split 0's sink range: pages [0, nsp) staged first, blocks [0, nsb) of it
+  const int nsp = split == 0 ? (sink_hi + P - 1) / P : 0;
+  const int nsb = split == 0 ? (sink_hi + 15) / 16 : 0;
+  int lp0 = lpb + split * a.pages_per_split;
+  int lp1 = max(min(lp0 + a.pages_per_split, n_pages), lp0);
+  int tok_lo = max(lp0 * P, mlo);
+  int tok_hi = min(lp1 * P, ctx);
+  if (nsp + (lp1 - lp0) > a.tbl_cap) {
     // Cannot happen with the host's plan (the table slot holds tbl_cap pages);
     // kept so that no table read or write can leave the staged slot.
     if (threadIdx.x == 0) flag_error(a.d_err, PA_DERR_BAD_CTX);
-    lp1 = lp0 + a.tbl_cap;
+    lp1 = lp0 + max(a.tbl_cap - nsp, 0);
     tok_hi = min(tok_hi, lp1 * P);
   }
   const int blk0 = tok_lo & ~15;  // blocks stay 16-aligned inside their page
@@ -951,7 +947,7 @@ __global__ void __launch_bounds__(W * 32, kMinCtas<KVT>) decode_kernel(const Dec
   const int tok0 = blk0;
   const int tok1 = tok_hi;
 
-  if (nblk == 0) {
+  if (nblk == 0 && nsb == 0) {
     if (a.keep_partials) {  // an empty partial: o = 0, lse = -inf (weight 0)
       for (int e = threadIdx.x; e < G * D; e += W * 32) {
         const size_t row = (size_t)b * a.hq + (size_t)h * G + e / D;
@@ -986,8 +982,10 @@ __global__ void __launch_bounds__(W * 32, kMinCtas<KVT>) decode_kernel(const Dec
       }
     }
   } else {
-    for (int i = threadIdx.x; i < lp1 - lp0; i += W * 32) {
-      int pg = __ldg(a.block_tables + (size_t)b * a.max_pages + lp0 + i);
+    // entries [0, nsp): the sink pages; then the main range's pages
+    for (int i = threadIdx.x; i < nsp + lp1 - lp0; i += W * 32) {
+      const int lp = i < nsp ? i : lp0 + i - nsp;
+      int pg = __ldg(a.block_tables + (size_t)b * a.max_pages + lp);
       if (pg < 0 || pg >= a.num_pages) {
         flag_error(a.d_err, PA_DERR_BAD_PAGE);
         pg = -1;
@@ -1002,7 +1000,7 @@ __global__ void __launch_bounds__(W * 32, kMinCtas<KVT>) decode_kernel(const Dec
   if (a.k_new != nullptr && ctx > 0 && split < a.S_main) {
     const int lp_new = (ctx - 1) / P;
     if (lp_new >= lp0 && lp_new < lp1) {  // CTA-uniform
-      const int page = tbl[lp_new - lp0];
+      const int page = tbl[nsp + lp_new - lp0];
       if (page >= 0)
         append_new_row<D, KVT>(a, b, h, ((size_t)page * a.hkv + h) * P + (ctx - 1) % P);
       __syncthreads();  // the row is stored before the page is copied in
@@ -1016,17 +1014,23 @@ __global__ void __launch_bounds__(W * 32, kMinCtas<KVT>) decode_kernel(const Dec
   const uint32_t ring = smem_u32(smem) + warp * SM::kRingBytesPerWarp;
   const unsigned char *kbase = static_cast<const unsigned char *>(a.k_pool);
   const unsigned char *vbase = static_cast<const unsigned char *>(a.v_pool);
-  const int nmine = nblk > warp ? (nblk - warp + W - 1) / W : 0;
   const LaneMap<D, KVT> lm(lane);
   const float *sz_base = lane < 8 ? a.k_sz : a.v_sz;
-  auto issue = [&](int kb, int st) {
-    const int btok = tok0 + kb * 16;
+  // A token range of this CTA: blocks [0, nblk) starting at token tok0, tokens
+  // [lo, hi) attended, table entry tb + token / P. Warp w takes blocks (pairs)
+  // w, w + W, ... of each range.
+  struct Range {
+    int tok0, nblk, lo, hi, tb;
+  };
+  const Range sinks_r = {0, nsb, 0, sink_hi, 0};
+  auto issue = [&](const Range &r, int kb, int st) {
+    const int btok = r.tok0 + kb * 16;
     const int lp = btok / P;
-    const int page = tbl[lp - lp0];
+    const int page = tbl[r.tb + lp];
     const int in_page = btok - lp * P;
     // rows [rlo, rhi) of the block hold tokens of this range
-    const int rlo = page >= 0 ? max(0, tok_lo - btok) : 16;
-    const int rhi = page >= 0 ? min(16, tok1 - btok) : 0;
+    const int rlo = page >= 0 ? max(0, r.lo - btok) : 16;
+    const int rhi = page >= 0 ? min(16, r.hi - btok) : 0;
     // rows of an invalid page are zero-filled; the address stays inside page 0
     const size_t row0 = ((size_t)(page >= 0 ? page : 0) * a.hkv + h) * P + in_page;
     issue_block<D, KVT>(lm, ring + st * T::kStageBytes, kbase, vbase, sz_base, row0, rlo, rhi,
@@ -1041,29 +1045,36 @@ __global__ void __launch_bounds__(W * 32, kMinCtas<KVT>) decode_kernel(const Dec
   if constexpr (KVT == PA_KV_BF16) {
     WarpAcc<D> acc;
     acc.reset();
+    // one range through the warp's ring; the online softmax state carries over
+    auto pass = [&](const Range &r) {
+      const int wr = warp;
+      const int nmine = r.nblk > wr ? (r.nblk - wr + W - 1) / W : 0;
 #pragma unroll
-    for (int st = 0; st < NSTAGE - 1; ++st) {
-      if (st < nmine) issue(warp + st * W, st);
-      cp_async_commit();
-    }
-    for (int k = 0; k < nmine; ++k) {
-      __syncwarp();
-      {
-        const int kn = k + NSTAGE - 1;
-        if (kn < nmine) issue(warp + kn * W, kn % NSTAGE);
+      for (int st = 0; st < NSTAGE - 1; ++st) {
+        if (st < nmine) issue(r, wr + st * W, st);
         cp_async_commit();
       }
-      cp_async_wait<NSTAGE - 1>();
-      __syncwarp();  // every lane's pieces of this block are now visible to the warp
+      for (int k = 0; k < nmine; ++k) {
+        __syncwarp();
+        {
+          const int kn = k + NSTAGE - 1;
+          if (kn < nmine) issue(r, wr + kn * W, kn % NSTAGE);
+          cp_async_commit();
+        }
+        cp_async_wait<NSTAGE - 1>();
+        __syncwarp();  // every lane's pieces of this block are now visible to the warp
 
-      const int kb = warp + k * W;
-      const int btok = tok0 + kb * 16;
-      const bool pvalid = tbl[btok / P - lp0] >= 0;
-      const uint32_t src = ring + (k % NSTAGE) * T::kStageBytes;
-      block_step<D>(lm, src, btok, tok_lo, tok1, pvalid, a.scale_log2, qa, t, acc);
-    }
-    cp_async_wait<0>();
-    __syncwarp();
+        const int kb = wr + k * W;
+        const int btok = r.tok0 + kb * 16;
+        const bool pvalid = tbl[r.tb + btok / P] >= 0;
+        const uint32_t src = ring + (k % NSTAGE) * T::kStageBytes;
+        block_step<D>(lm, src, btok, r.lo, r.hi, pvalid, a.scale_log2, qa, t, acc);
+      }
+      cp_async_wait<0>();
+      __syncwarp();
+    };
+    if (nsb > 0) pass(sinks_r);  // CTA-uniform: split 0's sinks first
+    pass(Range{tok0, nblk, tok_lo, tok1, nsp - lp0});
     // lane (g, t) ends with head g's max and its share of head g's
     // denominator, and O^T columns of heads 2t, 2t + 1
     float l_run = acc.l_run;
@@ -1089,14 +1100,12 @@ __global__ void __launch_bounds__(W * 32, kMinCtas<KVT>) decode_kernel(const Dec
     // 2 kp + 1, kp = warp + k W; a ring stage holds one pair
     constexpr int NPS = NSTAGE / 2;
     static_assert(NSTAGE % 2 == 0 && NPS >= 2, "quantised pools stage pairs of blocks");
-    const int npair = (nblk + 1) / 2;
-    const int npmine = npair > warp ? (npair - warp + W - 1) / W : 0;
-    auto issue_pair = [&](int kp, int st) {
+    auto issue_pair = [&](const Range &r, int kp, int st) {
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int kb = 2 * kp + u;
-        if (kb < nblk) {
-          issue(kb, 2 * st + u);
+        if (kb < r.nblk) {
+          issue(r, kb, 2 * st + u);
         } else {  // no such block: zero-fill the stage (codes and scales 0)
           issue_block<D, KVT>(lm, ring + (2 * st + u) * T::kStageBytes, kbase, vbase, sz_base,
                               (size_t)h * P, 16, 0, lane);
@@ -1109,30 +1118,41 @@ __global__ void __launch_bounds__(W * 32, kMinCtas<KVT>) decode_kernel(const Dec
     const float qz[2] = {__shfl_sync(0xffffffffu, qsum, 8 * t) * a.scale_log2,
                          __shfl_sync(0xffffffffu, qsum, 8 * t + 4) * a.scale_log2};
     const float kscale = kCodeScale<KVT> * a.scale_log2;
-#pragma unroll
-    for (int st = 0; st < NPS - 1; ++st) {
-      if (st < npmine) issue_pair(warp + st * W, st);
-      cp_async_commit();
-    }
-    auto loop = [&](auto pack_c) {
+    // one range through the warp's ring; the online softmax state carries over
+    auto pass = [&](auto pack_c, const Range &r) {
       constexpr bool kPack = decltype(pack_c)::value;
+      const int wr = warp;
+      const int npair = (r.nblk + 1) / 2;
+      const int npmine = npair > wr ? (npair - wr + W - 1) / W : 0;
+#pragma unroll
+      for (int st = 0; st < NPS - 1; ++st) {
+        if (st < npmine) issue_pair(r, wr + st * W, st);
+        cp_async_commit();
+      }
       for (int k = 0; k < npmine; ++k) {
         __syncwarp();
         {
           const int kn = k + NPS - 1;
-          if (kn < npmine) issue_pair(warp + kn * W, kn % NPS);
+          if (kn < npmine) issue_pair(r, wr + kn * W, kn % NPS);
           cp_async_commit();
         }
         cp_async_wait<NPS - 1>();
         __syncwarp();
 
-        const int kb = 2 * (warp + k * W);
-        const int btok[2] = {tok0 + kb * 16, tok0 + kb * 16 + 16};
-        const bool pvalid[2] = {tbl[btok[0] / P - lp0] >= 0,
-                                kb + 1 < nblk && tbl[btok[1] / P - lp0] >= 0};
+        const int kb = 2 * (wr + k * W);
+        const int btok[2] = {r.tok0 + kb * 16, r.tok0 + kb * 16 + 16};
+        const bool pvalid[2] = {tbl[r.tb + btok[0] / P] >= 0,
+                                kb + 1 < r.nblk && tbl[r.tb + btok[1] / P] >= 0};
         const uint32_t src = ring + (k % NPS) * 2 * T::kStageBytes;
-        pair_step<D, KVT, kPack>(lm, src, btok, pvalid, tok_lo, tok1, kscale, qz, qa, g, t, acc);
+        pair_step<D, KVT, kPack>(lm, src, btok, pvalid, r.lo, r.hi, kscale, qz, qa, g, t, acc);
       }
+      cp_async_wait<0>();
+      __syncwarp();
+    };
+    auto loop = [&](auto pack_c) {
+      constexpr bool kPack = decltype(pack_c)::value;
+      if (nsb > 0) pass(pack_c, sinks_r);  // CTA-uniform: split 0's sinks first
+      pass(pack_c, Range{tok0, nblk, tok_lo, tok1, nsp - lp0});
       if constexpr (kPack) {
         // high + low halves: lanes t < 2 end with the full O^T of heads 2t, 2t + 1
 #pragma unroll

@@ -87,3 +87,19 @@ def test_window_covering_the_context_equals_plain_decode():
     device_append(pool, w, bt)
     plain = pa_decode(pool, q, bt, ctx, w.scale).cpu().numpy().reshape(-1, w.D)
     assert np.abs(got - plain).max() <= 1e-5
+
+
+@pytest.mark.parametrize("name", ["bf16-p16", "int8", "int4"])
+@pytest.mark.parametrize("num_splits", [2, 3])
+def test_window_sinks_share_the_first_split(name, num_splits):
+    """The sinks are a second token range of split 0 (no split of their own):
+    with forced splits, ragged contexts put sequences where split 0 holds only
+    sinks, sinks plus window tokens, or where later splits are empty; every
+    row equals the oracle's Eq. 5 over exactly the kept tokens."""
+    w = CASES[name]()
+    for sinks, window in ((16, 40), (5, 300), (40, 17)):
+        got = _run(w, sinks, window, num_splits=num_splits)
+        ref, _ = oracle.paged_attention_window(oracle_pool(w), bits(w.q), w.block_tables,
+                                               w.context_lens, w.scale, sinks, window)
+        err = np.abs(got - ref).max()
+        assert np.all(np.isfinite(got)) and err <= TOL, (sinks, window, err)
