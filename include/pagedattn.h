@@ -331,7 +331,9 @@ int32_t pa_prefix_plan_splits(int64_t units, int32_t tiles, int32_t num_sms,
  *   sinks  : >= 0; tokens [0, min(sinks, ctx)) are always kept
  *   workspace : >= pa_decode_window_workspace_bytes(...), zero-filled before
  *               its first use, 256-byte aligned (NULL if that is 0)
- * Other arguments and behaviour as for pa_decode (bf16 and INT8 pools).
+ * Other arguments and behaviour as for pa_decode (bf16, INT8, FP8 and INT4
+ * pools). The sinks are a second token range of the first split, so one
+ * split per (sequence, KV head) needs no workspace.
  */
 size_t pa_decode_window_workspace_bytes(const pa_kv_pool_t *pool,
                                         int32_t num_seqs, int32_t num_q_heads,
