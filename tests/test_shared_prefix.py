@@ -96,3 +96,43 @@ def test_cascade_captured_in_a_cuda_graph_replays_the_eager_bits():
         assert torch.equal(out, eager)
     ref, _ = oracle_decode(w, oracle_pool(w))
     assert np.abs(out.cpu().numpy().reshape(-1, w.D) - ref).max() <= 2e-3
+
+
+def test_cascade_from_two_host_threads_on_two_streams():
+    """Two host threads run the forked cascade on their own streams, over the
+    same batch with their own outputs and workspaces, many calls each: every
+    output equals the single-thread result bit for bit (the fork and join
+    are serialised per device; each call's work stays inside its own stream's
+    order)."""
+    import threading
+    w, _ = W.prefix(B=20, prefix_tokens=320, suffix_range=(1, 120))
+    pool, bt, ctx, q = device_inputs(w)
+    device_append(pool, w, bt)
+    pre = torch.from_numpy(np.ascontiguousarray(w.notes["prefix_pages"])).to(DEV)
+    want = pa_decode_shared_prefix(pool, q, pre, w.notes["prefix_tokens"], bt, ctx, w.scale)
+    torch.cuda.synchronize()
+    need = pa_decode_shared_prefix_workspace_bytes(pool, w.B, w.Hq, bt.shape[1],
+                                                   w.notes["prefix_tokens"], 0)
+    errors = []
+
+    def worker():
+        try:
+            s = torch.cuda.Stream()
+            out = torch.zeros_like(want)
+            ws = torch.zeros(need, dtype=torch.uint8, device=DEV)
+            with torch.cuda.stream(s):
+                for _ in range(50):
+                    pa_decode_shared_prefix(pool, q, pre, w.notes["prefix_tokens"], bt, ctx,
+                                            w.scale, out=out, workspace=ws, stream=s)
+            s.synchronize()
+            if not torch.equal(out, want):
+                errors.append("mismatch")
+        except Exception as e:  # pragma: no cover - reported below
+            errors.append(repr(e))
+
+    threads = [threading.Thread(target=worker) for _ in range(2)]
+    for th in threads:
+        th.start()
+    for th in threads:
+        th.join()
+    assert not errors, errors
