@@ -317,9 +317,11 @@ def config_of(w, args, n, S):
 
 
 def run_ours(args, rank, world, local_rank):
+    import numpy as np
     import torch
     import torch.distributed as dist
     from paged_kv_cache_466_b200 import (KVPool, pa_decode, pa_decode_num_splits,
+                                         pa_decode_num_splits_lens,
                                          pa_decode_shared_prefix,
                                          pa_decode_shared_prefix_workspace_bytes,
                                          pa_decode_window, pa_decode_window_workspace_bytes,
@@ -343,7 +345,13 @@ def run_ours(args, rank, world, local_rank):
     sk, sv = w.step_k.to(dev), w.step_v.to(dev)
     sseq = torch.from_numpy(w.step_seq).to(dev)
     spos = torch.from_numpy(w.step_pos).to(dev)
-    S = pa_decode_num_splits(pool, w.B, w.max_pages, args.splits)
+    # the library schedules the fused step from the host's context lengths
+    # (pa_decode_append with host_context_lens), as a serving loop that knows
+    # them would; S is the split count that then runs
+    host_lens = np.ascontiguousarray(w.context_lens, dtype=np.int32)
+    fused_step = not (args.cascade or args.window > 0 or args.separate_append)
+    S = (pa_decode_num_splits_lens(pool, w.B, w.max_pages, host_lens, args.splits) if fused_step
+         else pa_decode_num_splits(pool, w.B, w.max_pages, args.splits))
     if args.cascade:
         pre_len = int(w.notes["prefix_tokens"])
         # the suffix decode's split count, planned over the suffix pages as the
@@ -394,7 +402,7 @@ def run_ours(args, rank, world, local_rank):
             if ev0 is not None:
                 ev0.record(stream)
             pa_decode_append(pl, q, kn, vn, bt, ctx, w.scale, out=out, workspace=ws,
-                             num_splits=S)
+                             num_splits=args.splits, host_context_lens=host_lens)
         else:
             pa_kv_append(pl, sk, sv, sseq, spos, bt)
             if ev0 is not None:

@@ -137,6 +137,57 @@ pa_status_t pa_kv_append(const pa_kv_pool_t *pool, const void *k_new,
                          int32_t max_pages, int32_t *d_err, void *stream);
 
 /*
+ * pa_decode_append_lens — pa_decode_append with the context lengths also given
+ * in host memory (host_context_lens: int32 [num_seqs], the values in
+ * context_lens as the host knows them, e.g. from a serving scheduler; may be
+ * NULL, which is pa_decode_append). With num_splits == 0 and num_seqs <= 256
+ * the split count comes from pa_decode_plan_lens: a ragged batch that needs
+ * several waves of CTAs runs one CTA per (sequence, KV head), launched
+ * longest context first, and then needs no workspace. Host values that
+ * differ from the device ones change only the schedule: the result is
+ * always Eq. 1 over the device's context_lens. Other arguments, layouts and
+ * errors as for pa_decode_append; a workspace sized as for pa_decode_append
+ * (pa_decode_workspace_bytes with pa_decode_num_splits' count) always
+ * suffices (the split count here is 1 or that count).
+ */
+pa_status_t pa_decode_append_lens(const pa_kv_pool_t *pool, const void *q,
+                                  const void *k_new, const void *v_new,
+                                  int32_t num_seqs, int32_t num_q_heads,
+                                  const int32_t *block_tables, int32_t max_pages,
+                                  const int32_t *context_lens,
+                                  const int32_t *host_context_lens, float scale,
+                                  float *out, void *workspace,
+                                  size_t workspace_bytes, int32_t num_splits,
+                                  int32_t *d_err, void *stream);
+
+/*
+ * pa_decode_num_splits_lens — the split count pa_decode_append_lens uses
+ * (pa_decode_plan_lens with this device's SM count and decode occupancy);
+ * pa_decode_num_splits when host_context_lens is NULL, requested > 0 or
+ * num_seqs > 256. Returns <= 0 on invalid arguments.
+ */
+int32_t pa_decode_num_splits_lens(const pa_kv_pool_t *pool, int32_t num_seqs,
+                                  int32_t max_pages,
+                                  const int32_t *host_context_lens,
+                                  int32_t requested);
+
+/*
+ * pa_decode_plan_lens — host only: the split count pa_decode_append_lens
+ * uses for num_seqs sequences of host_context_lens tokens (values clamped to
+ * [0, max_pages * page_size]) over num_kv_heads KV heads, on num_sms SMs
+ * holding ctas_per_sm decode CTAs each, and in order[0 .. num_seqs) the
+ * sequences longest first (ties by index). Returns 1 when the (sequence, KV
+ * head) units fill more than one wave of the planner's slots (num_sms x
+ * min(ctas_per_sm, 3)), the longest context is at least 1.3 x the mean and
+ * max_pages <= 2048; otherwise pa_decode_plan_splits' automatic count.
+ * Returns <= 0 on invalid arguments (num_seqs outside 1..256 included).
+ */
+int32_t pa_decode_plan_lens(const int32_t *host_context_lens, int32_t num_seqs,
+                            int32_t num_kv_heads, int32_t max_pages,
+                            int32_t page_size, int32_t num_sms,
+                            int32_t ctas_per_sm, uint16_t *order);
+
+/*
  * pa_decode_num_splits — the split-KV partition count S pa_decode uses for
  * this pool shape, table width and request. requested == 0 picks S from the
  * number of (sequence, KV head) units, the table width and how many decode

@@ -30,6 +30,7 @@ from __future__ import annotations
 import ctypes
 from typing import Optional
 
+import numpy as np
 import torch
 
 from . import _lib
@@ -51,7 +52,7 @@ __all__ = ["KVPool", "pa_kv_append", "pa_decode", "pa_decode_append", "pa_decode
            "PA_DERR_BAD_PAGE",
            "PA_DERR_BAD_CTX",
            "PA_DERR_BAD_SEQ", "PA_DERR_BAD_POS",
-           "load_library"]
+           "load_library", "pa_decode_num_splits_lens"]
 
 
 def load_library() -> ctypes.CDLL:
@@ -157,6 +158,14 @@ def pa_decode_num_splits(pool: KVPool, num_seqs: int, max_pages: int, requested:
     return s
 
 
+def pa_decode_num_splits_lens(pool: KVPool, num_seqs: int, max_pages: int, host_context_lens,
+                              requested: int = 0) -> int:
+    """The split count pa_decode_append with host_context_lens uses."""
+    hl = np.ascontiguousarray(np.asarray(host_context_lens, dtype=np.int32))
+    return int(_lib.load().pa_decode_num_splits_lens(ctypes.byref(pool.c), num_seqs, max_pages,
+                                                     hl.ctypes.data, requested))
+
+
 def pa_decode_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int,
                               num_splits: int) -> int:
     return int(_lib.load().pa_decode_workspace_bytes(num_seqs, num_q_heads, head_dim, num_splits))
@@ -221,10 +230,14 @@ def pa_decode_append(pool: KVPool, q: torch.Tensor, k_new: torch.Tensor, v_new: 
                      block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
                      out: Optional[torch.Tensor] = None,
                      workspace: Optional[torch.Tensor] = None, num_splits: int = 0,
-                     d_err: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                     d_err: Optional[torch.Tensor] = None, stream=None,
+                     host_context_lens=None) -> torch.Tensor:
     """One decode step in one launch: store k_new / v_new [B, Hkv, D] bf16 at
     position context_lens[b] - 1 of each sequence (as pa_kv_append would),
-    then Eq. 1 over tokens 0 .. context_lens[b] - 1 (as pa_decode)."""
+    then Eq. 1 over tokens 0 .. context_lens[b] - 1 (as pa_decode).
+    host_context_lens (optional, int32 numpy array or CPU tensor of the same
+    values) lets the library schedule the launch from the real lengths
+    (pa_decode_append_lens); the result does not depend on it."""
     dev = pool.device
     _need(q, "q", torch.bfloat16, dev)
     _need(k_new, "k_new", torch.bfloat16, dev)
@@ -245,6 +258,18 @@ def pa_decode_append(pool: KVPool, q: torch.Tensor, k_new: torch.Tensor, v_new: 
         if need > 0:
             workspace = torch.zeros(need, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if host_context_lens is not None:
+        hl = host_context_lens
+        if not (isinstance(hl, np.ndarray) and hl.dtype == np.int32 and hl.flags.c_contiguous):
+            hl = np.ascontiguousarray(np.asarray(hl, dtype=np.int32))
+        if hl.shape != (B,):
+            raise ValueError("pa_decode_append: host_context_lens must hold one length per sequence")
+        st = _lib.load().pa_decode_append_lens(
+            ctypes.byref(pool.c), _ptr(q), _ptr(k_new), _ptr(v_new), B, Hq, _ptr(block_tables),
+            max_pages, _ptr(context_lens), hl.ctypes.data, float(scale), _ptr(out),
+            _ptr(workspace), ws_bytes, num_splits, _ptr(d_err), _stream(stream))
+        _lib.check(st, "pa_decode_append_lens")
+        return out
     st = _lib.load().pa_decode_append(ctypes.byref(pool.c), _ptr(q), _ptr(k_new), _ptr(v_new), B,
                                       Hq, _ptr(block_tables), max_pages, _ptr(context_lens),
                                       float(scale), _ptr(out), _ptr(workspace), ws_bytes,

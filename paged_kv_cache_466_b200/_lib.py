@@ -59,8 +59,12 @@ SIGNATURES = {
     "pa_decode_auto_splits": (_I, [_I, _I, _I, _I]),
     "pa_decode_append": (_I, [_POOL, _P, _P, _P, _I, _I, _P, _I, _P, ctypes.c_float, _P, _P,
                               ctypes.c_size_t, _I, _P, _P]),
+    "pa_decode_append_lens": (_I, [_POOL, _P, _P, _P, _I, _I, _P, _I, _P, _P, ctypes.c_float, _P, _P,
+                              ctypes.c_size_t, _I, _P, _P]),
     "pa_decode_plan_splits": (_I, [ctypes.c_int64, _I, _I, _I, _I, _I]),
     "pa_prefix_plan_splits": (_I, [ctypes.c_int64, _I, _I, _I, ctypes.c_double]),
+    "pa_decode_plan_lens": (_I, [_P, _I, _I, _I, _I, _I, _I, _P]),
+    "pa_decode_num_splits_lens": (_I, [_POOL, _I, _I, _P, _I]),
     "pa_decode_num_splits": (_I, [_POOL, _I, _I, _I]),
     "pa_decode_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "pa_decode": (_I, [_POOL, _P, _I, _I, _P, _I, _P, ctypes.c_float, _P, _P, ctypes.c_size_t,

@@ -4,6 +4,7 @@
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
+#include <cstring>
 #include <mutex>
 #include <new>
 #include <string>
@@ -287,6 +288,56 @@ int32_t pa_decode_plan_splits(int64_t num_units, int32_t max_pages, int32_t page
   return (max_pages + chunk - 1) / chunk;
 }
 
+int32_t pa_decode_plan_lens(const int32_t *host_context_lens, int32_t num_seqs,
+                            int32_t num_kv_heads, int32_t max_pages, int32_t page_size,
+                            int32_t num_sms, int32_t ctas_per_sm, uint16_t *order) {
+  if (host_context_lens == nullptr || order == nullptr || num_seqs <= 0 ||
+      num_seqs > kMaxOrdered || num_kv_heads <= 0 || max_pages <= 0 || page_size <= 0 ||
+      num_sms <= 0 || ctas_per_sm <= 0)
+    return -1;
+  // the planner's slot count (its constants were measured with three decode
+  // CTAs per SM, see pa_decode_num_splits)
+  const int cps = ctas_per_sm < 3 ? ctas_per_sm : 3;
+  const long long units = (long long)num_seqs * num_kv_heads;
+  const int S_plan = pa_decode_plan_splits(units, max_pages, page_size, num_sms, cps, 0);
+  // longest context first, ties by index (a stable sort of the indices)
+  const long long cap = (long long)max_pages * page_size;
+  auto len = [&](int i) {
+    const long long c = host_context_lens[i];
+    return c < 0 ? 0LL : (c > cap ? cap : c);
+  };
+  for (int i = 0; i < num_seqs; ++i) order[i] = (uint16_t)i;
+  std::stable_sort(order, order + num_seqs,
+                   [&](uint16_t x, uint16_t y) { return len(x) > len(y); });
+  long long sum = 0;
+  for (int i = 0; i < num_seqs; ++i) sum += len(i);
+  const long long longest = len(order[0]);
+  // Several waves of a ragged batch: one CTA per (sequence, KV head),
+  // launched longest first, so the short ones fill the last wave. Measured on
+  // the ragged Llama-3-8B-shaped step (contexts 242..4095, longest / mean =
+  // 1.9): INT8 63.7 us against 70.9 at four splits, FP8 64.3 / 72.0, INT4
+  // 57.7 / 62.0, bf16 96.7 / 98.6. Uniform batches keep the planner's splits:
+  // one split per unit just over one wave was 11-21 % slower there.
+  const bool several_waves = units >= (long long)num_sms * cps;
+  const bool ragged = longest * 10 * num_seqs >= sum * 13;  // longest >= 1.3 x mean
+  if (several_waves && ragged && max_pages <= kMaxPagesPerSplit) return 1;
+  return S_plan;
+}
+
+int32_t pa_decode_num_splits_lens(const pa_kv_pool_t *pool, int32_t num_seqs,
+                                  int32_t max_pages, const int32_t *host_context_lens,
+                                  int32_t requested) {
+  if (host_context_lens == nullptr || requested != 0 || num_seqs <= 0 || num_seqs > kMaxOrdered ||
+      pool == nullptr)
+    return pa_decode_num_splits(pool, num_seqs, max_pages, requested);
+  if (pa_decode_num_splits(pool, num_seqs, max_pages, 0) <= 0) return -1;  // argument checks
+  uint16_t order[kMaxOrdered];
+  return pa_decode_plan_lens(host_context_lens, num_seqs, pool->num_kv_heads, max_pages,
+                             pool->page_size, device_sm_count(),
+                             cached_ctas_per_sm(pool->head_dim, pool->page_size, pool->dtype),
+                             order);
+}
+
 int32_t pa_decode_num_splits(const pa_kv_pool_t *pool, int32_t num_seqs, int32_t max_pages,
                              int32_t requested) {
   if (pool == nullptr || num_seqs < 0 || max_pages <= 0 || requested < 0) return -1;
@@ -338,7 +389,8 @@ pa_status_t decode_impl(const pa_kv_pool_t *pool, const void *q, int32_t num_seq
                         int32_t num_q_heads, const int32_t *block_tables, int32_t max_pages,
                         const int32_t *context_lens, float scale, float *out, void *workspace,
                         size_t workspace_bytes, int32_t num_splits, int32_t *d_err,
-                        void *stream, const void *k_new, const void *v_new) {
+                        void *stream, const void *k_new, const void *v_new,
+                        const int32_t *host_lens = nullptr) {
   g_last_error.clear();
   pa_status_t st = check_pool(pool);
   if (st != PA_OK) return st;
@@ -361,7 +413,19 @@ pa_status_t decode_impl(const pa_kv_pool_t *pool, const void *q, int32_t num_seq
     return fail(PA_ERR_INVALID_ARG, "q, block_tables, context_lens and out are required");
   if (!aligned(q, 16) || !aligned(out, 16))
     return fail(PA_ERR_INVALID_ARG, "q and out must be 16-byte aligned");
-  const int S = pa_decode_num_splits(pool, num_seqs, max_pages, num_splits);
+  // with host context lengths (and automatic splits) the lengths choose the
+  // split count and, for one split, a longest-first launch order
+  uint16_t order[kMaxOrdered];
+  int S = 0;
+  bool ordered = false;
+  if (host_lens != nullptr && num_splits == 0 && num_seqs <= kMaxOrdered) {
+    S = pa_decode_plan_lens(host_lens, num_seqs, pool->num_kv_heads, max_pages, pool->page_size,
+                            device_sm_count(),
+                            cached_ctas_per_sm(pool->head_dim, pool->page_size, pool->dtype),
+                            order);
+    ordered = S == 1;
+  }
+  if (S <= 0) S = pa_decode_num_splits(pool, num_seqs, max_pages, num_splits);
   if (S <= 0) return fail(PA_ERR_INVALID_ARG, "could not plan splits");
   const int chunk = (max_pages + S - 1) / S;
   const size_t rows = (size_t)num_seqs * num_q_heads;
@@ -413,6 +477,9 @@ pa_status_t decode_impl(const pa_kv_pool_t *pool, const void *q, int32_t num_seq
   a.d_err = d_err;
   a.k_new = static_cast<const unsigned char *>(k_new);
   a.v_new = static_cast<const unsigned char *>(v_new);
+  a.ordered = ordered ? 1 : 0;
+  if (ordered)
+    for (int i = 0; i < num_seqs; ++i) a.order[i] = (uint8_t)order[i];
   return cuda_status(launch_decode(pool->head_dim, pool->page_size, pool->dtype, a,
                                    static_cast<cudaStream_t>(stream)),
                      k_new ? "pa_decode_append launch" : "pa_decode launch");
@@ -444,6 +511,24 @@ pa_status_t pa_decode_append(const pa_kv_pool_t *pool, const void *q, const void
   return decode_impl(pool, q, num_seqs, num_q_heads, block_tables, max_pages, context_lens,
                      scale, out, workspace, workspace_bytes, num_splits, d_err, stream,
                      num_seqs > 0 ? k_new : nullptr, num_seqs > 0 ? v_new : nullptr);
+}
+
+pa_status_t pa_decode_append_lens(const pa_kv_pool_t *pool, const void *q, const void *k_new,
+                                  const void *v_new, int32_t num_seqs, int32_t num_q_heads,
+                                  const int32_t *block_tables, int32_t max_pages,
+                                  const int32_t *context_lens,
+                                  const int32_t *host_context_lens, float scale, float *out,
+                                  void *workspace, size_t workspace_bytes, int32_t num_splits,
+                                  int32_t *d_err, void *stream) {
+  g_last_error.clear();
+  if (num_seqs > 0 && (k_new == nullptr || v_new == nullptr))
+    return fail(PA_ERR_INVALID_ARG, "k_new and v_new are required");
+  if (!aligned(k_new, 16) || !aligned(v_new, 16))
+    return fail(PA_ERR_INVALID_ARG, "k_new/v_new must be 16-byte aligned");
+  return decode_impl(pool, q, num_seqs, num_q_heads, block_tables, max_pages, context_lens,
+                     scale, out, workspace, workspace_bytes, num_splits, d_err, stream,
+                     num_seqs > 0 ? k_new : nullptr, num_seqs > 0 ? v_new : nullptr,
+                     host_context_lens);
 }
 
 // ---------------------------------------------------------------- shared prefix
@@ -846,18 +931,22 @@ pa_status_t pa_decode_step_host(const pa_kv_pool_t *pool, const void *packet_hos
   char *pd = static_cast<char *>(packet_dev);
   const int32_t *tables = reinterpret_cast<const int32_t *>(pd + off[5]);
   const int32_t *ctx = reinterpret_cast<const int32_t *>(pd + off[6]);
+  // the packet's context lengths are on the host too: they schedule the launch
+  const int32_t *host_ctx =
+      reinterpret_cast<const int32_t *>(static_cast<const char *>(packet_host) + off[6]);
   if (num_new == PA_STEP_NEWEST_PER_SEQ) {  // cache write fused into the decode
-    st = pa_decode_append(pool, pd + off[0], pd + off[1], pd + off[2], num_seqs, num_q_heads,
-                          tables, max_pages, ctx, scale, out_dev, workspace, workspace_bytes,
-                          num_splits, d_err, stream);
+    st = pa_decode_append_lens(pool, pd + off[0], pd + off[1], pd + off[2], num_seqs,
+                               num_q_heads, tables, max_pages, ctx, host_ctx, scale, out_dev,
+                               workspace, workspace_bytes, num_splits, d_err, stream);
   } else {
     st = pa_kv_append(pool, pd + off[1], pd + off[2],
                       reinterpret_cast<const int32_t *>(pd + off[3]),
                       reinterpret_cast<const int32_t *>(pd + off[4]), num_new, tables, num_seqs,
                       max_pages, d_err, stream);
     if (st == PA_OK)
-      st = pa_decode(pool, pd + off[0], num_seqs, num_q_heads, tables, max_pages, ctx, scale,
-                     out_dev, workspace, workspace_bytes, num_splits, d_err, stream);
+      st = decode_impl(pool, pd + off[0], num_seqs, num_q_heads, tables, max_pages, ctx, scale,
+                       out_dev, workspace, workspace_bytes, num_splits, d_err, stream, nullptr,
+                       nullptr, host_ctx);
   }
   if (st != PA_OK || num_seqs == 0) return st;
   st = cuda_status(cudaMemcpyAsync(out_host, out_dev,

@@ -868,7 +868,7 @@ __global__ void __launch_bounds__(W * 32, kMinCtas<KVT>) decode_kernel(const Dec
 
   const int split = blockIdx.x;
   const int h = blockIdx.y;
-  const int b = blockIdx.z;
+  const int b = a.ordered ? (int)a.order[blockIdx.z] : (int)blockIdx.z;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2;

@@ -10,6 +10,10 @@
 
 namespace pa {
 
+// Most sequences a longest-first launch order can name (the order travels as
+// a kernel parameter of one byte per sequence).
+constexpr int kMaxOrdered = 256;
+
 // Largest GQA group a decode CTA serves (query heads per KV head).
 constexpr int kMaxGroup = 8;
 // Page-table entries one decode CTA stages in shared memory; a split covers at
@@ -52,6 +56,10 @@ struct DecodeArgs {
   int32_t range_mode;       // 1: a context shorter than tok_begin is an empty range,
                             //    not an error
   int32_t *d_err;
+  // 1: blockIdx.z is a launch rank and order[rank] the sequence it serves
+  // (longest context first); 0: blockIdx.z is the sequence
+  int32_t ordered = 0;
+  uint8_t order[kMaxOrdered];
   // fused cache write (pa_decode_append): bf16 [B][Hkv][D] rows of each
   // sequence's newest token, stored at position ctx - 1 before it is read
   const unsigned char *k_new = nullptr;

@@ -4,6 +4,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 from paged_kv_cache_466_b200 import _lib
@@ -242,6 +243,66 @@ def test_prefix_plan_invariants_for_any_shape(lib):
         assert 1 <= tp <= tiles and -(-tiles // tp) <= 256
         tp2 = lib.pa_prefix_plan_splits(units, tiles, sms, cps, mb * 1e6 * more)
         assert -(-tiles // tp2) <= -(-tiles // tp)
+
+    check()
+
+
+def _plan_lens(lib, lens, hkv=8, max_pages=256, P=16, sms=148, cps=3):
+    lens = np.ascontiguousarray(lens, dtype=np.int32)
+    order = np.zeros(max(len(lens), 1), dtype=np.uint16)
+    S = lib.pa_decode_plan_lens(lens.ctypes.data, len(lens), hkv, max_pages, P, sms, cps,
+                                order.ctypes.data)
+    return S, order[:len(lens)]
+
+
+def test_length_aware_plan_on_a_b200(lib):
+    """pa_decode_plan_lens with the B200's 148 SMs: a ragged batch that needs
+    several waves (64 x 8 = 512 units for 444 slots, contexts 242..4095 as in
+    the Llama-3-8B-shaped bench batch) runs one split, longest first; a
+    uniform one, a batch that fits one wave, and tables longer than one split
+    can stage keep the planner's count."""
+    rng = np.random.default_rng(0)
+    ragged = rng.integers(242, 4096, 64)
+    S, order = _plan_lens(lib, ragged)
+    assert S == 1
+    assert sorted(order.tolist()) == list(range(64))
+    assert all(ragged[order[i]] >= ragged[order[i + 1]] for i in range(63))
+    uniform = np.full(64, 4095)
+    assert _plan_lens(lib, uniform)[0] == lib.pa_decode_plan_splits(512, 256, 16, 148, 3, 0) == 4
+    assert _plan_lens(lib, ragged[:32])[0] == lib.pa_decode_plan_splits(256, 256, 16, 148, 3, 0)
+    assert _plan_lens(lib, ragged, max_pages=4096)[0] == \
+        lib.pa_decode_plan_splits(512, 4096, 16, 148, 3, 0)
+    # four CTAs per SM are planned as three (the planner's calibration)
+    assert _plan_lens(lib, ragged, cps=4)[0] == 1
+    # ties keep index order; values are clamped to the table
+    S, order = _plan_lens(lib, [5, 7, 7, 1 << 30, -3])
+    assert order.tolist() == [3, 1, 2, 0, 4]
+    bad = np.zeros(4, dtype=np.int32)
+    o = np.zeros(4, dtype=np.uint16)
+    assert lib.pa_decode_plan_lens(None, 4, 8, 256, 16, 148, 3, o.ctypes.data) <= 0
+    assert lib.pa_decode_plan_lens(bad.ctypes.data, 0, 8, 256, 16, 148, 3, o.ctypes.data) <= 0
+    big = np.zeros(257, dtype=np.int32)
+    ob = np.zeros(257, dtype=np.uint16)
+    assert lib.pa_decode_plan_lens(big.ctypes.data, 257, 8, 256, 16, 148, 3, ob.ctypes.data) <= 0
+
+
+def test_length_aware_plan_invariants(lib):
+    """Any lengths: the order is a permutation sorted longest first (ties by
+    index), and the count is 1 or the planner's automatic count."""
+    from hypothesis import given, settings, strategies as st
+
+    @settings(max_examples=300, deadline=None)
+    @given(lens=st.lists(st.integers(-10, 100000), min_size=1, max_size=256),
+           hkv=st.integers(1, 16), pages=st.integers(1, 3000), sms=st.integers(1, 200),
+           cps=st.integers(1, 6))
+    def check(lens, hkv, pages, sms, cps):
+        S, order = _plan_lens(lib, lens, hkv=hkv, max_pages=pages, sms=sms, cps=cps)
+        assert S in (1, lib.pa_decode_plan_splits(len(lens) * hkv, pages, 16, sms, min(cps, 3), 0))
+        assert sorted(order.tolist()) == list(range(len(lens)))
+        clamp = [min(max(x, 0), pages * 16) for x in lens]
+        for i in range(len(lens) - 1):
+            a, b = order[i], order[i + 1]
+            assert clamp[a] > clamp[b] or (clamp[a] == clamp[b] and a < b)
 
     check()
 

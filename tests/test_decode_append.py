@@ -103,3 +103,27 @@ def test_fused_step_with_rows_of_huge_span(kind):
         e = np.abs(g - ref).max()
         print(f"{kind} span {span:.0e}: max |gpu - oracle| = {e:.3e}")
         assert e <= 2e-6 * span + 2e-3
+
+
+@pytest.mark.parametrize("kv", ["bf16", "u8", "fp8", "u4"])
+def test_host_lengths_schedule_the_step_without_changing_it(kv):
+    """pa_decode_append with host_context_lens: a ragged batch over several
+    waves (64 sequences x 8 KV heads for 444 slots) runs one split, longest
+    context first. The output equals the one-split step bit for bit (the same
+    CTAs, launched in another order) and the oracle within 2e-3; host lengths
+    that are wrong (reversed) change only the schedule."""
+    w = W.llama8b(B=64, ctx_range=(242, 4095), kv=kv,
+                  outlier_frac=0.01 if kv != "bf16" else 0.0)
+    k_new, v_new = w.step_rows_by_sequence()
+    outs = []
+    for lens, splits in ((w.context_lens, 0), (w.context_lens[::-1], 0), (None, 1)):
+        pool, bt, ctx, q = device_inputs(w)
+        device_append(pool, w, bt, rows="prefill")
+        outs.append(pa_decode_append(pool, q, k_new.to(DEV), v_new.to(DEV), bt, ctx, w.scale,
+                                     num_splits=splits, host_context_lens=lens))
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0], outs[2])
+    ref, _ = oracle.paged_attention(oracle_pool(w), bits(w.q), w.block_tables, w.context_lens,
+                                    w.scale)
+    for o in outs[:2]:
+        assert np.abs(o.cpu().numpy().reshape(ref.shape) - ref).max() <= 2e-3
