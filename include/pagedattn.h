@@ -313,14 +313,16 @@ pa_status_t pa_decode_append(const pa_kv_pool_t *pool, const void *q,
  * K/V row once per 128 query rows instead of once per request; (2) the paged
  * decode over each request's own tokens [prefix_len, context_lens[b]),
  * writing its split partials; (3) the log-sum-exp merge of (2) and (1) per
- * row, in that order (deterministic). (1) runs on `stream` and (2) on a
- * second stream the library keeps per device, forked from `stream` before
- * (1) and joined back before (3), so the prefix pass (tensor-core and L2
- * bound) overlaps the suffix decode (HBM bound); the split count of (1) is
- * pa_prefix_plan_splits'. The call stays one unit of `stream` (all three
- * complete before later work on it; it can be captured in a CUDA graph, the
- * fork and join becoming graph edges). Calls from several host threads are
- * serialised around the fork.
+ * row, in that order (deterministic). (1) and (2) run side by side, so the
+ * prefix pass (tensor-core and L2 bound) overlaps the suffix decode (HBM
+ * bound); the split count of (1) is pa_prefix_plan_splits'. Called eagerly,
+ * all three run on `stream` as programmatic dependent launches ((1) lets (2)
+ * start once the work before the call has finished; (3) starts after both).
+ * While `stream` is being captured into a CUDA graph, (2) runs on a second
+ * stream the library keeps per device, forked from `stream` before (1) and
+ * joined back before (3) (the fork and join become graph edges; calls from
+ * several host threads are serialised around the fork). Either way the call
+ * is one unit of `stream`: all three complete before later work on it.
  *
  *   prefix_pages : (device) int32 [prefix_len / P] physical pages of the prefix
  *   prefix_len   : tokens in the prefix; a multiple of the page size (0 falls

@@ -535,8 +535,9 @@ pa_status_t pa_decode_append_lens(const pa_kv_pool_t *pool, const void *q, const
 namespace {
 
 // The cascade's second stream and its fork and join events, per device,
-// created on first use (a device whose creation failed runs the three
-// launches on the caller's stream). g_fork_mu serialises the fork sequence.
+// created on first use, for calls captured into a CUDA graph (a device whose
+// creation failed runs the three launches on the caller's stream).
+// g_fork_mu serialises the fork sequence.
 struct Fork {
   cudaStream_t s2 = nullptr;
   cudaEvent_t forked = nullptr, joined = nullptr;
@@ -714,20 +715,35 @@ pa_status_t pa_decode_shared_prefix(const pa_kv_pool_t *pool, const void *q, int
   a.sinks = 0;
   a.tok_begin = prefix_len;
   a.d_err = d_err;
-  // Three launches: the prefix pass on `stream`; the suffix decode, which
-  // writes its split partials (an empty split writes lse = -inf) instead of
-  // merging, on the second stream (forked after the work already on
-  // `stream`, the prefix pass launched first so that its CTAs are placed
-  // first); then, joined back on `stream`, one merge of the suffix splits and
-  // the prefix splits per row, with its loads batched (a decode CTA merging
-  // prefix partials in its epilogue measured slower).
+  // Three launches: the prefix pass, the suffix decode (which writes its split
+  // partials, an empty split lse = -inf, instead of merging), then one merge
+  // of the suffix splits and the prefix splits per row with its loads batched
+  // (a decode CTA merging prefix partials in its epilogue measured slower).
+  // The prefix pass and the decode run side by side, the prefix CTAs placed
+  // first. Called eagerly, all three go on `stream`, each a programmatic
+  // dependent of the one before: the prefix pass releases the decode as soon
+  // as its own wait for the earlier work returns, and the decode's last CTA
+  // waits for the prefix pass, so the merge follows both with no event
+  // between streams. Captured into a CUDA graph, the decode goes on a second
+  // stream forked from `stream` and joined back before the merge: there the
+  // fork and join are graph edges, and the two branches start at once.
   a.prior_o = nullptr;
   a.prior_lse = nullptr;
   a.n_prior = 0;
   a.keep_partials = 1;
   a.tok_end = 0x7fffffff;
   a.range_mode = 0;
-  {
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  st = cuda_status(cudaStreamIsCapturing(s, &cap), "pa_decode_shared_prefix capture query");
+  if (st != PA_OK) return st;
+  if (cap == cudaStreamCaptureStatusNone) {
+    a.pdl_defer = 1;
+    st = cuda_status(launch_prefix(pool->head_dim, pool->page_size, pa, true, s),
+                     "pa_decode_shared_prefix prefix launch");
+    if (st == PA_OK)
+      st = cuda_status(launch_decode(pool->head_dim, pool->page_size, pool->dtype, a, s),
+                       "pa_decode_shared_prefix suffix launch");
+  } else {
     std::lock_guard<std::mutex> lock(g_fork_mu);
     Fork *f = fork_for_device();
     if (f != nullptr) {

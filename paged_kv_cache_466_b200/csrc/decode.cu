@@ -864,7 +864,13 @@ __global__ void __launch_bounds__(W * 32, kMinCtas<KVT>) decode_kernel(const Dec
 
   // Launched as a programmatic dependent: wait until the previous kernel on
   // the stream (e.g. the cache write) has finished and its writes are visible.
-  pdl_wait_primary();
+  // Behind the cascade's prefix pass, which releases its dependents only after
+  // its own wait for the work before it, nothing this grid reads is still
+  // being written: one CTA (the last launched) waits, so that a kernel after
+  // this grid also finds the prefix pass finished.
+  if (!a.pdl_defer || (blockIdx.x == gridDim.x - 1 && blockIdx.y == gridDim.y - 1 &&
+                       blockIdx.z == gridDim.z - 1))
+    pdl_wait_primary();
 
   const int split = blockIdx.x;
   const int h = blockIdx.y;

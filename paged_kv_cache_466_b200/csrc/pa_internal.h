@@ -56,6 +56,10 @@ struct DecodeArgs {
   int32_t range_mode;       // 1: a context shorter than tok_begin is an empty range,
                             //    not an error
   int32_t *d_err;
+  // 1: launched as a programmatic dependent of a kernel whose output this
+  // grid does not read (the cascade's prefix pass): only the grid's last CTA
+  // waits for it, so the grid still ends after it
+  int32_t pdl_defer = 0;
   // 1: blockIdx.z is a launch rank and order[rank] the sequence it serves
   // (longest context first); 0: blockIdx.z is the sequence
   int32_t ordered = 0;

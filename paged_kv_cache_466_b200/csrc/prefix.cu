@@ -181,6 +181,9 @@ __global__ void __launch_bounds__(kThreads, 2)
   // the swizzled tiles need 1024-byte aligned atoms
   unsigned char *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   pdl_wait_primary();
+  // the work before this pass is finished and visible: the suffix decode,
+  // which does not read this pass's output, may start beside it now
+  pdl_launch_dependents();
 
   const int mt = blockIdx.x;
   const int h = blockIdx.y;
