@@ -6,7 +6,7 @@ import pytest
 import torch
 
 from paged_kv_cache_466_b200 import (pa_decode, pa_decode_shared_prefix,
-                                     pa_decode_shared_prefix_workspace_bytes)
+                                     pa_decode_shared_prefix_workspace_bytes, pa_kv_append)
 from paged_kv_cache_466_b200 import workloads as W
 from tests.helpers import (DEV, device_append, device_inputs, full_size_reference,
                            oracle_decode, oracle_pool)
@@ -68,10 +68,38 @@ def test_cascade_full_size_prefix_workload():
     assert np.abs(casc - plain).max() <= 1e-4
 
 
+def test_cascade_reads_rows_appended_just_before_it():
+    """The suffix decode skips its own programmatic wait (only the prefix pass
+    waits for the work before the call): rows that pa_kv_append writes right
+    before the call, on the same stream with nothing between, must still be
+    read. Unwritten slots hold the byte 0xFF (bf16 NaN), so a read that beat
+    the append would show; the suffixes are a few tokens, the newest one a
+    large part of each."""
+    w, _ = W.prefix(B=24, prefix_tokens=128, suffix_range=(1, 6))
+    pool, bt, ctx, q = device_inputs(w, fill_byte=0xFF)
+    pre = torch.from_numpy(np.ascontiguousarray(w.notes["prefix_pages"])).to(DEV)
+    ref, _ = oracle_decode(w, oracle_pool(w))
+    sk, sv = w.step_k.to(DEV), w.step_v.to(DEV)
+    sseq, spos = torch.from_numpy(w.step_seq).to(DEV), torch.from_numpy(w.step_pos).to(DEV)
+    for it in range(3):
+        for t in (pool.k, pool.v):
+            t.view(torch.uint8).fill_(0xFF)
+        device_append(pool, w, bt, rows="prefill")
+        torch.cuda.synchronize()
+        pa_kv_append(pool, sk, sv, sseq, spos, bt)  # the newest rows, then at once:
+        out = pa_decode_shared_prefix(pool, q, pre, w.notes["prefix_tokens"], bt, ctx, w.scale)
+        torch.cuda.synchronize()
+        got = out.cpu().numpy().reshape(-1, w.D)
+        assert np.all(np.isfinite(got)), f"call {it}: a row was read before the append wrote it"
+        err = np.abs(got - ref).max()
+        assert err <= 2e-3, f"call {it}: max |gpu - oracle| = {err:.3e}"
+
+
 def test_cascade_captured_in_a_cuda_graph_replays_the_eager_bits():
-    """The prefix pass and the suffix decode run on two streams (forked from
-    and joined back to the caller's stream); captured in a CUDA graph, the
-    call replays to the eager call's bits, twice in a row."""
+    """Called eagerly, the prefix pass, the suffix decode and the merge are one
+    chain of programmatic launches on the caller's stream; captured in a CUDA
+    graph, the suffix decode is a branch forked from and joined back to it.
+    The graph replays to the eager call's bits, twice in a row."""
     w, _ = W.prefix(B=33, prefix_tokens=1008, suffix_range=(1, 200))
     pool, bt, ctx, q = device_inputs(w)
     device_append(pool, w, bt)
@@ -99,11 +127,10 @@ def test_cascade_captured_in_a_cuda_graph_replays_the_eager_bits():
 
 
 def test_cascade_from_two_host_threads_on_two_streams():
-    """Two host threads run the forked cascade on their own streams, over the
-    same batch with their own outputs and workspaces, many calls each: every
-    output equals the single-thread result bit for bit (the fork and join
-    are serialised per device; each call's work stays inside its own stream's
-    order)."""
+    """Two host threads run the cascade on their own streams, over the same
+    batch with their own outputs and workspaces, many calls each: every output
+    equals the single-thread result bit for bit (each call's launches stay
+    inside its own stream's order)."""
     import threading
     w, _ = W.prefix(B=20, prefix_tokens=320, suffix_range=(1, 120))
     pool, bt, ctx, q = device_inputs(w)
