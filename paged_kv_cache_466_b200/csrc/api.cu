@@ -417,13 +417,16 @@ pa_status_t decode_impl(const pa_kv_pool_t *pool, const void *q, int32_t num_seq
   // split count and, for one split, a longest-first launch order
   uint16_t order[kMaxOrdered];
   int S = 0;
-  bool ordered = false;
+  int ordered = 0;  // 1: longest first; 2: and the units fill several waves
   if (host_lens != nullptr && num_splits == 0 && num_seqs <= kMaxOrdered) {
+    const int cps = cached_ctas_per_sm(pool->head_dim, pool->page_size, pool->dtype);
     S = pa_decode_plan_lens(host_lens, num_seqs, pool->num_kv_heads, max_pages, pool->page_size,
-                            device_sm_count(),
-                            cached_ctas_per_sm(pool->head_dim, pool->page_size, pool->dtype),
-                            order);
-    ordered = S == 1;
+                            device_sm_count(), cps, order);
+    if (S == 1)
+      ordered = (long long)num_seqs * pool->num_kv_heads >=
+                        (long long)device_sm_count() * (cps < 3 ? cps : 3)
+                    ? 2
+                    : 1;
   }
   if (S <= 0) S = pa_decode_num_splits(pool, num_seqs, max_pages, num_splits);
   if (S <= 0) return fail(PA_ERR_INVALID_ARG, "could not plan splits");
@@ -477,7 +480,7 @@ pa_status_t decode_impl(const pa_kv_pool_t *pool, const void *q, int32_t num_seq
   a.d_err = d_err;
   a.k_new = static_cast<const unsigned char *>(k_new);
   a.v_new = static_cast<const unsigned char *>(v_new);
-  a.ordered = ordered ? 1 : 0;
+  a.ordered = ordered;
   if (ordered)
     for (int i = 0; i < num_seqs; ++i) a.order[i] = (uint8_t)order[i];
   return cuda_status(launch_decode(pool->head_dim, pool->page_size, pool->dtype, a,

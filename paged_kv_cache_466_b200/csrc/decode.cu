@@ -63,6 +63,9 @@
 #ifndef PA_DECODE_STAGES_U8
 #define PA_DECODE_STAGES_U8 4
 #endif
+#ifndef PA_DECODE_STAGES_BF16_LPT  // bf16 launched longest unit first (see launch_t)
+#define PA_DECODE_STAGES_BF16_LPT 3
+#endif
 #ifndef PA_DECODE_MIN_CTAS
 #define PA_DECODE_MIN_CTAS 3
 #endif
@@ -1272,12 +1275,14 @@ __global__ void __launch_bounds__(W * 32, kMinCtas<KVT>) decode_kernel(const Dec
   if (threadIdx.x == 0) a.counters[(size_t)b * a.hkv + h] = 0;
 }
 
-template <int D, int P, int KVT>
+template <int D, int P, int KVT,
+          int NS = KVT != PA_KV_BF16 ? PA_DECODE_STAGES_U8 : PA_DECODE_STAGES_BF16>
 struct Config {
   static constexpr int W = PA_DECODE_WARPS;
-  static constexpr int NSTAGE = KVT != PA_KV_BF16 ? PA_DECODE_STAGES_U8 : PA_DECODE_STAGES_BF16;
+  static constexpr int NSTAGE = NS;
   using SM = Smem<D, KVT, W, NSTAGE>;
-  static void *fn() { return reinterpret_cast<void *>(&decode_kernel<D, P, KVT, W, NSTAGE>); }
+  static auto kernel() { return &decode_kernel<D, P, KVT, W, NSTAGE>; }
+  static void *fn() { return reinterpret_cast<void *>(kernel()); }
 };
 
 // Largest dynamic shared memory a decode CTA may request (ring + table slice).
@@ -1300,9 +1305,8 @@ cudaError_t ensure_smem_attr() {
   return e;
 }
 
-template <int D, int P, int KVT>
-cudaError_t launch_t(const DecodeArgs &a, cudaStream_t stream) {
-  using C = Config<D, P, KVT>;
+template <class C>
+cudaError_t launch_cfg(const DecodeArgs &a, cudaStream_t stream) {
   cudaError_t e = ensure_smem_attr<C>();
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -1315,7 +1319,21 @@ cudaError_t launch_t(const DecodeArgs &a, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = PA_DECODE_PDL ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<D, P, KVT, C::W, C::NSTAGE>, a);
+  return cudaLaunchKernelEx(&cfg, C::kernel(), a);
+}
+
+template <int D, int P, int KVT>
+cudaError_t launch_t(const DecodeArgs &a, cudaStream_t stream) {
+  // A ragged batch launched longest unit first over several waves of CTAs
+  // (ordered == 2) runs one CTA per (sequence, KV head), each streaming its
+  // whole unit: there a
+  // bf16 ring of three blocks per warp (two CTAs per SM) measured 3 % faster
+  // than two blocks (three CTAs per SM) on the Llama-3-8B-shaped step, and
+  // 5 % slower on one wave of equal units (the Llama-3-70B step), which keeps
+  // two.
+  if constexpr (KVT == PA_KV_BF16)
+    if (a.ordered == 2) return launch_cfg<Config<D, P, KVT, PA_DECODE_STAGES_BF16_LPT>>(a, stream);
+  return launch_cfg<Config<D, P, KVT>>(a, stream);
 }
 
 template <int D, int P, int KVT>

@@ -61,7 +61,9 @@ struct DecodeArgs {
   // waits for it, so the grid still ends after it
   int32_t pdl_defer = 0;
   // 1: blockIdx.z is a launch rank and order[rank] the sequence it serves
-  // (longest context first); 0: blockIdx.z is the sequence
+  // (longest context first); 2: the same, the units filling several waves of
+  // CTAs (the launch may then pick a deeper ring); 0: blockIdx.z is the
+  // sequence
   int32_t ordered = 0;
   uint8_t order[kMaxOrdered];
   // fused cache write (pa_decode_append): bf16 [B][Hkv][D] rows of each
