@@ -66,6 +66,9 @@
 #ifndef PA_DECODE_STAGES_BF16_LPT  // bf16 launched longest unit first (see launch_t)
 #define PA_DECODE_STAGES_BF16_LPT 3
 #endif
+#ifndef PA_DECODE_STAGES_U8_LPT  // INT8 / FP8 launched longest unit first
+#define PA_DECODE_STAGES_U8_LPT 6
+#endif
 #ifndef PA_DECODE_MIN_CTAS
 #define PA_DECODE_MIN_CTAS 3
 #endif
@@ -1326,13 +1329,16 @@ template <int D, int P, int KVT>
 cudaError_t launch_t(const DecodeArgs &a, cudaStream_t stream) {
   // A ragged batch launched longest unit first over several waves of CTAs
   // (ordered == 2) runs one CTA per (sequence, KV head), each streaming its
-  // whole unit: there a
-  // bf16 ring of three blocks per warp (two CTAs per SM) measured 3 % faster
-  // than two blocks (three CTAs per SM) on the Llama-3-8B-shaped step, and
-  // 5 % slower on one wave of equal units (the Llama-3-70B step), which keeps
-  // two.
+  // whole unit: there deeper rings (two CTAs per SM instead of three) pay.
+  // Measured on the Llama-3-8B-shaped step: bf16 with three blocks per warp
+  // instead of two 2-6 % faster (and 5 % slower on one wave of equal units,
+  // the Llama-3-70B step, which keeps two); INT8 and FP8 with three pairs
+  // instead of two 0.7-2.7 % faster on two B200s, 0.5 % slower on a third.
+  // INT4 keeps its ring (four CTAs per SM fit only with it).
   if constexpr (KVT == PA_KV_BF16)
     if (a.ordered == 2) return launch_cfg<Config<D, P, KVT, PA_DECODE_STAGES_BF16_LPT>>(a, stream);
+  if constexpr (KVT == PA_KV_U8_PER_TOKEN || KVT == PA_KV_FP8_PER_TOKEN)
+    if (a.ordered == 2) return launch_cfg<Config<D, P, KVT, PA_DECODE_STAGES_U8_LPT>>(a, stream);
   return launch_cfg<Config<D, P, KVT>>(a, stream);
 }
 
