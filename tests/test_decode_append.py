@@ -109,9 +109,11 @@ def test_fused_step_with_rows_of_huge_span(kind):
 def test_host_lengths_schedule_the_step_without_changing_it(kv):
     """pa_decode_append with host_context_lens: a ragged batch over several
     waves (64 sequences x 8 KV heads for 444 slots) runs one split, longest
-    context first. The output equals the one-split step bit for bit (the same
-    CTAs, launched in another order) and the oracle within 2e-3; host lengths
-    that are wrong (reversed) change only the schedule."""
+    context first (bf16, INT8 and FP8 with a deeper shared-memory ring). The
+    output equals the plain one-split step bit for bit (the same arithmetic
+    per CTA, launched in another order from another ring depth) and the
+    oracle within 2e-3; host lengths that are wrong (reversed) change only
+    the schedule."""
     w = W.llama8b(B=64, ctx_range=(242, 4095), kv=kv,
                   outlier_frac=0.01 if kv != "bf16" else 0.0)
     k_new, v_new = w.step_rows_by_sequence()
