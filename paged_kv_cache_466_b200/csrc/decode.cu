@@ -584,9 +584,9 @@ __device__ __forceinline__ void scores_t(const LaneMap<D, KVT> &lm, uint32_t src
         const uint32_t a0 = kIsFp8<KVT> ? e4m3x2_to_f16x2(w0[w]) : u8x2_to_f16x2(w0[w], 0x4140);
         const uint32_t a1 = kIsFp8<KVT> ? e4m3x2_to_f16x2(w1[w]) : u8x2_to_f16x2(w1[w], 0x4140);
         const uint32_t a2 =
-            kIsFp8<KVT> ? e4m3x2_to_f16x2(w0[w] >> 16) : u8x2_to_f16x2(w0[w], 0x4342);
+            kIsFp8<KVT> ? e4m3x2_hi_to_f16x2(w0[w]) : u8x2_to_f16x2(w0[w], 0x4342);
         const uint32_t a3 =
-            kIsFp8<KVT> ? e4m3x2_to_f16x2(w1[w] >> 16) : u8x2_to_f16x2(w1[w], 0x4342);
+            kIsFp8<KVT> ? e4m3x2_hi_to_f16x2(w1[w]) : u8x2_to_f16x2(w1[w], 0x4342);
         mma_f16_16816((w & 1) ? s2 : s, a0, a1, a2, a3, qa[4 * i + w][0], qa[4 * i + w][1]);
       }
     }
@@ -657,9 +657,9 @@ __device__ __forceinline__ void pv_quant(const LaneMap<D, KVT> &lm, uint32_t src
       const uint32_t xa = __byte_perm(w0, w1, sel);
       const uint32_t xb = __byte_perm(w2, w3, sel);
       const uint32_t a0 = kIsFp8<KVT> ? e4m3x2_to_f16x2(xa) : u8x2_to_f16x2(xa, 0x4140);
-      const uint32_t a1 = kIsFp8<KVT> ? e4m3x2_to_f16x2(xa >> 16) : u8x2_to_f16x2(xa, 0x4342);
+      const uint32_t a1 = kIsFp8<KVT> ? e4m3x2_hi_to_f16x2(xa) : u8x2_to_f16x2(xa, 0x4342);
       const uint32_t a2 = kIsFp8<KVT> ? e4m3x2_to_f16x2(xb) : u8x2_to_f16x2(xb, 0x4140);
-      const uint32_t a3 = kIsFp8<KVT> ? e4m3x2_to_f16x2(xb >> 16) : u8x2_to_f16x2(xb, 0x4342);
+      const uint32_t a3 = kIsFp8<KVT> ? e4m3x2_hi_to_f16x2(xb) : u8x2_to_f16x2(xb, 0x4342);
       mma_f16_16816(o[j], a0, a1, a2, a3, bh0, bh1);
       if constexpr (kTwo) mma_f16_16816(o[j], a0, a1, a2, a3, bl0, bl1);
     }

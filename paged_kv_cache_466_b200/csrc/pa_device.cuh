@@ -176,6 +176,15 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t pair) {
       : "r"(pair));
   return r;
 }
+// The same for the two codes in bits 16..31 (the upper half of the register,
+// read in place: no shift).
+__device__ __forceinline__ uint32_t e4m3x2_hi_to_f16x2(uint32_t pair) {
+  uint32_t r;
+  asm("{\n .reg .b16 lo, hi;\n mov.b32 {lo, hi}, %1;\n cvt.rn.f16x2.e4m3x2 %0, hi;\n}\n"
+      : "=r"(r)
+      : "r"(pair));
+  return r;
+}
 
 // Two fp32 -> two E4M3 codes (round to nearest even, saturate to +-448), the
 // code of `lo` in bits 0..7.
